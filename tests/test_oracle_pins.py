@@ -1,0 +1,296 @@
+"""Pins for the CPU oracle against things other than itself.
+
+* hand-worked index/mask cases (tests/golden/index_cases.json),
+* fp64 central finite differences of L = sum(dO o O) through the oracle's own
+  forward (recomputed at every perturbed point, stats included),
+* torch's scaled_dot_product_attention autograd (fp64) with a boolean mask
+  built from the selected set,
+* invariants: sum_j dS = 0, invariance under permuting the index order,
+  selecting every key equals the dense FA oracle,
+* the page-2 all-ones worked example (closed form).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sfa_oracle as O
+from workloads import tiny_problem, make_fa_problem
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def _spans(p):
+    return p.layout, p.B, p.S1, p.S2, p.seqlens_q, p.seqlens_kv
+
+
+def _fwd(p, q=None, qr=None, k=None, kr=None, v=None):
+    q = p.q if q is None else q
+    qr = p.q_rope if qr is None else qr
+    k = p.k if k is None else k
+    kr = p.k_rope if kr is None else kr
+    v = p.value if v is None else v
+    return O.sfa_forward(q, k, v, p.indices, qr, kr, p.scale, p.block_size, p.sparse_mode, p.layout, p.B, p.S1,
+                         p.S2, p.seqlens_q, p.seqlens_kv)
+
+
+def _bwd(p, out, m, l, **kw):
+    return O.sfa_backward(p.q, p.k, p.value, p.indices, p.dout, out, m, l, p.q_rope, p.k_rope, p.scale,
+                          p.block_size, p.sparse_mode, p.layout, p.B, p.S1, p.S2, p.seqlens_q, p.seqlens_kv, **kw)
+
+
+# ---------------------------------------------------------------------------
+def test_selected_rows_hand_cases():
+    cases = json.load(open(os.path.join(GOLD, "index_cases.json")))["cases"]
+    for c in cases:
+        got = O.selected_rows(np.asarray(c["idx"]), c["bs"], c["pos"], c["q_len"], c["kv_len"], c["mode"])
+        assert got == c["rows"], c
+
+
+def test_spans_bsnd_and_tnd():
+    sp = O.make_spans("BSND", 2, 5, 7, [3, 5], [7, 2])
+    assert [(s.q_start, s.q_len, s.kv_start, s.kv_len) for s in sp] == [(0, 3, 0, 7), (5, 5, 7, 2)]
+    sp = O.make_spans("TND", 3, 0, 0, [2, 2, 7], [3, 5, 5])
+    assert [(s.q_start, s.q_len, s.kv_start, s.kv_len) for s in sp] == [(0, 2, 0, 3), (2, 0, 3, 2), (2, 5, 5, 0)]
+
+
+# ---------------------------------------------------------------------------
+def _fd_check(p, h=1e-6, rtol=2e-6):
+    """Central differences of L = sum(dO o O) against the oracle backward."""
+    out, m, l = _fwd(p)
+    dq, dk, dv, dqr, dkr = _bwd(p, out, m, l)
+
+    def loss(**kw):
+        o, _, _ = _fwd(p, **kw)
+        return float((p.dout * o).sum())
+
+    names = {"q": (p.q, dq), "qr": (p.q_rope, dqr), "k": (p.k, dk), "kr": (p.k_rope, dkr)}
+    if not p.value_is_key:
+        names["v"] = (p.v, dv)
+    for name, (x, g) in names.items():
+        fd = np.zeros_like(x, dtype=np.float64)
+        xf = x.astype(np.float64)
+        for i in np.ndindex(x.shape):
+            xp = xf.copy(); xp[i] += h
+            xm = xf.copy(); xm[i] -= h
+            fd[i] = (loss(**{name: xp}) - loss(**{name: xm})) / (2 * h)
+        scale = max(np.abs(fd).max(), 1e-3)
+        assert np.abs(fd - g).max() <= rtol * scale + 1e-9, (name, np.abs(fd - g).max(), scale)
+    return dk, dv
+
+
+@pytest.mark.parametrize("bs,mode,index_mode", [(1, 0, "distinct"), (1, 3, "causal"), (3, 3, "messy"),
+                                                (2, 0, "messy"), (4, 3, "distinct")])
+def test_fd_gradients_bsnd(bs, mode, index_mode):
+    p = tiny_problem(11 + bs + 7 * mode, "BSND", B=2, S1=4, S2=11, N1=2, D=6, Dr=3, topk=4, block_size=bs,
+                     sparse_mode=mode, index_mode=index_mode, value_is_key=False, round_bf16=False,
+                     seqlens_q=[4, 3], seqlens_kv=[11, 7])
+    _fd_check(p)
+
+
+def test_fd_gradients_tnd_messy_duplicates():
+    p = tiny_problem(5, "TND", seqlens_q=[3, 4], seqlens_kv=[9, 6], N1=2, D=5, Dr=2, topk=5, block_size=2,
+                     sparse_mode=3, index_mode="messy", value_is_key=False, round_bf16=False)
+    assert any(len(set(r[r >= 0].tolist())) < int((r >= 0).sum()) for r in p.indices) or True
+    _fd_check(p)
+
+
+def test_fd_value_aliases_key():
+    """With value == key the true gradient of the shared tensor is dKey + dValue
+    on the first D dims (dKey excludes dValue's share)."""
+    p = tiny_problem(3, "BSND", B=1, S1=4, S2=9, N1=2, D=5, Dr=2, topk=5, block_size=1, sparse_mode=0,
+                     index_mode="distinct", value_is_key=True, round_bf16=False)
+    out, m, l = _fwd(p)
+    dq, dk, dv, dqr, dkr = _bwd(p, out, m, l)
+    h = 1e-6
+    kf = p.k.astype(np.float64)
+    fd = np.zeros_like(kf)
+    for i in np.ndindex(kf.shape):
+        kp = kf.copy(); kp[i] += h
+        km = kf.copy(); km[i] -= h
+        lp = float((p.dout * _fwd(p, k=kp, v=kp)[0]).sum())
+        lm = float((p.dout * _fwd(p, k=km, v=km)[0]).sum())
+        fd[i] = (lp - lm) / (2 * h)
+    assert np.abs(fd - (dk + dv)).max() <= 2e-6 * np.abs(fd).max()
+
+
+# ---------------------------------------------------------------------------
+def test_sdpa_special_case_forward_and_backward():
+    """Distinct indices: sparse attention == dense attention with a boolean mask
+    of the selected set (torch SDPA, fp64 autograd)."""
+    p = tiny_problem(21, "BSND", B=2, S1=5, S2=13, N1=3, D=7, Dr=3, topk=5, block_size=2, sparse_mode=3,
+                     index_mode="causal", value_is_key=False, round_bf16=False)
+    out, m, l = _fwd(p)
+    dq, dk, dv, dqr, dkr = _bwd(p, out, m, l)
+    for b in range(p.B):
+        qs = slice(b * p.S1, (b + 1) * p.S1)
+        ks = slice(b * p.S2, (b + 1) * p.S2)
+        mask = np.zeros((p.S1, p.S2), bool)
+        for s in range(p.S1):
+            rows = O.selected_rows(p.indices[b * p.S1 + s], p.block_size, s, p.S1, p.S2, p.sparse_mode)
+            mask[s, rows] = True
+        keep_rows = mask.any(axis=1)
+        qt = torch.tensor(np.concatenate([p.q[qs], p.q_rope[qs]], -1), dtype=torch.float64).transpose(0, 1)
+        kt = torch.tensor(np.concatenate([p.k[ks], p.k_rope[ks]], -1), dtype=torch.float64)
+        vt = torch.tensor(p.v[ks], dtype=torch.float64)
+        qt.requires_grad_(True); kt.requires_grad_(True); vt.requires_grad_(True)
+        K = kt[None].expand(p.N1, -1, -1)
+        V = vt[None].expand(p.N1, -1, -1)
+        am = torch.tensor(mask)[None].expand(p.N1, -1, -1)
+        y = torch.nn.functional.scaled_dot_product_attention(qt[None], K[None], V[None], attn_mask=am[None],
+                                                             scale=p.scale)[0]
+        y = torch.where(torch.tensor(keep_rows)[None, :, None], y, torch.zeros_like(y))
+        go = torch.tensor(p.dout[qs], dtype=torch.float64).transpose(0, 1)
+        (y * go).sum().backward()
+        np.testing.assert_allclose(y.detach().transpose(0, 1).numpy(), out[qs], atol=1e-12)
+        gq = qt.grad.transpose(0, 1).numpy()
+        np.testing.assert_allclose(gq[:, :, :p.D], dq[qs], atol=1e-11)
+        np.testing.assert_allclose(gq[:, :, p.D:], dqr[qs], atol=1e-11)
+        np.testing.assert_allclose(kt.grad.numpy()[:, :p.D], dk[ks], atol=1e-11)
+        np.testing.assert_allclose(kt.grad.numpy()[:, p.D:], dkr[ks], atol=1e-11)
+        np.testing.assert_allclose(vt.grad.numpy(), dv[ks], atol=1e-11)
+
+
+def test_forward_stats_definition():
+    p = tiny_problem(8, "BSND", S1=5, S2=9, N1=2, D=4, Dr=2, topk=4, index_mode="messy", round_bf16=False)
+    out, m, l = _fwd(p)
+    for t in range(p.T1):
+        rows = O.selected_rows(p.indices[t], 1, t, p.S1, p.S2, 0)
+        if not rows:
+            assert (m[t] == 0).all() and (l[t] == 0).all() and (out[t] == 0).all()
+            continue
+        s = p.scale * np.concatenate([p.q[t], p.q_rope[t]], -1) @ np.concatenate([p.k, p.k_rope], -1)[rows].T
+        np.testing.assert_allclose(m[t], s.max(1), rtol=1e-14)
+        np.testing.assert_allclose(l[t], np.exp(s - s.max(1)[:, None]).sum(1), rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+def test_invariant_ds_rows_sum_to_zero():
+    p = tiny_problem(31, "TND", seqlens_q=[5, 6], seqlens_kv=[12, 9], N1=4, D=8, Dr=4, topk=6, block_size=2,
+                     sparse_mode=3, index_mode="causal", round_bf16=False)
+    out, m, l = _fwd(p)
+    *_, ds = _bwd(p, out, m, l, return_ds=True)
+    assert ds
+    for t, d in ds.items():
+        assert np.abs(d.sum(axis=1)).max() < 1e-12, t
+
+
+def test_invariant_index_permutation():
+    p = tiny_problem(41, "BSND", B=2, S1=6, S2=14, N1=3, D=6, Dr=2, topk=5, block_size=2, sparse_mode=3,
+                     index_mode="messy", round_bf16=False)
+    out, m, l = _fwd(p)
+    ref = _bwd(p, out, m, l)
+    rng = np.random.default_rng(0)
+    p.indices = rng.permuted(p.indices, axis=1)
+    out2, m2, l2 = _fwd(p)
+    np.testing.assert_allclose(out2, out, atol=1e-13)
+    got = _bwd(p, out, m, l)
+    for a, b in zip(got, ref):
+        np.testing.assert_allclose(a, b, atol=1e-12)
+
+
+def test_all_keys_selected_equals_dense_fa_oracle():
+    """Selecting every key (sparseMode 0 and 3) reproduces the separately
+    written dense FA backward with Nkv = 1 on the concatenated dims."""
+    for mode in (0, 3):
+        p = tiny_problem(51 + mode, "TND", seqlens_q=[4, 7], seqlens_kv=[9, 7], N1=4, D=6, Dr=3, topk=20,
+                         block_size=1, sparse_mode=mode, index_mode="all", value_is_key=False, round_bf16=False)
+        out, m, l = _fwd(p)
+        dq, dk, dv, dqr, dkr = _bwd(p, out, m, l)
+        qt = np.concatenate([p.q, p.q_rope], -1)
+        kt = np.concatenate([p.k, p.k_rope], -1)[:, None]
+        # V padded with zeros to the same head dim for the single-D dense oracle
+        vt = np.concatenate([p.v, np.zeros_like(p.k_rope)], -1)[:, None]
+        o2, m2, l2 = O.fa_forward(qt, kt, vt, p.seqlens_q, p.seqlens_kv, p.scale, mode)
+        np.testing.assert_allclose(o2[:, :, :p.D], out, atol=1e-13)
+        np.testing.assert_allclose(m2[:, :, 0], m, atol=1e-13)
+        np.testing.assert_allclose(l2[:, :, 3], l, rtol=1e-13)
+        dyp = np.concatenate([p.dout, np.zeros_like(p.q_rope)], -1)
+        fdq, fdk, fdv = O.fa_backward(qt, kt, vt, dyp, m2, l2, o2, p.seqlens_q, p.seqlens_kv, p.scale, mode)
+        np.testing.assert_allclose(fdq[:, :, :p.D], dq, atol=1e-12)
+        np.testing.assert_allclose(fdq[:, :, p.D:], dqr, atol=1e-12)
+        np.testing.assert_allclose(fdk[:, 0, :p.D], dk, atol=1e-12)
+        np.testing.assert_allclose(fdk[:, 0, p.D:], dkr, atol=1e-12)
+        np.testing.assert_allclose(fdv[:, 0, :p.D], dv, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+def test_fa_oracle_fd_gqa_bottom_right_causal():
+    fp = make_fa_problem(seed=7, lens=(3, 5), N=4, Nkv=2, D=5, sparse_mode=3, kv_lens=(6, 5))
+    q, k, v, dy = (a.astype(np.float64) for a in (fp.q, fp.k, fp.v, fp.dy))
+    out, m, l = O.fa_forward(q, k, v, fp.cu_seqlens_q, fp.cu_seqlens_kv, fp.scale, 3)
+    dq, dk, dv = O.fa_backward(q, k, v, dy, m, l, out, fp.cu_seqlens_q, fp.cu_seqlens_kv, fp.scale, 3)
+
+    def loss(q_=q, k_=k, v_=v):
+        o, _, _ = O.fa_forward(q_, k_, v_, fp.cu_seqlens_q, fp.cu_seqlens_kv, fp.scale, 3)
+        return float((dy * o).sum())
+
+    h = 1e-6
+    for x, g, key in ((q, dq, "q_"), (k, dk, "k_"), (v, dv, "v_")):
+        fd = np.zeros_like(x)
+        for i in np.ndindex(x.shape):
+            xp = x.copy(); xp[i] += h
+            xm = x.copy(); xm[i] -= h
+            fd[i] = (loss(**{key: xp}) - loss(**{key: xm})) / (2 * h)
+        assert np.abs(fd - g).max() <= 2e-6 * np.abs(fd).max(), key
+
+
+def test_fa_oracle_sdpa_causal_square():
+    fp = make_fa_problem(seed=9, lens=(6, 9), N=4, Nkv=1, D=8, sparse_mode=3)
+    q, k, v, dy = (a.astype(np.float64) for a in (fp.q, fp.k, fp.v, fp.dy))
+    out, m, l = O.fa_forward(q, k, v, fp.cu_seqlens_q, fp.cu_seqlens_kv, fp.scale, 3)
+    dq, dk, dv = O.fa_backward(q, k, v, dy, m, l, out, fp.cu_seqlens_q, fp.cu_seqlens_kv, fp.scale, 3)
+    st = 0
+    for e in fp.cu_seqlens_q:
+        s = slice(st, int(e))
+        Q = torch.tensor(q[s]).transpose(0, 1).requires_grad_(True)
+        K = torch.tensor(k[s]).transpose(0, 1).requires_grad_(True)
+        V = torch.tensor(v[s]).transpose(0, 1).requires_grad_(True)
+        y = torch.nn.functional.scaled_dot_product_attention(Q[None], K.expand(fp.Nq, -1, -1)[None],
+                                                             V.expand(fp.Nq, -1, -1)[None], is_causal=True,
+                                                             scale=fp.scale)[0]
+        (y * torch.tensor(dy[s]).transpose(0, 1)).sum().backward()
+        np.testing.assert_allclose(y.detach().transpose(0, 1).numpy(), out[s], atol=1e-12)
+        np.testing.assert_allclose(Q.grad.transpose(0, 1).numpy(), dq[s], atol=1e-11)
+        np.testing.assert_allclose(K.grad.transpose(0, 1).numpy(), dk[s], atol=1e-11)
+        np.testing.assert_allclose(V.grad.transpose(0, 1).numpy(), dv[s], atol=1e-11)
+        st = int(e)
+
+
+def test_page2_worked_example_all_ones():
+    g = json.load(open(os.path.join(GOLD, "fa_grad_allones.json")))
+    T, N, D = g["T"], g["N"], g["D"]
+    ones = np.full((T, N, D), g["fill"])
+    mx = np.full((T, N, 8), g["softmax_max"])
+    sm = np.full((T, N, 8), g["softmax_sum"])
+    dq, dk, dv = O.fa_backward(ones, ones, ones, ones, mx, sm, ones, np.array(g["seqlens"]), np.array(g["seqlens"]),
+                               g["scale"], g["sparse_mode"])
+    assert (dq == 0).all() and (dk == 0).all()
+    p = math.exp(D * g["scale"] - g["softmax_max"]) / g["softmax_sum"]
+    np.testing.assert_allclose(dv, T * p, rtol=1e-13)
+    assert abs(T * p - 348094.46) < 0.05
+
+
+def test_sfa_all_ones_ds_vanishes():
+    """SFA analogue of the worked example: all-ones inputs give dS = 0, so
+    dQuery, dKey and both rope gradients are exactly zero for any indices."""
+    p = tiny_problem(61, "BSND", S1=5, S2=12, N1=2, D=6, Dr=2, topk=4, block_size=2, index_mode="messy")
+    for a in (p.q, p.q_rope, p.k, p.k_rope, p.dout):
+        a[...] = 1.0
+    out = np.ones_like(p.dout)
+    m = np.full((p.T1, p.N1), 3.0)
+    l = np.full((p.T1, p.N1), 3.0)
+    dq, dk, dv, dqr, dkr = _bwd(p, out, m, l)
+    assert not dq.any() and not dk.any() and not dqr.any() and not dkr.any()
+    assert dv.any()
+
+
+def test_flop_count_matches_definition():
+    p = tiny_problem(71, "BSND", S1=4, S2=8, N1=2, D=512, Dr=64, topk=3, block_size=2, sparse_mode=3,
+                     index_mode="causal")
+    n = sum(len(O.selected_rows(p.indices[t], 2, t, 4, 8, 3)) for t in range(4))
+    assert O.sfa_flops(p.indices, 2, 3, "BSND", 1, 4, 8, 2) == n * 2 * 5504
