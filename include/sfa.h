@@ -1,0 +1,242 @@
+/*
+ * sfa.h - C ABI of libsfa: top-k sparse attention backward (SparseFlashAttentionGrad)
+ * and the dense varlen FlashAttention backward (FlashAttentionUnpaddingScoreGrad)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor argument is a DEVICE pointer to densely packed (contiguous,
+ *    row-major) memory in the layout stated for it, unless the comment says
+ *    "host".  The caller owns every buffer: inputs, outputs and workspace.
+ *    The library allocates nothing and never synchronizes the stream.
+ *  - Inputs are never written.  `value` may be the same pointer as `key`.
+ *  - Outputs are fully overwritten (no accumulation into caller memory).
+ *  - Two phases, as in the aclnn convention of the FlashAttentionUnpaddingScoreGrad
+ *    page (函数原型 / 返回值): *_workspace_size() validates the arguments on the host
+ *    and returns the workspace size; the compute call re-validates, then enqueues
+ *    kernels on `stream` (a cudaStream_t; NULL = legacy default stream) and returns.
+ *  - Errors are reported before any launch and leave outputs untouched:
+ *      SFA_ERR_NULLPTR   a required pointer is NULL
+ *      SFA_ERR_INVALID   shape / attribute outside the supported set
+ *      SFA_ERR_WORKSPACE workspace_bytes smaller than the size query returned
+ *      SFA_ERR_CUDA      a CUDA launch or copy failed (see sfa_last_error_string)
+ *  - Out-of-range sparse index values and inconsistent sequence lengths are
+ *    masked on the device (the affected keys are skipped); they never fault.
+ *  - Not thread-safe for concurrent calls that share one workspace.
+ */
+#ifndef SFA_H_
+#define SFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t sfa_status;
+#define SFA_OK 0
+#define SFA_ERR_NULLPTR 161001   /* same codes as ACLNN_ERR_PARAM_NULLPTR / _INVALID */
+#define SFA_ERR_INVALID 161002
+#define SFA_ERR_WORKSPACE 161003
+#define SFA_ERR_CUDA 161004
+#define SFA_ERR_TIMEOUT 161005
+
+#define SFA_LAYOUT_BSND 0
+#define SFA_LAYOUT_TND 1
+
+#define SFA_DTYPE_BF16 0
+#define SFA_DTYPE_FP16 1
+
+typedef struct CUstream_st *sfa_stream_t; /* == cudaStream_t */
+
+/*
+ * Problem sizes of a sparse attention call (SparseFlashAttentionGrad README,
+ * 参数说明 and 约束说明).
+ *   layout  SFA_LAYOUT_BSND: query [B,S1,N1,D], key/value [B,S2,N2,D],
+ *                            queryRope [B,S1,N1,Dr], keyRope [B,S2,N2,Dr],
+ *                            sparseIndices [B,S1,N2,topk], softmax stats [B,S1,N1];
+ *                            T1/T2 are ignored (taken as B*S1, B*S2).
+ *           SFA_LAYOUT_TND:  query [T1,N1,D], key/value [T2,N2,D], queryRope
+ *                            [T1,N1,Dr], keyRope [T2,N2,Dr], sparseIndices
+ *                            [T1,N2,topk], softmax stats [T1,N1]; S1/S2 ignored.
+ *   dtype   SFA_DTYPE_BF16 or SFA_DTYPE_FP16 for every 16-bit tensor.
+ *   Supported: N2 = 1, D = 512, Dr = 64, N1 in {1,2,4,...,128}, B in [1,256],
+ *   S1, S2 (or per-sequence lengths) in [1, 128K], topk >= 1.
+ */
+typedef struct sfa_shape {
+    int32_t layout;
+    int32_t dtype;
+    int64_t B;
+    int64_t S1, S2;
+    int64_t T1, T2;
+    int64_t N1, N2;
+    int64_t D, Dr;
+    int64_t topk;
+} sfa_shape;
+
+/* ------------------------------------------------------------------------- */
+/* Sparse attention backward                                                  */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Phase 1 of sfa_grad: validate `shape` and the attributes, return the device
+ * workspace size in *workspace_bytes.  Host only, no device work.
+ * sparse_mode: 0 (no mask) or 3 (lower triangle split at the right vertex,
+ * i.e. key j kept for query position i iff j <= i + S2_b - S1_b), per the
+ * 约束说明 of the SparseFlashAttentionGrad README.
+ */
+sfa_status sfa_grad_workspace_size(const sfa_shape *shape, int64_t sparse_block_size, int64_t sparse_mode,
+                                   int32_t deterministic, size_t *workspace_bytes);
+
+/*
+ * Phase 2: the training backward of top-k sparse attention (SparseFlashAttentionGrad
+ * README, 功能说明): per query token, gather the key/value rows named by
+ * sparseIndices in blocks of sparse_block_size, recompute
+ *     P  = exp(scale * [q||qRope].[k||kRope]^T - softmaxMax) / softmaxSum,
+ * then dP = dOut.V^T, dS = P o (dP - rowsum(dOut o out)),
+ *      dQuery||dQueryRope = scale * dS.[k||kRope],
+ *      dKey||dKeyRope    += scale * dS^T.[q||qRope],   dValue += P^T.dOut,
+ * the key-side sums scatter-added in fp32 and cast once at the end.
+ *
+ *   query, query_rope, d_out, out   [.., N1, D|Dr] 16-bit, see sfa_shape
+ *   key, value, key_rope            [.., N2=1, D|Dr] 16-bit; value may == key
+ *   sparse_indices                  int32 [.., N2, topk]; entry i selects rows
+ *                                   [i*bs, i*bs+bs) of the token's own batch
+ *                                   (BSND) or sequence (TND); negative entries
+ *                                   and blocks starting at/after S2_b are skipped,
+ *                                   duplicates count with multiplicity
+ *   softmax_max, softmax_sum        fp32 [.., N1]: max of the scaled scores and
+ *                                   sum of exp(scaled - max) from the forward,
+ *                                   used as given; softmax_sum == 0 gives P = 0
+ *   actual_seq_lengths_q / _kv      int32, device.  BSND: per-batch valid lengths
+ *                                   (length B) or NULL for S1/S2.  TND: required,
+ *                                   cumulative end offsets (length B, last = T1/T2)
+ *   scale                           scaleValue (applied in S, dQuery, dKey)
+ *   pre_tokens, next_tokens         accepted and ignored (no effect for modes 0/3)
+ *   deterministic                   0: fp32 atomic scatter (run-to-run order may
+ *                                   differ); 1: bit-identical results run to run
+ *                                   (64-bit fixed-point scatter, 32 fraction bits;
+ *                                   every partial sum of a dKey/dValue element
+ *                                   must stay below 2^31 in magnitude)
+ *   workspace, workspace_bytes      >= sfa_grad_workspace_size(); 256-byte aligned
+ *   d_query, d_query_rope           [.., N1, D|Dr] 16-bit outputs; rows of BSND
+ *                                   padding tokens (position >= S1_b) are zero
+ *   d_key, d_value, d_key_rope      [.., N2, D|Dr] 16-bit outputs; d_key excludes
+ *                                   d_value's share even when value == key
+ */
+sfa_status sfa_grad(const void *query, const void *key, const void *value, const int32_t *sparse_indices,
+                    const void *d_out, const void *out, const float *softmax_max, const float *softmax_sum,
+                    const int32_t *actual_seq_lengths_q, const int32_t *actual_seq_lengths_kv,
+                    const void *query_rope, const void *key_rope, float scale, int64_t sparse_block_size,
+                    int64_t sparse_mode, int64_t pre_tokens, int64_t next_tokens, int32_t deterministic,
+                    const sfa_shape *shape, void *workspace, size_t workspace_bytes, sfa_stream_t stream,
+                    void *d_query, void *d_key, void *d_value, void *d_query_rope, void *d_key_rope);
+
+/* ------------------------------------------------------------------------- */
+/* Sparse attention forward (produces the inputs `out`, softmax_max/_sum)     */
+/* ------------------------------------------------------------------------- */
+
+sfa_status sfa_fwd_workspace_size(const sfa_shape *shape, int64_t sparse_block_size, int64_t sparse_mode,
+                                  size_t *workspace_bytes);
+
+/*
+ * Forward of the same attention (FlashAttentionUnpaddingScoreGrad page, 计算公式:
+ * S = scale*Q.K^T, P = Softmax(S), Y = P.V) over the gathered rows:
+ *   out [.., N1, D] 16-bit, softmax_max / softmax_sum fp32 [.., N1] (max of the
+ *   scaled scores, sum of exp(scaled - max)).  A query row with no valid key
+ *   gets out = 0, softmax_max = 0, softmax_sum = 0.  Arguments as in sfa_grad.
+ */
+sfa_status sfa_fwd(const void *query, const void *key, const void *value, const int32_t *sparse_indices,
+                   const int32_t *actual_seq_lengths_q, const int32_t *actual_seq_lengths_kv,
+                   const void *query_rope, const void *key_rope, float scale, int64_t sparse_block_size,
+                   int64_t sparse_mode, const sfa_shape *shape, void *workspace, size_t workspace_bytes,
+                   sfa_stream_t stream, void *out, float *softmax_max, float *softmax_sum);
+
+/* ------------------------------------------------------------------------- */
+/* Hot-path sub-steps, exported for bit-exact testing and reuse               */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Index compaction (the Gather of the SparseFlashAttentionGrad README, 功能说明,
+ * with the sparseMode mask of its 约束说明): for each query row t, copy the valid
+ * block indices of sparse_indices[t, 0, :] in their original order to
+ * blocks_out[t*topk + 0 .. n-1] (the rest is left unwritten), the count n to
+ * nblocks_out[t] and the number of valid key rows (after the S2_b cut and the
+ * mode-3 causal cut, row by row) to nrows_out[t].  A block is valid iff its
+ * index i >= 0, i*bs < S2_b and, in mode 3, i*bs <= pos + S2_b - S1_b.  BSND
+ * padding rows (position >= S1_b) get n = 0.  All outputs int32, device.
+ */
+sfa_status sfa_compact_indices(const int32_t *sparse_indices, const int32_t *actual_seq_lengths_q,
+                               const int32_t *actual_seq_lengths_kv, int64_t sparse_block_size, int64_t sparse_mode,
+                               const sfa_shape *shape, sfa_stream_t stream, int32_t *blocks_out,
+                               int32_t *nblocks_out, int32_t *nrows_out);
+
+/*
+ * FlashSoftmaxGrad(dO, O) of stage 2 (SparseFlashAttentionGrad README): the fp32
+ * row sum over the D value dims of dOut o out, one value per (query row, head):
+ * rowsum_out fp32 [T1, N1] (BSND: [B*S1, N1]).
+ */
+sfa_status sfa_softmax_grad_rowsum(const void *d_out, const void *out, const sfa_shape *shape, sfa_stream_t stream,
+                                   float *rowsum_out);
+
+/* ------------------------------------------------------------------------- */
+/* Dense varlen FlashAttention backward (TND), FlashAttentionUnpaddingScoreGrad */
+/* ------------------------------------------------------------------------- */
+
+typedef struct fa_shape {
+    int32_t dtype; /* SFA_DTYPE_BF16 | SFA_DTYPE_FP16 */
+    int32_t reserved;
+    int64_t B;     /* number of sequences */
+    int64_t T1, T2;
+    int64_t Nq, Nkv; /* Nq % Nkv == 0 (GQA), 1..256 */
+    int64_t D;       /* head dim, multiple of 8, 8..256 */
+} fa_shape;
+
+sfa_status fa_grad_workspace_size(const fa_shape *shape, int64_t sparse_mode, int32_t deterministic,
+                                  size_t *workspace_bytes);
+
+/*
+ * aclnnFlashAttentionUnpaddingScoreGrad (计算公式): with S = scale*Q.K^T (kept pairs
+ * only), P = exp(S - softmaxMax)/softmaxSum, dV = P^T.dY,
+ * dS = P o (dY.V^T - rowsum(dY o attentionIn)), dQ = scale*dS.K, dK = scale*dS^T.Q;
+ * query head h uses kv head h / (Nq/Nkv) and kv gradients sum over their heads.
+ *   q, dy, attention_in [T1, Nq, D]; k, v [T2, Nkv, D]; dq [T1,Nq,D]; dk, dv
+ *   [T2,Nkv,D] (16-bit).  softmax_max / softmax_sum fp32 [T1, Nq, 8] (8 equal
+ *   copies, lane 0 read), as in 关于softmaxMax与softmaxSum参数的约束.
+ *   actual_seq_qlen / actual_seq_kvlen: HOST int64 arrays of length B holding
+ *   cumulative end offsets (last = T1 / T2); copied into the workspace before
+ *   the call returns.  keep_prob must be 1 (no dropout); pre/next_tokens are
+ *   ignored for sparse_mode 0 / 3; head_num must equal Nq.
+ */
+sfa_status fa_grad(const void *q, const void *k, const void *v, const void *dy, const float *softmax_max,
+                   const float *softmax_sum, const void *attention_in, const int64_t *actual_seq_qlen,
+                   const int64_t *actual_seq_kvlen, double scale, double keep_prob, int64_t pre_tokens,
+                   int64_t next_tokens, int64_t head_num, int64_t sparse_mode, int32_t deterministic,
+                   const fa_shape *shape, void *workspace, size_t workspace_bytes, sfa_stream_t stream, void *dq,
+                   void *dk, void *dv);
+
+sfa_status fa_fwd_workspace_size(const fa_shape *shape, int64_t sparse_mode, size_t *workspace_bytes);
+
+/* Forward of the dense attention above: out [T1,Nq,D] 16-bit, softmax_max /
+ * softmax_sum fp32 [T1, Nq, 8] (8 equal copies).  Host cumulative seqlens as in fa_grad. */
+sfa_status fa_fwd(const void *q, const void *k, const void *v, const int64_t *actual_seq_qlen,
+                  const int64_t *actual_seq_kvlen, double scale, int64_t sparse_mode, const fa_shape *shape,
+                  void *workspace, size_t workspace_bytes, sfa_stream_t stream, void *out, float *softmax_max,
+                  float *softmax_sum);
+
+/* ------------------------------------------------------------------------- */
+/* Diagnostics                                                                */
+/* ------------------------------------------------------------------------- */
+
+/* Static string naming a status code. */
+const char *sfa_status_string(sfa_status status);
+/* Message of the last error on the calling thread ("" if none). */
+const char *sfa_last_error_string(void);
+/* Library version, "major.minor.patch". */
+const char *sfa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SFA_H_ */

@@ -1,0 +1,16 @@
+"""B200 (sm_100a) top-k sparse attention backward (SparseFlashAttentionGrad) and dense
+varlen FlashAttention backward, behind the C ABI of libsfa (include/sfa.h)."""
+from ._native import SfaError, load  # noqa: F401
+from .ops import (  # noqa: F401
+    compact_indices,
+    fa_fwd,
+    fa_grad,
+    sfa_fwd,
+    sfa_grad,
+    sfa_grad_workspace_size,
+    sfa_shape,
+    softmax_grad_rowsum,
+)
+
+__all__ = ["sfa_grad", "sfa_fwd", "fa_grad", "fa_fwd", "compact_indices", "softmax_grad_rowsum",
+           "sfa_grad_workspace_size", "sfa_shape", "SfaError", "load"]

@@ -1,0 +1,376 @@
+// C ABI of libsfa: argument validation, workspace sizing and kernel dispatch.
+// The argument set follows the SparseFlashAttentionGrad README (参数说明) and the
+// two-phase aclnn convention of aclnnFlashAttentionUnpaddingScoreGrad (函数原型).
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "sfa_internal.cuh"
+
+using namespace sfa;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sfa_status fail(sfa_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+sfa_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(SFA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define SFA_CUDA(expr, where)                              \
+    do {                                                   \
+        cudaError_t _e = (expr);                           \
+        if (_e != cudaSuccess) return cuda_fail(_e, where); \
+    } while (0)
+
+bool n1_supported(int64_t n) {
+    // 1/2/4/.../128 (SparseFlashAttentionGrad 约束说明) plus 3/6/12/24/48 (Ascend 950 list)
+    static const int64_t ok[] = {1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 48, 64, 128};
+    for (int64_t v : ok)
+        if (v == n) return true;
+    return false;
+}
+
+struct Sizes {
+    int64_t T1, T2;
+};
+
+sfa_status check_shape(const sfa_shape* s, int64_t bs, int64_t mode, Sizes* out) {
+    if (!s) return fail(SFA_ERR_NULLPTR, "shape is NULL");
+    if (s->layout != SFA_LAYOUT_BSND && s->layout != SFA_LAYOUT_TND)
+        return fail(SFA_ERR_INVALID, "layout %d: only BSND (0) or TND (1)", s->layout);
+    if (s->dtype != SFA_DTYPE_BF16 && s->dtype != SFA_DTYPE_FP16)
+        return fail(SFA_ERR_INVALID, "dtype %d: only bf16 (0) or fp16 (1)", s->dtype);
+    if (s->N2 != 1) return fail(SFA_ERR_INVALID, "N2=%lld: only 1 is supported", (long long)s->N2);
+    if (s->D != kD) return fail(SFA_ERR_INVALID, "D=%lld: only 512 is supported", (long long)s->D);
+    if (s->Dr != kDr) return fail(SFA_ERR_INVALID, "Dr=%lld: only 64 is supported", (long long)s->Dr);
+    if (!n1_supported(s->N1)) return fail(SFA_ERR_INVALID, "N1=%lld not supported", (long long)s->N1);
+    if (s->B < 1 || s->B > 256) return fail(SFA_ERR_INVALID, "B=%lld outside [1,256]", (long long)s->B);
+    if (s->topk < 1) return fail(SFA_ERR_INVALID, "topk=%lld < 1", (long long)s->topk);
+    if (bs < 1 || bs > (1 << 20)) return fail(SFA_ERR_INVALID, "sparse_block_size=%lld", (long long)bs);
+    if (mode != 0 && mode != 3) return fail(SFA_ERR_INVALID, "sparse_mode=%lld: only 0 or 3", (long long)mode);
+    const int64_t kMaxS = 128 * 1024;
+    if (s->layout == SFA_LAYOUT_BSND) {
+        if (s->S1 < 1 || s->S1 > kMaxS || s->S2 < 1 || s->S2 > kMaxS)
+            return fail(SFA_ERR_INVALID, "S1=%lld S2=%lld outside [1,128K]", (long long)s->S1, (long long)s->S2);
+        out->T1 = s->B * s->S1;
+        out->T2 = s->B * s->S2;
+    } else {
+        if (s->T1 < 1 || s->T2 < 1 || s->T1 > s->B * kMaxS || s->T2 > s->B * kMaxS)
+            return fail(SFA_ERR_INVALID, "T1=%lld T2=%lld out of range", (long long)s->T1, (long long)s->T2);
+        out->T1 = s->T1;
+        out->T2 = s->T2;
+    }
+    if (out->T1 * s->topk > (int64_t)INT32_MAX * 64)
+        return fail(SFA_ERR_INVALID, "T1*topk too large");
+    return SFA_OK;
+}
+
+SeqDesc seq_desc(const sfa_shape* s, const Sizes& z, const int32_t* sq, const int32_t* skv) {
+    SeqDesc d;
+    d.layout = s->layout;
+    d.B = (int32_t)s->B;
+    d.S1 = s->S1;
+    d.S2 = s->S2;
+    d.T1 = z.T1;
+    d.T2 = z.T2;
+    d.seq_q = sq;
+    d.seq_kv = skv;
+    return d;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sfa_version(void) { return "0.1.0"; }
+
+const char* sfa_last_error_string(void) { return g_last_error.c_str(); }
+
+const char* sfa_status_string(sfa_status st) {
+    switch (st) {
+        case SFA_OK: return "SFA_OK";
+        case SFA_ERR_NULLPTR: return "SFA_ERR_NULLPTR";
+        case SFA_ERR_INVALID: return "SFA_ERR_INVALID";
+        case SFA_ERR_WORKSPACE: return "SFA_ERR_WORKSPACE";
+        case SFA_ERR_CUDA: return "SFA_ERR_CUDA";
+        case SFA_ERR_TIMEOUT: return "SFA_ERR_TIMEOUT";
+        default: return "SFA_ERR_UNKNOWN";
+    }
+}
+
+sfa_status sfa_grad_workspace_size(const sfa_shape* shape, int64_t sparse_block_size, int64_t sparse_mode,
+                                   int32_t deterministic, size_t* workspace_bytes) {
+    g_last_error.clear();
+    if (!workspace_bytes) return fail(SFA_ERR_NULLPTR, "workspace_bytes is NULL");
+    Sizes z;
+    sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
+    if (st != SFA_OK) return st;
+    *workspace_bytes = grad_ws_layout(z.T1, z.T2, shape->N1, shape->topk, deterministic != 0,
+                                      fused_supported(shape->N1)).total;
+    return SFA_OK;
+}
+
+sfa_status sfa_grad(const void* query, const void* key, const void* value, const int32_t* sparse_indices,
+                    const void* d_out, const void* out, const float* softmax_max, const float* softmax_sum,
+                    const int32_t* actual_seq_lengths_q, const int32_t* actual_seq_lengths_kv,
+                    const void* query_rope, const void* key_rope, float scale, int64_t sparse_block_size,
+                    int64_t sparse_mode, int64_t pre_tokens, int64_t next_tokens, int32_t deterministic,
+                    const sfa_shape* shape, void* workspace, size_t workspace_bytes, sfa_stream_t stream,
+                    void* d_query, void* d_key, void* d_value, void* d_query_rope, void* d_key_rope) {
+    (void)pre_tokens;
+    (void)next_tokens;
+    g_last_error.clear();
+    Sizes z;
+    sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
+    if (st != SFA_OK) return st;
+    if (!query || !key || !value || !sparse_indices || !d_out || !out || !softmax_max || !softmax_sum ||
+        !query_rope || !key_rope || !d_query || !d_key || !d_value || !d_query_rope || !d_key_rope || !workspace)
+        return fail(SFA_ERR_NULLPTR, "a required tensor pointer is NULL");
+    if (shape->layout == SFA_LAYOUT_TND && (!actual_seq_lengths_q || !actual_seq_lengths_kv))
+        return fail(SFA_ERR_NULLPTR, "TND needs actual_seq_lengths_q and actual_seq_lengths_kv");
+    if (!(scale == scale)) return fail(SFA_ERR_INVALID, "scale is NaN");
+    if (((uintptr_t)workspace & 255u) != 0) return fail(SFA_ERR_INVALID, "workspace not 256-byte aligned");
+    const bool det = deterministic != 0;
+    const bool fused_shape = fused_supported(shape->N1);
+    const GradWs ws = grad_ws_layout(z.T1, z.T2, shape->N1, shape->topk, det, fused_shape);
+    if (workspace_bytes < ws.total)
+        return fail(SFA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, ws.total);
+    cudaStream_t s = (cudaStream_t)stream;
+    char* w = (char*)workspace;
+
+    GradArgs a;
+    a.q = query; a.qr = query_rope; a.k = key; a.kr = key_rope; a.v = value;
+    a.dout = d_out; a.out = out; a.smax = softmax_max; a.ssum = softmax_sum; a.idx = sparse_indices;
+    a.sd = seq_desc(shape, z, actual_seq_lengths_q, actual_seq_lengths_kv);
+    a.N1 = shape->N1; a.topk = shape->topk; a.bs = (int)sparse_block_size; a.mode = (int)sparse_mode;
+    a.scale = scale; a.det = det;
+    a.blocks = (int32_t*)(w + ws.blocks); a.nblk = (int32_t*)(w + ws.nblk); a.nrows = (int32_t*)(w + ws.nrows);
+    a.order = (int32_t*)(w + ws.order); a.rowsum = (float*)(w + ws.rowsum);
+    a.dkv_acc = w + ws.dkv; a.dq_acc = (float*)(w + ws.dq); a.ctrl = (int32_t*)(w + ws.ctrl);
+    a.dq = d_query; a.dqr = d_query_rope;
+
+    SFA_CUDA(cudaMemsetAsync(a.dkv_acc, 0, (size_t)z.T2 * kAccW * (det ? 8 : 4), s), "zero dK/dV accumulator");
+    SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, (int32_t*)a.blocks, (int32_t*)a.nblk,
+                            (int32_t*)a.nrows, s), "index compaction");
+    const bool fused = fused_shape && value == key;
+    if (fused) {
+        SFA_CUDA(cudaMemsetAsync(a.dq_acc, 0, (size_t)z.T1 * shape->N1 * kDK * 4, s), "zero dQ accumulator");
+        SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, z.T1, shape->N1, (float*)a.rowsum, s), "rowsum(dO*O)");
+        SFA_CUDA(launch_order(a.nrows, z.T1, (int32_t*)a.order, a.ctrl, s), "work order");
+        SFA_CUDA(launch_bwd_fused(shape->dtype, a, s), "fused backward");
+        SFA_CUDA(launch_cast_dq(shape->dtype, a.dq_acc, z.T1, shape->N1, d_query, d_query_rope, s), "cast dQuery");
+    } else {
+        SFA_CUDA(launch_bwd_generic(shape->dtype, a, s), "backward");
+    }
+    SFA_CUDA(launch_cast_dkv(shape->dtype, det, a.dkv_acc, z.T2, d_key, d_key_rope, d_value, s), "cast dKey/dValue");
+    return SFA_OK;
+}
+
+sfa_status sfa_fwd_workspace_size(const sfa_shape* shape, int64_t sparse_block_size, int64_t sparse_mode,
+                                  size_t* workspace_bytes) {
+    g_last_error.clear();
+    if (!workspace_bytes) return fail(SFA_ERR_NULLPTR, "workspace_bytes is NULL");
+    Sizes z;
+    sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
+    if (st != SFA_OK) return st;
+    *workspace_bytes = align256((size_t)z.T1 * shape->topk * 4) + 2 * align256((size_t)z.T1 * 4);
+    return SFA_OK;
+}
+
+sfa_status sfa_fwd(const void* query, const void* key, const void* value, const int32_t* sparse_indices,
+                   const int32_t* actual_seq_lengths_q, const int32_t* actual_seq_lengths_kv,
+                   const void* query_rope, const void* key_rope, float scale, int64_t sparse_block_size,
+                   int64_t sparse_mode, const sfa_shape* shape, void* workspace, size_t workspace_bytes,
+                   sfa_stream_t stream, void* out, float* softmax_max, float* softmax_sum) {
+    g_last_error.clear();
+    Sizes z;
+    sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
+    if (st != SFA_OK) return st;
+    if (!query || !key || !value || !sparse_indices || !query_rope || !key_rope || !out || !softmax_max ||
+        !softmax_sum || !workspace)
+        return fail(SFA_ERR_NULLPTR, "a required tensor pointer is NULL");
+    if (shape->layout == SFA_LAYOUT_TND && (!actual_seq_lengths_q || !actual_seq_lengths_kv))
+        return fail(SFA_ERR_NULLPTR, "TND needs actual_seq_lengths_q and actual_seq_lengths_kv");
+    size_t need = align256((size_t)z.T1 * shape->topk * 4) + 2 * align256((size_t)z.T1 * 4);
+    if (workspace_bytes < need) return fail(SFA_ERR_WORKSPACE, "workspace %zu < %zu", workspace_bytes, need);
+    cudaStream_t s = (cudaStream_t)stream;
+    char* w = (char*)workspace;
+    FwdArgs a;
+    a.q = query; a.qr = query_rope; a.k = key; a.kr = key_rope; a.v = value;
+    a.sd = seq_desc(shape, z, actual_seq_lengths_q, actual_seq_lengths_kv);
+    a.N1 = shape->N1; a.topk = shape->topk; a.bs = (int)sparse_block_size; a.mode = (int)sparse_mode;
+    a.scale = scale;
+    int32_t* blocks = (int32_t*)w;
+    int32_t* nblk = (int32_t*)(w + align256((size_t)z.T1 * shape->topk * 4));
+    int32_t* nrows = (int32_t*)((char*)nblk + align256((size_t)z.T1 * 4));
+    a.blocks = blocks; a.nblk = nblk;
+    a.out = out; a.smax = softmax_max; a.ssum = softmax_sum;
+    SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, blocks, nblk, nrows, s), "index compaction");
+    SFA_CUDA(launch_fwd_generic(shape->dtype, a, s), "forward");
+    return SFA_OK;
+}
+
+sfa_status sfa_compact_indices(const int32_t* sparse_indices, const int32_t* actual_seq_lengths_q,
+                               const int32_t* actual_seq_lengths_kv, int64_t sparse_block_size, int64_t sparse_mode,
+                               const sfa_shape* shape, sfa_stream_t stream, int32_t* blocks_out, int32_t* nblocks_out,
+                               int32_t* nrows_out) {
+    g_last_error.clear();
+    Sizes z;
+    sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
+    if (st != SFA_OK) return st;
+    if (!sparse_indices || !blocks_out || !nblocks_out || !nrows_out)
+        return fail(SFA_ERR_NULLPTR, "a required pointer is NULL");
+    if (shape->layout == SFA_LAYOUT_TND && (!actual_seq_lengths_q || !actual_seq_lengths_kv))
+        return fail(SFA_ERR_NULLPTR, "TND needs actual_seq_lengths_q and actual_seq_lengths_kv");
+    SeqDesc sd = seq_desc(shape, z, actual_seq_lengths_q, actual_seq_lengths_kv);
+    SFA_CUDA(launch_compact(sparse_indices, sd, shape->topk, (int)sparse_block_size, (int)sparse_mode, blocks_out,
+                            nblocks_out, nrows_out, (cudaStream_t)stream), "index compaction");
+    return SFA_OK;
+}
+
+sfa_status sfa_softmax_grad_rowsum(const void* d_out, const void* out, const sfa_shape* shape, sfa_stream_t stream,
+                                   float* rowsum_out) {
+    g_last_error.clear();
+    Sizes z;
+    sfa_status st = check_shape(shape, 1, 0, &z);
+    if (st != SFA_OK) return st;
+    if (!d_out || !out || !rowsum_out) return fail(SFA_ERR_NULLPTR, "a required pointer is NULL");
+    SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, z.T1, shape->N1, rowsum_out, (cudaStream_t)stream),
+             "rowsum(dO*O)");
+    return SFA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Dense varlen FlashAttention (TND)
+// ---------------------------------------------------------------------------
+static sfa_status check_fa(const fa_shape* s, int64_t mode) {
+    if (!s) return fail(SFA_ERR_NULLPTR, "shape is NULL");
+    if (s->dtype != SFA_DTYPE_BF16 && s->dtype != SFA_DTYPE_FP16)
+        return fail(SFA_ERR_INVALID, "dtype %d: only bf16 (0) or fp16 (1)", s->dtype);
+    if (s->B < 1) return fail(SFA_ERR_INVALID, "B=%lld < 1", (long long)s->B);
+    if (s->T1 < 1 || s->T2 < 1 || s->T1 > (1 << 20) || s->T2 > (1 << 20))
+        return fail(SFA_ERR_INVALID, "T1=%lld T2=%lld outside [1,1M]", (long long)s->T1, (long long)s->T2);
+    if (s->Nq < 1 || s->Nq > 256 || s->Nkv < 1 || s->Nq % s->Nkv != 0)
+        return fail(SFA_ERR_INVALID, "Nq=%lld Nkv=%lld: need 1<=Nq<=256 and Nq%%Nkv==0", (long long)s->Nq,
+                    (long long)s->Nkv);
+    if (s->D < 8 || s->D > 256 || s->D % 8 != 0) return fail(SFA_ERR_INVALID, "D=%lld: multiple of 8 in [8,256]",
+                                                             (long long)s->D);
+    if (mode != 0 && mode != 3) return fail(SFA_ERR_INVALID, "sparse_mode=%lld: only 0 or 3", (long long)mode);
+    return SFA_OK;
+}
+
+static sfa_status check_cu(const int64_t* cu, int64_t B, int64_t T, const char* name) {
+    if (!cu) return fail(SFA_ERR_NULLPTR, "%s is NULL", name);
+    int64_t prev = 0;
+    for (int64_t b = 0; b < B; ++b) {
+        if (cu[b] < prev) return fail(SFA_ERR_INVALID, "%s not non-decreasing at %lld", name, (long long)b);
+        prev = cu[b];
+    }
+    if (prev != T) return fail(SFA_ERR_INVALID, "%s last entry %lld != T %lld", name, (long long)prev, (long long)T);
+    return SFA_OK;
+}
+
+static size_t fa_cu_bytes(int64_t B) { return 2 * align256((size_t)B * 8); }
+
+sfa_status fa_grad_workspace_size(const fa_shape* shape, int64_t sparse_mode, int32_t deterministic,
+                                  size_t* workspace_bytes) {
+    g_last_error.clear();
+    if (!workspace_bytes) return fail(SFA_ERR_NULLPTR, "workspace_bytes is NULL");
+    sfa_status st = check_fa(shape, sparse_mode);
+    if (st != SFA_OK) return st;
+    *workspace_bytes = fa_cu_bytes(shape->B) +
+                       align256((size_t)2 * shape->T2 * shape->Nkv * shape->D * (deterministic ? 8 : 4));
+    return SFA_OK;
+}
+
+sfa_status fa_grad(const void* q, const void* k, const void* v, const void* dy, const float* softmax_max,
+                   const float* softmax_sum, const void* attention_in, const int64_t* actual_seq_qlen,
+                   const int64_t* actual_seq_kvlen, double scale, double keep_prob, int64_t pre_tokens,
+                   int64_t next_tokens, int64_t head_num, int64_t sparse_mode, int32_t deterministic,
+                   const fa_shape* shape, void* workspace, size_t workspace_bytes, sfa_stream_t stream, void* dq,
+                   void* dk, void* dv) {
+    (void)pre_tokens;
+    (void)next_tokens;
+    g_last_error.clear();
+    sfa_status st = check_fa(shape, sparse_mode);
+    if (st != SFA_OK) return st;
+    if (!q || !k || !v || !dy || !softmax_max || !softmax_sum || !attention_in || !dq || !dk || !dv || !workspace)
+        return fail(SFA_ERR_NULLPTR, "a required tensor pointer is NULL");
+    if ((st = check_cu(actual_seq_qlen, shape->B, shape->T1, "actual_seq_qlen")) != SFA_OK) return st;
+    if ((st = check_cu(actual_seq_kvlen, shape->B, shape->T2, "actual_seq_kvlen")) != SFA_OK) return st;
+    if (keep_prob != 1.0) return fail(SFA_ERR_INVALID, "keep_prob=%g: only 1 (no dropout)", keep_prob);
+    if (head_num != shape->Nq) return fail(SFA_ERR_INVALID, "head_num %lld != Nq %lld", (long long)head_num,
+                                           (long long)shape->Nq);
+    const bool det = deterministic != 0;
+    size_t acc_bytes = (size_t)2 * shape->T2 * shape->Nkv * shape->D * (det ? 8 : 4);
+    size_t need = fa_cu_bytes(shape->B) + align256(acc_bytes);
+    if (workspace_bytes < need) return fail(SFA_ERR_WORKSPACE, "workspace %zu < %zu", workspace_bytes, need);
+    cudaStream_t s = (cudaStream_t)stream;
+    char* w = (char*)workspace;
+    int64_t* cuq = (int64_t*)w;
+    int64_t* cukv = (int64_t*)(w + align256((size_t)shape->B * 8));
+    void* acc = w + fa_cu_bytes(shape->B);
+    SFA_CUDA(cudaMemcpyAsync(cuq, actual_seq_qlen, shape->B * 8, cudaMemcpyHostToDevice, s), "copy seqlens");
+    SFA_CUDA(cudaMemcpyAsync(cukv, actual_seq_kvlen, shape->B * 8, cudaMemcpyHostToDevice, s), "copy seqlens");
+    SFA_CUDA(cudaMemsetAsync(acc, 0, acc_bytes, s), "zero dK/dV accumulator");
+    FaArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = q; a.k = k; a.v = v; a.dy = dy; a.o = attention_in; a.smax = softmax_max; a.ssum = softmax_sum;
+    a.cu_q = cuq; a.cu_kv = cukv; a.B = shape->B; a.T1 = shape->T1; a.T2 = shape->T2; a.Nq = shape->Nq;
+    a.Nkv = shape->Nkv; a.D = shape->D; a.mode = (int)sparse_mode; a.scale = (float)scale; a.det = det;
+    a.dkv_acc = acc; a.dq = dq; a.dk = dk; a.dv = dv;
+    SFA_CUDA(launch_fa_bwd(shape->dtype, a, s), "fa backward");
+    return SFA_OK;
+}
+
+sfa_status fa_fwd_workspace_size(const fa_shape* shape, int64_t sparse_mode, size_t* workspace_bytes) {
+    g_last_error.clear();
+    if (!workspace_bytes) return fail(SFA_ERR_NULLPTR, "workspace_bytes is NULL");
+    sfa_status st = check_fa(shape, sparse_mode);
+    if (st != SFA_OK) return st;
+    *workspace_bytes = fa_cu_bytes(shape->B);
+    return SFA_OK;
+}
+
+sfa_status fa_fwd(const void* q, const void* k, const void* v, const int64_t* actual_seq_qlen,
+                  const int64_t* actual_seq_kvlen, double scale, int64_t sparse_mode, const fa_shape* shape,
+                  void* workspace, size_t workspace_bytes, sfa_stream_t stream, void* out, float* softmax_max,
+                  float* softmax_sum) {
+    g_last_error.clear();
+    sfa_status st = check_fa(shape, sparse_mode);
+    if (st != SFA_OK) return st;
+    if (!q || !k || !v || !out || !softmax_max || !softmax_sum || !workspace)
+        return fail(SFA_ERR_NULLPTR, "a required tensor pointer is NULL");
+    if ((st = check_cu(actual_seq_qlen, shape->B, shape->T1, "actual_seq_qlen")) != SFA_OK) return st;
+    if ((st = check_cu(actual_seq_kvlen, shape->B, shape->T2, "actual_seq_kvlen")) != SFA_OK) return st;
+    size_t need = fa_cu_bytes(shape->B);
+    if (workspace_bytes < need) return fail(SFA_ERR_WORKSPACE, "workspace %zu < %zu", workspace_bytes, need);
+    cudaStream_t s = (cudaStream_t)stream;
+    char* w = (char*)workspace;
+    int64_t* cuq = (int64_t*)w;
+    int64_t* cukv = (int64_t*)(w + align256((size_t)shape->B * 8));
+    SFA_CUDA(cudaMemcpyAsync(cuq, actual_seq_qlen, shape->B * 8, cudaMemcpyHostToDevice, s), "copy seqlens");
+    SFA_CUDA(cudaMemcpyAsync(cukv, actual_seq_kvlen, shape->B * 8, cudaMemcpyHostToDevice, s), "copy seqlens");
+    FaArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = q; a.k = k; a.v = v;
+    a.cu_q = cuq; a.cu_kv = cukv; a.B = shape->B; a.T1 = shape->T1; a.T2 = shape->T2; a.Nq = shape->Nq;
+    a.Nkv = shape->Nkv; a.D = shape->D; a.mode = (int)sparse_mode; a.scale = (float)scale;
+    a.out = out; a.smax_out = softmax_max; a.ssum_out = softmax_sum;
+    SFA_CUDA(launch_fa_fwd(shape->dtype, a, s), "fa forward");
+    return SFA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,181 @@
+// Internal declarations shared by the libsfa translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sfa.h"
+
+namespace sfa {
+
+constexpr int kD = 512;    // latent head dim (SparseFlashAttentionGrad 约束说明: D only 512)
+constexpr int kDr = 64;    // rope dim (Drope only 64)
+constexpr int kDK = kD + kDr;   // 576: width of a gathered key row [key || keyRope]
+constexpr int kAccW = kDK + kD; // 1088: fp32/int64 accumulator row = [dKey | dKeyRope | dValue]
+
+// 64-bit fixed point used by the deterministic scatter: value * 2^32, rounded.
+constexpr float kFixScale = 4294967296.0f;
+constexpr double kFixInv = 1.0 / 4294967296.0;
+
+// ---------------------------------------------------------------------------
+// 16-bit element access
+// ---------------------------------------------------------------------------
+template <typename T> __device__ __forceinline__ float to_f(T x);
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <> __device__ __forceinline__ float to_f<__half>(__half x) { return __half2float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+template <> __device__ __forceinline__ __half from_f<__half>(float x) { return __float2half_rn(x); }
+
+// ---------------------------------------------------------------------------
+// Query row -> batch / sequence span
+// ---------------------------------------------------------------------------
+struct SeqDesc {
+    int32_t layout;   // SFA_LAYOUT_BSND | SFA_LAYOUT_TND
+    int32_t B;
+    int64_t S1, S2;   // BSND padded lengths
+    int64_t T1, T2;
+    const int32_t* seq_q;   // BSND: per-batch lengths or null; TND: cumulative ends
+    const int32_t* seq_kv;
+};
+
+struct TokInfo {
+    int64_t kv_start;  // first key row of the span in the flattened [T2] view
+    int32_t pos;       // position of the query inside its span
+    int32_t q_len;     // S1_b
+    int32_t kv_len;    // S2_b (clamped to the tensor)
+    bool valid;        // false for BSND padding rows / rows beyond the TND total
+};
+
+__device__ __forceinline__ int64_t clamp64(int64_t x, int64_t lo, int64_t hi) {
+    return x < lo ? lo : (x > hi ? hi : x);
+}
+
+// Inconsistent lengths are clamped into the tensors, never trusted for addressing.
+__device__ __forceinline__ TokInfo tok_info(const SeqDesc& s, int64_t t) {
+    TokInfo r;
+    if (s.layout == SFA_LAYOUT_BSND) {
+        int64_t b = t / s.S1;
+        r.pos = (int32_t)(t - b * s.S1);
+        int64_t lq = s.seq_q ? clamp64(s.seq_q[b], 0, s.S1) : s.S1;
+        int64_t lk = s.seq_kv ? clamp64(s.seq_kv[b], 0, s.S2) : s.S2;
+        r.q_len = (int32_t)lq;
+        r.kv_len = (int32_t)lk;
+        r.kv_start = b * s.S2;
+        r.valid = r.pos < lq;
+        return r;
+    }
+    // TND: first b with cum_q[b] > t
+    int lo = 0, hi = s.B;
+    while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if ((int64_t)s.seq_q[mid] > t) hi = mid; else lo = mid + 1;
+    }
+    if (lo >= s.B) { r.valid = false; r.pos = 0; r.q_len = 0; r.kv_len = 0; r.kv_start = 0; return r; }
+    int b = lo;
+    int64_t qs = b ? clamp64(s.seq_q[b - 1], 0, s.T1) : 0;
+    int64_t qe = clamp64(s.seq_q[b], 0, s.T1);
+    int64_t ks = b ? clamp64(s.seq_kv[b - 1], 0, s.T2) : 0;
+    int64_t ke = clamp64(s.seq_kv[b], 0, s.T2);
+    r.pos = (int32_t)(t - qs);
+    r.q_len = (int32_t)(qe > qs ? qe - qs : 0);
+    r.kv_start = ks;
+    r.kv_len = (int32_t)(ke > ks ? ke - ks : 0);
+    r.valid = t >= qs && t < qe;
+    return r;
+}
+
+// Number of leading rows of block `blk` (bs rows) a query keeps: rows past S2_b
+// and, in sparse mode 3, rows past pos + S2_b - S1_b are dropped.
+__device__ __forceinline__ int block_rows(int64_t blk, int bs, const TokInfo& ti, int mode) {
+    int64_t start = blk * (int64_t)bs;
+    int64_t end = start + bs;
+    if (end > ti.kv_len) end = ti.kv_len;
+    if (mode == 3) {
+        int64_t lim = (int64_t)ti.pos + ti.kv_len - ti.q_len;  // last kept row
+        if (end > lim + 1) end = lim + 1;
+    }
+    int64_t n = end - start;
+    return n > 0 ? (int)n : 0;
+}
+
+// ---------------------------------------------------------------------------
+// Workspace layout of sfa_grad
+// ---------------------------------------------------------------------------
+struct GradWs {
+    size_t dkv;     // [T2][1088] fp32 (atomic) or int64 (deterministic)
+    size_t dq;      // [T1][N1][576] fp32, fused tensor-core path only
+    size_t blocks;  // [T1][topk] int32 compacted block indices
+    size_t nblk;    // [T1] int32
+    size_t nrows;   // [T1] int32
+    size_t order;   // [T1] int32 work order (longest first)
+    size_t rowsum;  // [T1][N1] fp32 FlashSoftmaxGrad
+    size_t ctrl;    // 256 B of counters / flags
+    size_t total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+inline GradWs grad_ws_layout(int64_t T1, int64_t T2, int64_t N1, int64_t topk, bool det, bool fused) {
+    GradWs w;
+    size_t o = 0;
+    w.dkv = o;    o = align256(o + (size_t)T2 * kAccW * (det ? 8 : 4));
+    w.dq = o;     o = align256(o + (fused ? (size_t)T1 * N1 * kDK * 4 : 0));
+    w.blocks = o; o = align256(o + (size_t)T1 * topk * 4);
+    w.nblk = o;   o = align256(o + (size_t)T1 * 4);
+    w.nrows = o;  o = align256(o + (size_t)T1 * 4);
+    w.order = o;  o = align256(o + (size_t)T1 * 4);
+    w.rowsum = o; o = align256(o + (size_t)T1 * N1 * 4);
+    w.ctrl = o;   o = align256(o + 256);
+    w.total = o;
+    return w;
+}
+
+// ---------------------------------------------------------------------------
+// Launchers (defined in the .cu files; all return cudaGetLastError())
+// ---------------------------------------------------------------------------
+cudaError_t launch_compact(const int32_t* idx, const SeqDesc& sd, int64_t topk, int bs, int mode, int32_t* blocks,
+                           int32_t* nblk, int32_t* nrows, cudaStream_t st);
+cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t T1, int64_t N1, float* rowsum,
+                          cudaStream_t st);
+cudaError_t launch_order(const int32_t* nrows, int64_t T1, int32_t* order, int32_t* ctrl, cudaStream_t st);
+cudaError_t launch_cast_dkv(int dtype, bool det, const void* acc, int64_t T2, void* dk, void* dkr, void* dv,
+                            cudaStream_t st);
+cudaError_t launch_cast_dq(int dtype, const float* acc, int64_t T1, int64_t N1, void* dq, void* dqr,
+                           cudaStream_t st);
+
+struct GradArgs {
+    const void* q; const void* qr; const void* k; const void* kr; const void* v;
+    const void* dout; const void* out; const float* smax; const float* ssum;
+    const int32_t* idx; SeqDesc sd; int64_t N1; int64_t topk; int bs; int mode; float scale; bool det;
+    const int32_t* blocks; const int32_t* nblk; const int32_t* nrows; const int32_t* order;
+    const float* rowsum; void* dkv_acc; float* dq_acc; int32_t* ctrl;
+    void* dq; void* dqr;
+};
+cudaError_t launch_bwd_generic(int dtype, const GradArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_fused(int dtype, const GradArgs& a, cudaStream_t st);
+bool fused_supported(int64_t N1);
+
+struct FwdArgs {
+    const void* q; const void* qr; const void* k; const void* kr; const void* v;
+    SeqDesc sd; int64_t N1; int64_t topk; int bs; int mode; float scale;
+    const int32_t* blocks; const int32_t* nblk;
+    void* out; float* smax; float* ssum;
+};
+cudaError_t launch_fwd_generic(int dtype, const FwdArgs& a, cudaStream_t st);
+
+struct FaArgs {
+    const void* q; const void* k; const void* v; const void* dy; const void* o;
+    const float* smax; const float* ssum;  // [T1][Nq][8]
+    const int64_t* cu_q; const int64_t* cu_kv;  // device copies, length B
+    int64_t B, T1, T2, Nq, Nkv, D; int mode; float scale; bool det;
+    void* dkv_acc;  // [2][T2][Nkv][D] fp32 or int64
+    void* dq; void* dk; void* dv;
+    void* out; float* smax_out; float* ssum_out;
+};
+cudaError_t launch_fa_bwd(int dtype, const FaArgs& a, cudaStream_t st);
+cudaError_t launch_fa_fwd(int dtype, const FaArgs& a, cudaStream_t st);
+
+}  // namespace sfa

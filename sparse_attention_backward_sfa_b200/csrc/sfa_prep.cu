@@ -1,0 +1,175 @@
+// Preparation and finishing kernels of the sparse attention backward:
+//   - index compaction (the Gather of SparseFlashAttentionGrad README, 功能说明, with
+//     the sparseMode 3 mask of 约束说明),
+//   - FlashSoftmaxGrad(dO, O) = rowsum(dO o O) of stage 2,
+//   - the work order of the fused kernel,
+//   - the final fp32 / fixed-point -> 16-bit casts of the scattered gradients.
+#include "sfa_internal.cuh"
+
+namespace sfa {
+
+// One warp per query row: keep the valid block indices in their original order.
+__global__ void compact_kernel(const int32_t* __restrict__ idx, SeqDesc sd, int64_t topk, int bs, int mode,
+                               int32_t* __restrict__ blocks, int32_t* __restrict__ nblk,
+                               int32_t* __restrict__ nrows) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= sd.T1) return;
+    TokInfo ti = tok_info(sd, t);
+    int count = 0, rows = 0;
+    if (ti.valid) {
+        const int32_t* src = idx + t * topk;
+        int32_t* dst = blocks + t * topk;
+        for (int64_t c = 0; c < topk; c += 32) {
+            int64_t i = c + lane;
+            int n = 0;
+            int32_t b = -1;
+            if (i < topk) {
+                b = src[i];
+                if (b >= 0) n = block_rows(b, bs, ti, mode);
+            }
+            // a block is kept iff it has at least one row before the cuts
+            bool keep = n > 0;
+            unsigned m = __ballot_sync(0xffffffffu, keep);
+            int before = __popc(m & ((1u << lane) - 1u));
+            if (keep) dst[count + before] = b;
+            count += __popc(m);
+            rows += n;
+        }
+    }
+    for (int o = 16; o; o >>= 1) rows += __shfl_xor_sync(0xffffffffu, rows, o);
+    if (lane == 0) {
+        nblk[t] = count;
+        nrows[t] = rows;
+    }
+}
+
+cudaError_t launch_compact(const int32_t* idx, const SeqDesc& sd, int64_t topk, int bs, int mode, int32_t* blocks,
+                           int32_t* nblk, int32_t* nrows, cudaStream_t st) {
+    const int warps = 8;
+    int64_t grid = (sd.T1 + warps - 1) / warps;
+    if (grid > 0) compact_kernel<<<(unsigned)grid, warps * 32, 0, st>>>(idx, sd, topk, bs, mode, blocks, nblk, nrows);
+    return cudaGetLastError();
+}
+
+// One warp per (row, head): sum over the 512 value dims of dO * O in fp32.
+template <typename T>
+__global__ void rowsum_kernel(const T* __restrict__ dout, const T* __restrict__ out, int64_t rows,
+                              float* __restrict__ res) {
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    const uint4* a = reinterpret_cast<const uint4*>(dout + r * kD);
+    const uint4* b = reinterpret_cast<const uint4*>(out + r * kD);
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < kD / 8 / 32; ++c) {
+        uint4 x = a[c * 32 + lane], y = b[c * 32 + lane];
+        const T* xp = reinterpret_cast<const T*>(&x);
+        const T* yp = reinterpret_cast<const T*>(&y);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s = fmaf(to_f(xp[e]), to_f(yp[e]), s);
+    }
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) res[r] = s;
+}
+
+cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t T1, int64_t N1, float* rowsum,
+                          cudaStream_t st) {
+    int64_t rows = T1 * N1;
+    const int warps = 8;
+    unsigned grid = (unsigned)((rows + warps - 1) / warps);
+    if (rows == 0) return cudaGetLastError();
+    if (dtype == SFA_DTYPE_BF16)
+        rowsum_kernel<__nv_bfloat16><<<grid, warps * 32, 0, st>>>((const __nv_bfloat16*)dout,
+                                                                  (const __nv_bfloat16*)out, rows, rowsum);
+    else
+        rowsum_kernel<__half><<<grid, warps * 32, 0, st>>>((const __half*)dout, (const __half*)out, rows, rowsum);
+    return cudaGetLastError();
+}
+
+// Work order for the persistent fused kernel: later rows first (under the causal
+// masks they carry the most keys, so the largest work items start first).
+__global__ void order_kernel(int64_t T1, int32_t* __restrict__ order, int32_t* __restrict__ ctrl) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < T1) order[i] = (int32_t)(T1 - 1 - i);
+    if (i < 64) ctrl[i] = 0;
+}
+
+cudaError_t launch_order(const int32_t* nrows, int64_t T1, int32_t* order, int32_t* ctrl, cudaStream_t st) {
+    (void)nrows;
+    int64_t n = T1 > 64 ? T1 : 64;
+    order_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(T1, order, ctrl);
+    return cudaGetLastError();
+}
+
+// [T2][1088] accumulator -> dKey [T2][512], dKeyRope [T2][64], dValue [T2][512].
+template <typename T, bool DET>
+__global__ void cast_dkv_kernel(const void* __restrict__ acc, int64_t T2, T* __restrict__ dk, T* __restrict__ dkr,
+                                T* __restrict__ dv) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // group of 4 columns
+    const int64_t per_row = kAccW / 4;
+    if (i >= T2 * per_row) return;
+    int64_t r = i / per_row;
+    int c = (int)(i - r * per_row) * 4;
+    float v[4];
+    if (DET) {
+        const long long* a = reinterpret_cast<const long long*>(acc) + r * kAccW + c;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = (float)((double)a[e] * kFixInv);
+    } else {
+        float4 x = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(acc) + r * kAccW + c);
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    }
+    T* dst;
+    if (c < kD) dst = dk + r * kD + c;
+    else if (c < kDK) dst = dkr + r * kDr + (c - kD);
+    else dst = dv + r * kD + (c - kDK);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[e] = from_f<T>(v[e]);
+}
+
+cudaError_t launch_cast_dkv(int dtype, bool det, const void* acc, int64_t T2, void* dk, void* dkr, void* dv,
+                            cudaStream_t st) {
+    int64_t n = T2 * (kAccW / 4);
+    if (n == 0) return cudaGetLastError();
+    unsigned grid = (unsigned)((n + 255) / 256);
+    if (dtype == SFA_DTYPE_BF16) {
+        using T = __nv_bfloat16;
+        if (det) cast_dkv_kernel<T, true><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv);
+        else cast_dkv_kernel<T, false><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv);
+    } else {
+        using T = __half;
+        if (det) cast_dkv_kernel<T, true><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv);
+        else cast_dkv_kernel<T, false><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv);
+    }
+    return cudaGetLastError();
+}
+
+// [T1][N1][576] fp32 -> dQuery [T1][N1][512], dQueryRope [T1][N1][64].
+template <typename T>
+__global__ void cast_dq_kernel(const float* __restrict__ acc, int64_t rows, T* __restrict__ dq, T* __restrict__ dqr) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t per_row = kDK / 4;
+    if (i >= rows * per_row) return;
+    int64_t r = i / per_row;
+    int c = (int)(i - r * per_row) * 4;
+    float4 x = *reinterpret_cast<const float4*>(acc + r * kDK + c);
+    T* dst = c < kD ? dq + r * kD + c : dqr + r * kDr + (c - kD);
+    dst[0] = from_f<T>(x.x); dst[1] = from_f<T>(x.y); dst[2] = from_f<T>(x.z); dst[3] = from_f<T>(x.w);
+}
+
+cudaError_t launch_cast_dq(int dtype, const float* acc, int64_t T1, int64_t N1, void* dq, void* dqr,
+                           cudaStream_t st) {
+    int64_t rows = T1 * N1;
+    int64_t n = rows * (kDK / 4);
+    if (n == 0) return cudaGetLastError();
+    unsigned grid = (unsigned)((n + 255) / 256);
+    if (dtype == SFA_DTYPE_BF16)
+        cast_dq_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(acc, rows, (__nv_bfloat16*)dq, (__nv_bfloat16*)dqr);
+    else
+        cast_dq_kernel<__half><<<grid, 256, 0, st>>>(acc, rows, (__half*)dq, (__half*)dqr);
+    return cudaGetLastError();
+}
+
+}  // namespace sfa

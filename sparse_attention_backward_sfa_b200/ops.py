@@ -1,0 +1,216 @@
+"""PyTorch-facing binding of libsfa: argument marshalling only.
+
+Tensors supply device memory and the current CUDA stream; every step of the
+computation runs in the library's kernels.  Each function mirrors the C entry
+point of the same name in include/sfa.h.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import _native as N
+
+_DT = {torch.bfloat16: N.DTYPE_BF16, torch.float16: N.DTYPE_FP16}
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _check16(name, t, dtype):
+    _need(t.is_cuda and t.is_contiguous(), f"{name} must be a contiguous CUDA tensor")
+    _need(t.dtype == dtype, f"{name} must be {dtype}")
+
+
+def sfa_shape(query: torch.Tensor, key: torch.Tensor, query_rope: torch.Tensor, sparse_indices: torch.Tensor,
+              layout: str, actual_seq_lengths_q=None) -> N.SfaShape:
+    s = N.SfaShape()
+    _need(query.dtype in _DT, "query must be bf16 or fp16")
+    s.dtype = _DT[query.dtype]
+    if layout == "BSND":
+        _need(query.dim() == 4 and key.dim() == 4, "BSND tensors are 4-D")
+        s.layout = N.LAYOUT_BSND
+        s.B, s.S1, s.N1, s.D = query.shape
+        _, s.S2, s.N2, _ = key.shape
+        s.T1, s.T2 = s.B * s.S1, s.B * s.S2
+    elif layout == "TND":
+        _need(query.dim() == 3 and key.dim() == 3, "TND tensors are 3-D")
+        s.layout = N.LAYOUT_TND
+        s.T1, s.N1, s.D = query.shape
+        s.T2, s.N2, _ = key.shape
+        s.S1 = s.S2 = 0
+        _need(actual_seq_lengths_q is not None, "TND needs actual sequence lengths")
+        s.B = actual_seq_lengths_q.numel()
+    else:
+        raise ValueError(f"layout {layout!r}")
+    s.Dr = query_rope.shape[-1]
+    s.topk = sparse_indices.shape[-1]
+    return s
+
+
+def _seqlens(x, layout, B):
+    if x is None:
+        _need(layout == "BSND", "TND needs actual sequence lengths")
+        return None
+    _need(x.is_cuda and x.dtype == torch.int32 and x.numel() == B, "seq lengths: int32 CUDA tensor of length B")
+    return x
+
+
+def sfa_grad_workspace_size(shape: N.SfaShape, sparse_block_size: int, sparse_mode: int, deterministic: bool) -> int:
+    lib = N.load()
+    n = ctypes.c_size_t()
+    N.check(lib.sfa_grad_workspace_size(ctypes.byref(shape), sparse_block_size, sparse_mode, int(deterministic),
+                                        ctypes.byref(n)))
+    return n.value
+
+
+def sfa_grad(query, key, value, sparse_indices, d_out, out, softmax_max, softmax_sum, query_rope, key_rope, *,
+             scale: float, sparse_block_size: int, layout: str, sparse_mode: int, deterministic: bool = False,
+             actual_seq_lengths_q=None, actual_seq_lengths_kv=None, pre_tokens: int = 2 ** 31 - 1,
+             next_tokens: int = 2 ** 31 - 1, workspace: Optional[torch.Tensor] = None, outputs=None, stream=None):
+    """Backward of top-k sparse attention; returns (dQuery, dKey, dValue, dQueryRope, dKeyRope)."""
+    lib = N.load()
+    dt = query.dtype
+    for name, t in (("query", query), ("key", key), ("value", value), ("d_out", d_out), ("out", out),
+                    ("query_rope", query_rope), ("key_rope", key_rope)):
+        _check16(name, t, dt)
+    _need(sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(), "sparse_indices: int32 contiguous")
+    _need(softmax_max.dtype == torch.float32 and softmax_sum.dtype == torch.float32, "softmax stats must be fp32")
+    shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
+    skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
+    ws_bytes = sfa_grad_workspace_size(shape, sparse_block_size, sparse_mode, deterministic)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=query.device)
+    if outputs is None:
+        outputs = (torch.empty_like(query), torch.empty_like(key), torch.empty_like(key),
+                   torch.empty_like(query_rope), torch.empty_like(key_rope))
+    dq, dk, dv, dqr, dkr = outputs
+    N.check(lib.sfa_grad(_p(query), _p(key), _p(value), _p(sparse_indices), _p(d_out), _p(out), _p(softmax_max),
+                         _p(softmax_sum), _p(sq), _p(skv), _p(query_rope), _p(key_rope), float(scale),
+                         int(sparse_block_size), int(sparse_mode), int(pre_tokens), int(next_tokens),
+                         int(deterministic), ctypes.byref(shape), _p(workspace), workspace.numel(), _stream(stream),
+                         _p(dq), _p(dk), _p(dv), _p(dqr), _p(dkr)))
+    return dq, dk, dv, dqr, dkr
+
+
+def sfa_fwd(query, key, value, sparse_indices, query_rope, key_rope, *, scale: float, sparse_block_size: int,
+            layout: str, sparse_mode: int, actual_seq_lengths_q=None, actual_seq_lengths_kv=None, stream=None):
+    """Forward of top-k sparse attention; returns (out, softmaxMax, softmaxSum)."""
+    lib = N.load()
+    dt = query.dtype
+    for name, t in (("query", query), ("key", key), ("value", value), ("query_rope", query_rope),
+                    ("key_rope", key_rope)):
+        _check16(name, t, dt)
+    shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
+    skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
+    n = ctypes.c_size_t()
+    N.check(lib.sfa_fwd_workspace_size(ctypes.byref(shape), sparse_block_size, sparse_mode, ctypes.byref(n)))
+    ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=query.device)
+    out = torch.empty_like(query)
+    stat_shape = query.shape[:-1]
+    smax = torch.empty(stat_shape, dtype=torch.float32, device=query.device)
+    ssum = torch.empty(stat_shape, dtype=torch.float32, device=query.device)
+    N.check(lib.sfa_fwd(_p(query), _p(key), _p(value), _p(sparse_indices), _p(sq), _p(skv), _p(query_rope),
+                        _p(key_rope), float(scale), int(sparse_block_size), int(sparse_mode), ctypes.byref(shape),
+                        _p(ws), ws.numel(), _stream(stream), _p(out), _p(smax), _p(ssum)))
+    return out, smax, ssum
+
+
+def compact_indices(sparse_indices, key, query, query_rope, *, sparse_block_size: int, layout: str,
+                    sparse_mode: int, actual_seq_lengths_q=None, actual_seq_lengths_kv=None, stream=None):
+    """Index compaction step; returns (blocks [T1, topk], nblocks [T1], nrows [T1]) int32."""
+    lib = N.load()
+    shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
+    skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
+    dev = sparse_indices.device
+    blocks = torch.full((shape.T1, shape.topk), -7, dtype=torch.int32, device=dev)
+    nb = torch.empty(shape.T1, dtype=torch.int32, device=dev)
+    nr = torch.empty(shape.T1, dtype=torch.int32, device=dev)
+    N.check(lib.sfa_compact_indices(_p(sparse_indices), _p(sq), _p(skv), int(sparse_block_size), int(sparse_mode),
+                                    ctypes.byref(shape), _stream(stream), _p(blocks), _p(nb), _p(nr)))
+    return blocks, nb, nr
+
+
+def softmax_grad_rowsum(d_out, out, key, query_rope, sparse_indices, *, layout: str, actual_seq_lengths_q=None,
+                        stream=None):
+    """FlashSoftmaxGrad(dO, O): fp32 [T1, N1] row sums of dO o O."""
+    lib = N.load()
+    shape = sfa_shape(d_out, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    res = torch.empty(shape.T1 * shape.N1, dtype=torch.float32, device=d_out.device)
+    N.check(lib.sfa_softmax_grad_rowsum(_p(d_out), _p(out), ctypes.byref(shape), _stream(stream), _p(res)))
+    return res.view(shape.T1, shape.N1)
+
+
+def _fa_shape(q, k, cu_q, cu_kv) -> N.FaShape:
+    s = N.FaShape()
+    _need(q.dtype in _DT, "q must be bf16 or fp16")
+    s.dtype = _DT[q.dtype]
+    s.B = len(cu_q)
+    s.T1, s.Nq, s.D = q.shape
+    s.T2, s.Nkv, _ = k.shape
+    return s
+
+
+def _host_i64(x: Sequence[int]):
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.int64))
+    return a, a.ctypes.data_as(ctypes.c_void_p)
+
+
+def fa_grad(q, k, v, dy, softmax_max, softmax_sum, attention_in, cu_seqlens_q, cu_seqlens_kv, *, scale: float,
+            sparse_mode: int, deterministic: bool = False, keep_prob: float = 1.0, pre_tokens: int = 65536,
+            next_tokens: int = 65536, workspace=None, outputs=None, stream=None):
+    """Dense varlen FA backward (TND); cu_seqlens_* are host cumulative end offsets. Returns (dq, dk, dv)."""
+    lib = N.load()
+    for name, t in (("q", q), ("k", k), ("v", v), ("dy", dy), ("attention_in", attention_in)):
+        _check16(name, t, q.dtype)
+    shape = _fa_shape(q, k, cu_seqlens_q, cu_seqlens_kv)
+    n = ctypes.c_size_t()
+    N.check(lib.fa_grad_workspace_size(ctypes.byref(shape), int(sparse_mode), int(deterministic), ctypes.byref(n)))
+    if workspace is None or workspace.numel() < n.value:
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
+    if outputs is None:
+        outputs = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    dq, dk, dv = outputs
+    aq, pq = _host_i64(cu_seqlens_q)
+    akv, pkv = _host_i64(cu_seqlens_kv)
+    N.check(lib.fa_grad(_p(q), _p(k), _p(v), _p(dy), _p(softmax_max), _p(softmax_sum), _p(attention_in), pq, pkv,
+                        float(scale), float(keep_prob), int(pre_tokens), int(next_tokens), int(shape.Nq),
+                        int(sparse_mode), int(deterministic), ctypes.byref(shape), _p(workspace), workspace.numel(),
+                        _stream(stream), _p(dq), _p(dk), _p(dv)))
+    del aq, akv
+    return dq, dk, dv
+
+
+def fa_fwd(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, scale: float, sparse_mode: int, stream=None):
+    """Dense varlen FA forward (TND). Returns (out, softmaxMax [T1,Nq,8], softmaxSum [T1,Nq,8])."""
+    lib = N.load()
+    shape = _fa_shape(q, k, cu_seqlens_q, cu_seqlens_kv)
+    n = ctypes.c_size_t()
+    N.check(lib.fa_fwd_workspace_size(ctypes.byref(shape), int(sparse_mode), ctypes.byref(n)))
+    ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
+    out = torch.empty_like(q)
+    smax = torch.empty(q.shape[0], q.shape[1], 8, dtype=torch.float32, device=q.device)
+    ssum = torch.empty_like(smax)
+    aq, pq = _host_i64(cu_seqlens_q)
+    akv, pkv = _host_i64(cu_seqlens_kv)
+    N.check(lib.fa_fwd(_p(q), _p(k), _p(v), pq, pkv, float(scale), int(sparse_mode), ctypes.byref(shape), _p(ws),
+                       ws.numel(), _stream(stream), _p(out), _p(smax), _p(ssum)))
+    del aq, akv
+    return out, smax, ssum
