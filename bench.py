@@ -1,0 +1,352 @@
+"""Benchmark of the sparse attention backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 4]
+
+One step = one full sfa_grad call (zero-init, index compaction, rowsum(dO*O),
+key-row expansion, the fused tensor-core backward, the dQuery and dKey/dValue
+casts) over one batch of the workload, inputs resident in HBM.  The metric is
+TFLOP/s with the 5-GEMM count (5504 FLOP per valid (query row, head, key)).
+
+N > 1 (torchrun): every rank runs its own independent copy of the workload
+(seed + rank); no data-path collective; value = total FLOP of all ranks / the
+max over ranks of the timed region ("scaling": "weak").
+
+--impl reference times the CPU oracle (the plain numpy definition) on a
+bounded sample of the same workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn backward TFLOP/s (bf16, 5-GEMM count) and % of B200 tensor peak"
+FLOP_PER_TRIPLE = 5504
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks / throttle reasons in the background."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+                if out.returncode == 0 and out.stdout.strip():
+                    self.rows.append([x.strip() for x in out.stdout.strip().split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=6)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.rows)}
+
+
+# ---------------------------------------------------------------------------
+def build_problem(workload: int, seed_offset: int, device):
+    from workloads import make_device_problem
+    p = make_device_problem(workload, device=device,
+                            seed=None if seed_offset == 0 else 2000 + workload + 7919 * seed_offset)
+    return p
+
+
+def kw(p):
+    return dict(scale=p.scale, sparse_block_size=p.block_size, layout=p.layout, sparse_mode=p.sparse_mode,
+                actual_seq_lengths_q=p.seqlens_q, actual_seq_lengths_kv=p.seqlens_kv)
+
+
+def count_triples(p):
+    import sparse_attention_backward_sfa_b200 as S
+    _, _, nr = S.compact_indices(p.indices, p.k, p.q, p.q_rope, sparse_block_size=p.block_size, layout=p.layout,
+                                 sparse_mode=p.sparse_mode, actual_seq_lengths_q=p.seqlens_q,
+                                 actual_seq_lengths_kv=p.seqlens_kv)
+    return int(nr.to(dtype=__import__("torch").int64).sum().item()) * p.N1
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import sparse_attention_backward_sfa_b200 as S
+    from sparse_attention_backward_sfa_b200 import _native as N
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lib = N.load()
+    p = build_problem(args.workload, rank, dev)
+    out, smax, ssum = S.sfa_fwd(p.q, p.k, p.k, p.indices, p.q_rope, p.k_rope, **kw(p))
+    triples = count_triples(p)
+    flop = triples * FLOP_PER_TRIPLE
+    shape = S.sfa_shape(p.q, p.k, p.q_rope, p.indices, p.layout, p.seqlens_q)
+    ws_bytes = S.sfa_grad_workspace_size(shape, p.block_size, p.sparse_mode, p.deterministic)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    outs = (torch.empty_like(p.q), torch.empty_like(p.k), torch.empty_like(p.k), torch.empty_like(p.q_rope),
+            torch.empty_like(p.k_rope))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            N.check(lib.sfa_set_kernel_events(ctypes_ptr(ev[0]), ctypes_ptr(ev[1])))
+        S.sfa_grad(p.q, p.k, p.k, p.indices, p.dout, out, smax, ssum, p.q_rope, p.k_rope,
+                   deterministic=p.deterministic, workspace=ws, outputs=outs, **kw(p))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank) as clk:
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+    kern_ms = [a.elapsed_time(b) for a, b in evs]
+    err = ws[-256:].view(torch.int32)  # device error word of the fused kernel (workspace control area)
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    # end-to-end through the public API with host buffers: H2D of the step's
+    # inputs from pinned memory, the call, D2H of the five gradients
+    e2e = None
+    if not args.no_e2e:
+        host_in = [x.cpu().pin_memory() for x in (p.q, p.q_rope, p.k, p.k_rope, p.dout, out, smax, ssum, p.indices)]
+        if p.seqlens_q is not None:
+            host_in.append(p.seqlens_q.cpu().pin_memory())
+        dev_in = [torch.empty_like(x, device=dev) for x in host_in]
+        host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+        h2d = sum(x.numel() * x.element_size() for x in host_in)
+        d2h = sum(x.numel() * x.element_size() for x in host_out)
+
+        def e2e_step():
+            for d, h in zip(dev_in, host_in):
+                d.copy_(h, non_blocking=True)
+            q, qr, k, kr, do, o, mx, sm, idx = dev_in[:9]
+            sq = dev_in[9] if len(dev_in) > 9 else None
+            S.sfa_grad(q, k, k, idx, do, o, mx, sm, qr, kr, deterministic=p.deterministic, workspace=ws,
+                       outputs=outs, scale=p.scale, sparse_block_size=p.block_size, layout=p.layout,
+                       sparse_mode=p.sparse_mode, actual_seq_lengths_q=sq, actual_seq_lengths_kv=sq)
+            for h, o2 in zip(host_out, outs):
+                h.copy_(o2, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(2, min(args.steps, 5))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = a.elapsed_time(b) / n_e2e
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": flop * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    err_word = int(err[0].item())
+    return dict(flop=flop, triples=triples, ms_step=ms_step, kern_ms=kern_ms, clocks=clk.summary(), e2e=e2e,
+                ws_bytes=ws_bytes, err_word=err_word, p=p)
+
+
+def ctypes_ptr(ev):
+    import ctypes
+    return ctypes.c_void_p(ev.cuda_event)
+
+
+def cpu_baseline(workload: int, budget_s: float):
+    """Time the oracle (fp64 numpy, as it stands) on a bounded sample of query
+    rows of the same workload on this host's cores."""
+    import torch
+    from oracle import sfa_oracle as O
+    from workloads import RowView
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    p = build_problem(workload, 0, dev)
+    import sparse_attention_backward_sfa_b200 as S
+    if dev == "cuda":
+        out, smax, ssum = S.sfa_fwd(p.q, p.k, p.k, p.indices, p.q_rope, p.k_rope, **kw(p))
+    else:
+        out = torch.zeros_like(p.q)
+        smax = torch.zeros(p.q.shape[:-1])
+        ssum = torch.ones(p.q.shape[:-1])
+    rng = np.random.default_rng(12345)
+    T1 = p.T1
+    k = p.k.reshape(p.T2, p.D).float().cpu().numpy()
+    kr = p.k_rope.reshape(p.T2, p.Dr).float().cpu().numpy()
+    sq = None if p.seqlens_q is None else p.seqlens_q.cpu().numpy()
+    done_tokens, elapsed, flop = 0, 0.0, 0
+    n = 2
+    while elapsed < budget_s and done_tokens < T1:
+        toks = np.sort(rng.choice(T1, size=n, replace=False))
+        views = [RowView(x, toks, T1) for x in (p.q, p.q_rope, p.dout, out, smax, ssum, p.indices)]
+        qv, qrv, dov, ov, mv, lv, iv = views
+        c0 = time.perf_counter()
+        O.sfa_backward(qv, k, k, iv, dov, ov, mv, lv, qrv, kr, p.scale, p.block_size, p.sparse_mode, p.layout,
+                       p.B, p.S1, p.S2, sq, sq, tokens=toks)
+        elapsed += time.perf_counter() - c0
+        for t in toks:
+            nrow = 0
+            row = iv[t]
+            # rows of this token (same rule as the oracle)
+            sp = [s for s in O.make_spans(p.layout, p.B, p.S1, p.S2, sq, sq) if s.q_start <= t < s.q_start + s.q_len]
+            if sp:
+                s = sp[0]
+                nrow = len(O.selected_rows(np.asarray(row).ravel(), p.block_size, int(t) - s.q_start, s.q_len,
+                                           s.kv_len, p.sparse_mode))
+            flop += nrow * p.N1 * FLOP_PER_TRIPLE
+        done_tokens += n
+        n = min(2 * n, 64)
+    cores = len(os.sched_getaffinity(0))
+    return {"value": flop / elapsed / 1e12 if elapsed > 0 else 0.0, "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle", "sample": f"{done_tokens} query rows of workload {workload} "
+                                        f"(fp64 numpy oracle, {elapsed:.1f} s)", "seconds": elapsed}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=4, choices=[3, 4, 5])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from workloads import WORKLOADS
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        per_step = []
+        res = None
+        budget = 20.0
+        for i in range(args.warmup + args.steps):
+            res = cpu_baseline(args.workload, budget if i >= args.warmup else 2.0)
+            if i >= args.warmup:
+                per_step.append(res)
+        val = statistics.mean(r["value"] for r in per_step)
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": statistics.mean(r["seconds"] for r in per_step) * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": WORKLOADS[args.workload], "sample": per_step[-1]["sample"]},
+                "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": per_step[-1]["cores"], "kind": "oracle",
+                                 "sample": per_step[-1]["sample"]},
+                "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    r = run_ours(args, rank, world, local_rank)
+    peaks, src = load_peaks()
+    value = r["flop"] * world / (r["ms_step"] * 1e-3) / 1e12
+    kern = statistics.mean(r["kern_ms"])
+    achieved = r["flop"] / (kern * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, args.cpu_budget)
+        cpu.pop("seconds", None)
+    if rank == 0:
+        p = r["p"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["ms_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "pct_of_peak": 100.0 * value / world / peak,
+            "config": {"workload": WORKLOADS[args.workload], "layout": p.layout, "N1": p.N1, "topk": p.topk,
+                       "sparse_block_size": p.block_size, "deterministic": p.deterministic,
+                       "valid_triples": r["triples"], "gflop_per_step": r["flop"] / 1e9,
+                       "l2": "inputs larger than L2 (q+dO+O %.1f GB per step)" % (3 * p.q.numel() * 2 / 1e9),
+                       "parallelism": f"independent replica per GPU x{world}"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_source": f"{src} bf16 burst",
+                         "peak_sustained": float(peaks.get("bf16_tflops_sustained", peak)),
+                         "frac_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                         "kernel": "sfa_bwd_fused_kernel", "kernel_ms": kern, "traffic": None},
+            "cpu_baseline": cpu,
+            "e2e": r["e2e"],
+            "gpu_launches": 7 * args.steps,
+            "clocks": r["clocks"],
+            "device_error_word": r["err_word"],
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

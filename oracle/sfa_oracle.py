@@ -126,6 +126,10 @@ def _as(x, dtype):
     return np.asarray(x, dtype=dtype)
 
 
+def _row(x, t, dtype):
+    return np.asarray(x[t], dtype=dtype)
+
+
 def sfa_forward(q, k, v, indices, q_rope, k_rope, scale: float, block_size: int, sparse_mode: int,
                 layout: str, B: int, S1: int, S2: int,
                 seqlens_q=None, seqlens_kv=None, dtype=np.float64, tokens=None):
@@ -133,36 +137,42 @@ def sfa_forward(q, k, v, indices, q_rope, k_rope, scale: float, block_size: int,
 
     q: [T1, N1, D], k/v: [T2, D] (N2 = 1 squeezed), q_rope: [T1, N1, Dr],
     k_rope: [T2, Dr], indices: [T1, topk] (N2 squeezed); BSND tensors are passed
-    flattened to T1 = B*S1 / T2 = B*S2 rows.
+    flattened to T1 = B*S1 / T2 = B*S2 rows.  Query-side arguments only need
+    ``len()`` and row indexing, and are converted one row at a time.
     Forward of the attention structure (aclnnFlashAttentionUnpaddingScoreGrad,
     计算公式: S = QK^T*scale, P = Softmax(S), Y = PV) restricted to the gathered
-    rows.  ``tokens`` restricts the work to a subset of flattened query rows.
+    rows.  ``tokens`` restricts the work to a subset of flattened query rows; the
+    outputs then hold only those rows, in ascending row order.
     Returns out [T1, N1, Dv], softmax_max [T1, N1], softmax_sum [T1, N1].
     """
-    q, k, v, q_rope, k_rope = (_as(a, dtype) for a in (q, k, v, q_rope, k_rope))
-    T1, N1, _ = q.shape
+    k, v, k_rope = (_as(a, dtype) for a in (k, v, k_rope))
+    T1 = len(q)
+    N1 = _row(q, 0, dtype).shape[0]
     Dv = v.shape[1]
-    out = np.zeros((T1, N1, Dv), dtype)
-    smax = np.zeros((T1, N1), dtype)
-    ssum = np.zeros((T1, N1), dtype)
-    qt_all = np.concatenate([q, q_rope], axis=2)
+    sel = list(range(T1)) if tokens is None else sorted(int(t) for t in tokens)
+    where = {t: i for i, t in enumerate(sel)}
+    out = np.zeros((len(sel), N1, Dv), dtype)
+    smax = np.zeros((len(sel), N1), dtype)
+    ssum = np.zeros((len(sel), N1), dtype)
     kt_all = np.concatenate([k, k_rope], axis=1)
     for sp in make_spans(layout, B, S1, S2, seqlens_q, seqlens_kv):
         for pos in range(sp.q_len):
             t = sp.q_start + pos
-            if tokens is not None and t not in tokens:
+            if t not in where:
                 continue
             rows = selected_rows(np.asarray(indices[t]), block_size, pos, sp.q_len, sp.kv_len, sparse_mode)
             if not rows:
                 continue
+            i = where[t]
             g = sp.kv_start + np.asarray(rows)
-            s = scale * (qt_all[t] @ kt_all[g].T)  # [N1, n]
+            qt = np.concatenate([_row(q, t, dtype), _row(q_rope, t, dtype)], axis=1)
+            s = scale * (qt @ kt_all[g].T)  # [N1, n]
             m = s.max(axis=1)
             e = np.exp(s - m[:, None])
             l = e.sum(axis=1)
-            out[t] = (e / l[:, None]) @ v[g]
-            smax[t] = m
-            ssum[t] = l
+            out[i] = (e / l[:, None]) @ v[g]
+            smax[i] = m
+            ssum[i] = l
     return out, smax, ssum
 
 
@@ -178,41 +188,45 @@ def sfa_backward(q, k, v, indices, d_out, out, softmax_max, softmax_sum, q_rope,
       dS = P o (dP - rowsum(dO o O))                              (stage 2)
       dQ~ = scale*dS.K~ ;  dK~[J_t] += scale*dS^T.Q~              (stage 3)
     Scatter-adds go through ``np.add.at`` so repeated rows accumulate.
-    ``tokens`` restricts the sum to a subset of query rows (sub-problem checks).
+    Query-side arguments only need ``len()`` and row indexing.  ``tokens``
+    restricts the sums to a subset of query rows (sub-problem checks); dQuery /
+    dQueryRope then hold only those rows, in ascending row order.
     """
-    q, k, v, d_out, out, q_rope, k_rope = (_as(a, dtype) for a in (q, k, v, d_out, out, q_rope, k_rope))
-    softmax_max = _as(softmax_max, dtype)
-    softmax_sum = _as(softmax_sum, dtype)
-    T1, N1, D = q.shape
-    Dr = q_rope.shape[2]
+    k, v, k_rope = (_as(a, dtype) for a in (k, v, k_rope))
+    T1 = len(q)
+    N1, D = _row(q, 0, dtype).shape
+    Dr = _row(q_rope, 0, dtype).shape[1]
     T2 = k.shape[0]
-    qt_all = np.concatenate([q, q_rope], axis=2)
+    sel = list(range(T1)) if tokens is None else sorted(int(t) for t in tokens)
+    where = {t: i for i, t in enumerate(sel)}
     kt_all = np.concatenate([k, k_rope], axis=1)
-    dqt = np.zeros((T1, N1, D + Dr), dtype)
+    dqt = np.zeros((len(sel), N1, D + Dr), dtype)
     dkt = np.zeros((T2, D + Dr), dtype)
     dv = np.zeros_like(v)
     ds_rows = {}
     for sp in make_spans(layout, B, S1, S2, seqlens_q, seqlens_kv):
         for pos in range(sp.q_len):
             t = sp.q_start + pos
-            if tokens is not None and t not in tokens:
+            if t not in where:
                 continue
             rows = selected_rows(np.asarray(indices[t]), block_size, pos, sp.q_len, sp.kv_len, sparse_mode)
             if not rows:
                 continue
             g = sp.kv_start + np.asarray(rows)
+            qt = np.concatenate([_row(q, t, dtype), _row(q_rope, t, dtype)], axis=1)  # [N1, D+Dr]
+            do = _row(d_out, t, dtype)
             kt = kt_all[g]  # [n, D+Dr]
             vt = v[g]  # [n, Dv]
-            s = scale * (qt_all[t] @ kt.T)  # [N1, n]
-            l = softmax_sum[t]
+            s = scale * (qt @ kt.T)  # [N1, n]
+            l = _row(softmax_sum, t, dtype)
             inv_l = np.where(l == 0, 0.0, 1.0 / np.where(l == 0, 1.0, l))
-            p = np.exp(s - softmax_max[t][:, None]) * inv_l[:, None]
-            dp = d_out[t] @ vt.T  # stage 1
-            np.add.at(dv, g, p.T @ d_out[t])  # stage 1
-            dsum = (d_out[t] * out[t]).sum(axis=1)  # FlashSoftmaxGrad(dO, O)
+            p = np.exp(s - _row(softmax_max, t, dtype)[:, None]) * inv_l[:, None]
+            dp = do @ vt.T  # stage 1
+            np.add.at(dv, g, p.T @ do)  # stage 1
+            dsum = (do * _row(out, t, dtype)).sum(axis=1)  # FlashSoftmaxGrad(dO, O)
             ds = p * (dp - dsum[:, None])  # stage 2
-            dqt[t] = scale * (ds @ kt)  # stage 3
-            np.add.at(dkt, g, scale * (ds.T @ qt_all[t]))  # stage 3
+            dqt[where[t]] = scale * (ds @ kt)  # stage 3
+            np.add.at(dkt, g, scale * (ds.T @ qt))  # stage 3
             if return_ds:
                 ds_rows[t] = ds
     res = (dqt[:, :, :D], dkt[:, :D], dv, dqt[:, :, D:], dkt[:, D:])

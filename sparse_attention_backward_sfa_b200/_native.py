@@ -64,6 +64,7 @@ SIGNATURES = {
                 _V, _V, _V],
     "fa_fwd_workspace_size": [_PFA, _I64, _PSZ],
     "fa_fwd": [_V, _V, _V, _V, _V, _Dbl, _I64, _PFA, _V, _SZ, _V, _V, _V, _V],
+    "sfa_set_kernel_events": [_V, _V],
     "sfa_status_string": [_I32],
     "sfa_last_error_string": [],
     "sfa_version": [],

@@ -13,6 +13,20 @@ using namespace sfa;
 namespace {
 
 thread_local std::string g_last_error;
+thread_local cudaEvent_t g_ev_before = nullptr, g_ev_after = nullptr;
+
+// Records the timing-hook events (if set) around the main kernel launch.
+struct KernelEvents {
+    cudaEvent_t a, b;
+    cudaStream_t s;
+    KernelEvents(cudaStream_t st) : a(g_ev_before), b(g_ev_after), s(st) {
+        g_ev_before = g_ev_after = nullptr;
+        if (a) cudaEventRecord(a, s);
+    }
+    ~KernelEvents() {
+        if (b) cudaEventRecord(b, s);
+    }
+};
 
 sfa_status fail(sfa_status st, const char* fmt, ...) {
     char buf[512];
@@ -98,6 +112,12 @@ const char* sfa_version(void) { return "0.1.0"; }
 
 const char* sfa_last_error_string(void) { return g_last_error.c_str(); }
 
+sfa_status sfa_set_kernel_events(void* event_before, void* event_after) {
+    g_ev_before = (cudaEvent_t)event_before;
+    g_ev_after = (cudaEvent_t)event_after;
+    return SFA_OK;
+}
+
 const char* sfa_status_string(sfa_status st) {
     switch (st) {
         case SFA_OK: return "SFA_OK";
@@ -117,7 +137,7 @@ sfa_status sfa_grad_workspace_size(const sfa_shape* shape, int64_t sparse_block_
     Sizes z;
     sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
     if (st != SFA_OK) return st;
-    *workspace_bytes = grad_ws_layout(z.T1, z.T2, shape->N1, shape->topk, deterministic != 0,
+    *workspace_bytes = grad_ws_layout(z.T1, z.T2, shape->N1, shape->topk, sparse_block_size, deterministic != 0,
                                       fused_supported(shape->N1)).total;
     return SFA_OK;
 }
@@ -144,7 +164,7 @@ sfa_status sfa_grad(const void* query, const void* key, const void* value, const
     if (((uintptr_t)workspace & 255u) != 0) return fail(SFA_ERR_INVALID, "workspace not 256-byte aligned");
     const bool det = deterministic != 0;
     const bool fused_shape = fused_supported(shape->N1);
-    const GradWs ws = grad_ws_layout(z.T1, z.T2, shape->N1, shape->topk, det, fused_shape);
+    const GradWs ws = grad_ws_layout(z.T1, z.T2, shape->N1, shape->topk, sparse_block_size, det, fused_shape);
     if (workspace_bytes < ws.total)
         return fail(SFA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, ws.total);
     cudaStream_t s = (cudaStream_t)stream;
@@ -160,6 +180,7 @@ sfa_status sfa_grad(const void* query, const void* key, const void* value, const
     a.order = (int32_t*)(w + ws.order); a.rowsum = (float*)(w + ws.rowsum);
     a.dkv_acc = w + ws.dkv; a.dq_acc = (float*)(w + ws.dq); a.ctrl = (int32_t*)(w + ws.ctrl);
     a.dq = d_query; a.dqr = d_query_rope;
+    a.dtype = shape->dtype; a.rowlist = (int32_t*)(w + ws.rowlist); a.rowcap = shape->topk * sparse_block_size;
 
     SFA_CUDA(cudaMemsetAsync(a.dkv_acc, 0, (size_t)z.T2 * kAccW * (det ? 8 : 4), s), "zero dK/dV accumulator");
     SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, (int32_t*)a.blocks, (int32_t*)a.nblk,
@@ -169,9 +190,15 @@ sfa_status sfa_grad(const void* query, const void* key, const void* value, const
         SFA_CUDA(cudaMemsetAsync(a.dq_acc, 0, (size_t)z.T1 * shape->N1 * kDK * 4, s), "zero dQ accumulator");
         SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, z.T1, shape->N1, (float*)a.rowsum, s), "rowsum(dO*O)");
         SFA_CUDA(launch_order(a.nrows, z.T1, (int32_t*)a.order, a.ctrl, s), "work order");
-        SFA_CUDA(launch_bwd_fused(shape->dtype, a, s), "fused backward");
+        SFA_CUDA(launch_expand(a.blocks, a.nblk, a.sd, a.topk, a.bs, a.mode, a.rowcap, (int32_t*)a.rowlist, s),
+                 "key row expansion");
+        {
+            KernelEvents ev(s);
+            SFA_CUDA(launch_bwd_fused(shape->dtype, a, s), "fused backward");
+        }
         SFA_CUDA(launch_cast_dq(shape->dtype, a.dq_acc, z.T1, shape->N1, d_query, d_query_rope, s), "cast dQuery");
     } else {
+        KernelEvents ev(s);
         SFA_CUDA(launch_bwd_generic(shape->dtype, a, s), "backward");
     }
     SFA_CUDA(launch_cast_dkv(shape->dtype, det, a.dkv_acc, z.T2, d_key, d_key_rope, d_value, s), "cast dKey/dValue");
@@ -331,6 +358,7 @@ sfa_status fa_grad(const void* q, const void* k, const void* v, const void* dy, 
     a.cu_q = cuq; a.cu_kv = cukv; a.B = shape->B; a.T1 = shape->T1; a.T2 = shape->T2; a.Nq = shape->Nq;
     a.Nkv = shape->Nkv; a.D = shape->D; a.mode = (int)sparse_mode; a.scale = (float)scale; a.det = det;
     a.dkv_acc = acc; a.dq = dq; a.dk = dk; a.dv = dv;
+    KernelEvents ev(s);
     SFA_CUDA(launch_fa_bwd(shape->dtype, a, s), "fa backward");
     return SFA_OK;
 }

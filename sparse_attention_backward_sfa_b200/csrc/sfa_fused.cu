@@ -1,18 +1,662 @@
-// Fused tensor-core sparse attention backward (tcgen05 / TMEM / TMA) for sm_100a.
+// Fused tensor-core sparse attention backward for sm_100a (tcgen05 MMA, TMEM
+// accumulators, TMA tile and gather4 loads, mbarrier pipelines).
+//
+// What it computes (SparseFlashAttentionGrad README, 功能说明, stages 1-3), per
+// query row t with its gathered key rows j (value == key, first 512 dims):
+//   S^T  = K~ . Q~^T                      [keys x heads], K = 576
+//   dP^T = V  . dO^T                      [keys x heads], K = 512
+//   P    = exp2(S*scale*log2e - max*log2e) / sum,  dS = P o (dP - rowsum(dO o O))
+//   dV^T = dO^T . P^T  -> red into dValue rows      [dims x keys], K = heads
+//   dK~^T= Q~^T . dS^T -> red into dKey||dKeyRope   [dims x keys], K = heads
+//   dQ~^T= K~^T . dS   -> red into the dQuery rows  [dims x heads], K = keys
+//
+// Layout decisions (B200):
+//  * Work item = one query row (all N1 heads share the single KV head), key
+//    tiles of 128 gathered rows.  MMA M is always 128: keys for S^T/dP^T, output
+//    dims for every gradient block, so TMEM lane = key during the softmax (per
+//    thread masking) and lane = output dim during the flush (each warp-level red
+//    covers 32 consecutive fp32 = one 128-byte line).
+//  * Every operand is a "chunk" of 128 dims (64 for the rope) held as two
+//    128-byte-row SW128 halves 16 KB apart; the same bytes serve as a K-major
+//    operand (S^T, dP^T) and as an MN-major one (gradients).  Chunks stream
+//    through a ring of 32 KB slots: key rows by TMA tile::gather4, the query
+//    row's q / qRope / dO by 2-D TMA tiles.
+//  * P and dS live in shared memory as bf16 [keys x heads] (SW128 halves of 64
+//    heads); S^T / dP^T and two 128-column staging accumulators live in TMEM
+//    (all 512 columns).
+//  * Warp roles: 0-3 softmax/dS (TMEM lanes = keys), 4-7 flush (TMEM lanes =
+//    dims), 8 TMA producer, 9 MMA issuer.  Every mbarrier wait is bounded; on
+//    timeout the kernel records an error word, stops issuing, drains what it
+//    issued and frees its TMEM.
+#include <cuda.h>
+
+#include <cstring>
+#include <type_traits>
+
 #include "sfa_internal.cuh"
 
 namespace sfa {
 
-bool fused_supported(int64_t N1) {
-    (void)N1;
-    return false;
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kSlotBytes = 32768;
+constexpr int kHalf = 16384;
+constexpr int kKeys = 128;          // key rows per tile (MMA M)
+constexpr int kItemsPerTile = 28;   // 14 for S/dP, 14 for the gradient blocks
+
+template <int N1> struct Cfg {
+    static constexpr int kSlots = N1 == 128 ? 5 : 6;
+    static constexpr int kRing = kSlots * kSlotBytes;
+    static constexpr int kPBytes = N1 * 2 * kKeys;   // bf16 [128 keys x N1 heads]
+    static constexpr int kOffP = kRing;
+    static constexpr int kOffDS = kOffP + (N1 == 128 ? 32768 : 16384);
+    static constexpr int kOffRows = kOffDS + (N1 == 128 ? 32768 : 16384);  // int32 [2][128]
+    static constexpr int kOffConst = kOffRows + 2 * kKeys * 4;              // float [3][128]
+    static constexpr int kOffBar = kOffConst + 3 * 128 * 4;
+    static constexpr int kNumBars = 2 * kSlots + 12;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kSmem = kOffMisc + 16;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
 }
 
+// Bounded wait: gives up after ~4 s (or as soon as another role aborted),
+// recording `code` in the device error word.
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err, int code) {
+    if (mbar_try(bar, parity)) return true;
+    uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try(bar, parity)) return true;
+        if ((it & 63) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > 4000000000ull) {
+                *abort_flag = 1;
+                atomicCAS(err, 0, code);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void fence_view_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t c0, int32_t c1,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int32_t col, int32_t r0, int32_t r1,
+                                            int32_t r2, int32_t r3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        ::"r"(dst), "l"((uint64_t)map), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+        : "memory");
+}
+
+// SW128 shared-memory matrix descriptor (tcgen05): start>>4 in [0,14), LBO>>4 in
+// [16,30), SBO>>4 in [32,46), version 1 in [46,48), layout SWIZZLE_128B (2) in [61,64).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor, kind::f16 with fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc(int M, int N, bool a_mn, bool b_mn, bool f16) {
+    return (1u << 4) |                              // D = f32
+           ((f16 ? 0u : 1u) << 7) |                 // A format: f16 = 0, bf16 = 1
+           ((f16 ? 0u : 1u) << 10) |                // B format
+           ((a_mn ? 1u : 0u) << 15) |               // A major: 0 K, 1 MN
+           ((b_mn ? 1u : 0u) << 16) |               // B major
+           ((uint32_t)(N >> 3) << 17) |             // N >> 3
+           ((uint32_t)(M >> 4) << 24);              // M >> 4
+}
+
+__device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(id), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+template <typename T> __device__ __forceinline__ uint32_t pack2(float a, float b);
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+struct FusedParams {
+    CUtensorMap mapQ, mapQr, mapO, mapK, mapKr;  // dO shares mapO
+    const int32_t* rowlist;  // [T1][cap] global key rows of each query row
+    const int32_t* nrows;    // [T1]
+    const int32_t* order;    // [T1] work order
+    const float* smax;       // [T1][N1]
+    const float* ssum;
+    const float* rowsum;     // [T1][N1]
+    void* dkv_acc;           // [T2][1088] fp32 or int64
+    float* dq_acc;           // [T1][N1][576]
+    int* err;                // device error word
+    int64_t T1;
+    int64_t cap;
+    float scale;
+    int det;
+};
+
+// Item i of a tile's load schedule: kind (0 key chunk, 1 q chunk, 2 dO chunk) and chunk c.
+__device__ __forceinline__ void item_of(int i, int& kind, int& c) {
+    if (i < 14) {  // S / dP phase: K0 Q0 O0 K1 Q1 O1 ... K3 Q3 O3 K4 Q4
+        c = i / 3;
+        kind = i - 3 * c;
+        return;
+    }
+    i -= 14;       // gradient phase: O0..O3 (dV), Q0..Q4 (dK), K0..K4 (dQ)
+    if (i < 4) { kind = 2; c = i; return; }
+    if (i < 9) { kind = 1; c = i - 4; return; }
+    kind = 0; c = i - 9;
+}
+
+template <typename T, int N1>
+__global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid_constant__ FusedParams prm) {
+    using C = Cfg<N1>;
+    constexpr bool kF16 = std::is_same<T, __half>::value;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_u32(smem);
+    if (sbase & 1023u) {  // the SW128 layouts need a 1024-byte aligned base
+        if (threadIdx.x == 0) atomicCAS(prm.err, 0, 7);
+        return;
+    }
+    int32_t* rowids = reinterpret_cast<int32_t*>(smem + C::kOffRows);
+    float* cst = reinterpret_cast<float*>(smem + C::kOffConst);
+    const uint32_t bar0 = sbase + C::kOffBar;
+    auto FULL = [&](int s) { return bar0 + 8u * s; };
+    auto EMPTY = [&](int s) { return bar0 + 8u * (C::kSlots + s); };
+    const uint32_t SDP_FULL = bar0 + 8u * (2 * C::kSlots + 0);
+    const uint32_t PDS_FULL = bar0 + 8u * (2 * C::kSlots + 1);
+    const uint32_t PDS_FREE = bar0 + 8u * (2 * C::kSlots + 2);
+    auto STG_FULL = [&](int s) { return bar0 + 8u * (2 * C::kSlots + 3 + s); };
+    auto STG_EMPTY = [&](int s) { return bar0 + 8u * (2 * C::kSlots + 5 + s); };
+    auto ROWS_FULL = [&](int s) { return bar0 + 8u * (2 * C::kSlots + 7 + s); };
+    auto ROWS_EMPTY = [&](int s) { return bar0 + 8u * (2 * C::kSlots + 9 + s); };
+    const uint32_t DONE = bar0 + 8u * (2 * C::kSlots + 11);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kSlots; ++s) {
+            mbar_init(FULL(s), 1);
+            mbar_init(EMPTY(s), 1);
+        }
+        mbar_init(SDP_FULL, 1);
+        mbar_init(PDS_FULL, 128);
+        mbar_init(PDS_FREE, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(STG_FULL(s), 1);
+            mbar_init(STG_EMPTY(s), 128);
+            mbar_init(ROWS_FULL(s), 1);
+            mbar_init(ROWS_EMPTY(s), 128);
+        }
+        mbar_init(DONE, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {  // whole TMEM: S^T [0,128), dP^T [128,256), staging [256,384) and [384,512)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tmem_slot))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t T_S = tmem, T_DP = tmem + 128;
+    auto T_STG = [&](int s) { return tmem + 256u + 128u * s; };
+
+    const int nwork = (int)prm.T1;
+    const float scale = prm.scale;
+
+    if (warp == 8) {
+        // =================== TMA producer ===================
+        int slot = 0;
+        uint32_t sphase = 0;
+        int tile_ctr = 0;
+        bool ok = true;
+        int issued_full[8];  // slots whose loads may still be in flight
+        for (int s = 0; s < 8; ++s) issued_full[s] = 0;
+        for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
+            const int t = prm.order[w];
+            const int n = prm.nrows[t];
+            if (n <= 0) continue;
+            const int32_t* rl = prm.rowlist + (int64_t)t * prm.cap;
+            const int ntiles = (n + kKeys - 1) / kKeys;
+            for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
+                const int rb = tile_ctr & 1;
+                ok = wait_bar(ROWS_EMPTY(rb), ((tile_ctr >> 1) & 1) ^ 1, abort_flag, prm.err, 1);
+                if (!ok) break;
+                int32_t* rid = rowids + rb * kKeys;
+                const int first = rl[0];
+                for (int r = lane; r < kKeys; r += 32) {
+                    const int s = tile * kKeys + r;
+                    rid[r] = s < n ? rl[s] : first;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(ROWS_FULL(rb));
+                for (int it = 0; it < kItemsPerTile && ok; ++it) {
+                    int kind, c;
+                    item_of(it, kind, c);
+                    if (lane == 0) ok = wait_bar(EMPTY(slot), sphase ^ 1, abort_flag, prm.err, 2);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    if (lane == 0) {
+                        const uint32_t dst = sbase + slot * kSlotBytes;
+                        const int halves = c < 4 ? 2 : 1;
+                        const uint32_t rows = kind == 0 ? kKeys : N1;
+                        mbar_expect_tx(FULL(slot), halves * rows * 128u);
+                        for (int h = 0; h < halves; ++h) {
+                            const uint32_t d = dst + h * kHalf;
+                            if (kind == 0) {
+                                const CUtensorMap* map = c < 4 ? &prm.mapK : &prm.mapKr;
+                                const int col = c < 4 ? c * 128 + h * 64 : 0;
+                                for (int g = 0; g < kKeys / 4; ++g)
+                                    tma_gather4(d + g * 512, map, col, rid[4 * g], rid[4 * g + 1], rid[4 * g + 2],
+                                                rid[4 * g + 3], FULL(slot));
+                            } else {
+                                const CUtensorMap* map = kind == 1 ? (c < 4 ? &prm.mapQ : &prm.mapQr) : &prm.mapO;
+                                const int col = c < 4 ? c * 128 + h * 64 : 0;
+                                tma_load_2d(d, map, col, t * N1, FULL(slot));
+                            }
+                        }
+                        issued_full[slot] = 1;
+                    }
+                    if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+                }
+            }
+        }
+        // drain: every issued load must land before the CTA can exit
+        if (lane == 0) {
+            for (int k = 0; k < C::kSlots; ++k) {
+                // the most recent use of each slot is the one still possibly in flight
+                const int s = (slot + k) % C::kSlots;
+                const uint32_t ph = s < slot ? sphase : sphase ^ 1;
+                if (issued_full[s]) {
+                    uint64_t t0 = globaltimer();
+                    while (!mbar_try(FULL(s), ph) && globaltimer() - t0 < 1000000000ull) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 9) {
+        // =================== MMA issuer ===================
+        const uint32_t ID_S = idesc(128, N1, false, false, kF16);      // S^T, dP^T
+        const uint32_t ID_G = idesc(128, 128, true, false, kF16);      // dV^T, dK~^T (N = keys)
+        const uint32_t ID_Q = idesc(128, N1, true, true, kF16);        // dQ~^T (N = heads)
+        const uint32_t sP = sbase + C::kOffP, sDS = sbase + C::kOffDS;
+        int slot = 0;
+        uint32_t sphase = 0;
+        int tile_ctr = 0;
+        int blk_ctr = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
+            const int t = prm.order[w];
+            const int n = prm.nrows[t];
+            if (n <= 0) continue;
+            const int ntiles = (n + kKeys - 1) / kKeys;
+            for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
+                // ---- S^T and dP^T over the 5 / 4 chunks ----
+                uint32_t slotK = 0, slotQ = 0;
+                for (int it = 0; it < 14 && ok; ++it) {
+                    int kind, c;
+                    item_of(it, kind, c);
+                    if (lane == 0) ok = wait_bar(FULL(slot), sphase, abort_flag, prm.err, 3);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t sa = sbase + slot * kSlotBytes;
+                    if (kind == 0) slotK = sa;
+                    else if (kind == 1) slotQ = sa;
+                    const int ksteps = c < 4 ? 8 : 4;
+                    if (lane == 0 && kind != 0) {
+                        const uint32_t dst = kind == 1 ? T_S : T_DP;
+                        for (int ks = 0; ks < ksteps; ++ks) {
+                            const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                            const uint64_t a = sdesc(slotK + off, 16, 1024);
+                            const uint64_t b = sdesc(sa + off, 16, 1024);
+                            mma(dst, a, b, ID_S, (c > 0 || ks > 0) ? 1u : 0u);
+                        }
+                    }
+                    // a slot is released once the MMAs that read it have completed
+                    const bool release_k = (kind == 2) || (kind == 1 && c == 4);
+                    if (lane == 0 && kind != 0) mma_commit(EMPTY(slot));
+                    if (lane == 0 && release_k) mma_commit(EMPTY((slotK - sbase) / kSlotBytes));
+                    __syncwarp();
+                    if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+                }
+                if (!ok) break;
+                if (lane == 0) mma_commit(SDP_FULL);
+                // ---- gradient blocks ----
+                if (lane == 0) ok = wait_bar(PDS_FULL, tile_ctr & 1, abort_flag, prm.err, 4);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                tc_fence_after();
+                for (int bi = 0; bi < 14 && ok; ++bi, ++blk_ctr) {
+                    const int stg = blk_ctr & 1;
+                    if (lane == 0) ok = wait_bar(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, abort_flag, prm.err, 5);
+                    if (lane == 0 && ok) ok = wait_bar(FULL(slot), sphase, abort_flag, prm.err, 6);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t sa = sbase + slot * kSlotBytes;
+                    if (lane == 0) {
+                        const uint32_t dst = T_STG(stg);
+                        if (bi < 9) {
+                            // dV^T (A = dO chunk) or dK~^T (A = q chunk): [128 dims x 128 keys], K = heads
+                            const uint32_t bsrc = bi < 4 ? sP : sDS;
+                            for (int ks = 0; ks < N1 / 16; ++ks) {
+                                const uint64_t a = sdesc(sa + ks * 2048, kHalf, 1024);
+                                const uint64_t b = sdesc(bsrc + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
+                                mma(dst, a, b, ID_G, ks > 0 ? 1u : 0u);
+                            }
+                        } else {
+                            // dQ~^T: A = key chunk [128 dims x 128 keys] (MN), B = dS [heads x keys] (MN)
+                            for (int ks = 0; ks < kKeys / 16; ++ks) {
+                                const uint64_t a = sdesc(sa + ks * 2048, kHalf, 1024);
+                                const uint64_t b = sdesc(sDS + ks * 2048, kHalf, 1024);
+                                mma(dst, a, b, ID_Q, ks > 0 ? 1u : 0u);
+                            }
+                        }
+                        mma_commit(EMPTY(slot));
+                        mma_commit(STG_FULL(stg));
+                    }
+                    __syncwarp();
+                    if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+                }
+                if (lane == 0 && ok) mma_commit(PDS_FREE);
+            }
+        }
+        if (lane == 0) {
+            mma_commit(DONE);
+            uint64_t t0 = globaltimer();
+            while (!mbar_try(DONE, 0) && globaltimer() - t0 < 1000000000ull) {
+            }
+        }
+    } else if (warp < 4) {
+        // =================== softmax / dS (TMEM lane = key) ===================
+        const int j = threadIdx.x;  // key slot within the tile
+        const float c1 = scale * 1.4426950408889634f;
+        uint8_t* sPp = smem + C::kOffP;
+        uint8_t* sDSp = smem + C::kOffDS;
+        int tile_ctr = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
+            const int t = prm.order[w];
+            const int n = prm.nrows[t];
+            if (n <= 0) continue;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (j < N1) {
+                const float m = prm.smax[(int64_t)t * N1 + j];
+                const float l = prm.ssum[(int64_t)t * N1 + j];
+                cst[j] = m * 1.4426950408889634f;
+                cst[128 + j] = l == 0.f ? 0.f : 1.f / l;
+                cst[256 + j] = prm.rowsum[(int64_t)t * N1 + j];
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            const int ntiles = (n + kKeys - 1) / kKeys;
+            for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
+                const bool valid = tile * kKeys + j < n;
+                ok = wait_bar(SDP_FULL, tile_ctr & 1, abort_flag, prm.err, 8);
+                if (ok && tile_ctr > 0) ok = wait_bar(PDS_FREE, (tile_ctr - 1) & 1, abort_flag, prm.err, 9);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+#pragma unroll 1
+                for (int cc = 0; cc < N1 / 32; ++cc) {
+                    float s[32], dp[32];
+                    tmem_ld32(T_S + lane_base + cc * 32, s);
+                    tmem_ld32(T_DP + lane_base + cc * 32, dp);
+                    tmem_wait_ld();
+                    uint32_t pw[16], dw[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int h = cc * 32 + e;
+                        float p0 = valid ? exp2f(fmaf(s[e], c1, -cst[h])) * cst[128 + h] : 0.f;
+                        float p1 = valid ? exp2f(fmaf(s[e + 1], c1, -cst[h + 1])) * cst[128 + h + 1] : 0.f;
+                        float d0 = p0 * (dp[e] - cst[256 + h]);
+                        float d1 = p1 * (dp[e + 1] - cst[256 + h + 1]);
+                        pw[e >> 1] = pack2<T>(p0, p1);
+                        dw[e >> 1] = pack2<T>(d0, d1);
+                    }
+                    const int half = cc >> 1;
+                    const int u0 = (cc & 1) * 4;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t off = half * kHalf + j * 128 + (((u0 + u) ^ (j & 7)) << 4);
+                        *reinterpret_cast<uint4*>(sPp + off) =
+                            make_uint4(pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
+                        *reinterpret_cast<uint4*>(sDSp + off) =
+                            make_uint4(dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
+                    }
+                }
+                fence_view_async_shared();
+                tc_fence_before();
+                mbar_arrive(PDS_FULL);
+            }
+        }
+    } else {
+        // =================== flush (TMEM lane = output dim) ===================
+        const int q = warp - 4;  // lane quarter
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        int tile_ctr = 0;
+        int blk_ctr = 0;
+        bool ok = true;
+        float* dkv32 = reinterpret_cast<float*>(prm.dkv_acc);
+        unsigned long long* dkv64 = reinterpret_cast<unsigned long long*>(prm.dkv_acc);
+        for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
+            const int t = prm.order[w];
+            const int n = prm.nrows[t];
+            if (n <= 0) continue;
+            const int ntiles = (n + kKeys - 1) / kKeys;
+            for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
+                const int rb = tile_ctr & 1;
+                ok = wait_bar(ROWS_FULL(rb), (tile_ctr >> 1) & 1, abort_flag, prm.err, 10);
+                if (!ok) break;
+                const int32_t* rid = rowids + rb * kKeys;
+                const int nvalid = min(kKeys, n - tile * kKeys);
+                for (int bi = 0; bi < 14 && ok; ++bi, ++blk_ctr) {
+                    const int stg = blk_ctr & 1;
+                    ok = wait_bar(STG_FULL(stg), (blk_ctr >> 1) & 1, abort_flag, prm.err, 11);
+                    if (!ok) break;
+                    tc_fence_after();
+                    // which output block and which dims this lane quarter holds
+                    int kind, b;
+                    if (bi < 4) { kind = 2; b = bi; }
+                    else if (bi < 9) { kind = 1; b = bi - 4; }
+                    else { kind = 0; b = bi - 9; }
+                    const bool active = b < 4 || q < 2;  // rope blocks: 64 valid dims
+                    const int dim = (b < 4 ? b * 128 : kD) + q * 32 + lane;
+                    if (active) {
+                        const int ncols = kind == 0 ? N1 : kKeys;
+                        for (int cc = 0; cc < ncols / 32; ++cc) {
+                            float v[32];
+                            tmem_ld32(T_STG(stg) + lane_base + cc * 32, v);
+                            tmem_wait_ld();
+                            if (kind == 0) {
+                                // dQ~^T: column = head
+                                float* dst = prm.dq_acc + ((int64_t)t * N1 + cc * 32) * kDK + dim;
+#pragma unroll 8
+                                for (int e = 0; e < 32; ++e) atomicAdd(dst + (int64_t)e * kDK, v[e] * scale);
+                            } else {
+                                // dV^T / dK~^T: column = key
+                                const int col = kind == 2 ? kDK + dim : dim;
+                                const float mul = kind == 2 ? 1.f : scale;
+                                const int lim = min(32, nvalid - cc * 32);
+#pragma unroll 4
+                                for (int e = 0; e < lim; ++e) {
+                                    const int64_t off = (int64_t)rid[cc * 32 + e] * kAccW + col;
+                                    if (prm.det)
+                                        atomicAdd(dkv64 + off, (unsigned long long)__float2ll_rn(v[e] * mul * kFixScale));
+                                    else
+                                        atomicAdd(dkv32 + off, v[e] * mul);
+                                }
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive(STG_EMPTY(stg));
+                }
+                if (ok) mbar_arrive(ROWS_EMPTY(rb));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, int dtype, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, dtype == SFA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                    const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename T, int N1>
+cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
+    FusedParams p;
+    memset(&p, 0, sizeof p);
+    const int64_t T1 = a.sd.T1, T2 = a.sd.T2;
+    if (!make_map(&p.mapQ, a.q, a.dtype, kD, (uint64_t)T1 * N1, N1) ||
+        !make_map(&p.mapQr, a.qr, a.dtype, kDr, (uint64_t)T1 * N1, N1) ||
+        !make_map(&p.mapO, a.dout, a.dtype, kD, (uint64_t)T1 * N1, N1) ||
+        !make_map(&p.mapK, a.k, a.dtype, kD, (uint64_t)T2, 1) || !make_map(&p.mapKr, a.kr, a.dtype, kDr, (uint64_t)T2, 1))
+        return cudaErrorInvalidValue;
+    p.rowlist = a.rowlist;
+    p.nrows = a.nrows;
+    p.order = a.order;
+    p.smax = a.smax;
+    p.ssum = a.ssum;
+    p.rowsum = a.rowsum;
+    p.dkv_acc = a.dkv_acc;
+    p.dq_acc = a.dq_acc;
+    p.err = a.ctrl;
+    p.T1 = T1;
+    p.cap = a.rowcap;
+    p.scale = a.scale;
+    p.det = a.det ? 1 : 0;
+    auto kern = sfa_bwd_fused_kernel<T, N1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<N1>::kSmem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int grid = (int)(T1 < sms ? T1 : sms);
+    if (grid < 1) return cudaSuccess;
+    kern<<<grid, kThreads, Cfg<N1>::kSmem, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool fused_supported(int64_t N1) { return N1 == 64 || N1 == 128; }
+
 cudaError_t launch_bwd_fused(int dtype, const GradArgs& a, cudaStream_t st) {
-    (void)dtype;
-    (void)a;
-    (void)st;
-    return cudaErrorNotSupported;
+    if (dtype == SFA_DTYPE_BF16)
+        return a.N1 == 128 ? launch_t<__nv_bfloat16, 128>(a, st) : launch_t<__nv_bfloat16, 64>(a, st);
+    return a.N1 == 128 ? launch_t<__half, 128>(a, st) : launch_t<__half, 64>(a, st);
 }
 
 }  // namespace sfa

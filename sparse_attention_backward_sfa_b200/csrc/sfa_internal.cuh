@@ -112,13 +112,14 @@ struct GradWs {
     size_t nrows;   // [T1] int32
     size_t order;   // [T1] int32 work order (longest first)
     size_t rowsum;  // [T1][N1] fp32 FlashSoftmaxGrad
+    size_t rowlist; // [T1][topk*bs] int32 gathered key rows, fused path only
     size_t ctrl;    // 256 B of counters / flags
     size_t total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-inline GradWs grad_ws_layout(int64_t T1, int64_t T2, int64_t N1, int64_t topk, bool det, bool fused) {
+inline GradWs grad_ws_layout(int64_t T1, int64_t T2, int64_t N1, int64_t topk, int64_t bs, bool det, bool fused) {
     GradWs w;
     size_t o = 0;
     w.dkv = o;    o = align256(o + (size_t)T2 * kAccW * (det ? 8 : 4));
@@ -128,6 +129,7 @@ inline GradWs grad_ws_layout(int64_t T1, int64_t T2, int64_t N1, int64_t topk, b
     w.nrows = o;  o = align256(o + (size_t)T1 * 4);
     w.order = o;  o = align256(o + (size_t)T1 * 4);
     w.rowsum = o; o = align256(o + (size_t)T1 * N1 * 4);
+    w.rowlist = o; o = align256(o + (fused ? (size_t)T1 * topk * bs * 4 : 0));
     w.ctrl = o;   o = align256(o + 256);
     w.total = o;
     return w;
@@ -141,6 +143,8 @@ cudaError_t launch_compact(const int32_t* idx, const SeqDesc& sd, int64_t topk, 
 cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t T1, int64_t N1, float* rowsum,
                           cudaStream_t st);
 cudaError_t launch_order(const int32_t* nrows, int64_t T1, int32_t* order, int32_t* ctrl, cudaStream_t st);
+cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs, int mode,
+                          int64_t cap, int32_t* rowlist, cudaStream_t st);
 cudaError_t launch_cast_dkv(int dtype, bool det, const void* acc, int64_t T2, void* dk, void* dkr, void* dv,
                             cudaStream_t st);
 cudaError_t launch_cast_dq(int dtype, const float* acc, int64_t T1, int64_t N1, void* dq, void* dqr,
@@ -153,6 +157,7 @@ struct GradArgs {
     const int32_t* blocks; const int32_t* nblk; const int32_t* nrows; const int32_t* order;
     const float* rowsum; void* dkv_acc; float* dq_acc; int32_t* ctrl;
     void* dq; void* dqr;
+    int dtype; const int32_t* rowlist; int64_t rowcap;
 };
 cudaError_t launch_bwd_generic(int dtype, const GradArgs& a, cudaStream_t st);
 cudaError_t launch_bwd_fused(int dtype, const GradArgs& a, cudaStream_t st);

@@ -103,6 +103,42 @@ cudaError_t launch_order(const int32_t* nrows, int64_t T1, int32_t* order, int32
     return cudaGetLastError();
 }
 
+// Expand each query row's compacted block list into its gathered key rows
+// (global row ids, in index order), one warp per query row.
+__global__ void expand_kernel(const int32_t* __restrict__ blocks, const int32_t* __restrict__ nblk, SeqDesc sd,
+                              int64_t topk, int bs, int mode, int64_t cap, int32_t* __restrict__ rowlist) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= sd.T1) return;
+    const TokInfo ti = tok_info(sd, t);
+    const int nb = nblk[t];
+    int32_t* dst = rowlist + t * cap;
+    int64_t base = 0;
+    for (int c = 0; c < nb; c += 32) {
+        const int i = c + lane;
+        const int64_t blk = i < nb ? blocks[t * topk + i] : 0;
+        const int n = i < nb ? block_rows(blk, bs, ti, mode) : 0;
+        int x = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        const int total = __shfl_sync(0xffffffffu, x, 31);
+        const int64_t first = ti.kv_start + blk * bs;
+        for (int r = 0; r < n; ++r) dst[base + (x - n) + r] = (int32_t)(first + r);
+        base += total;
+    }
+}
+
+cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs, int mode,
+                          int64_t cap, int32_t* rowlist, cudaStream_t st) {
+    const int warps = 8;
+    int64_t grid = (sd.T1 + warps - 1) / warps;
+    if (grid > 0) expand_kernel<<<(unsigned)grid, warps * 32, 0, st>>>(blocks, nblk, sd, topk, bs, mode, cap, rowlist);
+    return cudaGetLastError();
+}
+
 // [T2][1088] accumulator -> dKey [T2][512], dKeyRope [T2][64], dValue [T2][512].
 template <typename T, bool DET>
 __global__ void cast_dkv_kernel(const void* __restrict__ acc, int64_t T2, T* __restrict__ dk, T* __restrict__ dkr,

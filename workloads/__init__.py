@@ -12,6 +12,8 @@ from .gen import (  # noqa: F401
     bf16_bits,
     make_problem,
     make_fa_problem,
+    make_device_problem,
+    RowView,
     FAProblem,
     tiny_problem,
     subproblem,

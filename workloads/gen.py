@@ -274,3 +274,101 @@ WORKLOADS = {
     4: "sfa_tnd_2048-4096-4096-6144_n128_topk1024x16_causal_deterministic",
     5: "sfa_bsnd_s32768_n128_topk8192_bs1_causal_atomic",
 }
+
+
+# ---------------------------------------------------------------------------
+# Device-side generation of the large workloads (3, 4, 5)
+# ---------------------------------------------------------------------------
+def _dev_causal_distinct(gen: torch.Generator, n_valid: torch.Tensor, topk: int, chunk: int) -> torch.Tensor:
+    """Row t: min(n_valid[t], topk) distinct values uniform in [0, n_valid[t]),
+    random order, then -1 padding (same distribution as the host generator)."""
+    T = n_valid.numel()
+    dev = n_valid.device
+    hi = int(n_valid.max().item())
+    kk = min(topk, hi)
+    out = torch.full((T, topk), -1, dtype=torch.int32, device=dev)
+    ar = torch.arange(hi, device=dev)[None, :]
+    for s in range(0, T, chunk):
+        nv = n_valid[s:s + chunk]
+        keys = torch.rand((nv.numel(), hi), generator=gen, device=dev)
+        keys.masked_fill_(ar >= nv[:, None], 2.0)
+        val, pos = torch.topk(keys, kk, dim=1, largest=False, sorted=True)
+        pos = torch.where(val < 1.5, pos, torch.full_like(pos, -1))
+        out[s:s + chunk, :kk] = pos.to(torch.int32)
+    return out
+
+
+def make_device_problem(cfg: int, device="cuda", seed: Optional[int] = None) -> Problem:
+    """Workloads 3, 4, 5 generated directly on the device as torch tensors in the
+    library's layouts (q [B,S1,N1,D] or [T1,N1,D], key [..,1,D], indices
+    [..,1,topk]); value is key.  Seed defaults to 2000 + cfg."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(2000 + cfg if seed is None else seed)
+    D, Dr = 512, 64
+    if cfg == 3:
+        B, S, N1, topk, bs = 1, 8192, 64, 2048, 1
+        layout, lens = "BSND", None
+    elif cfg == 4:
+        lens = [2048, 4096, 4096, 6144]
+        B, N1, topk, bs = 4, 128, 1024, 16
+        layout = "TND"
+    elif cfg == 5:
+        B, S, N1, topk, bs = 1, 32768, 128, 8192, 1
+        layout, lens = "BSND", None
+    else:
+        raise ValueError(cfg)
+    if layout == "BSND":
+        T1 = T2 = B * S
+        S1 = S2 = S
+        nvalid = torch.arange(1, S + 1, device=device).repeat(B)
+        sq = skv = None
+        qs, ks, ish = (B, S, N1), (B, S, 1), (B, S, 1, topk)
+    else:
+        T1 = T2 = int(sum(lens))
+        S1 = S2 = 0
+        nvalid = torch.cat([torch.arange(L, device=device) // bs + 1 for L in lens])
+        cu = torch.tensor(np.cumsum(lens), dtype=torch.int32, device=device)
+        sq = skv = cu
+        qs, ks, ish = (T1, N1), (T2, 1), (T1, 1, topk)
+    idx = _dev_causal_distinct(gen, nvalid, topk, chunk=max(1, (1 << 25) // int(nvalid.max().item()))).reshape(ish)
+
+    def rnd(*shape):
+        return torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+    q = rnd(*qs, D)
+    qr = rnd(*qs, Dr)
+    k = rnd(*ks, D)
+    kr = rnd(*ks, Dr)
+    do = rnd(*qs, D)
+    det = cfg == 4
+    return Problem(f"cfg{cfg}", layout, B, S1, S2, T1, T2, N1, D, Dr, topk, bs, 3, det, _scale(D, Dr), sq, skv,
+                   q, qr, k, kr, do, idx, meta={"seed": 2000 + cfg if seed is None else seed, "device": True})
+
+
+class RowView:
+    """Row access t -> numpy row for a subset of rows of a large device tensor,
+    so the oracle can run on sampled query rows without a full host copy."""
+
+    def __init__(self, tensor: torch.Tensor, rows, flat_rows: int):
+        flat = tensor.reshape(flat_rows, -1)
+        self._shape = tensor.shape[tensor.dim() - _row_rank(tensor, flat_rows):]
+        rows = sorted(int(r) for r in rows)
+        sel = flat[torch.tensor(rows, device=tensor.device, dtype=torch.long)].float().cpu().numpy()
+        self._rows = {r: sel[i].reshape(self._shape) for i, r in enumerate(rows)}
+        self._n = flat_rows
+
+    def __len__(self):
+        return self._n
+
+    def __getitem__(self, t):
+        return self._rows[int(t)]
+
+
+def _row_rank(tensor: torch.Tensor, flat_rows: int) -> int:
+    """Number of trailing dims that make up one flattened row."""
+    n = 1
+    for r in range(tensor.dim() - 1, -1, -1):
+        lead = int(np.prod(tensor.shape[:r])) if r else 1
+        if lead == flat_rows:
+            return tensor.dim() - r
+    raise ValueError("row count does not match a leading product of the shape")
