@@ -146,6 +146,9 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:  # torch creates the CUDA event on first record; the hook needs real handles
+        a.record(stream)
+        b.record(stream)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank) as clk:
         torch.cuda.synchronize(dev)
@@ -286,9 +289,9 @@ def main():
             return
         per_step = []
         res = None
-        budget = 20.0
+        budget = max(2.0, min(20.0, 90.0 / max(1, args.steps)))  # whole run ~1.5-2 min
         for i in range(args.warmup + args.steps):
-            res = cpu_baseline(args.workload, budget if i >= args.warmup else 2.0)
+            res = cpu_baseline(args.workload, budget if i >= args.warmup else 1.0)
             if i >= args.warmup:
                 per_step.append(res)
         val = statistics.mean(r["value"] for r in per_step)

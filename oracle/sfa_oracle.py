@@ -147,9 +147,9 @@ def sfa_forward(q, k, v, indices, q_rope, k_rope, scale: float, block_size: int,
     """
     k, v, k_rope = (_as(a, dtype) for a in (k, v, k_rope))
     T1 = len(q)
-    N1 = _row(q, 0, dtype).shape[0]
-    Dv = v.shape[1]
     sel = list(range(T1)) if tokens is None else sorted(int(t) for t in tokens)
+    N1 = _row(q, sel[0] if sel else 0, dtype).shape[0]
+    Dv = v.shape[1]
     where = {t: i for i, t in enumerate(sel)}
     out = np.zeros((len(sel), N1, Dv), dtype)
     smax = np.zeros((len(sel), N1), dtype)
@@ -194,10 +194,10 @@ def sfa_backward(q, k, v, indices, d_out, out, softmax_max, softmax_sum, q_rope,
     """
     k, v, k_rope = (_as(a, dtype) for a in (k, v, k_rope))
     T1 = len(q)
-    N1, D = _row(q, 0, dtype).shape
-    Dr = _row(q_rope, 0, dtype).shape[1]
-    T2 = k.shape[0]
     sel = list(range(T1)) if tokens is None else sorted(int(t) for t in tokens)
+    N1, D = _row(q, sel[0] if sel else 0, dtype).shape
+    Dr = _row(q_rope, sel[0] if sel else 0, dtype).shape[1]
+    T2 = k.shape[0]
     where = {t: i for i, t in enumerate(sel)}
     kt_all = np.concatenate([k, k_rope], axis=1)
     dqt = np.zeros((len(sel), N1, D + Dr), dtype)

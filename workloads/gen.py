@@ -353,7 +353,8 @@ class RowView:
         flat = tensor.reshape(flat_rows, -1)
         self._shape = tensor.shape[tensor.dim() - _row_rank(tensor, flat_rows):]
         rows = sorted(int(r) for r in rows)
-        sel = flat[torch.tensor(rows, device=tensor.device, dtype=torch.long)].float().cpu().numpy()
+        sel = flat[torch.tensor(rows, device=tensor.device, dtype=torch.long)]
+        sel = (sel.float() if sel.is_floating_point() else sel).cpu().numpy()
         self._rows = {r: sel[i].reshape(self._shape) for i, r in enumerate(rows)}
         self._n = flat_rows
 
