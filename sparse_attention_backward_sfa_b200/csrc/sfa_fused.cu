@@ -24,8 +24,10 @@
 //  * P and dS live in shared memory as bf16 [keys x heads] (SW128 halves of 64
 //    heads); S^T / dP^T and two 128-column staging accumulators live in TMEM
 //    (all 512 columns).
-//  * Warp roles: 0-3 softmax/dS (TMEM lanes = keys), 4-7 flush (TMEM lanes =
-//    dims), 8 TMA producer, 9 MMA issuer.  Every mbarrier wait is bounded; on
+//  * Warp roles: 0-3 softmax/dS (TMEM lanes = keys), 4-11 flush (TMEM lanes =
+//    dims; two warps per lane quarter, each taking half of a block's columns),
+//    12 TMA producer, 13 MMA issuer.  dS is stored pre-multiplied by scale so
+//    the flush is a bare reduction.  Every mbarrier wait is bounded; on
 //    timeout the kernel records an error word, stops issuing, drains what it
 //    issued and frees its TMEM.
 #include <cuda.h>
@@ -39,7 +41,7 @@ namespace sfa {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;   // 4 softmax + 8 flush + 1 TMA + 1 MMA warps
 constexpr int kSlotBytes = 32768;
 constexpr int kHalf = 16384;
 constexpr int kKeys = 128;          // key rows per tile (MMA M)
@@ -220,7 +222,7 @@ __device__ __forceinline__ void item_of(int i, int& kind, int& c) {
     kind = 0; c = i - 9;
 }
 
-template <typename T, int N1>
+template <typename T, int N1, bool DET>
 __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid_constant__ FusedParams prm) {
     using C = Cfg<N1>;
     constexpr bool kF16 = std::is_same<T, __half>::value;
@@ -258,9 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
         mbar_init(PDS_FREE, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(STG_FULL(s), 1);
-            mbar_init(STG_EMPTY(s), 128);
+            mbar_init(STG_EMPTY(s), 256);
             mbar_init(ROWS_FULL(s), 1);
-            mbar_init(ROWS_EMPTY(s), 128);
+            mbar_init(ROWS_EMPTY(s), 256);
         }
         mbar_init(DONE, 1);
         *abort_flag = 0;
@@ -281,14 +283,13 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
     const int nwork = (int)prm.T1;
     const float scale = prm.scale;
 
-    if (warp == 8) {
+    if (warp == 12) {
         // =================== TMA producer ===================
         int slot = 0;
         uint32_t sphase = 0;
         int tile_ctr = 0;
         bool ok = true;
-        int issued_full[8];  // slots whose loads may still be in flight
-        for (int s = 0; s < 8; ++s) issued_full[s] = 0;
+        uint32_t issued_mask = 0;  // slots that have received loads
         for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
             const int t = prm.order[w];
             const int n = prm.nrows[t];
@@ -332,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                                 tma_load_2d(d, map, col, t * N1, FULL(slot));
                             }
                         }
-                        issued_full[slot] = 1;
+                        issued_mask |= 1u << slot;
                     }
                     if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
                 }
@@ -344,14 +345,14 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 // the most recent use of each slot is the one still possibly in flight
                 const int s = (slot + k) % C::kSlots;
                 const uint32_t ph = s < slot ? sphase : sphase ^ 1;
-                if (issued_full[s]) {
+                if (issued_mask & (1u << s)) {
                     uint64_t t0 = globaltimer();
                     while (!mbar_try(FULL(s), ph) && globaltimer() - t0 < 1000000000ull) {
                     }
                 }
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == 13) {
         // =================== MMA issuer ===================
         const uint32_t ID_S = idesc(128, N1, false, false, kF16);      // S^T, dP^T
         const uint32_t ID_G = idesc(128, 128, true, false, kF16);      // dV^T, dK~^T (N = keys)
@@ -486,8 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                         const int h = cc * 32 + e;
                         float p0 = valid ? exp2f(fmaf(s[e], c1, -cst[h])) * cst[128 + h] : 0.f;
                         float p1 = valid ? exp2f(fmaf(s[e + 1], c1, -cst[h + 1])) * cst[128 + h + 1] : 0.f;
-                        float d0 = p0 * (dp[e] - cst[256 + h]);
-                        float d1 = p1 * (dp[e + 1] - cst[256 + h + 1]);
+                        float d0 = p0 * (dp[e] - cst[256 + h]) * scale;
+                        float d1 = p1 * (dp[e + 1] - cst[256 + h + 1]) * scale;
                         pw[e >> 1] = pack2<T>(p0, p1);
                         dw[e >> 1] = pack2<T>(d0, d1);
                     }
@@ -509,7 +510,8 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
         }
     } else {
         // =================== flush (TMEM lane = output dim) ===================
-        const int q = warp - 4;  // lane quarter
+        const int q = warp & 3;                 // TMEM lane quarter of this warp
+        const int hsel = (warp - 4) >> 2;       // which half of each block's columns
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         int tile_ctr = 0;
         int blk_ctr = 0;
@@ -540,28 +542,31 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                     const bool active = b < 4 || q < 2;  // rope blocks: 64 valid dims
                     const int dim = (b < 4 ? b * 128 : kD) + q * 32 + lane;
                     if (active) {
-                        const int ncols = kind == 0 ? N1 : kKeys;
-                        for (int cc = 0; cc < ncols / 32; ++cc) {
+                        const int nch = (kind == 0 ? N1 : kKeys) / 32;
+                        const int c0 = hsel * (nch >> 1);
+                        for (int cc = c0; cc < c0 + (nch >> 1); ++cc) {
                             float v[32];
                             tmem_ld32(T_STG(stg) + lane_base + cc * 32, v);
                             tmem_wait_ld();
                             if (kind == 0) {
-                                // dQ~^T: column = head
+                                // dQ~^T: column = head; rows of dq_acc are 576 floats apart
                                 float* dst = prm.dq_acc + ((int64_t)t * N1 + cc * 32) * kDK + dim;
-#pragma unroll 8
-                                for (int e = 0; e < 32; ++e) atomicAdd(dst + (int64_t)e * kDK, v[e] * scale);
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) atomicAdd(dst + e * kDK, v[e]);
                             } else {
-                                // dV^T / dK~^T: column = key
-                                const int col = kind == 2 ? kDK + dim : dim;
-                                const float mul = kind == 2 ? 1.f : scale;
-                                const int lim = min(32, nvalid - cc * 32);
-#pragma unroll 4
-                                for (int e = 0; e < lim; ++e) {
-                                    const int64_t off = (int64_t)rid[cc * 32 + e] * kAccW + col;
-                                    if (prm.det)
-                                        atomicAdd(dkv64 + off, (unsigned long long)__float2ll_rn(v[e] * mul * kFixScale));
-                                    else
-                                        atomicAdd(dkv32 + off, v[e] * mul);
+                                // dV^T / dK~^T: column = key; skip the padding keys of the last tile
+                                const size_t col = kind == 2 ? kDK + dim : dim;
+                                const int32_t* r = rid + cc * 32;
+                                const int lim = nvalid - cc * 32;
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) {
+                                    if (e < lim) {
+                                        const size_t off = (size_t)(uint32_t)r[e] * kAccW + col;
+                                        if (DET)
+                                            atomicAdd(dkv64 + off, (unsigned long long)__float2ll_rn(v[e] * kFixScale));
+                                        else
+                                            atomicAdd(dkv32 + off, v[e]);
+                                    }
                                 }
                             }
                         }
@@ -614,7 +619,7 @@ bool make_map(CUtensorMap* m, const void* base, int dtype, uint64_t cols, uint64
     return r == CUDA_SUCCESS;
 }
 
-template <typename T, int N1>
+template <typename T, int N1, bool DET>
 cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
     FusedParams p;
     memset(&p, 0, sizeof p);
@@ -636,8 +641,8 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
     p.T1 = T1;
     p.cap = a.rowcap;
     p.scale = a.scale;
-    p.det = a.det ? 1 : 0;
-    auto kern = sfa_bwd_fused_kernel<T, N1>;
+    p.det = DET ? 1 : 0;
+    auto kern = sfa_bwd_fused_kernel<T, N1, DET>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<N1>::kSmem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -653,10 +658,14 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
 
 bool fused_supported(int64_t N1) { return N1 == 64 || N1 == 128; }
 
+template <typename T>
+cudaError_t launch_n1(const GradArgs& a, cudaStream_t st) {
+    if (a.N1 == 128) return a.det ? launch_t<T, 128, true>(a, st) : launch_t<T, 128, false>(a, st);
+    return a.det ? launch_t<T, 64, true>(a, st) : launch_t<T, 64, false>(a, st);
+}
+
 cudaError_t launch_bwd_fused(int dtype, const GradArgs& a, cudaStream_t st) {
-    if (dtype == SFA_DTYPE_BF16)
-        return a.N1 == 128 ? launch_t<__nv_bfloat16, 128>(a, st) : launch_t<__nv_bfloat16, 64>(a, st);
-    return a.N1 == 128 ? launch_t<__half, 128>(a, st) : launch_t<__half, 64>(a, st);
+    return dtype == SFA_DTYPE_BF16 ? launch_n1<__nv_bfloat16>(a, st) : launch_n1<__half>(a, st);
 }
 
 }  // namespace sfa
