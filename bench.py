@@ -94,10 +94,14 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+SEQS = None  # optional override of workload 4's sequence lengths (--seqs, for profiling captures)
+
+
 def build_problem(workload: int, seed_offset: int, device):
     from workloads import make_device_problem
     p = make_device_problem(workload, device=device,
-                            seed=None if seed_offset == 0 else 2000 + workload + 7919 * seed_offset)
+                            seed=None if seed_offset == 0 else 2000 + workload + 7919 * seed_offset,
+                            seqs=SEQS if workload == 4 else None)
     return p
 
 
@@ -275,7 +279,12 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqs", default=None,
+                    help="comma-separated sequence lengths replacing workload 4's (smaller profiling case)")
     args = ap.parse_args()
+    global SEQS
+    if args.seqs:
+        SEQS = [int(x) for x in args.seqs.split(",")]
     if args.warmup < 3:
         args.warmup = 3
 
@@ -329,7 +338,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": r["ms_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "pct_of_peak": 100.0 * value / world / peak,
-            "config": {"workload": WORKLOADS[args.workload], "layout": p.layout, "N1": p.N1, "topk": p.topk,
+            "config": {"workload": WORKLOADS[args.workload] + (f" seqs={args.seqs}" if args.seqs else ""),
+                       "layout": p.layout, "N1": p.N1, "topk": p.topk,
                        "sparse_block_size": p.block_size, "deterministic": p.deterministic,
                        "valid_triples": r["triples"], "gflop_per_step": r["flop"] / 1e9,
                        "l2": "inputs larger than L2 (q+dO+O %.1f GB per step)" % (3 * p.q.numel() * 2 / 1e9),

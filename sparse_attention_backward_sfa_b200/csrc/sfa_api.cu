@@ -187,7 +187,6 @@ sfa_status sfa_grad(const void* query, const void* key, const void* value, const
                             (int32_t*)a.nrows, s), "index compaction");
     const bool fused = fused_shape && value == key;
     if (fused) {
-        SFA_CUDA(cudaMemsetAsync(a.dq_acc, 0, (size_t)z.T1 * shape->N1 * kDK * 4, s), "zero dQ accumulator");
         SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, z.T1, shape->N1, (float*)a.rowsum, s), "rowsum(dO*O)");
         SFA_CUDA(launch_order(a.nrows, z.T1, (int32_t*)a.order, a.ctrl, s), "work order");
         SFA_CUDA(launch_expand(a.blocks, a.nblk, a.sd, a.topk, a.bs, a.mode, a.rowcap, (int32_t*)a.rowlist, s),
@@ -196,7 +195,6 @@ sfa_status sfa_grad(const void* query, const void* key, const void* value, const
             KernelEvents ev(s);
             SFA_CUDA(launch_bwd_fused(shape->dtype, a, s), "fused backward");
         }
-        SFA_CUDA(launch_cast_dq(shape->dtype, a.dq_acc, z.T1, shape->N1, d_query, d_query_rope, s), "cast dQuery");
     } else {
         KernelEvents ev(s);
         SFA_CUDA(launch_bwd_generic(shape->dtype, a, s), "backward");

@@ -45,12 +45,10 @@ constexpr int kThreads = 448;   // 4 softmax + 8 flush + 1 TMA + 1 MMA warps
 constexpr int kSlotBytes = 32768;
 constexpr int kHalf = 16384;
 constexpr int kKeys = 128;          // key rows per tile (MMA M)
-constexpr int kItemsPerTile = 28;   // 14 for S/dP, 14 for the gradient blocks
 
 template <int N1> struct Cfg {
     static constexpr int kSlots = N1 == 128 ? 5 : 6;
     static constexpr int kRing = kSlots * kSlotBytes;
-    static constexpr int kPBytes = N1 * 2 * kKeys;   // bf16 [128 keys x N1 heads]
     static constexpr int kOffP = kRing;
     static constexpr int kOffDS = kOffP + (N1 == 128 ? 32768 : 16384);
     static constexpr int kOffRows = kOffDS + (N1 == 128 ? 32768 : 16384);  // int32 [2][128]
@@ -201,7 +199,9 @@ struct FusedParams {
     const float* ssum;
     const float* rowsum;     // [T1][N1]
     void* dkv_acc;           // [T2][1088] fp32 or int64
-    float* dq_acc;           // [T1][N1][576]
+    float* dq_scratch;       // [gridDim.x][N1][576] fp32 per-CTA partial dQ~ of the current row
+    void* dq_out;            // dQuery [T1][N1][512]
+    void* dqr_out;           // dQueryRope [T1][N1][64]
     int* err;                // device error word
     int64_t T1;
     int64_t cap;
@@ -220,6 +220,89 @@ __device__ __forceinline__ void item_of(int i, int& kind, int& c) {
     if (i < 4) { kind = 2; c = i; return; }
     if (i < 9) { kind = 1; c = i - 4; return; }
     kind = 0; c = i - 9;
+}
+
+// Reductions of one 32-column chunk of a staged gradient block held by this
+// thread (its TMEM lane = output dim `dim`).  kind 0: dQ~ (column = head);
+// kind 1 / 2: dK~ / dV (column = key, padding keys of the last tile skipped).
+enum { DQ_SINGLE = 0, DQ_FIRST = 1, DQ_MID = 2, DQ_LAST = 3 };
+
+__device__ __forceinline__ void st_relaxed(float* a, float v) {
+    asm volatile("st.relaxed.gpu.global.f32 [%0], %1;" ::"l"(a), "f"(v) : "memory");
+}
+__device__ __forceinline__ float ld_relaxed(const float* a) {
+    float v;
+    asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(a) : "memory");
+    return v;
+}
+
+// dQ~ of one query row accumulates across its key tiles in this CTA's scratch:
+// the first tile stores, middle tiles reduce, the last tile reads back, adds and
+// writes the 16-bit dQuery / dQueryRope; a single-tile row is written directly.
+// Every element is handled by the same thread in tile order.
+template <typename T, int N1>
+__device__ __forceinline__ void flush_dq(const float (&v)[32], int mode, int cc, int t, int dim, const FusedParams& prm) {
+    float* sc = prm.dq_scratch + ((size_t)blockIdx.x * N1 + cc * 32) * kDK + dim;
+    if (mode == DQ_FIRST) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) st_relaxed(sc + e * kDK, v[e]);
+        return;
+    }
+    if (mode == DQ_MID) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) atomicAdd(sc + e * kDK, v[e]);
+        return;
+    }
+    float x[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = v[e];
+    if (mode == DQ_LAST) {
+#pragma unroll
+        for (int h = 0; h < 32; h += 16) {
+            float y[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) y[e] = ld_relaxed(sc + (h + e) * kDK);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) x[h + e] += y[e];
+        }
+    }
+    const int64_t row0 = (int64_t)t * N1 + cc * 32;
+    if (dim < kD) {
+        T* o = reinterpret_cast<T*>(prm.dq_out) + row0 * kD + dim;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e * kD] = from_f<T>(x[e]);
+    } else {
+        T* o = reinterpret_cast<T*>(prm.dqr_out) + row0 * kDr + (dim - kD);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e * kDr] = from_f<T>(x[e]);
+    }
+}
+
+template <bool DET, int N1>
+__device__ __forceinline__ void flush_chunk(const float (&v)[32], int kind, int cc, int t, int dim, const int32_t* rid,
+                                            int nvalid, const FusedParams& prm) {
+    const size_t col = kind == 2 ? kDK + dim : dim;
+    const int32_t* r = rid + cc * 32;
+    const int lim = nvalid - cc * 32;
+    float* d32 = reinterpret_cast<float*>(prm.dkv_acc) + col;
+    unsigned long long* d64 = reinterpret_cast<unsigned long long*>(prm.dkv_acc) + col;
+    if (lim >= 32) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const size_t off = (size_t)(uint32_t)r[e] * kAccW;
+            if (DET) atomicAdd(d64 + off, (unsigned long long)__float2ll_rn(v[e] * kFixScale));
+            else atomicAdd(d32 + off, v[e]);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            if (e < lim) {
+                const size_t off = (size_t)(uint32_t)r[e] * kAccW;
+                if (DET) atomicAdd(d64 + off, (unsigned long long)__float2ll_rn(v[e] * kFixScale));
+                else atomicAdd(d32 + off, v[e]);
+            }
+        }
+    }
 }
 
 template <typename T, int N1, bool DET>
@@ -298,7 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
             const int ntiles = (n + kKeys - 1) / kKeys;
             for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
                 const int rb = tile_ctr & 1;
-                ok = wait_bar(ROWS_EMPTY(rb), ((tile_ctr >> 1) & 1) ^ 1, abort_flag, prm.err, 1);
+                if (lane == 0) ok = wait_bar(ROWS_EMPTY(rb), ((tile_ctr >> 1) & 1) ^ 1, abort_flag, prm.err, 1);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 int32_t* rid = rowids + rb * kKeys;
                 const int first = rl[0];
@@ -308,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ROWS_FULL(rb));
-                for (int it = 0; it < kItemsPerTile && ok; ++it) {
+                for (int it = 0; it < 28 && ok; ++it) {
                     int kind, c;
                     item_of(it, kind, c);
                     if (lane == 0) ok = wait_bar(EMPTY(slot), sphase ^ 1, abort_flag, prm.err, 2);
@@ -370,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
             const int ntiles = (n + kKeys - 1) / kKeys;
             for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
                 // ---- S^T and dP^T over the 5 / 4 chunks ----
-                uint32_t slotK = 0, slotQ = 0;
+                uint32_t slotK = 0;
                 for (int it = 0; it < 14 && ok; ++it) {
                     int kind, c;
                     item_of(it, kind, c);
@@ -380,21 +464,19 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                     tc_fence_after();
                     const uint32_t sa = sbase + slot * kSlotBytes;
                     if (kind == 0) slotK = sa;
-                    else if (kind == 1) slotQ = sa;
-                    const int ksteps = c < 4 ? 8 : 4;
                     if (lane == 0 && kind != 0) {
                         const uint32_t dst = kind == 1 ? T_S : T_DP;
+                        const int ksteps = c < 4 ? 8 : 4;
                         for (int ks = 0; ks < ksteps; ++ks) {
                             const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
                             const uint64_t a = sdesc(slotK + off, 16, 1024);
                             const uint64_t b = sdesc(sa + off, 16, 1024);
                             mma(dst, a, b, ID_S, (c > 0 || ks > 0) ? 1u : 0u);
                         }
+                        // a slot is released once the MMAs that read it have completed
+                        mma_commit(EMPTY(slot));
+                        if (kind == 2 || c == 4) mma_commit(EMPTY((slotK - sbase) / kSlotBytes));
                     }
-                    // a slot is released once the MMAs that read it have completed
-                    const bool release_k = (kind == 2) || (kind == 1 && c == 4);
-                    if (lane == 0 && kind != 0) mma_commit(EMPTY(slot));
-                    if (lane == 0 && release_k) mma_commit(EMPTY((slotK - sbase) / kSlotBytes));
                     __syncwarp();
                     if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
                 }
@@ -516,14 +598,22 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
         int tile_ctr = 0;
         int blk_ctr = 0;
         bool ok = true;
-        float* dkv32 = reinterpret_cast<float*>(prm.dkv_acc);
-        unsigned long long* dkv64 = reinterpret_cast<unsigned long long*>(prm.dkv_acc);
+        const int ep = threadIdx.x - 128;  // 0..255 across the flush warps
         for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
             const int t = prm.order[w];
             const int n = prm.nrows[t];
-            if (n <= 0) continue;
+            if (n <= 0) {
+                // no key for this query row (or a BSND padding row): dQuery = 0
+                uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<T*>(prm.dq_out) + (int64_t)t * N1 * kD);
+                uint4* orp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(prm.dqr_out) + (int64_t)t * N1 * kDr);
+                for (int i = ep; i < N1 * kD / 8; i += 256) o[i] = make_uint4(0, 0, 0, 0);
+                for (int i = ep; i < N1 * kDr / 8; i += 256) orp[i] = make_uint4(0, 0, 0, 0);
+                continue;
+            }
             const int ntiles = (n + kKeys - 1) / kKeys;
             for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
+                const int dqmode = ntiles == 1 ? DQ_SINGLE
+                                   : (tile == 0 ? DQ_FIRST : (tile == ntiles - 1 ? DQ_LAST : DQ_MID));
                 const int rb = tile_ctr & 1;
                 ok = wait_bar(ROWS_FULL(rb), (tile_ctr >> 1) & 1, abort_flag, prm.err, 10);
                 if (!ok) break;
@@ -544,31 +634,13 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                     if (active) {
                         const int nch = (kind == 0 ? N1 : kKeys) / 32;
                         const int c0 = hsel * (nch >> 1);
-                        for (int cc = c0; cc < c0 + (nch >> 1); ++cc) {
+                        const int c1 = c0 + (nch >> 1);
+                        for (int cc = c0; cc < c1; ++cc) {
                             float v[32];
                             tmem_ld32(T_STG(stg) + lane_base + cc * 32, v);
                             tmem_wait_ld();
-                            if (kind == 0) {
-                                // dQ~^T: column = head; rows of dq_acc are 576 floats apart
-                                float* dst = prm.dq_acc + ((int64_t)t * N1 + cc * 32) * kDK + dim;
-#pragma unroll
-                                for (int e = 0; e < 32; ++e) atomicAdd(dst + e * kDK, v[e]);
-                            } else {
-                                // dV^T / dK~^T: column = key; skip the padding keys of the last tile
-                                const size_t col = kind == 2 ? kDK + dim : dim;
-                                const int32_t* r = rid + cc * 32;
-                                const int lim = nvalid - cc * 32;
-#pragma unroll
-                                for (int e = 0; e < 32; ++e) {
-                                    if (e < lim) {
-                                        const size_t off = (size_t)(uint32_t)r[e] * kAccW + col;
-                                        if (DET)
-                                            atomicAdd(dkv64 + off, (unsigned long long)__float2ll_rn(v[e] * kFixScale));
-                                        else
-                                            atomicAdd(dkv32 + off, v[e]);
-                                    }
-                                }
-                            }
+                            if (kind == 0) flush_dq<T, N1>(v, dqmode, cc, t, dim, prm);
+                            else flush_chunk<DET, N1>(v, kind, cc, t, dim, rid, nvalid, prm);
                         }
                     }
                     tc_fence_before();
@@ -636,12 +708,15 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
     p.ssum = a.ssum;
     p.rowsum = a.rowsum;
     p.dkv_acc = a.dkv_acc;
-    p.dq_acc = a.dq_acc;
+    p.dq_scratch = a.dq_acc;
+    p.dq_out = a.dq;
+    p.dqr_out = a.dqr;
     p.err = a.ctrl;
     p.T1 = T1;
     p.cap = a.rowcap;
     p.scale = a.scale;
     p.det = DET ? 1 : 0;
+
     auto kern = sfa_bwd_fused_kernel<T, N1, DET>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<N1>::kSmem);
     if (e != cudaSuccess) return e;
@@ -649,6 +724,7 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int grid = (int)(T1 < sms ? T1 : sms);
+    if (grid > kMaxFusedGrid) grid = kMaxFusedGrid;
     if (grid < 1) return cudaSuccess;
     kern<<<grid, kThreads, Cfg<N1>::kSmem, st>>>(p);
     return cudaGetLastError();

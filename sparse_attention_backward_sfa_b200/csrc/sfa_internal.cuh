@@ -106,7 +106,7 @@ __device__ __forceinline__ int block_rows(int64_t blk, int bs, const TokInfo& ti
 // ---------------------------------------------------------------------------
 struct GradWs {
     size_t dkv;     // [T2][1088] fp32 (atomic) or int64 (deterministic)
-    size_t dq;      // [T1][N1][576] fp32, fused tensor-core path only
+    size_t dq;      // [kMaxFusedGrid][N1][576] fp32 per-CTA dQ~ partial sums, fused path only
     size_t blocks;  // [T1][topk] int32 compacted block indices
     size_t nblk;    // [T1] int32
     size_t nrows;   // [T1] int32
@@ -119,11 +119,13 @@ struct GradWs {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+constexpr int kMaxFusedGrid = 256;  // persistent CTAs of the fused kernel (one per SM)
+
 inline GradWs grad_ws_layout(int64_t T1, int64_t T2, int64_t N1, int64_t topk, int64_t bs, bool det, bool fused) {
     GradWs w;
     size_t o = 0;
     w.dkv = o;    o = align256(o + (size_t)T2 * kAccW * (det ? 8 : 4));
-    w.dq = o;     o = align256(o + (fused ? (size_t)T1 * N1 * kDK * 4 : 0));
+    w.dq = o;     o = align256(o + (fused ? (size_t)kMaxFusedGrid * N1 * kDK * 4 : 0));
     w.blocks = o; o = align256(o + (size_t)T1 * topk * 4);
     w.nblk = o;   o = align256(o + (size_t)T1 * 4);
     w.nrows = o;  o = align256(o + (size_t)T1 * 4);

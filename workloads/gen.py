@@ -298,10 +298,12 @@ def _dev_causal_distinct(gen: torch.Generator, n_valid: torch.Tensor, topk: int,
     return out
 
 
-def make_device_problem(cfg: int, device="cuda", seed: Optional[int] = None) -> Problem:
+def make_device_problem(cfg: int, device="cuda", seed: Optional[int] = None, seqs=None) -> Problem:
     """Workloads 3, 4, 5 generated directly on the device as torch tensors in the
     library's layouts (q [B,S1,N1,D] or [T1,N1,D], key [..,1,D], indices
-    [..,1,topk]); value is key.  Seed defaults to 2000 + cfg."""
+    [..,1,topk]); value is key.  Seed defaults to 2000 + cfg.  `seqs` replaces
+    workload 4's sequence lengths (a smaller case of the same shape, used for
+    profiling captures)."""
     gen = torch.Generator(device=device)
     gen.manual_seed(2000 + cfg if seed is None else seed)
     D, Dr = 512, 64
@@ -309,8 +311,8 @@ def make_device_problem(cfg: int, device="cuda", seed: Optional[int] = None) -> 
         B, S, N1, topk, bs = 1, 8192, 64, 2048, 1
         layout, lens = "BSND", None
     elif cfg == 4:
-        lens = [2048, 4096, 4096, 6144]
-        B, N1, topk, bs = 4, 128, 1024, 16
+        lens = [2048, 4096, 4096, 6144] if seqs is None else [int(x) for x in seqs]
+        B, N1, topk, bs = len(lens), 128, 1024, 16
         layout = "TND"
     elif cfg == 5:
         B, S, N1, topk, bs = 1, 32768, 128, 8192, 1
