@@ -133,6 +133,38 @@ sfa_status sfa_grad(const void *query, const void *key, const void *value, const
                     const sfa_shape *shape, void *workspace, size_t workspace_bytes, sfa_stream_t stream,
                     void *d_query, void *d_key, void *d_value, void *d_query_rope, void *d_key_rope);
 
+/*
+ * sfa_grad_noalloc - sfa_grad for callers that cannot allocate device memory.
+ * (The source pages have no counterpart: it exists for this library's callers.)
+ *
+ * Some callers cannot supply a workspace: code running under another
+ * framework's memory pool (a raw allocation would escape its accounting),
+ * plugins and embedded runtimes that are handed only input and output buffers,
+ * and code where allocating would synchronize the device.  This call takes the
+ * same arguments as sfa_grad minus the workspace, and allocates nothing: its
+ * scratch is a 64 MiB array that is part of the library's device image, so
+ * every GPU that loads the library holds those 64 MiB until the process exits.
+ *  - Computes with the CUDA-core backward kernel; results match sfa_grad within
+ *    the bf16 tolerance (and are bit-identical run to run when deterministic).
+ *  - Problems whose scratch would exceed 64 MiB (the dKey/dValue accumulator,
+ *    T2 x 1088 x 4 bytes, or x 8 when deterministic, plus T1 x topk x 4 bytes of
+ *    index tables) are rejected with SFA_ERR_WORKSPACE before any device work.
+ *  - The first call on each device looks up the array's device address with
+ *    cudaGetSymbolAddress (with that device current); make that first call
+ *    before any stream capture on the device.
+ *  - All calls on a device share the array, which keeps the previous call's
+ *    contents (the accumulator is cleared on the call's stream).  Calls whose
+ *    work overlaps on the GPU (other streams, other threads) race on it and
+ *    must be serialized by the caller.
+ */
+sfa_status sfa_grad_noalloc(const void *query, const void *key, const void *value, const int32_t *sparse_indices,
+                            const void *d_out, const void *out, const float *softmax_max, const float *softmax_sum,
+                            const int32_t *actual_seq_lengths_q, const int32_t *actual_seq_lengths_kv,
+                            const void *query_rope, const void *key_rope, float scale, int64_t sparse_block_size,
+                            int64_t sparse_mode, int64_t pre_tokens, int64_t next_tokens, int32_t deterministic,
+                            const sfa_shape *shape, sfa_stream_t stream, void *d_query, void *d_key, void *d_value,
+                            void *d_query_rope, void *d_key_rope);
+
 /* ------------------------------------------------------------------------- */
 /* Sparse attention forward (produces the inputs `out`, softmax_max/_sum)     */
 /* ------------------------------------------------------------------------- */

@@ -106,6 +106,8 @@ SeqDesc seq_desc(const sfa_shape* s, const Sizes& z, const int32_t* sq, const in
 
 }  // namespace
 
+void sfa::set_last_error(const char* msg) { g_last_error = msg; }
+
 extern "C" {
 
 const char* sfa_version(void) { return "0.1.0"; }

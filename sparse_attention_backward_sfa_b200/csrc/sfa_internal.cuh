@@ -183,6 +183,8 @@ struct FaArgs {
     void* out; float* smax_out; float* ssum_out;
 };
 cudaError_t launch_fa_bwd(int dtype, const FaArgs& a, cudaStream_t st);
+// Sets the message returned by sfa_last_error_string() on the calling thread.
+void set_last_error(const char* msg);
 cudaError_t launch_fa_fwd(int dtype, const FaArgs& a, cudaStream_t st);
 
 }  // namespace sfa
