@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -33,6 +34,36 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-attn backward TFLOP/s (bf16, 5-GEMM count) and % of B200 tensor peak"
 FLOP_PER_TRIPLE = 5504
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "sfa_bwd_fused_kernel_workload4.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "sparse_attention_backward_sfa_b200", "csrc", f)
+                  for f in ("sfa_fused.cu", "tc_common.cuh")]
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the fused kernel on workload 4 from the committed
+    ncu summary, or None when the kernel sources changed since the capture."""
+    try:
+        txt = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    vals = dict(re.findall(r"^(traffic_bytes_per_launch|kernel_source_sha256):\s*(\S+)", txt, re.M))
+    if vals.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def load_peaks():
@@ -216,6 +247,59 @@ def run_ours(args, rank, world, local_rank):
                 ws_bytes=ws_bytes, err_word=err_word, p=p)
 
 
+def run_fa(args, rank, world, local_rank):
+    """Workload 2: dense varlen FA backward (TND, causal); 1280 FLOP per valid
+    (query row, head, key) triple."""
+    import torch
+    import torch.distributed as dist
+    import sparse_attention_backward_sfa_b200 as S
+    from sparse_attention_backward_sfa_b200 import _native as N
+    from workloads import make_fa_problem
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lib = N.load()
+    fp = make_fa_problem(seed=1002 + 7919 * rank)
+    t = lambda a: torch.from_numpy(a).to(device=dev, dtype=torch.bfloat16)
+    q, k, v, dy = t(fp.q), t(fp.k), t(fp.v), t(fp.dy)
+    out, smax, ssum = S.fa_fwd(q, k, v, fp.cu_seqlens_q, fp.cu_seqlens_kv, scale=fp.scale, sparse_mode=3)
+    lens = np.diff(np.concatenate([[0], fp.cu_seqlens_q]))
+    triples = int(sum(L * (L + 1) // 2 for L in lens)) * fp.Nq
+    flop = triples * 1280
+    outs = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            N.check(lib.sfa_set_kernel_events(ctypes_ptr(ev[0]), ctypes_ptr(ev[1])))
+        S.fa_grad(q, k, v, dy, smax, ssum, out, fp.cu_seqlens_q, fp.cu_seqlens_kv, scale=fp.scale, sparse_mode=3,
+                  outputs=outs)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        a.record(stream)
+        b.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms_step = t0.elapsed_time(t1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_step = float(tt.item())
+    kern_ms = [a.elapsed_time(b) for a, b in evs]
+    return dict(flop=flop, triples=triples, ms_step=ms_step, kern_ms=kern_ms, clocks=clk.summary(), e2e=None,
+                ws_bytes=0, err_word=0, p=None)
+
+
 def ctypes_ptr(ev):
     import ctypes
     return ctypes.c_void_p(ev.cuda_event)
@@ -275,7 +359,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", type=int, default=4, choices=[3, 4, 5])
+    ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -321,17 +405,27 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    r = run_ours(args, rank, world, local_rank)
+    r = run_fa(args, rank, world, local_rank) if args.workload == 2 else run_ours(args, rank, world, local_rank)
     peaks, src = load_peaks()
     value = r["flop"] * world / (r["ms_step"] * 1e-3) / 1e12
     kern = statistics.mean(r["kern_ms"])
     achieved = r["flop"] / (kern * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload != 2:
         cpu = cpu_baseline(args.workload, args.cpu_budget)
         cpu.pop("seconds", None)
-    if rank == 0:
+    if rank == 0 and args.workload == 2:
+        line = {"metric": "dense varlen FA backward TFLOP/s (bf16, 5-GEMM count, D=128)", "value": value,
+                "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": r["ms_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOADS[2], "valid_triples": r["triples"], "gflop_per_step": r["flop"] / 1e9},
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                             "frac": achieved / peak, "kernel": "fa_bwd_kernel", "kernel_ms": kern, "traffic": None},
+                "gpu_launches": 2 * args.steps, "clocks": r["clocks"]}
+        print(json.dumps(line), flush=True)
+    elif rank == 0:
         p = r["p"]
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -348,7 +442,8 @@ def main():
                          "frac": achieved / peak, "peak_source": f"{src} bf16 burst",
                          "peak_sustained": float(peaks.get("bf16_tflops_sustained", peak)),
                          "frac_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
-                         "kernel": "sfa_bwd_fused_kernel", "kernel_ms": kern, "traffic": None},
+                         "kernel": "sfa_bwd_fused_kernel", "kernel_ms": kern,
+                         "traffic": recorded_traffic() if args.workload == 4 and not args.seqs else None},
             "cpu_baseline": cpu,
             "e2e": r["e2e"],
             "gpu_launches": 7 * args.steps,

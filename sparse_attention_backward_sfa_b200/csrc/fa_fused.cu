@@ -1,0 +1,511 @@
+// Tensor-core dense varlen FlashAttention backward for sm_100a, head dim 128
+// (aclnnFlashAttentionUnpaddingScoreGrad, 计算公式: dV = P^T.dY, dQ = scale*dS.K,
+// dK = scale*dS^T.Q with dS = P o (dY.V^T - rowsum(dY o attentionIn)) and
+// P = exp(scale*Q.K^T - softmaxMax) / softmaxSum; TND layout, GQA, sparseMode 0 / 3).
+//
+// Key-major: a work item is one 128-key block of one KV head of one sequence.
+// The CTA loops over the query heads of that KV head's group and over the
+// 128-row query blocks that can see the key block, and accumulates dK and dV
+// for its keys in TMEM (so they are written once, without atomics).  Per
+// (query head, query block):
+//   S^T  = K . Q^T,  dP^T = V . dY^T        [128 keys x 128 queries] in TMEM
+//   P, dS (scale folded in) by the softmax warps (TMEM lane = key) -> SW128 smem
+//   dV  += P  . dY,   dK += dS . Q          [128 keys x 128 dims] in TMEM
+//   dQ^T = K^T . dS^T                        [128 dims x 128 queries], reusing
+//        S^T's columns, reduced into an fp32 (or 64-bit fixed point) dQ buffer
+//        by the flush warps (TMEM lane = dim: 128-byte coalesced reductions).
+// Warps: 0-3 softmax + dK/dV write-out, 4-7 dQ flush, 8 TMA producer, 9 MMA.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cstring>
+#include <type_traits>
+#include <vector>
+
+#include "sfa_internal.cuh"
+#include "tc_common.cuh"
+
+namespace sfa {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kFaD = 128;
+constexpr int kBlk = 128;
+constexpr int kFaThreads = 320;
+constexpr int kOffK = 0, kOffV = 32768, kOffQ = 65536, kOffO = 98304, kOffP = 131072, kOffDS = 163840;
+constexpr int kOffCst = 196608;                 // float [3][128]: max*log2e, 1/sum, rowsum(dY o O)
+constexpr int kOffBar = kOffCst + 3 * 128 * 4;  // 11 mbarriers
+constexpr int kOffMisc = kOffBar + 16 * 8;
+constexpr int kFaSmem = kOffMisc + 16;
+
+struct FaItem {
+    int b, hk, kb, cost;
+};
+
+struct FaParams {
+    CUtensorMap mapQ, mapK, mapV, mapO;  // mapO = dY
+    const FaItem* items;
+    int nitems;
+    const int64_t* cu_q;
+    const int64_t* cu_kv;
+    const float* smax;    // [T1][Nq][8]
+    const float* ssum;
+    const float* rowsum;  // [T1][Nq]
+    void* dq_acc;         // [T1][Nq][128] fp32 or int64
+    void* dk;             // [T2][Nkv][128]
+    void* dv;
+    int* err;
+    int B, Nq, Nkv, mode;
+    float scale;
+};
+
+struct Seq {
+    int64_t qs, ql, ks, kl;
+};
+__device__ __forceinline__ Seq seq_of(const FaParams& p, int b) {
+    Seq s;
+    s.qs = b ? p.cu_q[b - 1] : 0;
+    s.ql = p.cu_q[b] - s.qs;
+    s.ks = b ? p.cu_kv[b - 1] : 0;
+    s.kl = p.cu_kv[b] - s.ks;
+    return s;
+}
+// first query block that can see key block kb (bottom-right causal in mode 3)
+__device__ __forceinline__ int first_qb(const Seq& s, int kb, int mode) {
+    if (mode != 3) return 0;
+    const int64_t lo = (int64_t)kb * kBlk - (s.kl - s.ql);  // smallest query row seeing the block's first key
+    return lo <= 0 ? 0 : (int)(lo / kBlk);
+}
+
+template <typename T, bool DET>
+__global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __grid_constant__ FaParams prm) {
+    constexpr bool kF16 = std::is_same<T, __half>::value;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_u32(smem);
+    if (sbase & 1023u) {
+        if (threadIdx.x == 0) atomicCAS(prm.err, 0, 7);
+        return;
+    }
+    float* cst = reinterpret_cast<float*>(smem + kOffCst);
+    const uint32_t bar0 = sbase + kOffBar;
+    const uint32_t KV_FULL = bar0, KV_EMPTY = bar0 + 8, QDO_FULL = bar0 + 16, QDO_EMPTY = bar0 + 24,
+                   SDP_FULL = bar0 + 32, PDS_FULL = bar0 + 40, PDS_FREE = bar0 + 48, DQ_FULL = bar0 + 56,
+                   S_FREE = bar0 + 64, ACC_FULL = bar0 + 72, ACC_EMPTY = bar0 + 80, DONE = bar0 + 88;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    if (threadIdx.x == 0) {
+        mbar_init(KV_FULL, 1);
+        mbar_init(KV_EMPTY, 1);
+        mbar_init(QDO_FULL, 1);
+        mbar_init(QDO_EMPTY, 1);
+        mbar_init(SDP_FULL, 1);
+        mbar_init(PDS_FULL, 128);
+        mbar_init(PDS_FREE, 1);
+        mbar_init(DQ_FULL, 1);
+        mbar_init(S_FREE, 128);
+        mbar_init(ACC_FULL, 1);
+        mbar_init(ACC_EMPTY, 128);
+        mbar_init(DONE, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {  // S^T / dQ^T [0,128), dP^T [128,256), dK [256,384), dV [384,512)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tmem_slot))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t T_S = tmem, T_DP = tmem + 128, T_DK = tmem + 256, T_DV = tmem + 384;
+    const int G = prm.Nq / prm.Nkv;
+    const float scale = prm.scale;
+
+    if (warp == 8) {
+        // =================== TMA producer ===================
+        int item_ctr = 0, pair_ctr = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < prm.nitems && ok; w += gridDim.x, ++item_ctr) {
+            const FaItem it = prm.items[w];
+            const Seq s = seq_of(prm, it.b);
+            if (lane == 0) {
+                ok = wait_bar(KV_EMPTY, (item_ctr & 1) ^ 1, abort_flag, prm.err, 21);
+                if (ok) {
+                    mbar_expect_tx(KV_FULL, 4 * kBlk * 128);
+                    const int row = (int)(s.ks + (int64_t)it.kb * kBlk);
+                    for (int h = 0; h < 2; ++h) {
+                        tma_load_2d(sbase + kOffK + h * 16384, &prm.mapK, it.hk * kFaD + h * 64, row, KV_FULL);
+                        tma_load_2d(sbase + kOffV + h * 16384, &prm.mapV, it.hk * kFaD + h * 64, row, KV_FULL);
+                    }
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            const int q0 = first_qb(s, it.kb, prm.mode), nqb = (int)((s.ql + kBlk - 1) / kBlk);
+            for (int h = it.hk * G; h < it.hk * G + G && ok; ++h) {
+                for (int qb = q0; qb < nqb && ok; ++qb, ++pair_ctr) {
+                    if (lane == 0) {
+                        ok = wait_bar(QDO_EMPTY, (pair_ctr & 1) ^ 1, abort_flag, prm.err, 22);
+                        if (ok) {
+                            mbar_expect_tx(QDO_FULL, 4 * kBlk * 128);
+                            const int row = (int)(s.qs + (int64_t)qb * kBlk);
+                            for (int hh = 0; hh < 2; ++hh) {
+                                tma_load_2d(sbase + kOffQ + hh * 16384, &prm.mapQ, h * kFaD + hh * 64, row, QDO_FULL);
+                                tma_load_2d(sbase + kOffO + hh * 16384, &prm.mapO, h * kFaD + hh * 64, row, QDO_FULL);
+                            }
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                }
+            }
+        }
+        if (lane == 0) {  // drain the last loads before exiting
+            uint64_t t0 = globaltimer();
+            if (item_ctr > 0)
+                while (!mbar_try(KV_FULL, (item_ctr - 1) & 1) && globaltimer() - t0 < 1000000000ull) {
+                }
+            if (pair_ctr > 0)
+                while (!mbar_try(QDO_FULL, (pair_ctr - 1) & 1) && globaltimer() - t0 < 1000000000ull) {
+                }
+        }
+    } else if (warp == 9) {
+        // =================== MMA issuer ===================
+        const uint32_t ID_S = idesc(128, 128, false, false, kF16);  // S^T, dP^T (A = K/V, B = Q/dY, both K-major)
+        const uint32_t ID_A = idesc(128, 128, false, true, kF16);   // dV, dK (A = P/dS K-major, B = dY/Q MN-major)
+        const uint32_t ID_Q = idesc(128, 128, true, true, kF16);    // dQ^T (A = K MN-major, B = dS MN-major)
+        const uint32_t sK = sbase + kOffK, sV = sbase + kOffV, sQ = sbase + kOffQ, sO = sbase + kOffO,
+                       sP = sbase + kOffP, sDS = sbase + kOffDS;
+        int item_ctr = 0, pair_ctr = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < prm.nitems && ok; w += gridDim.x, ++item_ctr) {
+            const FaItem it = prm.items[w];
+            const Seq s = seq_of(prm, it.b);
+            if (lane == 0) ok = wait_bar(KV_FULL, item_ctr & 1, abort_flag, prm.err, 23);
+            if (lane == 0 && ok) ok = wait_bar(ACC_EMPTY, (item_ctr & 1) ^ 1, abort_flag, prm.err, 24);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const int q0 = first_qb(s, it.kb, prm.mode), nqb = (int)((s.ql + kBlk - 1) / kBlk);
+            bool first = true;
+            for (int h = it.hk * G; h < it.hk * G + G && ok; ++h) {
+                for (int qb = q0; qb < nqb && ok; ++qb, ++pair_ctr) {
+                    if (lane == 0) ok = wait_bar(QDO_FULL, pair_ctr & 1, abort_flag, prm.err, 25);
+                    if (lane == 0 && ok) ok = wait_bar(S_FREE, (pair_ctr & 1) ^ 1, abort_flag, prm.err, 26);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                            mma(T_S, sdesc(sK + off, 16, 1024), sdesc(sQ + off, 16, 1024), ID_S, ks > 0);
+                        }
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                            mma(T_DP, sdesc(sV + off, 16, 1024), sdesc(sO + off, 16, 1024), ID_S, ks > 0);
+                        }
+                        mma_commit(SDP_FULL);
+                        ok = wait_bar(PDS_FULL, pair_ctr & 1, abort_flag, prm.err, 27);
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        for (int ks = 0; ks < 8; ++ks) {  // K = 128 queries, 16 per step
+                            const uint64_t aP = sdesc(sP + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                            const uint64_t aS = sdesc(sDS + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                            mma(T_DV, aP, sdesc(sO + ks * 2048, 16384, 1024), ID_A, (!first || ks > 0));
+                            mma(T_DK, aS, sdesc(sQ + ks * 2048, 16384, 1024), ID_A, (!first || ks > 0));
+                        }
+                        for (int ks = 0; ks < 8; ++ks)  // K = 128 keys
+                            mma(T_S, sdesc(sK + ks * 2048, 16384, 1024), sdesc(sDS + ks * 2048, 16384, 1024), ID_Q,
+                                ks > 0);
+                        mma_commit(QDO_EMPTY);
+                        mma_commit(PDS_FREE);
+                        mma_commit(DQ_FULL);
+                    }
+                    __syncwarp();
+                    first = false;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) {
+                mma_commit(KV_EMPTY);
+                mma_commit(ACC_FULL);
+            }
+        }
+        if (lane == 0) {
+            mma_commit(DONE);
+            uint64_t t0 = globaltimer();
+            while (!mbar_try(DONE, 0) && globaltimer() - t0 < 1000000000ull) {
+            }
+        }
+    } else if (warp < 4) {
+        // =================== softmax / dS, then dK / dV write-out (TMEM lane = key) ===================
+        const int j = threadIdx.x;
+        const float c1 = scale * 1.4426950408889634f;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        int item_ctr = 0, pair_ctr = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < prm.nitems && ok; w += gridDim.x, ++item_ctr) {
+            const FaItem it = prm.items[w];
+            const Seq s = seq_of(prm, it.b);
+            const int q0 = first_qb(s, it.kb, prm.mode), nqb = (int)((s.ql + kBlk - 1) / kBlk);
+            const int64_t jl = (int64_t)it.kb * kBlk + j;  // key position in the sequence
+            const bool key_ok = jl < s.kl;
+            const int64_t off = s.kl - s.ql;
+            int npairs = 0;
+            for (int h = it.hk * G; h < it.hk * G + G && ok; ++h) {
+                for (int qb = q0; qb < nqb && ok; ++qb, ++pair_ctr, ++npairs) {
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    {
+                        const int64_t il = (int64_t)qb * kBlk + j;
+                        const int64_t row = s.qs + il;
+                        if (il < s.ql) {
+                            const int64_t sidx = row * prm.Nq + h;
+                            const float l = prm.ssum[sidx * 8];
+                            cst[j] = prm.smax[sidx * 8] * 1.4426950408889634f;
+                            cst[128 + j] = l == 0.f ? 0.f : 1.f / l;
+                            cst[256 + j] = prm.rowsum[sidx];
+                        } else {
+                            cst[j] = 0.f;
+                            cst[128 + j] = 0.f;
+                            cst[256 + j] = 0.f;
+                        }
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    ok = wait_bar(SDP_FULL, pair_ctr & 1, abort_flag, prm.err, 28);
+                    if (ok && pair_ctr > 0) ok = wait_bar(PDS_FREE, (pair_ctr - 1) & 1, abort_flag, prm.err, 29);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const int64_t ibase = (int64_t)qb * kBlk;
+#pragma unroll 1
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float sv[32], dp[32];
+                        tmem_ld32(T_S + lane_base + cc * 32, sv);
+                        tmem_ld32(T_DP + lane_base + cc * 32, dp);
+                        tmem_wait_ld();
+                        uint32_t pw[16], dw[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const int i = cc * 32 + e;
+                            // key kept for query il iff il < ql, key valid, and (mode 3) jl <= il + off
+                            const bool v0 = key_ok && (ibase + i < s.ql) && (prm.mode != 3 || jl <= ibase + i + off);
+                            const bool v1 = key_ok && (ibase + i + 1 < s.ql) &&
+                                            (prm.mode != 3 || jl <= ibase + i + 1 + off);
+                            const float p0 = v0 ? exp2f(fmaf(sv[e], c1, -cst[i])) * cst[128 + i] : 0.f;
+                            const float p1 = v1 ? exp2f(fmaf(sv[e + 1], c1, -cst[i + 1])) * cst[128 + i + 1] : 0.f;
+                            pw[e >> 1] = pack2<T>(p0, p1);
+                            dw[e >> 1] = pack2<T>(p0 * (dp[e] - cst[256 + i]) * scale,
+                                                  p1 * (dp[e + 1] - cst[256 + i + 1]) * scale);
+                        }
+                        const int half = cc >> 1, u0 = (cc & 1) * 4;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t o = half * 16384 + j * 128 + (((u0 + u) ^ (j & 7)) << 4);
+                            *reinterpret_cast<uint4*>(smem + kOffP + o) =
+                                make_uint4(pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
+                            *reinterpret_cast<uint4*>(smem + kOffDS + o) =
+                                make_uint4(dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
+                        }
+                    }
+                    fence_view_async_shared();
+                    tc_fence_before();
+                    mbar_arrive(PDS_FULL);
+                }
+            }
+            if (!ok) break;
+            // dK / dV rows of this key block (zero when no query sees the block)
+            ok = wait_bar(ACC_FULL, item_ctr & 1, abort_flag, prm.err, 30);
+            if (!ok) break;
+            tc_fence_after();
+            const int64_t orow = ((s.ks + jl) * prm.Nkv + it.hk) * kFaD;
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                T* dst = reinterpret_cast<T*>(which ? prm.dv : prm.dk) + orow;
+                const uint32_t src = which ? T_DV : T_DK;
+#pragma unroll 1
+                for (int cc = 0; cc < 4; ++cc) {
+                    float v[32];
+                    tmem_ld32(src + lane_base + cc * 32, v);
+                    tmem_wait_ld();
+                    if (key_ok) {
+                        uint32_t wv[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2)
+                            wv[e >> 1] = npairs ? pack2<T>(v[e], v[e + 1]) : 0u;
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) d4[u] = make_uint4(wv[4 * u], wv[4 * u + 1], wv[4 * u + 2], wv[4 * u + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(ACC_EMPTY);
+        }
+    } else {
+        // =================== dQ flush (TMEM lane = dim) ===================
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const int dim = q * 32 + lane;
+        int pair_ctr = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < prm.nitems && ok; w += gridDim.x) {
+            const FaItem it = prm.items[w];
+            const Seq s = seq_of(prm, it.b);
+            const int q0 = first_qb(s, it.kb, prm.mode), nqb = (int)((s.ql + kBlk - 1) / kBlk);
+            for (int h = it.hk * G; h < it.hk * G + G && ok; ++h) {
+                for (int qb = q0; qb < nqb && ok; ++qb, ++pair_ctr) {
+                    ok = wait_bar(DQ_FULL, pair_ctr & 1, abort_flag, prm.err, 31);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const int64_t nq = min((int64_t)kBlk, s.ql - (int64_t)qb * kBlk);
+                    const int64_t row0 = s.qs + (int64_t)qb * kBlk;
+#pragma unroll 1
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float v[32];
+                        tmem_ld32(T_S + lane_base + cc * 32, v);
+                        tmem_wait_ld();
+                        const int64_t lim = nq - cc * 32;
+                        const size_t base = ((size_t)(row0 + cc * 32) * prm.Nq + h) * kFaD + dim;
+                        const size_t step = (size_t)prm.Nq * kFaD;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            if (e < lim) {
+                                if (DET)
+                                    atomicAdd(reinterpret_cast<unsigned long long*>(prm.dq_acc) + base + e * step,
+                                              (unsigned long long)__float2ll_rn(v[e] * kFixScale));
+                                else
+                                    atomicAdd(reinterpret_cast<float*>(prm.dq_acc) + base + e * step, v[e]);
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive(S_FREE);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    }
+}
+
+template <typename T>
+__global__ void fa_rowsum_kernel(const T* __restrict__ dy, const T* __restrict__ o, int64_t rows,
+                                 float* __restrict__ res) {
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    const uint2 a = reinterpret_cast<const uint2*>(dy + r * kFaD)[lane];
+    const uint2 b = reinterpret_cast<const uint2*>(o + r * kFaD)[lane];
+    const T* ap = reinterpret_cast<const T*>(&a);
+    const T* bp = reinterpret_cast<const T*>(&b);
+    float sum = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sum = fmaf(to_f(ap[e]), to_f(bp[e]), sum);
+#pragma unroll
+    for (int k = 16; k; k >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, k);
+    if (lane == 0) res[r] = sum;
+}
+
+template <typename T, bool DET>
+__global__ void fa_cast_dq_kernel(const void* __restrict__ acc, int64_t n, T* __restrict__ dq) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const float x = DET ? (float)((double)reinterpret_cast<const long long*>(acc)[i] * kFixInv)
+                        : reinterpret_cast<const float*>(acc)[i];
+    dq[i] = from_f<T>(x);
+}
+
+template <typename T, bool DET>
+cudaError_t launch_fa_t(const FaFusedArgs& a, cudaStream_t st) {
+    FaParams p;
+    memset(&p, 0, sizeof p);
+    const uint64_t qcols = (uint64_t)a.Nq * kFaD, kcols = (uint64_t)a.Nkv * kFaD;
+    if (!make_map(&p.mapQ, a.q, a.dtype, qcols, a.T1, qcols, kBlk) ||
+        !make_map(&p.mapO, a.dy, a.dtype, qcols, a.T1, qcols, kBlk) ||
+        !make_map(&p.mapK, a.k, a.dtype, kcols, a.T2, kcols, kBlk) ||
+        !make_map(&p.mapV, a.v, a.dtype, kcols, a.T2, kcols, kBlk))
+        return cudaErrorInvalidValue;
+    p.items = reinterpret_cast<const FaItem*>(a.items);
+    p.nitems = a.nitems;
+    p.cu_q = a.cu_q;
+    p.cu_kv = a.cu_kv;
+    p.smax = a.smax;
+    p.ssum = a.ssum;
+    p.rowsum = a.rowsum;
+    p.dq_acc = a.dq_acc;
+    p.dk = a.dk;
+    p.dv = a.dv;
+    p.err = a.err;
+    p.B = (int)a.B;
+    p.Nq = (int)a.Nq;
+    p.Nkv = (int)a.Nkv;
+    p.mode = a.mode;
+    p.scale = a.scale;
+    const int64_t rows = a.T1 * a.Nq;
+    if (rows > 0)
+        fa_rowsum_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>((const T*)a.dy, (const T*)a.o, rows,
+                                                                        (float*)a.rowsum);
+    auto kern = fa_bwd_fused_kernel<T, DET>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFaSmem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = std::min(sms, a.nitems);
+    if (grid > 0) kern<<<grid, kFaThreads, kFaSmem, st>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int64_t n = a.T1 * a.Nq * kFaD;
+    if (n > 0)
+        fa_cast_dq_kernel<T, DET><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.dq_acc, n, (T*)a.dq);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t fa_fused_items(const int64_t* cu_q, const int64_t* cu_kv, int64_t B, int64_t Nq, int64_t Nkv, int mode,
+                      std::vector<int32_t>* out) {
+    std::vector<FaItem> items;
+    const int64_t G = Nq / Nkv;
+    int64_t pq = 0, pk = 0;
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t ql = cu_q[b] - pq, kl = cu_kv[b] - pk;
+        pq = cu_q[b];
+        pk = cu_kv[b];
+        const int64_t nkb = (kl + kBlk - 1) / kBlk, nqb = (ql + kBlk - 1) / kBlk;
+        for (int64_t kb = 0; kb < nkb; ++kb) {
+            int64_t q0 = 0;
+            if (mode == 3) {
+                const int64_t lo = kb * kBlk - (kl - ql);
+                q0 = lo <= 0 ? 0 : lo / kBlk;
+            }
+            const int cost = (int)(G * std::max<int64_t>(0, nqb - q0));
+            for (int64_t hk = 0; hk < Nkv; ++hk) items.push_back(FaItem{(int)b, (int)hk, (int)kb, cost});
+        }
+    }
+    // longest first, so the persistent CTAs finish together
+    std::stable_sort(items.begin(), items.end(), [](const FaItem& x, const FaItem& y) { return x.cost > y.cost; });
+    if (out) {
+        out->resize(items.size() * 4);
+        memcpy(out->data(), items.data(), items.size() * sizeof(FaItem));
+    }
+    return items.size();
+}
+
+bool fa_fused_supported(int64_t D) { return D == kFaD; }
+
+cudaError_t launch_fa_bwd_fused(int dtype, const FaFusedArgs& a, cudaStream_t st) {
+    if (dtype == SFA_DTYPE_BF16) return a.det ? launch_fa_t<__nv_bfloat16, true>(a, st) : launch_fa_t<__nv_bfloat16, false>(a, st);
+    return a.det ? launch_fa_t<__half, true>(a, st) : launch_fa_t<__half, false>(a, st);
+}
+
+}  // namespace sfa

@@ -3,7 +3,9 @@
 // two-phase aclnn convention of aclnnFlashAttentionUnpaddingScoreGrad (函数原型).
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
+#include <vector>
 #include <string>
 
 #include "sfa_internal.cuh"
@@ -311,6 +313,22 @@ static sfa_status check_cu(const int64_t* cu, int64_t B, int64_t T, const char* 
 
 static size_t fa_cu_bytes(int64_t B) { return 2 * align256((size_t)B * 8); }
 
+// Workspace of the tensor-core dense backward (head dim 128): cumulative lengths,
+// work list, rowsum(dY o O), dQ accumulator, control word.
+struct FaFusedWs {
+    size_t items, rowsum, dq, ctrl, total;
+};
+static FaFusedWs fa_fused_ws(const fa_shape* s, bool det) {
+    FaFusedWs w;
+    size_t o = fa_cu_bytes(s->B);
+    w.items = o;  o = align256(o + fa_fused_max_items(s->B, s->T2, s->Nkv) * 16);
+    w.rowsum = o; o = align256(o + (size_t)s->T1 * s->Nq * 4);
+    w.dq = o;     o = align256(o + (size_t)s->T1 * s->Nq * s->D * (det ? 8 : 4));
+    w.ctrl = o;   o = align256(o + 256);
+    w.total = o;
+    return w;
+}
+
 sfa_status fa_grad_workspace_size(const fa_shape* shape, int64_t sparse_mode, int32_t deterministic,
                                   size_t* workspace_bytes) {
     g_last_error.clear();
@@ -319,6 +337,10 @@ sfa_status fa_grad_workspace_size(const fa_shape* shape, int64_t sparse_mode, in
     if (st != SFA_OK) return st;
     *workspace_bytes = fa_cu_bytes(shape->B) +
                        align256((size_t)2 * shape->T2 * shape->Nkv * shape->D * (deterministic ? 8 : 4));
+    if (fa_fused_supported(shape->D)) {
+        const size_t f = fa_fused_ws(shape, deterministic != 0).total;
+        if (f > *workspace_bytes) *workspace_bytes = f;
+    }
     return SFA_OK;
 }
 
@@ -343,6 +365,8 @@ sfa_status fa_grad(const void* q, const void* k, const void* v, const void* dy, 
     const bool det = deterministic != 0;
     size_t acc_bytes = (size_t)2 * shape->T2 * shape->Nkv * shape->D * (det ? 8 : 4);
     size_t need = fa_cu_bytes(shape->B) + align256(acc_bytes);
+    const bool fused = fa_fused_supported(shape->D);
+    if (fused) need = std::max(need, fa_fused_ws(shape, det).total);
     if (workspace_bytes < need) return fail(SFA_ERR_WORKSPACE, "workspace %zu < %zu", workspace_bytes, need);
     cudaStream_t s = (cudaStream_t)stream;
     char* w = (char*)workspace;
@@ -351,6 +375,28 @@ sfa_status fa_grad(const void* q, const void* k, const void* v, const void* dy, 
     void* acc = w + fa_cu_bytes(shape->B);
     SFA_CUDA(cudaMemcpyAsync(cuq, actual_seq_qlen, shape->B * 8, cudaMemcpyHostToDevice, s), "copy seqlens");
     SFA_CUDA(cudaMemcpyAsync(cukv, actual_seq_kvlen, shape->B * 8, cudaMemcpyHostToDevice, s), "copy seqlens");
+    if (fused) {
+        const FaFusedWs fw = fa_fused_ws(shape, det);
+        std::vector<int32_t> items;
+        const size_t nitems = fa_fused_items(actual_seq_qlen, actual_seq_kvlen, shape->B, shape->Nq, shape->Nkv,
+                                             (int)sparse_mode, &items);
+        if (nitems)
+            SFA_CUDA(cudaMemcpyAsync(w + fw.items, items.data(), nitems * 16, cudaMemcpyHostToDevice, s),
+                     "copy work list");
+        SFA_CUDA(cudaMemsetAsync(w + fw.dq, 0, (size_t)shape->T1 * shape->Nq * shape->D * (det ? 8 : 4), s),
+                 "zero dQ accumulator");
+        SFA_CUDA(cudaMemsetAsync(w + fw.ctrl, 0, 256, s), "zero control word");
+        FaFusedArgs f;
+        memset(&f, 0, sizeof f);
+        f.q = q; f.k = k; f.v = v; f.dy = dy; f.o = attention_in; f.smax = softmax_max; f.ssum = softmax_sum;
+        f.cu_q = cuq; f.cu_kv = cukv; f.B = shape->B; f.T1 = shape->T1; f.T2 = shape->T2; f.Nq = shape->Nq;
+        f.Nkv = shape->Nkv; f.mode = (int)sparse_mode; f.scale = (float)scale; f.det = det; f.dtype = shape->dtype;
+        f.items = w + fw.items; f.nitems = (int)nitems; f.rowsum = (float*)(w + fw.rowsum); f.dq_acc = w + fw.dq;
+        f.err = (int*)(w + fw.ctrl); f.dq = dq; f.dk = dk; f.dv = dv;
+        KernelEvents ev(s);
+        SFA_CUDA(launch_fa_bwd_fused(shape->dtype, f, s), "fa backward (tensor cores)");
+        return SFA_OK;
+    }
     SFA_CUDA(cudaMemsetAsync(acc, 0, acc_bytes, s), "zero dK/dV accumulator");
     FaArgs a;
     memset(&a, 0, sizeof a);

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "../../include/sfa.h"
 
 namespace sfa {
@@ -183,6 +185,27 @@ struct FaArgs {
     void* out; float* smax_out; float* ssum_out;
 };
 cudaError_t launch_fa_bwd(int dtype, const FaArgs& a, cudaStream_t st);
+
+// Tensor-core dense backward (head dim 128): work list of (sequence, kv head,
+// 128-key block) items, built on the host and copied into the workspace.
+struct FaFusedArgs {
+    const void* q; const void* k; const void* v; const void* dy; const void* o;
+    const float* smax; const float* ssum;
+    const int64_t* cu_q; const int64_t* cu_kv;
+    int64_t B, T1, T2, Nq, Nkv; int mode; float scale; bool det; int dtype;
+    const void* items; int nitems;
+    float* rowsum;   // [T1][Nq]
+    void* dq_acc;    // [T1][Nq][128] fp32 or int64 (zeroed by the caller)
+    int* err;
+    void* dq; void* dk; void* dv;
+};
+bool fa_fused_supported(int64_t D);
+// Builds the work list (4 int32 per item) for the given host cumulative lengths
+// (when `out` is non-null) and returns the number of items.
+size_t fa_fused_items(const int64_t* cu_q, const int64_t* cu_kv, int64_t B, int64_t Nq, int64_t Nkv, int mode,
+                      std::vector<int32_t>* out);
+inline size_t fa_fused_max_items(int64_t B, int64_t T2, int64_t Nkv) { return (size_t)Nkv * (T2 / 128 + B + 1); }
+cudaError_t launch_fa_bwd_fused(int dtype, const FaFusedArgs& a, cudaStream_t st);
 // Sets the message returned by sfa_last_error_string() on the calling thread.
 void set_last_error(const char* msg);
 cudaError_t launch_fa_fwd(int dtype, const FaArgs& a, cudaStream_t st);
