@@ -258,9 +258,13 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 if (!ok) break;
                 int32_t* rid = rowids + rb * kKeys;
                 const int first = rl[0];
-                for (int r = lane; r < kKeys; r += 32) {
-                    const int s = tile * kKeys + r;
-                    rid[r] = s < n ? rl[s] : first;
+                // lane L owns key rows 4L..4L+3 of the tile (one gather4 per 64-dim half)
+                int32_t my[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int s = tile * kKeys + 4 * lane + e;
+                    my[e] = s < n ? rl[s] : first;
+                    rid[4 * lane + e] = my[e];
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ROWS_FULL(rb));
@@ -270,27 +274,25 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                     if (lane == 0) ok = wait_bar(EMPTY(slot), sphase ^ 1, abort_flag, prm.err, 2);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
+                    const uint32_t dst = sbase + slot * kSlotBytes;
+                    const int halves = c < 4 ? 2 : 1;
                     if (lane == 0) {
-                        const uint32_t dst = sbase + slot * kSlotBytes;
-                        const int halves = c < 4 ? 2 : 1;
                         const uint32_t rows = kind == 0 ? kKeys : N1;
                         mbar_expect_tx(FULL(slot), halves * rows * 128u);
-                        for (int h = 0; h < halves; ++h) {
-                            const uint32_t d = dst + h * kHalf;
-                            if (kind == 0) {
-                                const CUtensorMap* map = c < 4 ? &prm.mapK : &prm.mapKr;
-                                const int col = c < 4 ? c * 128 + h * 64 : 0;
-                                for (int g = 0; g < kKeys / 4; ++g)
-                                    tma_gather4(d + g * 512, map, col, rid[4 * g], rid[4 * g + 1], rid[4 * g + 2],
-                                                rid[4 * g + 3], FULL(slot));
-                            } else {
-                                const CUtensorMap* map = kind == 1 ? (c < 4 ? &prm.mapQ : &prm.mapQr) : &prm.mapO;
-                                const int col = c < 4 ? c * 128 + h * 64 : 0;
-                                tma_load_2d(d, map, col, t * N1, FULL(slot));
-                            }
-                        }
-                        issued_mask |= 1u << slot;
                     }
+                    __syncwarp();
+                    if (kind == 0) {
+                        // key rows: every lane gathers its own four rows, in parallel
+                        const CUtensorMap* map = c < 4 ? &prm.mapK : &prm.mapKr;
+                        for (int h = 0; h < halves; ++h)
+                            tma_gather4(dst + h * kHalf + lane * 512, map, c < 4 ? c * 128 + h * 64 : 0, my[0], my[1],
+                                        my[2], my[3], FULL(slot));
+                    } else if (lane == 0) {
+                        const CUtensorMap* map = kind == 1 ? (c < 4 ? &prm.mapQ : &prm.mapQr) : &prm.mapO;
+                        for (int h = 0; h < halves; ++h)
+                            tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, t * N1, FULL(slot));
+                    }
+                    if (lane == 0) issued_mask |= 1u << slot;
                     if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
                 }
             }
