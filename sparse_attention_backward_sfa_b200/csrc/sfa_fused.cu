@@ -425,7 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
             asm volatile("bar.sync 1, 128;" ::: "memory");
             const int ntiles = (n + kKeys - 1) / kKeys;
             for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
-                const bool valid = tile * kKeys + j < n;
+                // padding keys of the last tile get P = dS = 0 (their S is finite: a real gathered row)
+                const float vmul = tile * kKeys + j < n ? 1.f : 0.f;
                 ok = wait_bar(SDP_FULL, tile_ctr & 1, abort_flag, prm.err, 8);
                 if (ok && tile_ctr > 0) ok = wait_bar(PDS_FREE, (tile_ctr - 1) & 1, abort_flag, prm.err, 9);
                 if (!ok) break;
@@ -438,15 +439,25 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                     tmem_ld32(T_DP + lane_base + cc * 32, dp);
                     tmem_wait_ld();
                     uint32_t pw[16], dw[16];
+                    const float4* cm = reinterpret_cast<const float4*>(cst + cc * 32);        // max * log2e
+                    const float4* cl = reinterpret_cast<const float4*>(cst + 128 + cc * 32);  // 1 / sum
+                    const float4* cd = reinterpret_cast<const float4*>(cst + 256 + cc * 32);  // rowsum(dO o O)
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int h = cc * 32 + e;
-                        float p0 = valid ? exp2f(fmaf(s[e], c1, -cst[h])) * cst[128 + h] : 0.f;
-                        float p1 = valid ? exp2f(fmaf(s[e + 1], c1, -cst[h + 1])) * cst[128 + h + 1] : 0.f;
-                        float d0 = p0 * (dp[e] - cst[256 + h]) * scale;
-                        float d1 = p1 * (dp[e + 1] - cst[256 + h + 1]) * scale;
-                        pw[e >> 1] = pack2<T>(p0, p1);
-                        dw[e >> 1] = pack2<T>(d0, d1);
+                    for (int g = 0; g < 8; ++g) {
+                        const float4 m4 = cm[g], l4 = cl[g], d4 = cd[g];
+                        const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, ll[4] = {l4.x, l4.y, l4.z, l4.w},
+                                    dd[4] = {d4.x, d4.y, d4.z, d4.w};
+                        float pv[4], dv[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int e = 4 * g + k;
+                            pv[k] = ex2_approx(fmaf(s[e], c1, -mm[k])) * (ll[k] * vmul);
+                            dv[k] = pv[k] * (dp[e] - dd[k]) * scale;
+                        }
+                        pw[2 * g] = pack2<T>(pv[0], pv[1]);
+                        pw[2 * g + 1] = pack2<T>(pv[2], pv[3]);
+                        dw[2 * g] = pack2<T>(dv[0], dv[1]);
+                        dw[2 * g + 1] = pack2<T>(dv[2], dv[3]);
                     }
                     const int half = cc >> 1;
                     const int u0 = (cc & 1) * 4;

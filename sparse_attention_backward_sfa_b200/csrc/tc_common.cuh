@@ -126,6 +126,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
         : "r"(taddr)
         : "memory");
 }
+// 2^x with the hardware approximation (relative error ~2^-22; P is rounded to
+// 16 bits right after, so the approximation is invisible in the outputs).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 template <typename T> __device__ __forceinline__ uint32_t pack2(float a, float b);
