@@ -14,7 +14,8 @@
 //   dQ^T = K^T . dS^T                        [128 dims x 128 queries], reusing
 //        S^T's columns, reduced into an fp32 (or 64-bit fixed point) dQ buffer
 //        by the flush warps (TMEM lane = dim: 128-byte coalesced reductions).
-// Warps: 0-3 softmax + dK/dV write-out, 4-7 dQ flush, 8 TMA producer, 9 MMA.
+// Warps: 0-3 softmax + dK/dV write-out, 4-11 dQ flush (two per TMEM lane quarter,
+// each taking half of the query columns), 12 TMA producer, 13 MMA.
 #include <cuda.h>
 
 #include <algorithm>
@@ -33,7 +34,7 @@ using namespace tc;
 
 constexpr int kFaD = 128;
 constexpr int kBlk = 128;
-constexpr int kFaThreads = 320;
+constexpr int kFaThreads = 448;
 constexpr int kOffK = 0, kOffV = 32768, kOffQ = 65536, kOffO = 98304, kOffP = 131072, kOffDS = 163840;
 constexpr int kOffCst = 196608;                 // float [3][128]: max*log2e, 1/sum, rowsum(dY o O)
 constexpr int kOffBar = kOffCst + 3 * 128 * 4;  // 11 mbarriers
@@ -106,7 +107,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
         mbar_init(PDS_FULL, 128);
         mbar_init(PDS_FREE, 1);
         mbar_init(DQ_FULL, 1);
-        mbar_init(S_FREE, 128);
+        mbar_init(S_FREE, 256);
         mbar_init(ACC_FULL, 1);
         mbar_init(ACC_EMPTY, 128);
         mbar_init(DONE, 1);
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
     const int G = prm.Nq / prm.Nkv;
     const float scale = prm.scale;
 
-    if (warp == 8) {
+    if (warp == 12) {
         // =================== TMA producer ===================
         int item_ctr = 0, pair_ctr = 0;
         bool ok = true;
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                 while (!mbar_try(QDO_FULL, (pair_ctr - 1) & 1) && globaltimer() - t0 < 1000000000ull) {
                 }
         }
-    } else if (warp == 9) {
+    } else if (warp == 13) {
         // =================== MMA issuer ===================
         const uint32_t ID_S = idesc(128, 128, false, false, kF16);  // S^T, dP^T (A = K/V, B = Q/dY, both K-major)
         const uint32_t ID_A = idesc(128, 128, false, true, kF16);   // dV, dK (A = P/dS K-major, B = dY/Q MN-major)
@@ -277,34 +278,52 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                         }
                     }
                     asm volatile("bar.sync 1, 128;" ::: "memory");
+                    // queries i of this block that keep this key: lo <= i < hi (i < ql, and in
+                    // mode 3 jl <= qb*128 + i + off); none when the key is past the sequence
+                    const int64_t ibase = (int64_t)qb * kBlk;
+                    int64_t lo64 = prm.mode == 3 ? jl - off - ibase : 0;
+                    int64_t hi64 = s.ql - ibase;
+                    lo64 = lo64 < 0 ? 0 : (lo64 > kBlk ? kBlk : lo64);
+                    hi64 = hi64 > kBlk ? kBlk : hi64;
+                    const int lo = (int)lo64;
+                    const uint32_t span = key_ok && hi64 > lo64 ? (uint32_t)(hi64 - lo64) : 0u;
                     ok = wait_bar(SDP_FULL, pair_ctr & 1, abort_flag, prm.err, 28);
                     if (ok && pair_ctr > 0) ok = wait_bar(PDS_FREE, (pair_ctr - 1) & 1, abort_flag, prm.err, 29);
                     if (!ok) break;
                     tc_fence_after();
-                    const int64_t ibase = (int64_t)qb * kBlk;
 #pragma unroll 1
-                    for (int cc = 0; cc < 4; ++cc) {
-                        float sv[32], dp[32];
-                        tmem_ld32(T_S + lane_base + cc * 32, sv);
-                        tmem_ld32(T_DP + lane_base + cc * 32, dp);
+                    for (int cc = 0; cc < 8; ++cc) {  // 16 query columns at a time (keeps the loop in registers)
+                        float sv[16], dp[16];
+                        tmem_ld16(T_S + lane_base + cc * 16, sv);
+                        tmem_ld16(T_DP + lane_base + cc * 16, dp);
                         tmem_wait_ld();
-                        uint32_t pw[16], dw[16];
+                        uint32_t pw[8], dw[8];
+                        const float4* cm = reinterpret_cast<const float4*>(cst + cc * 16);        // max * log2e
+                        const float4* cl = reinterpret_cast<const float4*>(cst + 128 + cc * 16);  // 1 / sum
+                        const float4* cd = reinterpret_cast<const float4*>(cst + 256 + cc * 16);  // rowsum(dY o O)
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const int i = cc * 32 + e;
-                            // key kept for query il iff il < ql, key valid, and (mode 3) jl <= il + off
-                            const bool v0 = key_ok && (ibase + i < s.ql) && (prm.mode != 3 || jl <= ibase + i + off);
-                            const bool v1 = key_ok && (ibase + i + 1 < s.ql) &&
-                                            (prm.mode != 3 || jl <= ibase + i + 1 + off);
-                            const float p0 = v0 ? exp2f(fmaf(sv[e], c1, -cst[i])) * cst[128 + i] : 0.f;
-                            const float p1 = v1 ? exp2f(fmaf(sv[e + 1], c1, -cst[i + 1])) * cst[128 + i + 1] : 0.f;
-                            pw[e >> 1] = pack2<T>(p0, p1);
-                            dw[e >> 1] = pack2<T>(p0 * (dp[e] - cst[256 + i]) * scale,
-                                                  p1 * (dp[e + 1] - cst[256 + i + 1]) * scale);
+                        for (int g = 0; g < 4; ++g) {
+                            const float4 m4 = cm[g], l4 = cl[g], d4 = cd[g];
+                            const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, ll[4] = {l4.x, l4.y, l4.z, l4.w},
+                                        dd[4] = {d4.x, d4.y, d4.z, d4.w};
+                            float pv[4], dv[4];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const int e = 4 * g + k;
+                                const bool v = (uint32_t)(cc * 16 + e - lo) < span;
+                                // a select (not a product): masked scores may overflow exp2
+                                pv[k] = v ? ex2_approx(fmaf(sv[e], c1, -mm[k])) * ll[k] : 0.f;
+                                dv[k] = pv[k] * (dp[e] - dd[k]) * scale;
+                            }
+                            pw[2 * g] = pack2<T>(pv[0], pv[1]);
+                            pw[2 * g + 1] = pack2<T>(pv[2], pv[3]);
+                            dw[2 * g] = pack2<T>(dv[0], dv[1]);
+                            dw[2 * g + 1] = pack2<T>(dv[2], dv[3]);
                         }
-                        const int half = cc >> 1, u0 = (cc & 1) * 4;
+                        // columns [16cc, 16cc+16): SW128 half cc/4, 16-byte units 2(cc%4) and 2(cc%4)+1
+                        const int half = cc >> 2, u0 = (cc & 3) * 2;
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
+                        for (int u = 0; u < 2; ++u) {
                             const uint32_t o = half * 16384 + j * 128 + (((u0 + u) ^ (j & 7)) << 4);
                             *reinterpret_cast<uint4*>(smem + kOffP + o) =
                                 make_uint4(pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
@@ -348,7 +367,8 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
         }
     } else {
         // =================== dQ flush (TMEM lane = dim) ===================
-        const int q = warp & 3;
+        const int q = warp & 3;                 // TMEM lane quarter
+        const int hsel = (warp - 4) >> 2;       // which half of the query columns
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const int dim = q * 32 + lane;
         int pair_ctr = 0;
@@ -365,22 +385,24 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                     const int64_t nq = min((int64_t)kBlk, s.ql - (int64_t)qb * kBlk);
                     const int64_t row0 = s.qs + (int64_t)qb * kBlk;
 #pragma unroll 1
-                    for (int cc = 0; cc < 4; ++cc) {
+                    for (int cc = 2 * hsel; cc < 2 * hsel + 2; ++cc) {
                         float v[32];
                         tmem_ld32(T_S + lane_base + cc * 32, v);
                         tmem_wait_ld();
-                        const int64_t lim = nq - cc * 32;
+                        const int lim = (int)min((int64_t)32, nq - cc * 32);
                         const size_t base = ((size_t)(row0 + cc * 32) * prm.Nq + h) * kFaD + dim;
-                        const size_t step = (size_t)prm.Nq * kFaD;
+                        const uint32_t step = (uint32_t)prm.Nq * kFaD;  // elements between query rows
+                        // one running pointer (not 32 precomputed addresses) keeps the loop in registers
+                        if (DET) {
+                            unsigned long long* d = reinterpret_cast<unsigned long long*>(prm.dq_acc) + base;
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            if (e < lim) {
-                                if (DET)
-                                    atomicAdd(reinterpret_cast<unsigned long long*>(prm.dq_acc) + base + e * step,
-                                              (unsigned long long)__float2ll_rn(v[e] * kFixScale));
-                                else
-                                    atomicAdd(reinterpret_cast<float*>(prm.dq_acc) + base + e * step, v[e]);
-                            }
+                            for (int e = 0; e < 32; ++e, d += step)
+                                if (e < lim) atomicAdd(d, (unsigned long long)__float2ll_rn(v[e] * kFixScale));
+                        } else {
+                            float* d = reinterpret_cast<float*>(prm.dq_acc) + base;
+#pragma unroll
+                            for (int e = 0; e < 32; ++e, d += step)
+                                if (e < lim) atomicAdd(d, v[e]);
                         }
                     }
                     tc_fence_before();
