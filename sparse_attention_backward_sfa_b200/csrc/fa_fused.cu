@@ -14,8 +14,9 @@
 //   dQ^T = K^T . dS^T                        [128 dims x 128 queries], reusing
 //        S^T's columns, reduced into an fp32 (or 64-bit fixed point) dQ buffer
 //        by the flush warps (TMEM lane = dim: 128-byte coalesced reductions).
-// Warps: 0-3 softmax + dK/dV write-out, 4-11 dQ flush (two per TMEM lane quarter,
-// each taking half of the query columns), 12 TMA producer, 13 MMA.
+// Warps: 0-7 softmax (two per TMEM lane quarter, each taking half of the query
+// columns), 0-3 also the dK/dV write-out, 4-11 dQ flush (two per lane quarter,
+// halves of the query columns), 12 TMA producer, 13 MMA.
 #include <cuda.h>
 
 #include <algorithm>
@@ -36,8 +37,8 @@ constexpr int kFaD = 128;
 constexpr int kBlk = 128;
 constexpr int kFaThreads = 448;
 constexpr int kOffK = 0, kOffV = 32768, kOffQ = 65536, kOffO = 98304, kOffP = 131072, kOffDS = 163840;
-constexpr int kOffCst = 196608;                 // float [3][128]: max*log2e, 1/sum, rowsum(dY o O)
-constexpr int kOffBar = kOffCst + 3 * 128 * 4;  // 11 mbarriers
+constexpr int kOffCst = 196608;                     // float [2][3][128]: max*log2e, 1/sum, rowsum(dY o O)
+constexpr int kOffBar = kOffCst + 2 * 3 * 128 * 4;  // 14 mbarriers
 constexpr int kOffMisc = kOffBar + 16 * 8;
 constexpr int kFaSmem = kOffMisc + 16;
 
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
     const uint32_t KV_FULL = bar0, KV_EMPTY = bar0 + 8, QDO_FULL = bar0 + 16, QDO_EMPTY = bar0 + 24,
                    SDP_FULL = bar0 + 32, PDS_FULL = bar0 + 40, PDS_FREE = bar0 + 48, DQ_FULL = bar0 + 56,
                    S_FREE = bar0 + 64, ACC_FULL = bar0 + 72, ACC_EMPTY = bar0 + 80, DONE = bar0 + 88;
+    auto CST_FULL = [&](int x) { return bar0 + 96 + 8u * x; };  // per-pair softmax constants written
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     if (threadIdx.x == 0) {
@@ -104,7 +106,9 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
         mbar_init(QDO_FULL, 1);
         mbar_init(QDO_EMPTY, 1);
         mbar_init(SDP_FULL, 1);
-        mbar_init(PDS_FULL, 128);
+        mbar_init(PDS_FULL, 256);
+        mbar_init(CST_FULL(0), 128);
+        mbar_init(CST_FULL(1), 128);
         mbar_init(PDS_FREE, 1);
         mbar_init(DQ_FULL, 1);
         mbar_init(S_FREE, 256);
@@ -244,11 +248,16 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
             while (!mbar_try(DONE, 0) && globaltimer() - t0 < 1000000000ull) {
             }
         }
-    } else if (warp < 4) {
-        // =================== softmax / dS, then dK / dV write-out (TMEM lane = key) ===================
-        const int j = threadIdx.x;
+    } else {
+        // ====== warps 0-7: softmax / dS (TMEM lane = key; warp w takes query columns 64*(w/4)..+64);
+        // ====== warps 0-3: dK / dV write-out; warps 4-11: dQ flush (TMEM lane = dim) ======
+        const bool do_softmax = warp < 8, do_flush = warp >= 4, do_out = warp < 4;
+        const int quarter = warp & 3;                 // TMEM lane quarter of this warp
+        const int j = quarter * 32 + lane;            // key (softmax / write-out) or dim (flush)
+        const int cs = warp >> 2;                     // softmax: which half of the query columns
+        const int hsel = (warp - 4) >> 2;             // flush: which half of the query columns
         const float c1 = scale * 1.4426950408889634f;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         int item_ctr = 0, pair_ctr = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < prm.nitems && ok; w += gridDim.x, ++item_ctr) {
@@ -261,82 +270,119 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
             int npairs = 0;
             for (int h = it.hk * G; h < it.hk * G + G && ok; ++h) {
                 for (int qb = q0; qb < nqb && ok; ++qb, ++pair_ctr, ++npairs) {
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
-                    {
-                        const int64_t il = (int64_t)qb * kBlk + j;
-                        const int64_t row = s.qs + il;
-                        if (il < s.ql) {
-                            const int64_t sidx = row * prm.Nq + h;
-                            const float l = prm.ssum[sidx * 8];
-                            cst[j] = prm.smax[sidx * 8] * 1.4426950408889634f;
-                            cst[128 + j] = l == 0.f ? 0.f : 1.f / l;
-                            cst[256 + j] = prm.rowsum[sidx];
-                        } else {
-                            cst[j] = 0.f;
-                            cst[128 + j] = 0.f;
-                            cst[256 + j] = 0.f;
-                        }
-                    }
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
-                    // queries i of this block that keep this key: lo <= i < hi (i < ql, and in
-                    // mode 3 jl <= qb*128 + i + off); none when the key is past the sequence
-                    const int64_t ibase = (int64_t)qb * kBlk;
-                    int64_t lo64 = prm.mode == 3 ? jl - off - ibase : 0;
-                    int64_t hi64 = s.ql - ibase;
-                    lo64 = lo64 < 0 ? 0 : (lo64 > kBlk ? kBlk : lo64);
-                    hi64 = hi64 > kBlk ? kBlk : hi64;
-                    const int lo = (int)lo64;
-                    const uint32_t span = key_ok && hi64 > lo64 ? (uint32_t)(hi64 - lo64) : 0u;
-                    ok = wait_bar(SDP_FULL, pair_ctr & 1, abort_flag, prm.err, 28);
-                    if (ok && pair_ctr > 0) ok = wait_bar(PDS_FREE, (pair_ctr - 1) & 1, abort_flag, prm.err, 29);
-                    if (!ok) break;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int cc = 0; cc < 8; ++cc) {  // 16 query columns at a time (keeps the loop in registers)
-                        float sv[16], dp[16];
-                        tmem_ld16(T_S + lane_base + cc * 16, sv);
-                        tmem_ld16(T_DP + lane_base + cc * 16, dp);
-                        tmem_wait_ld();
-                        uint32_t pw[8], dw[8];
-                        const float4* cm = reinterpret_cast<const float4*>(cst + cc * 16);        // max * log2e
-                        const float4* cl = reinterpret_cast<const float4*>(cst + 128 + cc * 16);  // 1 / sum
-                        const float4* cd = reinterpret_cast<const float4*>(cst + 256 + cc * 16);  // rowsum(dY o O)
-#pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            const float4 m4 = cm[g], l4 = cl[g], d4 = cd[g];
-                            const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, ll[4] = {l4.x, l4.y, l4.z, l4.w},
-                                        dd[4] = {d4.x, d4.y, d4.z, d4.w};
-                            float pv[4], dv[4];
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const int e = 4 * g + k;
-                                const bool v = (uint32_t)(cc * 16 + e - lo) < span;
-                                // a select (not a product): masked scores may overflow exp2
-                                pv[k] = v ? ex2_approx(fmaf(sv[e], c1, -mm[k])) * ll[k] : 0.f;
-                                dv[k] = pv[k] * (dp[e] - dd[k]) * scale;
+                    if (do_softmax) {
+                        const int x = pair_ctr & 1, use = pair_ctr >> 1;
+                        float* cx = cst + x * 384;
+                        if (do_out) {
+                            // constants of query row j of this block (the buffer's previous pair,
+                            // pair_ctr - 2, finished its softmax before the gradients of pair_ctr - 1)
+                            const int64_t il = (int64_t)qb * kBlk + j;
+                            if (il < s.ql) {
+                                const int64_t sidx = (s.qs + il) * prm.Nq + h;
+                                const float l = prm.ssum[sidx * 8];
+                                cx[j] = prm.smax[sidx * 8] * 1.4426950408889634f;
+                                cx[128 + j] = l == 0.f ? 0.f : 1.f / l;
+                                cx[256 + j] = prm.rowsum[sidx];
+                            } else {
+                                cx[j] = 0.f;
+                                cx[128 + j] = 0.f;
+                                cx[256 + j] = 0.f;
                             }
-                            pw[2 * g] = pack2<T>(pv[0], pv[1]);
-                            pw[2 * g + 1] = pack2<T>(pv[2], pv[3]);
-                            dw[2 * g] = pack2<T>(dv[0], dv[1]);
-                            dw[2 * g + 1] = pack2<T>(dv[2], dv[3]);
+                            mbar_arrive(CST_FULL(x));
                         }
-                        // columns [16cc, 16cc+16): SW128 half cc/4, 16-byte units 2(cc%4) and 2(cc%4)+1
-                        const int half = cc >> 2, u0 = (cc & 3) * 2;
+                        // queries i of this block that keep this key: lo <= i < hi (i < ql, and in
+                        // mode 3 jl <= qb*128 + i + off); none when the key is past the sequence
+                        const int64_t ibase = (int64_t)qb * kBlk;
+                        int64_t lo64 = prm.mode == 3 ? jl - off - ibase : 0;
+                        int64_t hi64 = s.ql - ibase;
+                        lo64 = lo64 < 0 ? 0 : (lo64 > kBlk ? kBlk : lo64);
+                        hi64 = hi64 > kBlk ? kBlk : hi64;
+                        const int lo = (int)lo64;
+                        const uint32_t span = key_ok && hi64 > lo64 ? (uint32_t)(hi64 - lo64) : 0u;
+                        ok = wait_bar(CST_FULL(x), use & 1, abort_flag, prm.err, 32);
+                        if (ok) ok = wait_bar(SDP_FULL, pair_ctr & 1, abort_flag, prm.err, 28);
+                        if (ok && pair_ctr > 0) ok = wait_bar(PDS_FREE, (pair_ctr - 1) & 1, abort_flag, prm.err, 29);
+                        if (!ok) break;
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int cc = 4 * cs; cc < 4 * cs + 4; ++cc) {  // 16 query columns at a time
+                            float sv[16], dp[16];
+                            tmem_ld16(T_S + lane_base + cc * 16, sv);
+                            tmem_ld16(T_DP + lane_base + cc * 16, dp);
+                            tmem_wait_ld();
+                            uint32_t pw[8], dw[8];
+                            const float4* cm = reinterpret_cast<const float4*>(cx + cc * 16);        // max * log2e
+                            const float4* cl = reinterpret_cast<const float4*>(cx + 128 + cc * 16);  // 1 / sum
+                            const float4* cd = reinterpret_cast<const float4*>(cx + 256 + cc * 16);  // rowsum(dY o O)
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const uint32_t o = half * 16384 + j * 128 + (((u0 + u) ^ (j & 7)) << 4);
-                            *reinterpret_cast<uint4*>(smem + kOffP + o) =
-                                make_uint4(pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
-                            *reinterpret_cast<uint4*>(smem + kOffDS + o) =
-                                make_uint4(dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
+                            for (int g = 0; g < 4; ++g) {
+                                const float4 m4 = cm[g], l4 = cl[g], d4 = cd[g];
+                                const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, ll[4] = {l4.x, l4.y, l4.z, l4.w},
+                                            dd[4] = {d4.x, d4.y, d4.z, d4.w};
+                                float pv[4], dv[4];
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const int e = 4 * g + k;
+                                    const bool v = (uint32_t)(cc * 16 + e - lo) < span;
+                                    // a select (not a product): masked scores may overflow exp2
+                                    pv[k] = v ? ex2_approx(fmaf(sv[e], c1, -mm[k])) * ll[k] : 0.f;
+                                    dv[k] = pv[k] * (dp[e] - dd[k]) * scale;
+                                }
+                                pw[2 * g] = pack2<T>(pv[0], pv[1]);
+                                pw[2 * g + 1] = pack2<T>(pv[2], pv[3]);
+                                dw[2 * g] = pack2<T>(dv[0], dv[1]);
+                                dw[2 * g + 1] = pack2<T>(dv[2], dv[3]);
+                            }
+                            // columns [16cc, 16cc+16): SW128 half cc/4, 16-byte units 2(cc%4) and 2(cc%4)+1
+                            const int half = cc >> 2, u0 = (cc & 3) * 2;
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const uint32_t o = half * 16384 + j * 128 + (((u0 + u) ^ (j & 7)) << 4);
+                                *reinterpret_cast<uint4*>(smem + kOffP + o) =
+                                    make_uint4(pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
+                                *reinterpret_cast<uint4*>(smem + kOffDS + o) =
+                                    make_uint4(dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
+                            }
                         }
+                        fence_view_async_shared();
+                        tc_fence_before();
+                        mbar_arrive(PDS_FULL);
                     }
-                    fence_view_async_shared();
-                    tc_fence_before();
-                    mbar_arrive(PDS_FULL);
+                    if (do_flush) {
+                        ok = wait_bar(DQ_FULL, pair_ctr & 1, abort_flag, prm.err, 31);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const int dim = j;
+                        const int64_t nq = min((int64_t)kBlk, s.ql - (int64_t)qb * kBlk);
+                        const int64_t row0 = s.qs + (int64_t)qb * kBlk;
+#pragma unroll 1
+                        for (int cc = 2 * hsel; cc < 2 * hsel + 2; ++cc) {
+                            float v[32];
+                            tmem_ld32(T_S + lane_base + cc * 32, v);
+                            tmem_wait_ld();
+                            const int lim = (int)min((int64_t)32, nq - cc * 32);
+                            const size_t base = ((size_t)(row0 + cc * 32) * prm.Nq + h) * kFaD + dim;
+                            const uint32_t step = (uint32_t)prm.Nq * kFaD;  // elements between query rows
+                            // one running pointer (not 32 precomputed addresses) keeps the loop in registers
+                            if (DET) {
+                                unsigned long long* d = reinterpret_cast<unsigned long long*>(prm.dq_acc) + base;
+#pragma unroll
+                                for (int e = 0; e < 32; ++e, d += step)
+                                    if (e < lim) atomicAdd(d, (unsigned long long)__float2ll_rn(v[e] * kFixScale));
+                            } else {
+                                float* d = reinterpret_cast<float*>(prm.dq_acc) + base;
+#pragma unroll
+                                for (int e = 0; e < 32; ++e, d += step)
+                                    if (e < lim) atomicAdd(d, v[e]);
+                            }
+                        }
+                        tc_fence_before();
+                        mbar_arrive(S_FREE);
+                    }
                 }
             }
             if (!ok) break;
+            if (!do_out) continue;
             // dK / dV rows of this key block (zero when no query sees the block)
             ok = wait_bar(ACC_FULL, item_ctr & 1, abort_flag, prm.err, 30);
             if (!ok) break;
@@ -364,51 +410,6 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
             }
             tc_fence_before();
             mbar_arrive(ACC_EMPTY);
-        }
-    } else {
-        // =================== dQ flush (TMEM lane = dim) ===================
-        const int q = warp & 3;                 // TMEM lane quarter
-        const int hsel = (warp - 4) >> 2;       // which half of the query columns
-        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const int dim = q * 32 + lane;
-        int pair_ctr = 0;
-        bool ok = true;
-        for (int w = blockIdx.x; w < prm.nitems && ok; w += gridDim.x) {
-            const FaItem it = prm.items[w];
-            const Seq s = seq_of(prm, it.b);
-            const int q0 = first_qb(s, it.kb, prm.mode), nqb = (int)((s.ql + kBlk - 1) / kBlk);
-            for (int h = it.hk * G; h < it.hk * G + G && ok; ++h) {
-                for (int qb = q0; qb < nqb && ok; ++qb, ++pair_ctr) {
-                    ok = wait_bar(DQ_FULL, pair_ctr & 1, abort_flag, prm.err, 31);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const int64_t nq = min((int64_t)kBlk, s.ql - (int64_t)qb * kBlk);
-                    const int64_t row0 = s.qs + (int64_t)qb * kBlk;
-#pragma unroll 1
-                    for (int cc = 2 * hsel; cc < 2 * hsel + 2; ++cc) {
-                        float v[32];
-                        tmem_ld32(T_S + lane_base + cc * 32, v);
-                        tmem_wait_ld();
-                        const int lim = (int)min((int64_t)32, nq - cc * 32);
-                        const size_t base = ((size_t)(row0 + cc * 32) * prm.Nq + h) * kFaD + dim;
-                        const uint32_t step = (uint32_t)prm.Nq * kFaD;  // elements between query rows
-                        // one running pointer (not 32 precomputed addresses) keeps the loop in registers
-                        if (DET) {
-                            unsigned long long* d = reinterpret_cast<unsigned long long*>(prm.dq_acc) + base;
-#pragma unroll
-                            for (int e = 0; e < 32; ++e, d += step)
-                                if (e < lim) atomicAdd(d, (unsigned long long)__float2ll_rn(v[e] * kFixScale));
-                        } else {
-                            float* d = reinterpret_cast<float*>(prm.dq_acc) + base;
-#pragma unroll
-                            for (int e = 0; e < 32; ++e, d += step)
-                                if (e < lim) atomicAdd(d, v[e]);
-                        }
-                    }
-                    tc_fence_before();
-                    mbar_arrive(S_FREE);
-                }
-            }
         }
     }
 
