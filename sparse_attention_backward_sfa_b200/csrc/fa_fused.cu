@@ -9,11 +9,14 @@
 // for its keys in TMEM (so they are written once, without atomics).  Per
 // (query head, query block):
 //   S^T  = K . Q^T,  dP^T = V . dY^T        [128 keys x 128 queries] in TMEM
-//   P, dS (scale folded in) by the softmax warps (TMEM lane = key) -> SW128 smem
-//   dV  += P  . dY,   dK += dS . Q          [128 keys x 128 dims] in TMEM
+//   P (16-bit, written back into S^T's columns) and dS (scale folded in, SW128
+//        smem) by the softmax warps (TMEM lane = key)
+//   dV  += P  . dY  (A operand read from TMEM),   dK += dS . Q     [128 keys x 128 dims]
 //   dQ^T = K^T . dS^T                        [128 dims x 128 queries], reusing
-//        S^T's columns, reduced into an fp32 (or 64-bit fixed point) dQ buffer
+//        dP^T's columns, reduced into an fp32 (or 64-bit fixed point) dQ buffer
 //        by the flush warps (TMEM lane = dim: 128-byte coalesced reductions).
+// Q / dY are double-buffered, so the next pair's load overlaps this pair, and the
+// next S^T is issued as soon as this pair's gradient MMAs have read P.
 // Warps: 0-7 softmax (two per TMEM lane quarter, each taking half of the query
 // columns), 0-3 also the dK/dV write-out, 4-11 dQ flush (two per lane quarter,
 // halves of the query columns), 12 TMA producer, 13 MMA.
@@ -36,10 +39,11 @@ using namespace tc;
 constexpr int kFaD = 128;
 constexpr int kBlk = 128;
 constexpr int kFaThreads = 448;
-constexpr int kOffK = 0, kOffV = 32768, kOffQ = 65536, kOffO = 98304, kOffP = 131072, kOffDS = 163840;
-constexpr int kOffCst = 196608;                     // float [2][3][128]: max*log2e, 1/sum, rowsum(dY o O)
-constexpr int kOffBar = kOffCst + 2 * 3 * 128 * 4;  // 14 mbarriers
-constexpr int kOffMisc = kOffBar + 16 * 8;
+// K, V, then Q / dY of slot x at kOffQ / kOffO + x * 65536, dS, constants, barriers
+constexpr int kOffK = 0, kOffV = 32768, kOffQ = 65536, kOffO = 98304, kOffDS = 196608;
+constexpr int kOffCst = 229376;                     // float [2][2][128]: max*log2e + log2(sum), rowsum(dY o O)
+constexpr int kOffBar = kOffCst + 2 * 2 * 128 * 4;  // 17 mbarriers
+constexpr int kOffMisc = kOffBar + 18 * 8;
 constexpr int kFaSmem = kOffMisc + 16;
 
 struct FaItem {
@@ -94,31 +98,35 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
     }
     float* cst = reinterpret_cast<float*>(smem + kOffCst);
     const uint32_t bar0 = sbase + kOffBar;
-    const uint32_t KV_FULL = bar0, KV_EMPTY = bar0 + 8, QDO_FULL = bar0 + 16, QDO_EMPTY = bar0 + 24,
-                   SDP_FULL = bar0 + 32, PDS_FULL = bar0 + 40, PDS_FREE = bar0 + 48, DQ_FULL = bar0 + 56,
-                   S_FREE = bar0 + 64, ACC_FULL = bar0 + 72, ACC_EMPTY = bar0 + 80, DONE = bar0 + 88;
-    auto CST_FULL = [&](int x) { return bar0 + 96 + 8u * x; };  // per-pair softmax constants written
+    const uint32_t KV_FULL = bar0, KV_EMPTY = bar0 + 8, SDP_FULL = bar0 + 16, PDS_FULL = bar0 + 24,
+                   PDS_FREE = bar0 + 32, DQ_FULL = bar0 + 40, DQ_FREE = bar0 + 48, ACC_FULL = bar0 + 56,
+                   ACC_EMPTY = bar0 + 64, DONE = bar0 + 72;
+    auto CST_FULL = [&](int x) { return bar0 + 80 + 8u * x; };   // per-pair softmax constants written
+    auto QDO_FULL = [&](int x) { return bar0 + 96 + 8u * x; };   // Q / dY slot loaded
+    auto QDO_EMPTY = [&](int x) { return bar0 + 112 + 8u * x; }; // ... and consumed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     if (threadIdx.x == 0) {
         mbar_init(KV_FULL, 1);
         mbar_init(KV_EMPTY, 1);
-        mbar_init(QDO_FULL, 1);
-        mbar_init(QDO_EMPTY, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(QDO_FULL(x), 1);
+            mbar_init(QDO_EMPTY(x), 1);
+        }
         mbar_init(SDP_FULL, 1);
         mbar_init(PDS_FULL, 256);
         mbar_init(CST_FULL(0), 128);
         mbar_init(CST_FULL(1), 128);
         mbar_init(PDS_FREE, 1);
         mbar_init(DQ_FULL, 1);
-        mbar_init(S_FREE, 256);
+        mbar_init(DQ_FREE, 256);
         mbar_init(ACC_FULL, 1);
         mbar_init(ACC_EMPTY, 128);
         mbar_init(DONE, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) {  // S^T / dQ^T [0,128), dP^T [128,256), dK [256,384), dV [384,512)
+    if (warp == 0) {  // S^T / P [0,128), dP^T / dQ^T [128,256), dK [256,384), dV [384,512)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tmem_slot))
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -153,14 +161,17 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
             const int q0 = first_qb(s, it.kb, prm.mode), nqb = (int)((s.ql + kBlk - 1) / kBlk);
             for (int h = it.hk * G; h < it.hk * G + G && ok; ++h) {
                 for (int qb = q0; qb < nqb && ok; ++qb, ++pair_ctr) {
+                    const int x = pair_ctr & 1;
                     if (lane == 0) {
-                        ok = wait_bar(QDO_EMPTY, (pair_ctr & 1) ^ 1, abort_flag, prm.err, 22);
+                        ok = wait_bar(QDO_EMPTY(x), ((pair_ctr >> 1) & 1) ^ 1, abort_flag, prm.err, 22);
                         if (ok) {
-                            mbar_expect_tx(QDO_FULL, 4 * kBlk * 128);
+                            mbar_expect_tx(QDO_FULL(x), 4 * kBlk * 128);
                             const int row = (int)(s.qs + (int64_t)qb * kBlk);
                             for (int hh = 0; hh < 2; ++hh) {
-                                tma_load_2d(sbase + kOffQ + hh * 16384, &prm.mapQ, h * kFaD + hh * 64, row, QDO_FULL);
-                                tma_load_2d(sbase + kOffO + hh * 16384, &prm.mapO, h * kFaD + hh * 64, row, QDO_FULL);
+                                tma_load_2d(sbase + kOffQ + x * 65536 + hh * 16384, &prm.mapQ, h * kFaD + hh * 64, row,
+                                            QDO_FULL(x));
+                                tma_load_2d(sbase + kOffO + x * 65536 + hh * 16384, &prm.mapO, h * kFaD + hh * 64, row,
+                                            QDO_FULL(x));
                             }
                         }
                     }
@@ -173,17 +184,19 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
             if (item_ctr > 0)
                 while (!mbar_try(KV_FULL, (item_ctr - 1) & 1) && globaltimer() - t0 < 1000000000ull) {
                 }
-            if (pair_ctr > 0)
-                while (!mbar_try(QDO_FULL, (pair_ctr - 1) & 1) && globaltimer() - t0 < 1000000000ull) {
-                }
+            for (int k = 1; k <= 2; ++k) {
+                const int p = pair_ctr - k;
+                if (p >= 0)
+                    while (!mbar_try(QDO_FULL(p & 1), (p >> 1) & 1) && globaltimer() - t0 < 1000000000ull) {
+                    }
+            }
         }
     } else if (warp == 13) {
         // =================== MMA issuer ===================
         const uint32_t ID_S = idesc(128, 128, false, false, kF16);  // S^T, dP^T (A = K/V, B = Q/dY, both K-major)
-        const uint32_t ID_A = idesc(128, 128, false, true, kF16);   // dV, dK (A = P/dS K-major, B = dY/Q MN-major)
+        const uint32_t ID_A = idesc(128, 128, false, true, kF16);   // dV (A = P in TMEM), dK (A = dS K-major); B MN-major
         const uint32_t ID_Q = idesc(128, 128, true, true, kF16);    // dQ^T (A = K MN-major, B = dS MN-major)
-        const uint32_t sK = sbase + kOffK, sV = sbase + kOffV, sQ = sbase + kOffQ, sO = sbase + kOffO,
-                       sP = sbase + kOffP, sDS = sbase + kOffDS;
+        const uint32_t sK = sbase + kOffK, sV = sbase + kOffV, sDS = sbase + kOffDS;
         int item_ctr = 0, pair_ctr = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < prm.nitems && ok; w += gridDim.x, ++item_ctr) {
@@ -198,8 +211,13 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
             bool first = true;
             for (int h = it.hk * G; h < it.hk * G + G && ok; ++h) {
                 for (int qb = q0; qb < nqb && ok; ++qb, ++pair_ctr) {
-                    if (lane == 0) ok = wait_bar(QDO_FULL, pair_ctr & 1, abort_flag, prm.err, 25);
-                    if (lane == 0 && ok) ok = wait_bar(S_FREE, (pair_ctr & 1) ^ 1, abort_flag, prm.err, 26);
+                    const int x = pair_ctr & 1;
+                    const uint32_t sQ = sbase + kOffQ + x * 65536, sO = sbase + kOffO + x * 65536;
+                    if (lane == 0) {
+                        ok = wait_bar(QDO_FULL(x), (pair_ctr >> 1) & 1, abort_flag, prm.err, 25);
+                        // S^T overwrites P of the previous pair: its gradient MMAs must have completed
+                        if (ok && pair_ctr > 0) ok = wait_bar(PDS_FREE, (pair_ctr - 1) & 1, abort_flag, prm.err, 26);
+                    }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     tc_fence_after();
@@ -208,27 +226,33 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                             const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
                             mma(T_S, sdesc(sK + off, 16, 1024), sdesc(sQ + off, 16, 1024), ID_S, ks > 0);
                         }
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            mma(T_DP, sdesc(sV + off, 16, 1024), sdesc(sO + off, 16, 1024), ID_S, ks > 0);
+                        // dP^T overwrites the previous pair's dQ^T once the flush has read it
+                        ok = wait_bar(DQ_FREE, (pair_ctr & 1) ^ 1, abort_flag, prm.err, 33);
+                        if (ok) {
+                            tc_fence_after();
+                            for (int ks = 0; ks < 8; ++ks) {
+                                const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                                mma(T_DP, sdesc(sV + off, 16, 1024), sdesc(sO + off, 16, 1024), ID_S, ks > 0);
+                            }
+                            mma_commit(SDP_FULL);
+                            ok = wait_bar(PDS_FULL, pair_ctr & 1, abort_flag, prm.err, 27);
                         }
-                        mma_commit(SDP_FULL);
-                        ok = wait_bar(PDS_FULL, pair_ctr & 1, abort_flag, prm.err, 27);
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     tc_fence_after();
                     if (lane == 0) {
                         for (int ks = 0; ks < 8; ++ks) {  // K = 128 queries, 16 per step
-                            const uint64_t aP = sdesc(sP + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                            // P of queries 16ks..16ks+15: TMEM columns 64*(ks/4) + 8*(ks%4) (16-bit pairs)
+                            const uint32_t aP = T_S + 64u * (ks >> 2) + 8u * (ks & 3);
                             const uint64_t aS = sdesc(sDS + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                            mma(T_DV, aP, sdesc(sO + ks * 2048, 16384, 1024), ID_A, (!first || ks > 0));
+                            mma_ts(T_DV, aP, sdesc(sO + ks * 2048, 16384, 1024), ID_A, (!first || ks > 0));
                             mma(T_DK, aS, sdesc(sQ + ks * 2048, 16384, 1024), ID_A, (!first || ks > 0));
                         }
                         for (int ks = 0; ks < 8; ++ks)  // K = 128 keys
-                            mma(T_S, sdesc(sK + ks * 2048, 16384, 1024), sdesc(sDS + ks * 2048, 16384, 1024), ID_Q,
+                            mma(T_DP, sdesc(sK + ks * 2048, 16384, 1024), sdesc(sDS + ks * 2048, 16384, 1024), ID_Q,
                                 ks > 0);
-                        mma_commit(QDO_EMPTY);
+                        mma_commit(QDO_EMPTY(x));
                         mma_commit(PDS_FREE);
                         mma_commit(DQ_FULL);
                     }
@@ -272,21 +296,21 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                 for (int qb = q0; qb < nqb && ok; ++qb, ++pair_ctr, ++npairs) {
                     if (do_softmax) {
                         const int x = pair_ctr & 1, use = pair_ctr >> 1;
-                        float* cx = cst + x * 384;
+                        float* cx = cst + x * 256;
                         if (do_out) {
                             // constants of query row j of this block (the buffer's previous pair,
                             // pair_ctr - 2, finished its softmax before the gradients of pair_ctr - 1)
                             const int64_t il = (int64_t)qb * kBlk + j;
+                            // P = exp2(S*scale*log2e - (max*log2e + log2(sum))); an empty row (sum 0)
+                            // gets +inf, so P = 0
                             if (il < s.ql) {
                                 const int64_t sidx = (s.qs + il) * prm.Nq + h;
                                 const float l = prm.ssum[sidx * 8];
-                                cx[j] = prm.smax[sidx * 8] * 1.4426950408889634f;
-                                cx[128 + j] = l == 0.f ? 0.f : 1.f / l;
-                                cx[256 + j] = prm.rowsum[sidx];
+                                cx[j] = l > 0.f ? fmaf(prm.smax[sidx * 8], 1.4426950408889634f, log2f(l)) : INFINITY;
+                                cx[128 + j] = prm.rowsum[sidx];
                             } else {
-                                cx[j] = 0.f;
+                                cx[j] = INFINITY;
                                 cx[128 + j] = 0.f;
-                                cx[256 + j] = 0.f;
                             }
                             mbar_arrive(CST_FULL(x));
                         }
@@ -311,21 +335,19 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                             tmem_ld16(T_DP + lane_base + cc * 16, dp);
                             tmem_wait_ld();
                             uint32_t pw[8], dw[8];
-                            const float4* cm = reinterpret_cast<const float4*>(cx + cc * 16);        // max * log2e
-                            const float4* cl = reinterpret_cast<const float4*>(cx + 128 + cc * 16);  // 1 / sum
-                            const float4* cd = reinterpret_cast<const float4*>(cx + 256 + cc * 16);  // rowsum(dY o O)
+                            const float4* cm = reinterpret_cast<const float4*>(cx + cc * 16);        // log2 offset
+                            const float4* cd = reinterpret_cast<const float4*>(cx + 128 + cc * 16);  // rowsum(dY o O)
 #pragma unroll
                             for (int g = 0; g < 4; ++g) {
-                                const float4 m4 = cm[g], l4 = cl[g], d4 = cd[g];
-                                const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, ll[4] = {l4.x, l4.y, l4.z, l4.w},
-                                            dd[4] = {d4.x, d4.y, d4.z, d4.w};
+                                const float4 m4 = cm[g], d4 = cd[g];
+                                const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
                                 float pv[4], dv[4];
 #pragma unroll
                                 for (int k = 0; k < 4; ++k) {
                                     const int e = 4 * g + k;
                                     const bool v = (uint32_t)(cc * 16 + e - lo) < span;
                                     // a select (not a product): masked scores may overflow exp2
-                                    pv[k] = v ? ex2_approx(fmaf(sv[e], c1, -mm[k])) * ll[k] : 0.f;
+                                    pv[k] = v ? ex2_approx(fmaf(sv[e], c1, -mm[k])) : 0.f;
                                     dv[k] = pv[k] * (dp[e] - dd[k]) * scale;
                                 }
                                 pw[2 * g] = pack2<T>(pv[0], pv[1]);
@@ -333,17 +355,19 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                                 dw[2 * g] = pack2<T>(dv[0], dv[1]);
                                 dw[2 * g + 1] = pack2<T>(dv[2], dv[3]);
                             }
-                            // columns [16cc, 16cc+16): SW128 half cc/4, 16-byte units 2(cc%4) and 2(cc%4)+1
+                            // P -> TMEM columns 64*(cc/4) + 8*(cc%4): inside the S^T columns this warp
+                            // group reads, at or behind the ones it has already read
+                            tmem_st8(T_S + lane_base + 64u * (cc >> 2) + 8u * (cc & 3), pw);
+                            // dS columns [16cc, 16cc+16): SW128 half cc/4, 16-byte units 2(cc%4) and 2(cc%4)+1
                             const int half = cc >> 2, u0 = (cc & 3) * 2;
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
                                 const uint32_t o = half * 16384 + j * 128 + (((u0 + u) ^ (j & 7)) << 4);
-                                *reinterpret_cast<uint4*>(smem + kOffP + o) =
-                                    make_uint4(pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
                                 *reinterpret_cast<uint4*>(smem + kOffDS + o) =
                                     make_uint4(dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
                             }
                         }
+                        tmem_wait_st();
                         fence_view_async_shared();
                         tc_fence_before();
                         mbar_arrive(PDS_FULL);
@@ -358,7 +382,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
 #pragma unroll 1
                         for (int cc = 2 * hsel; cc < 2 * hsel + 2; ++cc) {
                             float v[32];
-                            tmem_ld32(T_S + lane_base + cc * 32, v);
+                            tmem_ld32(T_DP + lane_base + cc * 32, v);
                             tmem_wait_ld();
                             const int lim = (int)min((int64_t)32, nq - cc * 32);
                             const size_t base = ((size_t)(row0 + cc * 32) * prm.Nq + h) * kFaD + dim;
@@ -377,7 +401,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                             }
                         }
                         tc_fence_before();
-                        mbar_arrive(S_FREE);
+                        mbar_arrive(DQ_FREE);
                     }
                 }
             }
