@@ -36,29 +36,34 @@ FLOP_PER_TRIPLE = 5504
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "sfa_bwd_fused_kernel_workload4.md")
-KERNEL_SOURCES = [os.path.join(ROOT, "sparse_attention_backward_sfa_b200", "csrc", f)
-                  for f in ("sfa_fused.cu", "tc_common.cuh")]
+# committed ncu summaries: (summary file, kernel sources whose hash it records)
+PROFILE_SUMMARIES = {
+    4: ("sfa_bwd_fused_kernel_workload4.md", ("sfa_fused.cu", "tc_common.cuh")),
+    2: ("fa_bwd_fused_kernel_workload2.md", ("fa_fused.cu", "tc_common.cuh")),
+}
 
 
-def kernel_source_hash():
+def kernel_source_hash(sources):
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
-        with open(f, "rb") as fh:
+    for f in sources:
+        with open(os.path.join(ROOT, "sparse_attention_backward_sfa_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
 
 
-def recorded_traffic():
-    """DRAM bytes per launch of the fused kernel on workload 4 from the committed
-    ncu summary, or None when the kernel sources changed since the capture."""
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the workload's main kernel from the committed ncu
+    summary, or None when there is none or the kernel sources changed since the capture."""
+    if workload not in PROFILE_SUMMARIES:
+        return None
+    name, sources = PROFILE_SUMMARIES[workload]
     try:
-        txt = open(PROFILE_SUMMARY).read()
+        txt = open(os.path.join(ROOT, "profiles", name)).read()
     except OSError:
         return None
     vals = dict(re.findall(r"^(traffic_bytes_per_launch|kernel_source_sha256):\s*(\S+)", txt, re.M))
-    if vals.get("kernel_source_sha256") != kernel_source_hash():
+    if vals.get("kernel_source_sha256") != kernel_source_hash(sources):
         return None
     try:
         return float(vals["traffic_bytes_per_launch"])
@@ -422,8 +427,9 @@ def main():
                 "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": WORKLOADS[2], "valid_triples": r["triples"], "gflop_per_step": r["flop"] / 1e9},
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                             "frac": achieved / peak, "kernel": "fa_bwd_kernel", "kernel_ms": kern, "traffic": None},
-                "gpu_launches": 2 * args.steps, "clocks": r["clocks"]}
+                             "frac": achieved / peak, "kernel": "fa_bwd_fused_kernel", "kernel_ms": kern,
+                             "traffic": recorded_traffic(2)},
+                "gpu_launches": 3 * args.steps, "clocks": r["clocks"]}
         print(json.dumps(line), flush=True)
     elif rank == 0:
         p = r["p"]
@@ -443,7 +449,7 @@ def main():
                          "peak_sustained": float(peaks.get("bf16_tflops_sustained", peak)),
                          "frac_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                          "kernel": "sfa_bwd_fused_kernel", "kernel_ms": kern,
-                         "traffic": recorded_traffic() if args.workload == 4 and not args.seqs else None},
+                         "traffic": recorded_traffic(4) if args.workload == 4 and not args.seqs else None},
             "cpu_baseline": cpu,
             "e2e": r["e2e"],
             "gpu_launches": 7 * args.steps,
