@@ -7,9 +7,14 @@ key-row expansion, the fused tensor-core backward, the dQuery and dKey/dValue
 casts) over one batch of the workload, inputs resident in HBM.  The metric is
 TFLOP/s with the 5-GEMM count (5504 FLOP per valid (query row, head, key)).
 
-N > 1 (torchrun): every rank runs its own independent copy of the workload
-(seed + rank); no data-path collective; value = total FLOP of all ranks / the
-max over ranks of the timed region ("scaling": "weak").
+N > 1 (torchrun), sparse workloads: the workload's query rows are split into N
+contiguous ranges of equal work (valid (row, key) pairs); every rank holds the
+whole (identically generated) problem, runs the backward of its rows into a
+key-side accumulator (sfa_grad_rows), the ranks sum the accumulators with one
+NCCL all-reduce (int64 fixed point in deterministic mode: exact), and each rank
+casts it (sfa_dkv_finalize).  One step = that whole sharded backward; value =
+the workload's FLOP / the max over ranks of the timed region ("scaling":
+"strong").  The dense FA workload (2) runs independent replicas ("weak").
 
 --impl reference times the CPU oracle (the plain numpy definition) on a
 bounded sample of the same workload on the host cores (rank 0 only).
@@ -146,14 +151,6 @@ def kw(p):
                 actual_seq_lengths_q=p.seqlens_q, actual_seq_lengths_kv=p.seqlens_kv)
 
 
-def count_triples(p):
-    import sparse_attention_backward_sfa_b200 as S
-    _, _, nr = S.compact_indices(p.indices, p.k, p.q, p.q_rope, sparse_block_size=p.block_size, layout=p.layout,
-                                 sparse_mode=p.sparse_mode, actual_seq_lengths_q=p.seqlens_q,
-                                 actual_seq_lengths_kv=p.seqlens_kv)
-    return int(nr.to(dtype=__import__("torch").int64).sum().item()) * p.N1
-
-
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -163,22 +160,49 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     lib = N.load()
-    p = build_problem(args.workload, rank, dev)
+    sharded = world > 1
+    # sharded: every rank builds the same problem and takes its share of the rows
+    p = build_problem(args.workload, 0 if sharded else rank, dev)
     out, smax, ssum = S.sfa_fwd(p.q, p.k, p.k, p.indices, p.q_rope, p.k_rope, **kw(p))
-    triples = count_triples(p)
+    _, _, nr = S.compact_indices(p.indices, p.k, p.q, p.q_rope, sparse_block_size=p.block_size, layout=p.layout,
+                                 sparse_mode=p.sparse_mode, actual_seq_lengths_q=p.seqlens_q,
+                                 actual_seq_lengths_kv=p.seqlens_kv)
+    nr = nr.to(torch.int64).cpu().numpy()
+    triples = int(nr.sum()) * p.N1
     flop = triples * FLOP_PER_TRIPLE
+    T1 = nr.size
+    ranges = S.balanced_row_ranges(nr, world) if sharded else [(0, T1)]
+    rb, re_ = ranges[rank]
+    flop_rank = int(nr[rb:re_].sum()) * p.N1 * FLOP_PER_TRIPLE
     shape = S.sfa_shape(p.q, p.k, p.q_rope, p.indices, p.layout, p.seqlens_q)
     ws_bytes = S.sfa_grad_workspace_size(shape, p.block_size, p.sparse_mode, p.deterministic)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     outs = (torch.empty_like(p.q), torch.empty_like(p.k), torch.empty_like(p.k), torch.empty_like(p.q_rope),
             torch.empty_like(p.k_rope))
+    acc = S.sfa_dkv_accumulator(p.q, p.k, p.q_rope, p.indices, layout=p.layout, deterministic=p.deterministic,
+                                actual_seq_lengths_q=p.seqlens_q) if sharded else None
     stream = torch.cuda.current_stream(dev)
+
+    def grad(q, k, idx, do, o, mx, sm, qr, kr, sq, skv):
+        if not sharded:
+            S.sfa_grad(q, k, k, idx, do, o, mx, sm, qr, kr, deterministic=p.deterministic, workspace=ws, outputs=outs,
+                       scale=p.scale, sparse_block_size=p.block_size, layout=p.layout, sparse_mode=p.sparse_mode,
+                       actual_seq_lengths_q=sq, actual_seq_lengths_kv=skv)
+            return
+        dq, dk, dv, dqr, dkr = outs
+        acc.zero_()
+        S.sfa_grad_rows(q, k, k, idx, do, o, mx, sm, qr, kr, row_begin=rb, row_end=re_, dkv_accum=acc,
+                        deterministic=p.deterministic, workspace=ws, d_query=dq, d_query_rope=dqr, scale=p.scale,
+                        sparse_block_size=p.block_size, layout=p.layout, sparse_mode=p.sparse_mode,
+                        actual_seq_lengths_q=sq, actual_seq_lengths_kv=skv)
+        dist.all_reduce(acc, op=dist.ReduceOp.SUM)
+        S.sfa_dkv_finalize(acc, q, k, qr, idx, layout=p.layout, deterministic=p.deterministic,
+                           actual_seq_lengths_q=sq, outputs=(dk, dv, dkr))
 
     def step(ev=None):
         if ev is not None:
             N.check(lib.sfa_set_kernel_events(ctypes_ptr(ev[0]), ctypes_ptr(ev[1])))
-        S.sfa_grad(p.q, p.k, p.k, p.indices, p.dout, out, smax, ssum, p.q_rope, p.k_rope,
-                   deterministic=p.deterministic, workspace=ws, outputs=outs, **kw(p))
+        grad(p.q, p.k, p.indices, p.dout, out, smax, ssum, p.q_rope, p.k_rope, p.seqlens_q, p.seqlens_kv)
 
     for _ in range(args.warmup):
         step()
@@ -192,6 +216,8 @@ def run_ours(args, rank, world, local_rank):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank) as clk:
         torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
         t0.record(stream)
         for i in range(args.steps):
             step(evs[i])
@@ -209,32 +235,43 @@ def run_ours(args, rank, world, local_rank):
         ms_step = float(t.item())
 
     # end-to-end through the public API with host buffers: H2D of the step's
-    # inputs from pinned memory, the call, D2H of the five gradients
+    # inputs from pinned memory, the call(s), D2H of the gradients.  Sharded: each
+    # rank copies its rows of the query-side inputs plus the shared key side and
+    # indices, and reads back its dQuery rows and the summed key-side gradients.
     e2e = None
     if not args.no_e2e:
-        host_in = [x.cpu().pin_memory() for x in (p.q, p.q_rope, p.k, p.k_rope, p.dout, out, smax, ssum, p.indices)]
-        if p.seqlens_q is not None:
-            host_in.append(p.seqlens_q.cpu().pin_memory())
-        dev_in = [torch.empty_like(x, device=dev) for x in host_in]
-        host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
-        h2d = sum(x.numel() * x.element_size() for x in host_in)
+        qside = [p.q, p.q_rope, p.dout, out, smax, ssum]
+        shared = [p.k, p.k_rope, p.indices] + ([p.seqlens_q] if p.seqlens_q is not None else [])
+        rows = lambda x: x.reshape(T1, -1)[rb:re_]  # this rank's query rows of a [.., T1-row] tensor
+        host_q = [rows(x).cpu().pin_memory() for x in qside]
+        host_s = [x.cpu().pin_memory() for x in shared]
+        dev_q = [torch.zeros_like(x) for x in qside]
+        dev_s = [torch.empty_like(x) for x in shared]
+        dq, dk, dv, dqr, dkr = outs
+        host_out = [torch.empty_like(rows(dq), device="cpu").pin_memory(),
+                    torch.empty_like(rows(dqr), device="cpu").pin_memory()] + \
+                   [torch.empty_like(x, device="cpu").pin_memory() for x in (dk, dv, dkr)]
+        h2d = sum(x.numel() * x.element_size() for x in host_q + host_s)
         d2h = sum(x.numel() * x.element_size() for x in host_out)
 
         def e2e_step():
-            for d, h in zip(dev_in, host_in):
+            for d, h in zip(dev_q, host_q):
+                rows(d).copy_(h, non_blocking=True)
+            for d, h in zip(dev_s, host_s):
                 d.copy_(h, non_blocking=True)
-            q, qr, k, kr, do, o, mx, sm, idx = dev_in[:9]
-            sq = dev_in[9] if len(dev_in) > 9 else None
-            S.sfa_grad(q, k, k, idx, do, o, mx, sm, qr, kr, deterministic=p.deterministic, workspace=ws,
-                       outputs=outs, scale=p.scale, sparse_block_size=p.block_size, layout=p.layout,
-                       sparse_mode=p.sparse_mode, actual_seq_lengths_q=sq, actual_seq_lengths_kv=sq)
-            for h, o2 in zip(host_out, outs):
+            q, qr, do, o, mx, sm = dev_q
+            k, kr, idx = dev_s[:3]
+            sq = dev_s[3] if len(dev_s) > 3 else None
+            grad(q, k, idx, do, o, mx, sm, qr, kr, sq, sq)
+            for h, o2 in zip(host_out, (rows(dq), rows(dqr), dk, dv, dkr)):
                 h.copy_(o2, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize(dev)
         n_e2e = max(2, min(args.steps, 5))
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
         a.record(stream)
         for _ in range(n_e2e):
             e2e_step()
@@ -245,11 +282,12 @@ def run_ours(args, rank, world, local_rank):
             t = torch.tensor([e2e_ms], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e2e_ms = float(t.item())
-        e2e = {"value": flop * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e = {"value": flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     err_word = int(err[0].item())
-    return dict(flop=flop, triples=triples, ms_step=ms_step, kern_ms=kern_ms, clocks=clk.summary(), e2e=e2e,
-                ws_bytes=ws_bytes, err_word=err_word, p=p)
+    return dict(flop=flop, flop_rank=flop_rank, triples=triples, ms_step=ms_step, kern_ms=kern_ms,
+                clocks=clk.summary(), e2e=e2e, ws_bytes=ws_bytes, err_word=err_word, p=p, sharded=sharded,
+                rows=(rb, re_))
 
 
 def run_fa(args, rank, world, local_rank):
@@ -412,9 +450,11 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     r = run_fa(args, rank, world, local_rank) if args.workload == 2 else run_ours(args, rank, world, local_rank)
     peaks, src = load_peaks()
-    value = r["flop"] * world / (r["ms_step"] * 1e-3) / 1e12
+    sharded = bool(r.get("sharded"))
+    # sharded: r["flop"] is the whole workload, split over the ranks; replicas: per rank
+    value = r["flop"] * (1 if sharded else world) / (r["ms_step"] * 1e-3) / 1e12
     kern = statistics.mean(r["kern_ms"])
-    achieved = r["flop"] / (kern * 1e-3) / 1e12
+    achieved = r.get("flop_rank", r["flop"]) / (kern * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload != 2:
@@ -435,7 +475,8 @@ def main():
         p = r["p"]
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": r["ms_step"], "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": r["ms_step"], "higher_is_better": True,
+            "scaling": "strong" if sharded else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "pct_of_peak": 100.0 * value / world / peak,
             "config": {"workload": WORKLOADS[args.workload] + (f" seqs={args.seqs}" if args.seqs else ""),
@@ -443,16 +484,18 @@ def main():
                        "sparse_block_size": p.block_size, "deterministic": p.deterministic,
                        "valid_triples": r["triples"], "gflop_per_step": r["flop"] / 1e9,
                        "l2": "inputs larger than L2 (q+dO+O %.1f GB per step)" % (3 * p.q.numel() * 2 / 1e9),
-                       "parallelism": f"independent replica per GPU x{world}"},
+                       "parallelism": (f"query rows sharded over {world} GPUs by work, NCCL all-reduce of the "
+                                       f"dK/dV accumulator" if sharded else "single GPU")},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "peak_source": f"{src} bf16 burst",
                          "peak_sustained": float(peaks.get("bf16_tflops_sustained", peak)),
                          "frac_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                          "kernel": "sfa_bwd_fused_kernel", "kernel_ms": kern,
-                         "traffic": recorded_traffic(4) if args.workload == 4 and not args.seqs else None},
+                         "traffic": recorded_traffic(4) if args.workload == 4 and not args.seqs and not sharded
+                         else None},
             "cpu_baseline": cpu,
             "e2e": r["e2e"],
-            "gpu_launches": 7 * args.steps,
+            "gpu_launches": 6 * args.steps,  # compact, rowsum, order, expand, fused backward, cast
             "clocks": r["clocks"],
             "device_error_word": r["err_word"],
         }

@@ -134,6 +134,52 @@ sfa_status sfa_grad(const void *query, const void *key, const void *value, const
                     void *d_query, void *d_key, void *d_value, void *d_query_rope, void *d_key_rope);
 
 /*
+ * Query-row sharding of sfa_grad (for data parallelism over query rows with a
+ * replicated key/value: each GPU runs its own rows, then the key-side sums are
+ * added across GPUs).  The pages' operator runs all rows at once; splitting it
+ * this way computes the same sums (SparseFlashAttentionGrad README, 功能说明:
+ * dKey / dValue are sums over every query row that selected a key, so partial
+ * sums over disjoint row sets add up to the whole).
+ *
+ * sfa_dkv_accum_size - bytes of the key-side accumulator: [T2][1088] (columns
+ * dKey 0-511 | dKeyRope 512-575 | dValue 576-1087), fp32 when deterministic == 0,
+ * int64 fixed point (value * 2^32, rounded) when 1.  Host only.
+ */
+sfa_status sfa_dkv_accum_size(const sfa_shape *shape, int32_t deterministic, size_t *accum_bytes);
+
+/*
+ * sfa_grad_rows - sfa_grad restricted to query rows [row_begin, row_end) of the
+ * flattened [T1] row index (BSND: b * S1 + s; TND: the token index).
+ *   - Same inputs, workspace and validation as sfa_grad; 0 <= row_begin <=
+ *     row_end <= T1, else SFA_ERR_INVALID before any device work.
+ *   - d_query / d_query_rope: the rows in the range are written (zero for rows
+ *     with no selected key); rows outside the range are not touched.
+ *   - dkv_accum (caller-owned, 256-byte aligned, sfa_dkv_accum_size bytes): the
+ *     range's dKey | dKeyRope | dValue contributions are ADDED to it; the caller
+ *     zeroes it before the first range and may add accumulators of other ranges
+ *     (other GPUs) element-wise before sfa_dkv_finalize.  With deterministic == 1
+ *     the accumulator is integer, so that element-wise addition is exact and
+ *     order-independent and the final outputs are bit-identical to sfa_grad's.
+ *   - Enqueued on `stream`; nothing is allocated and nothing synchronizes.
+ */
+sfa_status sfa_grad_rows(const void *query, const void *key, const void *value, const int32_t *sparse_indices,
+                         const void *d_out, const void *out, const float *softmax_max, const float *softmax_sum,
+                         const int32_t *actual_seq_lengths_q, const int32_t *actual_seq_lengths_kv,
+                         const void *query_rope, const void *key_rope, float scale, int64_t sparse_block_size,
+                         int64_t sparse_mode, int32_t deterministic, int64_t row_begin, int64_t row_end,
+                         const sfa_shape *shape, void *workspace, size_t workspace_bytes, sfa_stream_t stream,
+                         void *dkv_accum, void *d_query, void *d_query_rope);
+
+/*
+ * sfa_dkv_finalize - casts a (summed) key-side accumulator into the 16-bit
+ * d_key [.., N2, D], d_value [.., N2, D] and d_key_rope [.., N2, Dr] outputs
+ * (round to nearest even; fixed point is divided by 2^32 first).  `shape` gives
+ * T2 and the dtype; `deterministic` selects the accumulator format.
+ */
+sfa_status sfa_dkv_finalize(const void *dkv_accum, const sfa_shape *shape, int32_t deterministic, sfa_stream_t stream,
+                            void *d_key, void *d_value, void *d_key_rope);
+
+/*
  * sfa_grad_noalloc - sfa_grad for callers that cannot allocate device memory.
  * (The source pages have no counterpart: it exists for this library's callers.)
  *

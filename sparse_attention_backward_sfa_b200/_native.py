@@ -65,6 +65,10 @@ SIGNATURES = {
     "fa_fwd_workspace_size": [_PFA, _I64, _PSZ],
     "fa_fwd": [_V, _V, _V, _V, _V, _Dbl, _I64, _PFA, _V, _SZ, _V, _V, _V, _V],
     "sfa_set_kernel_events": [_V, _V],
+    "sfa_dkv_accum_size": [_PSH, _I32, _PSZ],
+    "sfa_grad_rows": [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _F, _I64, _I64, _I32, _I64, _I64, _PSH, _V,
+                      _SZ, _V, _V, _V, _V],
+    "sfa_dkv_finalize": [_V, _PSH, _I32, _V, _V, _V, _V],
     "sfa_grad_noalloc": [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _F, _I64, _I64, _I64, _I64, _I32, _PSH, _V,
                          _V, _V, _V, _V, _V],
     "sfa_status_string": [_I32],

@@ -146,26 +146,38 @@ sfa_status sfa_grad_workspace_size(const sfa_shape* shape, int64_t sparse_block_
     return SFA_OK;
 }
 
-sfa_status sfa_grad(const void* query, const void* key, const void* value, const int32_t* sparse_indices,
-                    const void* d_out, const void* out, const float* softmax_max, const float* softmax_sum,
-                    const int32_t* actual_seq_lengths_q, const int32_t* actual_seq_lengths_kv,
-                    const void* query_rope, const void* key_rope, float scale, int64_t sparse_block_size,
-                    int64_t sparse_mode, int64_t pre_tokens, int64_t next_tokens, int32_t deterministic,
-                    const sfa_shape* shape, void* workspace, size_t workspace_bytes, sfa_stream_t stream,
-                    void* d_query, void* d_key, void* d_value, void* d_query_rope, void* d_key_rope) {
-    (void)pre_tokens;
-    (void)next_tokens;
+}  // extern "C"
+
+namespace {
+
+// Shared body of sfa_grad and sfa_grad_rows: rows [row_begin, row_end) of the
+// backward, with the dK/dV contributions added into `acc` (the workspace's own
+// accumulator when `acc` is null, which is then zeroed first and cast into the
+// three key-side outputs at the end).
+sfa_status grad_impl(const void* query, const void* key, const void* value, const int32_t* sparse_indices,
+                     const void* d_out, const void* out, const float* softmax_max, const float* softmax_sum,
+                     const int32_t* actual_seq_lengths_q, const int32_t* actual_seq_lengths_kv,
+                     const void* query_rope, const void* key_rope, float scale, int64_t sparse_block_size,
+                     int64_t sparse_mode, int32_t deterministic, const sfa_shape* shape, void* workspace,
+                     size_t workspace_bytes, sfa_stream_t stream, int64_t row_begin, int64_t row_end, void* acc,
+                     void* d_query, void* d_key, void* d_value, void* d_query_rope, void* d_key_rope) {
     g_last_error.clear();
     Sizes z;
     sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
     if (st != SFA_OK) return st;
+    const bool own_acc = acc == nullptr;
     if (!query || !key || !value || !sparse_indices || !d_out || !out || !softmax_max || !softmax_sum ||
-        !query_rope || !key_rope || !d_query || !d_key || !d_value || !d_query_rope || !d_key_rope || !workspace)
+        !query_rope || !key_rope || !d_query || !d_query_rope || !workspace ||
+        (own_acc && (!d_key || !d_value || !d_key_rope)))
         return fail(SFA_ERR_NULLPTR, "a required tensor pointer is NULL");
     if (shape->layout == SFA_LAYOUT_TND && (!actual_seq_lengths_q || !actual_seq_lengths_kv))
         return fail(SFA_ERR_NULLPTR, "TND needs actual_seq_lengths_q and actual_seq_lengths_kv");
     if (!(scale == scale)) return fail(SFA_ERR_INVALID, "scale is NaN");
+    if (row_begin < 0 || row_end < row_begin || row_end > z.T1)
+        return fail(SFA_ERR_INVALID, "row range [%lld, %lld) outside [0, %lld]", (long long)row_begin,
+                    (long long)row_end, (long long)z.T1);
     if (((uintptr_t)workspace & 255u) != 0) return fail(SFA_ERR_INVALID, "workspace not 256-byte aligned");
+    if (!own_acc && ((uintptr_t)acc & 255u) != 0) return fail(SFA_ERR_INVALID, "dkv_accum not 256-byte aligned");
     const bool det = deterministic != 0;
     const bool fused_shape = fused_supported(shape->N1);
     const GradWs ws = grad_ws_layout(z.T1, z.T2, shape->N1, shape->topk, sparse_block_size, det, fused_shape);
@@ -182,17 +194,21 @@ sfa_status sfa_grad(const void* query, const void* key, const void* value, const
     a.scale = scale; a.det = det;
     a.blocks = (int32_t*)(w + ws.blocks); a.nblk = (int32_t*)(w + ws.nblk); a.nrows = (int32_t*)(w + ws.nrows);
     a.order = (int32_t*)(w + ws.order); a.rowsum = (float*)(w + ws.rowsum);
-    a.dkv_acc = w + ws.dkv; a.dq_acc = (float*)(w + ws.dq); a.ctrl = (int32_t*)(w + ws.ctrl);
+    a.dkv_acc = own_acc ? (void*)(w + ws.dkv) : acc;
+    a.dq_acc = (float*)(w + ws.dq); a.ctrl = (int32_t*)(w + ws.ctrl);
     a.dq = d_query; a.dqr = d_query_rope;
     a.dtype = shape->dtype; a.rowlist = (int32_t*)(w + ws.rowlist); a.rowcap = shape->topk * sparse_block_size;
+    a.row_begin = row_begin; a.row_end = row_end;
 
-    SFA_CUDA(cudaMemsetAsync(a.dkv_acc, 0, (size_t)z.T2 * kAccW * (det ? 8 : 4), s), "zero dK/dV accumulator");
+    if (own_acc)
+        SFA_CUDA(cudaMemsetAsync(a.dkv_acc, 0, (size_t)z.T2 * kAccW * (det ? 8 : 4), s), "zero dK/dV accumulator");
     SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, (int32_t*)a.blocks, (int32_t*)a.nblk,
                             (int32_t*)a.nrows, s), "index compaction");
     const bool fused = fused_shape && value == key;
     if (fused) {
-        SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, z.T1, shape->N1, (float*)a.rowsum, s), "rowsum(dO*O)");
-        SFA_CUDA(launch_order(a.nrows, z.T1, (int32_t*)a.order, a.ctrl, s), "work order");
+        SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, row_begin, row_end, shape->N1, (float*)a.rowsum, s),
+                 "rowsum(dO*O)");
+        SFA_CUDA(launch_order(a.nrows, row_begin, row_end, (int32_t*)a.order, a.ctrl, s), "work order");
         SFA_CUDA(launch_expand(a.blocks, a.nblk, a.sd, a.topk, a.bs, a.mode, a.rowcap, (int32_t*)a.rowlist, s),
                  "key row expansion");
         {
@@ -203,7 +219,72 @@ sfa_status sfa_grad(const void* query, const void* key, const void* value, const
         KernelEvents ev(s);
         SFA_CUDA(launch_bwd_generic(shape->dtype, a, s), "backward");
     }
-    SFA_CUDA(launch_cast_dkv(shape->dtype, det, a.dkv_acc, z.T2, d_key, d_key_rope, d_value, s), "cast dKey/dValue");
+    if (own_acc)
+        SFA_CUDA(launch_cast_dkv(shape->dtype, det, a.dkv_acc, z.T2, d_key, d_key_rope, d_value, s),
+                 "cast dKey/dValue");
+    return SFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sfa_status sfa_grad(const void* query, const void* key, const void* value, const int32_t* sparse_indices,
+                    const void* d_out, const void* out, const float* softmax_max, const float* softmax_sum,
+                    const int32_t* actual_seq_lengths_q, const int32_t* actual_seq_lengths_kv,
+                    const void* query_rope, const void* key_rope, float scale, int64_t sparse_block_size,
+                    int64_t sparse_mode, int64_t pre_tokens, int64_t next_tokens, int32_t deterministic,
+                    const sfa_shape* shape, void* workspace, size_t workspace_bytes, sfa_stream_t stream,
+                    void* d_query, void* d_key, void* d_value, void* d_query_rope, void* d_key_rope) {
+    (void)pre_tokens;
+    (void)next_tokens;
+    Sizes z;
+    g_last_error.clear();
+    sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
+    if (st != SFA_OK) return st;
+    return grad_impl(query, key, value, sparse_indices, d_out, out, softmax_max, softmax_sum, actual_seq_lengths_q,
+                     actual_seq_lengths_kv, query_rope, key_rope, scale, sparse_block_size, sparse_mode, deterministic,
+                     shape, workspace, workspace_bytes, stream, 0, z.T1, nullptr, d_query, d_key, d_value,
+                     d_query_rope, d_key_rope);
+}
+
+sfa_status sfa_dkv_accum_size(const sfa_shape* shape, int32_t deterministic, size_t* accum_bytes) {
+    g_last_error.clear();
+    if (!accum_bytes) return fail(SFA_ERR_NULLPTR, "accum_bytes is NULL");
+    Sizes z;
+    sfa_status st = check_shape(shape, 1, 0, &z);
+    if (st != SFA_OK) return st;
+    *accum_bytes = (size_t)z.T2 * kAccW * (deterministic ? 8 : 4);
+    return SFA_OK;
+}
+
+sfa_status sfa_grad_rows(const void* query, const void* key, const void* value, const int32_t* sparse_indices,
+                         const void* d_out, const void* out, const float* softmax_max, const float* softmax_sum,
+                         const int32_t* actual_seq_lengths_q, const int32_t* actual_seq_lengths_kv,
+                         const void* query_rope, const void* key_rope, float scale, int64_t sparse_block_size,
+                         int64_t sparse_mode, int32_t deterministic, int64_t row_begin, int64_t row_end,
+                         const sfa_shape* shape, void* workspace, size_t workspace_bytes, sfa_stream_t stream,
+                         void* dkv_accum, void* d_query, void* d_query_rope) {
+    if (!dkv_accum) {
+        g_last_error = "dkv_accum is NULL";
+        return SFA_ERR_NULLPTR;
+    }
+    return grad_impl(query, key, value, sparse_indices, d_out, out, softmax_max, softmax_sum, actual_seq_lengths_q,
+                     actual_seq_lengths_kv, query_rope, key_rope, scale, sparse_block_size, sparse_mode, deterministic,
+                     shape, workspace, workspace_bytes, stream, row_begin, row_end, dkv_accum, d_query, nullptr,
+                     nullptr, d_query_rope, nullptr);
+}
+
+sfa_status sfa_dkv_finalize(const void* dkv_accum, const sfa_shape* shape, int32_t deterministic, sfa_stream_t stream,
+                            void* d_key, void* d_value, void* d_key_rope) {
+    g_last_error.clear();
+    Sizes z;
+    sfa_status st = check_shape(shape, 1, 0, &z);
+    if (st != SFA_OK) return st;
+    if (!dkv_accum || !d_key || !d_value || !d_key_rope) return fail(SFA_ERR_NULLPTR, "a required pointer is NULL");
+    if (((uintptr_t)dkv_accum & 255u) != 0) return fail(SFA_ERR_INVALID, "dkv_accum not 256-byte aligned");
+    SFA_CUDA(launch_cast_dkv(shape->dtype, deterministic != 0, dkv_accum, z.T2, d_key, d_key_rope, d_value,
+                             (cudaStream_t)stream), "cast dKey/dValue");
     return SFA_OK;
 }
 
@@ -276,7 +357,7 @@ sfa_status sfa_softmax_grad_rowsum(const void* d_out, const void* out, const sfa
     sfa_status st = check_shape(shape, 1, 0, &z);
     if (st != SFA_OK) return st;
     if (!d_out || !out || !rowsum_out) return fail(SFA_ERR_NULLPTR, "a required pointer is NULL");
-    SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, z.T1, shape->N1, rowsum_out, (cudaStream_t)stream),
+    SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, 0, z.T1, shape->N1, rowsum_out, (cudaStream_t)stream),
              "rowsum(dO*O)");
     return SFA_OK;
 }

@@ -76,6 +76,7 @@ struct FusedParams {
     void* dqr_out;           // dQueryRope [T1][N1][64]
     int* err;                // device error word
     int64_t T1;
+    int64_t nwork;           // entries of `order` (query rows processed by this launch)
     int64_t cap;
     float scale;
     int det;
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
     const uint32_t T_S = tmem, T_DP = tmem + 128;
     auto T_STG = [&](int s) { return tmem + 256u + 128u * s; };
 
-    const int nwork = (int)prm.T1;
+    const int nwork = (int)prm.nwork;
     const float scale = prm.scale;
 
     if (warp == 12) {
@@ -570,6 +571,7 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
     p.dqr_out = a.dqr;
     p.err = a.ctrl;
     p.T1 = T1;
+    p.nwork = a.row_end - a.row_begin;
     p.cap = a.rowcap;
     p.scale = a.scale;
     p.det = DET ? 1 : 0;
@@ -580,7 +582,7 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int grid = (int)(T1 < sms ? T1 : sms);
+    int grid = (int)(p.nwork < sms ? p.nwork : sms);
     if (grid > kMaxFusedGrid) grid = kMaxFusedGrid;
     if (grid < 1) return cudaSuccess;
     kern<<<grid, kThreads, Cfg<N1>::kSmem, st>>>(p);

@@ -37,8 +37,9 @@ __device__ __forceinline__ void scatter_add(void* acc, int64_t off, float x) {
 template <typename T, bool DET>
 __global__ void __launch_bounds__(256) sfa_bwd_generic_kernel(GradArgs a) {
     const int lane = threadIdx.x & 31;
-    const int64_t pair = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (pair >= a.sd.T1 * a.N1) return;
+    // (row, head) pair within the processed rows [row_begin, row_end)
+    const int64_t pair = a.row_begin * a.N1 + (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (pair >= a.row_end * a.N1) return;
     const int64_t t = pair / a.N1;
     const int h = (int)(pair - t * a.N1);
     const TokInfo ti = tok_info(a.sd, t);
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(256) sfa_bwd_generic_kernel(GradArgs a) {
 }
 
 cudaError_t launch_bwd_generic(int dtype, const GradArgs& a, cudaStream_t st) {
-    const int64_t pairs = a.sd.T1 * a.N1;
+    const int64_t pairs = (a.row_end - a.row_begin) * a.N1;
     if (pairs == 0) return cudaGetLastError();
     const int warps = 8;
     unsigned grid = (unsigned)((pairs + warps - 1) / warps);

@@ -144,9 +144,12 @@ inline GradWs grad_ws_layout(int64_t T1, int64_t T2, int64_t N1, int64_t topk, i
 // ---------------------------------------------------------------------------
 cudaError_t launch_compact(const int32_t* idx, const SeqDesc& sd, int64_t topk, int bs, int mode, int32_t* blocks,
                            int32_t* nblk, int32_t* nrows, cudaStream_t st);
-cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t T1, int64_t N1, float* rowsum,
-                          cudaStream_t st);
-cudaError_t launch_order(const int32_t* nrows, int64_t T1, int32_t* order, int32_t* ctrl, cudaStream_t st);
+// rowsum(dO o O) of query rows [row_begin, row_end) (rows outside are not written)
+cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t row_begin, int64_t row_end, int64_t N1,
+                          float* rowsum, cudaStream_t st);
+// work order of the fused kernel over query rows [row_begin, row_end) (row_end - row_begin entries)
+cudaError_t launch_order(const int32_t* nrows, int64_t row_begin, int64_t row_end, int32_t* order, int32_t* ctrl,
+                         cudaStream_t st);
 cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs, int mode,
                           int64_t cap, int32_t* rowlist, cudaStream_t st);
 cudaError_t launch_cast_dkv(int dtype, bool det, const void* acc, int64_t T2, void* dk, void* dkr, void* dv,
@@ -162,6 +165,7 @@ struct GradArgs {
     const float* rowsum; void* dkv_acc; float* dq_acc; int32_t* ctrl;
     void* dq; void* dqr;
     int dtype; const int32_t* rowlist; int64_t rowcap;
+    int64_t row_begin, row_end;  // query rows [row_begin, row_end) of the flattened [T1] view are processed
 };
 cudaError_t launch_bwd_generic(int dtype, const GradArgs& a, cudaStream_t st);
 cudaError_t launch_bwd_fused(int dtype, const GradArgs& a, cudaStream_t st);

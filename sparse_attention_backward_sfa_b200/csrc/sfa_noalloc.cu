@@ -112,6 +112,7 @@ sfa_status sfa_grad_noalloc(const void* query, const void* key, const void* valu
     a.dkv_acc = w + ws.dkv; a.dq_acc = nullptr; a.ctrl = (int32_t*)(w + ws.ctrl);
     a.dq = d_query; a.dqr = d_query_rope;
     a.dtype = shape->dtype; a.rowlist = nullptr; a.rowcap = 0;
+    a.row_begin = 0; a.row_end = T1;
 
     cudaError_t e;
     // the accumulator must start at zero; the rest of the scratch is fully rewritten

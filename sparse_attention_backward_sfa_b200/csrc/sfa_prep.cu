@@ -74,9 +74,14 @@ __global__ void rowsum_kernel(const T* __restrict__ dout, const T* __restrict__ 
     if (lane == 0) res[r] = s;
 }
 
-cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t T1, int64_t N1, float* rowsum,
-                          cudaStream_t st) {
-    int64_t rows = T1 * N1;
+cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t row_begin, int64_t row_end, int64_t N1,
+                          float* rowsum, cudaStream_t st) {
+    const int64_t rows = (row_end - row_begin) * N1;
+    const int64_t first = row_begin * N1;  // (row, head) pairs before the range
+    const size_t elem = 2;                  // bf16 / fp16
+    dout = (const char*)dout + first * kD * elem;
+    out = (const char*)out + first * kD * elem;
+    rowsum += first;
     const int warps = 8;
     unsigned grid = (unsigned)((rows + warps - 1) / warps);
     if (rows == 0) return cudaGetLastError();
@@ -90,16 +95,19 @@ cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t 
 
 // Work order for the persistent fused kernel: later rows first (under the causal
 // masks they carry the most keys, so the largest work items start first).
-__global__ void order_kernel(int64_t T1, int32_t* __restrict__ order, int32_t* __restrict__ ctrl) {
+__global__ void order_kernel(int64_t row_begin, int64_t row_end, int32_t* __restrict__ order,
+                             int32_t* __restrict__ ctrl) {
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < T1) order[i] = (int32_t)(T1 - 1 - i);
+    if (i < row_end - row_begin) order[i] = (int32_t)(row_end - 1 - i);
     if (i < 64) ctrl[i] = 0;
 }
 
-cudaError_t launch_order(const int32_t* nrows, int64_t T1, int32_t* order, int32_t* ctrl, cudaStream_t st) {
+cudaError_t launch_order(const int32_t* nrows, int64_t row_begin, int64_t row_end, int32_t* order, int32_t* ctrl,
+                         cudaStream_t st) {
     (void)nrows;
-    int64_t n = T1 > 64 ? T1 : 64;
-    order_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(T1, order, ctrl);
+    const int64_t cnt = row_end - row_begin;
+    int64_t n = cnt > 64 ? cnt : 64;
+    order_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(row_begin, row_end, order, ctrl);
     return cudaGetLastError();
 }
 

@@ -108,6 +108,68 @@ def sfa_grad(query, key, value, sparse_indices, d_out, out, softmax_max, softmax
     return dq, dk, dv, dqr, dkr
 
 
+def sfa_dkv_accumulator(query, key, query_rope, sparse_indices, *, layout: str, deterministic: bool,
+                        actual_seq_lengths_q=None):
+    """Zeroed key-side accumulator for sfa_grad_rows: [T2, 1088] (dKey | dKeyRope | dValue), fp32,
+    or int64 fixed point (value * 2^32) when deterministic."""
+    lib = N.load()
+    shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    n = ctypes.c_size_t()
+    N.check(lib.sfa_dkv_accum_size(ctypes.byref(shape), int(deterministic), ctypes.byref(n)))
+    dt = torch.int64 if deterministic else torch.float32
+    return torch.zeros(shape.T2, n.value // (shape.T2 * (8 if deterministic else 4)), dtype=dt, device=query.device)
+
+
+def sfa_grad_rows(query, key, value, sparse_indices, d_out, out, softmax_max, softmax_sum, query_rope, key_rope, *,
+                  row_begin: int, row_end: int, dkv_accum: torch.Tensor, scale: float, sparse_block_size: int,
+                  layout: str, sparse_mode: int, deterministic: bool = False, actual_seq_lengths_q=None,
+                  actual_seq_lengths_kv=None, workspace: Optional[torch.Tensor] = None, d_query=None,
+                  d_query_rope=None, stream=None):
+    """Backward of query rows [row_begin, row_end) (flattened row index): writes those rows of
+    (dQuery, dQueryRope) and adds their dKey / dKeyRope / dValue contributions into `dkv_accum`
+    (from sfa_dkv_accumulator). Returns (dQuery, dQueryRope)."""
+    lib = N.load()
+    dt = query.dtype
+    for name, t in (("query", query), ("key", key), ("value", value), ("d_out", d_out), ("out", out),
+                    ("query_rope", query_rope), ("key_rope", key_rope)):
+        _check16(name, t, dt)
+    _need(sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(), "sparse_indices: int32 contiguous")
+    _need(softmax_max.dtype == torch.float32 and softmax_sum.dtype == torch.float32, "softmax stats must be fp32")
+    _need(dkv_accum.is_contiguous() and dkv_accum.dtype == (torch.int64 if deterministic else torch.float32),
+          "dkv_accum: contiguous, int64 when deterministic else float32")
+    shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
+    skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
+    ws_bytes = sfa_grad_workspace_size(shape, sparse_block_size, sparse_mode, deterministic)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=query.device)
+    if d_query is None:
+        d_query = torch.zeros_like(query)
+    if d_query_rope is None:
+        d_query_rope = torch.zeros_like(query_rope)
+    N.check(lib.sfa_grad_rows(_p(query), _p(key), _p(value), _p(sparse_indices), _p(d_out), _p(out),
+                              _p(softmax_max), _p(softmax_sum), _p(sq), _p(skv), _p(query_rope), _p(key_rope),
+                              float(scale), int(sparse_block_size), int(sparse_mode), int(deterministic),
+                              int(row_begin), int(row_end), ctypes.byref(shape), _p(workspace), workspace.numel(),
+                              _stream(stream), _p(dkv_accum), _p(d_query), _p(d_query_rope)))
+    return d_query, d_query_rope
+
+
+def sfa_dkv_finalize(dkv_accum, query, key, query_rope, sparse_indices, *, layout: str, deterministic: bool,
+                     actual_seq_lengths_q=None, outputs=None, stream=None):
+    """Casts a (summed) key-side accumulator into 16-bit (dKey, dValue, dKeyRope)."""
+    lib = N.load()
+    shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    if outputs is None:
+        kr_shape = key.shape[:-1] + (query_rope.shape[-1],)
+        outputs = (torch.empty_like(key), torch.empty_like(key),
+                   torch.empty(kr_shape, dtype=key.dtype, device=key.device))
+    dk, dv, dkr = outputs
+    N.check(lib.sfa_dkv_finalize(_p(dkv_accum), ctypes.byref(shape), int(deterministic), _stream(stream), _p(dk),
+                                 _p(dv), _p(dkr)))
+    return dk, dv, dkr
+
+
 def sfa_fwd(query, key, value, sparse_indices, query_rope, key_rope, *, scale: float, sparse_block_size: int,
             layout: str, sparse_mode: int, actual_seq_lengths_q=None, actual_seq_lengths_kv=None, stream=None):
     """Forward of top-k sparse attention; returns (out, softmaxMax, softmaxSum)."""

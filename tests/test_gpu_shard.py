@@ -1,0 +1,114 @@
+"""GPU checks of the query-row sharded backward (sfa_grad_rows + sfa_dkv_finalize):
+the key-side accumulators of disjoint row ranges add up to sfa_grad's result —
+bit-identical in deterministic mode (64-bit fixed point) — and the dQuery rows of
+each range are the ones sfa_grad writes.  The ranges run one after another on one
+GPU; several GPUs would sum the same accumulators with an all-reduce."""
+import numpy as np
+import pytest
+import torch
+
+from workloads import tiny_problem
+from parity import DevProblem, compare_grads, grads_np, oracle_backward, prepare_oracle_forward
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_attention_backward_sfa_b200 import build
+    build.build()
+
+
+CASES = {
+    # CUDA-core path (N1 < 64)
+    "generic_n2_bsnd": dict(layout="BSND", B=2, S1=7, S2=90, N1=2, topk=30, block_size=1, sparse_mode=3,
+                            index_mode="causal"),
+    # fused tensor-core path, several tiles per row, block indices
+    "fused_n128_tnd_bs16": dict(layout="TND", seqlens_q=[70, 3, 150], seqlens_kv=[70, 260, 150], N1=128, topk=12,
+                                block_size=16, sparse_mode=3, index_mode="causal"),
+    "fused_n64_bsnd": dict(layout="BSND", B=1, S1=11, S2=400, N1=64, topk=300, block_size=1, sparse_mode=0),
+}
+
+
+def sharded(dp, ranges, det, separate=False):
+    """sfa_grad_rows over `ranges`; one shared accumulator, or one per range summed afterwards."""
+    import sparse_attention_backward_sfa_b200 as S
+    kw = dp.kw()
+    mk = lambda: S.sfa_dkv_accumulator(dp.q, dp.k, dp.qr, dp.idx, layout=kw["layout"], deterministic=det,
+                                       actual_seq_lengths_q=dp.sq)
+    acc = mk()
+    accs = []
+    dq = torch.zeros_like(dp.q)
+    dqr = torch.zeros_like(dp.qr)
+    for rb, re_ in ranges:
+        a = mk() if separate else acc
+        S.sfa_grad_rows(dp.q, dp.k, dp.v, dp.idx, dp.do, dp.out, dp.smax, dp.ssum, dp.qr, dp.kr, row_begin=rb,
+                        row_end=re_, dkv_accum=a, deterministic=det, d_query=dq, d_query_rope=dqr, **kw)
+        accs.append(a)
+    if separate:
+        acc = torch.stack(accs).sum(0)  # what an all-reduce of the ranks' accumulators computes
+    dk, dv, dkr = S.sfa_dkv_finalize(acc, dp.q, dp.k, dp.qr, dp.idx, layout=kw["layout"], deterministic=det,
+                                     actual_seq_lengths_q=dp.sq)
+    return dq, dk, dv, dqr, dkr
+
+
+def three_ranges(T1):
+    a, b = T1 // 3, (2 * T1) // 3 + 1
+    return [(0, a), (a, b), (b, T1)]
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_sharded_deterministic_is_bit_identical(case):
+    p = tiny_problem(311, D=512, Dr=64, **CASES[case])
+    dp = DevProblem(p)
+    prepare_oracle_forward(p, dp)
+    full = dp.grad_gpu(deterministic=True)
+    for separate in (False, True):
+        got = sharded(dp, three_ranges(p.T1), True, separate=separate)
+        for name, g, f in zip(("dQuery", "dKey", "dValue", "dQueryRope", "dKeyRope"), got, full):
+            assert torch.equal(g, f), f"{case}: {name} differs from sfa_grad (separate={separate})"
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_sharded_atomic_matches_oracle(case):
+    p = tiny_problem(313, D=512, Dr=64, **CASES[case])
+    dp = DevProblem(p)
+    out, m, l = prepare_oracle_forward(p, dp)
+    got = grads_np(sharded(dp, three_ranges(p.T1), False, separate=True), p)
+    compare_grads(got, oracle_backward(p, out, m, l), what=f"sharded {case}/")
+
+
+def test_rows_outside_range_untouched_and_range_checked():
+    import sparse_attention_backward_sfa_b200 as S
+    p = tiny_problem(317, D=512, Dr=64, **CASES["fused_n64_bsnd"])
+    dp = DevProblem(p)
+    prepare_oracle_forward(p, dp)
+    kw = dp.kw()
+    acc = S.sfa_dkv_accumulator(dp.q, dp.k, dp.qr, dp.idx, layout=kw["layout"], deterministic=False)
+    dq = torch.full_like(dp.q, 7.0)
+    dqr = torch.full_like(dp.qr, 7.0)
+    S.sfa_grad_rows(dp.q, dp.k, dp.v, dp.idx, dp.do, dp.out, dp.smax, dp.ssum, dp.qr, dp.kr, row_begin=3, row_end=5,
+                    dkv_accum=acc, d_query=dq, d_query_rope=dqr, **kw)
+    flat = dq.reshape(p.T1, -1)
+    assert bool((flat[:3] == 7).all()) and bool((flat[5:] == 7).all())
+    assert not bool((flat[3:5] == 7).all())
+    with pytest.raises(S.SfaError):
+        S.sfa_grad_rows(dp.q, dp.k, dp.v, dp.idx, dp.do, dp.out, dp.smax, dp.ssum, dp.qr, dp.kr, row_begin=2,
+                        row_end=p.T1 + 1, dkv_accum=acc, d_query=dq, d_query_rope=dqr, **kw)
+
+
+def test_balanced_split_of_real_counts():
+    """The bench's work split on a causal problem: contiguous, covering, and balanced within one row."""
+    import sparse_attention_backward_sfa_b200 as S
+    p = tiny_problem(319, D=512, Dr=64, **CASES["fused_n128_tnd_bs16"])
+    dp = DevProblem(p)
+    _, _, nr = S.compact_indices(dp.idx, dp.k, dp.q, dp.qr, sparse_block_size=p.block_size, layout=p.layout,
+                                 sparse_mode=p.sparse_mode, actual_seq_lengths_q=dp.sq, actual_seq_lengths_kv=dp.skv)
+    w = nr.cpu().numpy().astype(np.float64)
+    for parts in (2, 3, 8):
+        r = S.balanced_row_ranges(w, parts)
+        assert r[0][0] == 0 and r[-1][1] == p.T1 and all(r[i][1] == r[i + 1][0] for i in range(parts - 1))
+        sums = [w[a:b].sum() for a, b in r]
+        assert max(sums) - w.sum() / parts <= w.max() + 1e-9
