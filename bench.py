@@ -290,6 +290,60 @@ def run_ours(args, rank, world, local_rank):
                 rows=(rb, re_))
 
 
+def run_fwd(args, local_rank):
+    """The forward of a sparse workload (sfa_fwd), one GPU: 2176 FLOP per valid
+    (row, head, key) triple (S = Q~.K~^T over 576 dims, out = P.V over 512)."""
+    import torch
+    import sparse_attention_backward_sfa_b200 as S
+    from sparse_attention_backward_sfa_b200 import _native as N
+    from workloads import WORKLOADS
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lib = N.load()
+    p = build_problem(args.workload, 0, dev)
+    _, _, nr = S.compact_indices(p.indices, p.k, p.q, p.q_rope, sparse_block_size=p.block_size, layout=p.layout,
+                                 sparse_mode=p.sparse_mode, actual_seq_lengths_q=p.seqlens_q,
+                                 actual_seq_lengths_kv=p.seqlens_kv)
+    triples = int(nr.to(torch.int64).sum().item()) * p.N1
+    flop = triples * 2176
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            N.check(lib.sfa_set_kernel_events(ctypes_ptr(ev[0]), ctypes_ptr(ev[1])))
+        S.sfa_fwd(p.q, p.k, p.k, p.indices, p.q_rope, p.k_rope, **kw(p))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        a.record(stream)
+        b.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms_step = t0.elapsed_time(t1) / args.steps
+    kern = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    return {"metric": "sparse-attn forward TFLOP/s (bf16, S + P.V count, 2176 FLOP per triple)",
+            "value": flop / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload], "N1": p.N1, "valid_triples": triples,
+                       "path": "tcgen05 (N1 = 128)" if p.N1 == 128 else "CUDA-core"},
+            "roofline": {"bound": "tensor", "achieved": flop / (kern * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                         "frac": flop / (kern * 1e-3) / 1e12 / peak, "kernel_ms": kern, "traffic": None},
+            "gpu_launches": (4 if p.N1 == 128 else 2) * args.steps, "clocks": clk.summary()}
+
+
 def run_fa(args, rank, world, local_rank):
     """Workload 2: dense varlen FA backward (TND, causal); 1280 FLOP per valid
     (query row, head, key) triple."""
@@ -405,6 +459,8 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fwd", action="store_true",
+                    help="time the forward (sfa_fwd: out + softmax statistics) instead of the backward")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqs", default=None,
                     help="comma-separated sequence lengths replacing workload 4's (smaller profiling case)")
@@ -448,6 +504,11 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    if args.fwd:
+        if world > 1 or args.workload == 2:
+            raise SystemExit("--fwd: one GPU, sparse workloads (3, 4, 5)")
+        print(json.dumps(run_fwd(args, local_rank)), flush=True)
+        return
     r = run_fa(args, rank, world, local_rank) if args.workload == 2 else run_ours(args, rank, world, local_rank)
     peaks, src = load_peaks()
     sharded = bool(r.get("sharded"))

@@ -308,10 +308,10 @@ sfa_status fa_fwd(const void *q, const void *k, const void *v, const int64_t *ac
 /* ------------------------------------------------------------------------- */
 
 /*
- * Timing hook for benchmarks: the next sfa_grad / fa_grad call on the calling
- * thread records `event_before` immediately before and `event_after`
- * immediately after launching its main backward kernel (the fused tensor-core
- * kernel or the CUDA-core kernel), on that call's stream.  Both are cudaEvent_t
+ * Timing hook for benchmarks: the next sfa_grad / sfa_grad_rows / sfa_fwd /
+ * fa_grad call on the calling thread records `event_before` immediately before
+ * and `event_after` immediately after launching its main kernel (the fused
+ * tensor-core kernel or the CUDA-core kernel), on that call's stream.  Both are cudaEvent_t
  * handles created by the caller; NULL clears the hook.  Consumed by one call.
  */
 sfa_status sfa_set_kernel_events(void *event_before, void *event_after);

@@ -295,7 +295,7 @@ sfa_status sfa_fwd_workspace_size(const sfa_shape* shape, int64_t sparse_block_s
     Sizes z;
     sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
     if (st != SFA_OK) return st;
-    *workspace_bytes = align256((size_t)z.T1 * shape->topk * 4) + 2 * align256((size_t)z.T1 * 4);
+    *workspace_bytes = fwd_ws_layout(z.T1, shape->N1, shape->topk, sparse_block_size).total;
     return SFA_OK;
 }
 
@@ -313,8 +313,10 @@ sfa_status sfa_fwd(const void* query, const void* key, const void* value, const 
         return fail(SFA_ERR_NULLPTR, "a required tensor pointer is NULL");
     if (shape->layout == SFA_LAYOUT_TND && (!actual_seq_lengths_q || !actual_seq_lengths_kv))
         return fail(SFA_ERR_NULLPTR, "TND needs actual_seq_lengths_q and actual_seq_lengths_kv");
-    size_t need = align256((size_t)z.T1 * shape->topk * 4) + 2 * align256((size_t)z.T1 * 4);
-    if (workspace_bytes < need) return fail(SFA_ERR_WORKSPACE, "workspace %zu < %zu", workspace_bytes, need);
+    const FwdWs ws = fwd_ws_layout(z.T1, shape->N1, shape->topk, sparse_block_size);
+    if (workspace_bytes < ws.total)
+        return fail(SFA_ERR_WORKSPACE, "workspace %zu < %zu", workspace_bytes, ws.total);
+    if (((uintptr_t)workspace & 255u) != 0) return fail(SFA_ERR_INVALID, "workspace not 256-byte aligned");
     cudaStream_t s = (cudaStream_t)stream;
     char* w = (char*)workspace;
     FwdArgs a;
@@ -322,13 +324,37 @@ sfa_status sfa_fwd(const void* query, const void* key, const void* value, const 
     a.sd = seq_desc(shape, z, actual_seq_lengths_q, actual_seq_lengths_kv);
     a.N1 = shape->N1; a.topk = shape->topk; a.bs = (int)sparse_block_size; a.mode = (int)sparse_mode;
     a.scale = scale;
-    int32_t* blocks = (int32_t*)w;
-    int32_t* nblk = (int32_t*)(w + align256((size_t)z.T1 * shape->topk * 4));
-    int32_t* nrows = (int32_t*)((char*)nblk + align256((size_t)z.T1 * 4));
+    int32_t* blocks = (int32_t*)(w + ws.blocks);
+    int32_t* nblk = (int32_t*)(w + ws.nblk);
+    int32_t* nrows = (int32_t*)(w + ws.nrows);
     a.blocks = blocks; a.nblk = nblk;
     a.out = out; a.smax = softmax_max; a.ssum = softmax_sum;
     SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, blocks, nblk, nrows, s), "index compaction");
-    SFA_CUDA(launch_fwd_generic(shape->dtype, a, s), "forward");
+    if (ws.rowlist && value == key) {
+        // tensor-core path: expanded key-row lists, longest rows first
+        FwdFusedArgs f;
+        f.q = query; f.qr = query_rope; f.k = key; f.kr = key_rope;
+        f.rowlist = (int32_t*)(w + ws.rowlist); f.nrows = nrows; f.order = (int32_t*)(w + ws.order);
+        f.out = out; f.smax = softmax_max; f.ssum = softmax_sum; f.err = (int*)(w + ws.ctrl);
+        f.T1 = z.T1; f.T2 = z.T2; f.rowcap = shape->topk * sparse_block_size; f.scale = scale; f.dtype = shape->dtype;
+        SFA_CUDA(launch_order(nrows, 0, z.T1, (int32_t*)f.order, (int32_t*)(w + ws.ctrl), s), "work order");
+        f.blk16 = a.bs % 16 == 0 ? 1 : 0;
+        if (f.blk16) {  // runs of 16 contiguous key rows: 16-row 2-D tile loads instead of row gathers
+            f.nrows = (int32_t*)(w + ws.nslots);
+            SFA_CUDA(launch_expand_blocks(blocks, nblk, a.sd, a.topk, a.bs, a.mode, f.rowcap, (int32_t*)f.rowlist,
+                                          (int32_t*)f.nrows, s), "key row expansion");
+        } else {
+            SFA_CUDA(launch_expand(blocks, nblk, a.sd, a.topk, a.bs, a.mode, f.rowcap, (int32_t*)f.rowlist, s),
+                     "key row expansion");
+        }
+        KernelEvents ev(s);
+        SFA_CUDA(launch_fwd_fused(shape->dtype, f, s), "fused forward");
+        return SFA_OK;
+    }
+    {
+        KernelEvents ev(s);
+        SFA_CUDA(launch_fwd_generic(shape->dtype, a, s), "forward");
+    }
     return SFA_OK;
 }
 

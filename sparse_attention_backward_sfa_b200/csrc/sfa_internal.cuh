@@ -139,6 +139,26 @@ inline GradWs grad_ws_layout(int64_t T1, int64_t T2, int64_t N1, int64_t topk, i
     return w;
 }
 
+// Workspace layout of sfa_fwd (the expanded row lists, order and control word only
+// on the tensor-core path, N1 = 128)
+struct FwdWs {
+    size_t blocks, nblk, nrows, order, rowlist, nslots, ctrl, total;
+};
+inline FwdWs fwd_ws_layout(int64_t T1, int64_t N1, int64_t topk, int64_t bs) {
+    FwdWs w;
+    const bool fused = N1 == 128;
+    size_t o = 0;
+    w.blocks = o;  o = align256(o + (size_t)T1 * topk * 4);
+    w.nblk = o;    o = align256(o + (size_t)T1 * 4);
+    w.nrows = o;   o = align256(o + (size_t)T1 * 4);
+    w.order = o;   o = align256(o + (fused ? (size_t)T1 * 4 : 0));
+    w.rowlist = fused ? o : 0; o = align256(o + (fused ? (size_t)T1 * topk * bs * 4 : 0));
+    w.nslots = o;  o = align256(o + (fused ? (size_t)T1 * 4 : 0));
+    w.ctrl = o;    o = align256(o + 256);
+    w.total = o;
+    return w;
+}
+
 // ---------------------------------------------------------------------------
 // Launchers (defined in the .cu files; all return cudaGetLastError())
 // ---------------------------------------------------------------------------
@@ -152,6 +172,9 @@ cudaError_t launch_order(const int32_t* nrows, int64_t row_begin, int64_t row_en
                          cudaStream_t st);
 cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs, int mode,
                           int64_t cap, int32_t* rowlist, cudaStream_t st);
+// block-aligned key-row lists for sparse_block_size % 16 == 0 (invalid slots: bit 31 set)
+cudaError_t launch_expand_blocks(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs,
+                                 int mode, int64_t cap, int32_t* rowlist, int32_t* nslots, cudaStream_t st);
 cudaError_t launch_cast_dkv(int dtype, bool det, const void* acc, int64_t T2, void* dk, void* dkr, void* dv,
                             cudaStream_t st);
 cudaError_t launch_cast_dq(int dtype, const float* acc, int64_t T1, int64_t N1, void* dq, void* dqr,
@@ -178,6 +201,17 @@ struct FwdArgs {
     void* out; float* smax; float* ssum;
 };
 cudaError_t launch_fwd_generic(int dtype, const FwdArgs& a, cudaStream_t st);
+
+// Tensor-core forward (N1 = 128, value == key) over the expanded key-row lists.
+struct FwdFusedArgs {
+    const void* q; const void* qr; const void* k; const void* kr;
+    const int32_t* rowlist; const int32_t* nrows; const int32_t* order;
+    void* out; float* smax; float* ssum; int* err;
+    int64_t T1, T2, rowcap; float scale; int dtype;
+    int blk16;  // row lists are block-aligned runs of 16 contiguous rows (nrows = slots; invalid slots: bit 31)
+};
+bool fwd_fused_supported(int64_t N1);
+cudaError_t launch_fwd_fused(int dtype, const FwdFusedArgs& a, cudaStream_t st);
 
 struct FaArgs {
     const void* q; const void* k; const void* v; const void* dy; const void* o;

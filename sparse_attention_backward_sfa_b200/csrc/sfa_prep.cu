@@ -139,6 +139,40 @@ __global__ void expand_kernel(const int32_t* __restrict__ blocks, const int32_t*
     }
 }
 
+// Block-aligned expansion (sparse_block_size a multiple of 16): block i of row t
+// takes slots [i*bs, i*bs+bs) with the block's consecutive rows, so every
+// 16-slot group is one run of contiguous key rows (loadable as one 2-D tile);
+// slots past the block's kept rows (sequence end, causal bound) hold the row id
+// with bit 31 set.  nslots[t] = blocks x bs.
+__global__ void expand_blocks_kernel(const int32_t* __restrict__ blocks, const int32_t* __restrict__ nblk, SeqDesc sd,
+                                     int64_t topk, int bs, int mode, int64_t cap, int32_t* __restrict__ rowlist,
+                                     int32_t* __restrict__ nslots) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= sd.T1) return;
+    const TokInfo ti = tok_info(sd, t);
+    const int nb = nblk[t];
+    int32_t* dst = rowlist + t * cap;
+    for (int i = 0; i < nb; ++i) {
+        const int64_t blk = blocks[t * topk + i];
+        const int keep = block_rows(blk, bs, ti, mode);
+        const int64_t first = ti.kv_start + blk * bs;
+        for (int o = lane; o < bs; o += 32)
+            dst[(int64_t)i * bs + o] = (int32_t)((uint32_t)(first + o) | (o < keep ? 0u : 0x80000000u));
+    }
+    if (lane == 0) nslots[t] = (int32_t)(nb * bs);
+}
+
+cudaError_t launch_expand_blocks(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs,
+                                 int mode, int64_t cap, int32_t* rowlist, int32_t* nslots, cudaStream_t st) {
+    const int warps = 8;
+    const int64_t grid = (sd.T1 + warps - 1) / warps;
+    if (grid > 0)
+        expand_blocks_kernel<<<(unsigned)grid, warps * 32, 0, st>>>(blocks, nblk, sd, topk, bs, mode, cap, rowlist,
+                                                                    nslots);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs, int mode,
                           int64_t cap, int32_t* rowlist, cudaStream_t st) {
     const int warps = 8;

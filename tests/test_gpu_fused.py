@@ -35,6 +35,12 @@ FUSED = {
     "n64_tnd_messy_bs5": dict(layout="TND", seqlens_q=[9, 12], seqlens_kv=[333, 90], N1=64, topk=40, block_size=5,
                               sparse_mode=0, index_mode="messy"),
     "n128_exact_tile": dict(layout="BSND", B=1, S1=3, S2=256, N1=128, topk=128, block_size=1, sparse_mode=0),
+    # block-aligned row lists (block size a multiple of 16): 16-row tile loads, padding slots inside
+    # the lists (blocks cut by the sequence end or the causal bound, duplicates, -1, blocks past S2)
+    "n128_bsnd_bs16_messy": dict(layout="BSND", B=2, S1=5, S2=300, N1=128, topk=20, block_size=16, sparse_mode=3,
+                                 index_mode="messy", seqlens_q=[5, 4], seqlens_kv=[300, 37]),
+    "n64_tnd_bs32_causal": dict(layout="TND", seqlens_q=[40, 9], seqlens_kv=[200, 70], N1=64, topk=8, block_size=32,
+                                sparse_mode=3, index_mode="causal"),
 }
 
 
@@ -81,3 +87,45 @@ def test_fused_matches_generic_path():
     dp.v = dp.k.clone()
     generic = grads_np(dp.grad_gpu(), p)
     compare_grads(fused, generic, what="fused-vs-generic/")
+
+
+FWD = {
+    "n128_bsnd_mode0_3tiles": FUSED["n128_bsnd_mode0_bs1_3tiles"],
+    "n128_tnd_bs16_causal": FUSED["n128_tnd_bs16_causal"],
+    "n128_exact_tile": FUSED["n128_exact_tile"],
+    # empty rows (BSND padding positions, all-invalid index lists) and a short ragged tile
+    "n128_bsnd_messy_varlen": dict(layout="BSND", B=2, S1=6, S2=150, N1=128, topk=40, block_size=3, sparse_mode=3,
+                                   index_mode="messy", seqlens_q=[6, 2], seqlens_kv=[150, 9]),
+    # block-aligned row lists (16-row tile loads) with padding slots inside the lists
+    "n128_bsnd_bs16_messy": FUSED["n128_bsnd_bs16_messy"],
+    "n128_tnd_bs32_causal": dict(layout="TND", seqlens_q=[40, 9], seqlens_kv=[200, 70], N1=128, topk=8, block_size=32,
+                                 sparse_mode=3, index_mode="causal"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(FWD))
+def test_fused_fwd_parity(case):
+    """Tensor-core forward (N1 = 128, value == key): out, softmaxMax, softmaxSum against the oracle."""
+    from parity import assert_close, oracle_forward
+    p = tiny(107, **FWD[case])
+    dp = DevProblem(p)
+    dp.forward_gpu()
+    ro, rm, rl = oracle_forward(p)
+    go, gm, gl = dp.host_fwd_inputs()
+    assert_close("out", go, ro)
+    np.testing.assert_allclose(gm, rm, rtol=2e-5, atol=2e-5)
+    np.testing.assert_allclose(gl, rl, rtol=2e-5, atol=1e-6)
+
+
+def test_fused_fwd_fp16():
+    from parity import assert_close, oracle_forward
+    p = tiny(109, **FWD["n128_tnd_bs16_causal"])
+    for a in (p.q, p.q_rope, p.k, p.k_rope):
+        a[...] = a.astype(np.float16).astype(np.float32)
+    dp = DevProblem(p, dtype=torch.float16)
+    dp.forward_gpu()
+    ro, rm, rl = oracle_forward(p)
+    go, gm, gl = dp.host_fwd_inputs()
+    assert_close("out", go, ro)
+    np.testing.assert_allclose(gm, rm, rtol=2e-5, atol=2e-5)
+    np.testing.assert_allclose(gl, rl, rtol=2e-5, atol=1e-6)
