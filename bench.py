@@ -45,6 +45,7 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 PROFILE_SUMMARIES = {
     4: ("sfa_bwd_fused_kernel_workload4.md", ("sfa_fused.cu", "tc_common.cuh")),
     2: ("fa_bwd_fused_kernel_workload2.md", ("fa_fused.cu", "tc_common.cuh")),
+    "fwd4": ("sfa_fwd_fused_kernel_workload4.md", ("sfa_fwd_fused.cu", "tc_common.cuh")),
 }
 
 
@@ -340,7 +341,8 @@ def run_fwd(args, local_rank):
             "config": {"workload": WORKLOADS[args.workload], "N1": p.N1, "valid_triples": triples,
                        "path": "tcgen05 (N1 = 128)" if p.N1 == 128 else "CUDA-core"},
             "roofline": {"bound": "tensor", "achieved": flop / (kern * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
-                         "frac": flop / (kern * 1e-3) / 1e12 / peak, "kernel_ms": kern, "traffic": None},
+                         "frac": flop / (kern * 1e-3) / 1e12 / peak, "kernel_ms": kern,
+                         "traffic": recorded_traffic("fwd4") if args.workload == 4 and not args.seqs else None},
             "gpu_launches": (4 if p.N1 == 128 else 2) * args.steps, "clocks": clk.summary()}
 
 
