@@ -267,6 +267,27 @@ def run_ours(args, rank, world, local_rank):
             for h, o2 in zip(host_out, (rows(dq), rows(dqr), dk, dv, dkr)):
                 h.copy_(o2, non_blocking=True)
 
+        if not sharded:
+            # one GPU: the library's pipelined host API (chunked rows, copies overlapped with the kernels)
+            pl = S.HostPipeline(dev)
+            host_all = {n: x.cpu().pin_memory() for n, x in (("q", p.q), ("qr", p.q_rope), ("k", p.k),
+                                                             ("kr", p.k_rope), ("do", p.dout), ("o", out),
+                                                             ("mx", smax), ("sm", ssum), ("idx", p.indices))}
+            host_sq = p.seqlens_q.cpu().pin_memory() if p.seqlens_q is not None else None
+            host_res = tuple(torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+                             for x in (p.q, p.k, p.k, p.q_rope, p.k_rope))
+            h2d = sum(x.numel() * x.element_size() for x in host_all.values()) + \
+                (host_sq.numel() * host_sq.element_size() if host_sq is not None else 0)
+            d2h = sum(x.numel() * x.element_size() for x in host_res)
+
+            def e2e_step():
+                h = host_all
+                S.sfa_grad_host(h["q"], h["k"], True, h["idx"], h["do"], h["o"], h["mx"], h["sm"], h["qr"], h["kr"],
+                                scale=p.scale, sparse_block_size=p.block_size, layout=p.layout,
+                                sparse_mode=p.sparse_mode, deterministic=p.deterministic,
+                                actual_seq_lengths_q=host_sq, actual_seq_lengths_kv=host_sq, outputs=host_res,
+                                pipeline=pl, device=dev)
+
         e2e_step()
         torch.cuda.synchronize(dev)
         n_e2e = max(2, min(args.steps, 5))

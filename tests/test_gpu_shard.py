@@ -112,3 +112,23 @@ def test_balanced_split_of_real_counts():
         assert r[0][0] == 0 and r[-1][1] == p.T1 and all(r[i][1] == r[i + 1][0] for i in range(parts - 1))
         sums = [w[a:b].sum() for a, b in r]
         assert max(sums) - w.sum() / parts <= w.max() + 1e-9
+
+
+@pytest.mark.parametrize("case", ["generic_n2_bsnd", "fused_n128_tnd_bs16"])
+def test_host_pipeline_matches_sfa_grad(case):
+    """sfa_grad_host (pinned host tensors, chunked rows, copies overlapped) gives sfa_grad's
+    results: bit-identical in deterministic mode."""
+    import sparse_attention_backward_sfa_b200 as S
+    p = tiny_problem(331, D=512, Dr=64, **CASES[case])
+    dp = DevProblem(p)
+    prepare_oracle_forward(p, dp)
+    full = dp.grad_gpu(deterministic=True)
+    h = lambda x: None if x is None else x.cpu().pin_memory()
+    pl = S.HostPipeline(torch.device("cuda"))
+    for chunks in (1, 3):
+        got = S.sfa_grad_host(h(dp.q), h(dp.k), True, h(dp.idx), h(dp.do), h(dp.out), h(dp.smax), h(dp.ssum),
+                              h(dp.qr), h(dp.kr), scale=p.scale, sparse_block_size=p.block_size, layout=p.layout,
+                              sparse_mode=p.sparse_mode, deterministic=True, actual_seq_lengths_q=h(dp.sq),
+                              actual_seq_lengths_kv=h(dp.skv), chunks=chunks, pipeline=pl)
+        for name, g, f in zip(("dQuery", "dKey", "dValue", "dQueryRope", "dKeyRope"), got, full):
+            assert torch.equal(g, f.cpu()), f"{case}: {name} differs (chunks={chunks})"
