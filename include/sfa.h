@@ -316,6 +316,28 @@ sfa_status fa_fwd(const void *q, const void *k, const void *v, const int64_t *ac
  */
 sfa_status sfa_set_kernel_events(void *event_before, void *event_after);
 
+/*
+ * Failure detection.  Every wait of the fused kernels on an mbarrier (a load, an
+ * MMA or another warp role) is bounded: past the limit the kernel writes a
+ * non-zero wait-site code into its workspace's error word (the first 4 bytes of
+ * the workspace of sfa_grad / sfa_grad_rows / sfa_fwd / fa_grad / fa_fwd, zeroed
+ * at the start of each such call), stops issuing work, drains what it issued,
+ * frees its tensor memory and exits; the CUDA context stays usable.  (The pages
+ * name only an AI Core "timeout or trap" error for oversized problems, 约束说明 of
+ * aclnnFlashAttentionUnpaddingScoreGrad.)
+ *
+ * sfa_workspace_status - synchronizes `stream`, reads the error word of
+ * `workspace` (device pointer) and returns SFA_OK, or SFA_ERR_TIMEOUT with the
+ * wait-site code in *site_out (may be NULL) when the last call on it gave up.
+ *
+ * sfa_set_wait_limit - limit in nanoseconds of every such wait in fused kernels
+ * launched afterwards from the calling thread; 0 restores the default (4 s).
+ * A tiny limit (the tests use 1 ns) makes a launch give up at its first wait that is
+ * not already satisfied, which exercises the path above without any fault.
+ */
+sfa_status sfa_workspace_status(const void *workspace, sfa_stream_t stream, int32_t *site_out);
+sfa_status sfa_set_wait_limit(uint64_t limit_ns);
+
 /* Static string naming a status code. */
 const char *sfa_status_string(sfa_status status);
 /* Message of the last error on the calling thread ("" if none). */

@@ -12,11 +12,14 @@ from .ops import (  # noqa: F401
     sfa_grad_rows,
     sfa_grad_workspace_size,
     sfa_shape,
+    set_wait_limit,
     softmax_grad_rowsum,
+    workspace_status,
 )
 from .shard import balanced_row_ranges, sfa_grad_sharded  # noqa: F401
 from .host import HostPipeline, sfa_grad_host  # noqa: F401
 
 __all__ = ["sfa_grad", "sfa_fwd", "fa_grad", "fa_fwd", "compact_indices", "softmax_grad_rowsum",
            "sfa_grad_workspace_size", "sfa_shape", "SfaError", "load", "sfa_grad_rows", "sfa_dkv_accumulator",
-           "sfa_dkv_finalize", "sfa_grad_sharded", "balanced_row_ranges", "sfa_grad_host", "HostPipeline"]
+           "sfa_dkv_finalize", "sfa_grad_sharded", "balanced_row_ranges", "sfa_grad_host", "HostPipeline",
+           "workspace_status", "set_wait_limit"]

@@ -65,6 +65,8 @@ SIGNATURES = {
     "fa_fwd_workspace_size": [_PFA, _I64, _PSZ],
     "fa_fwd": [_V, _V, _V, _V, _V, _Dbl, _I64, _PFA, _V, _SZ, _V, _V, _V, _V],
     "sfa_set_kernel_events": [_V, _V],
+    "sfa_workspace_status": [_V, _V, ctypes.POINTER(ctypes.c_int32)],
+    "sfa_set_wait_limit": [ctypes.c_uint64],
     "sfa_dkv_accum_size": [_PSH, _I32, _PSZ],
     "sfa_grad_rows": [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _F, _I64, _I64, _I32, _I64, _I64, _PSH, _V,
                       _SZ, _V, _V, _V, _V],

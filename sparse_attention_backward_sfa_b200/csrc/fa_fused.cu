@@ -65,6 +65,7 @@ struct FaParams {
     int* err;
     int B, Nq, Nkv, mode;
     float scale;
+    uint64_t wait_ns;  // limit of every mbarrier wait
 };
 
 struct Seq {
@@ -106,6 +107,10 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
     auto QDO_EMPTY = [&](int x) { return bar0 + 112 + 8u * x; }; // ... and consumed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    // bounded mbarrier wait: past prm.wait_ns it records `code` in the error word and every role exits
+    auto WAIT = [&](uint32_t bar, uint32_t parity, int code) {
+        return wait_bar(bar, parity, abort_flag, prm.err, code, prm.wait_ns);
+    };
     if (threadIdx.x == 0) {
         mbar_init(KV_FULL, 1);
         mbar_init(KV_EMPTY, 1);
@@ -147,7 +152,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
             const FaItem it = prm.items[w];
             const Seq s = seq_of(prm, it.b);
             if (lane == 0) {
-                ok = wait_bar(KV_EMPTY, (item_ctr & 1) ^ 1, abort_flag, prm.err, 21);
+                ok = WAIT(KV_EMPTY, (item_ctr & 1) ^ 1, 21);
                 if (ok) {
                     mbar_expect_tx(KV_FULL, 4 * kBlk * 128);
                     const int row = (int)(s.ks + (int64_t)it.kb * kBlk);
@@ -163,7 +168,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                 for (int qb = q0; qb < nqb && ok; ++qb, ++pair_ctr) {
                     const int x = pair_ctr & 1;
                     if (lane == 0) {
-                        ok = wait_bar(QDO_EMPTY(x), ((pair_ctr >> 1) & 1) ^ 1, abort_flag, prm.err, 22);
+                        ok = WAIT(QDO_EMPTY(x), ((pair_ctr >> 1) & 1) ^ 1, 22);
                         if (ok) {
                             mbar_expect_tx(QDO_FULL(x), 4 * kBlk * 128);
                             const int row = (int)(s.qs + (int64_t)qb * kBlk);
@@ -202,8 +207,8 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
         for (int w = blockIdx.x; w < prm.nitems && ok; w += gridDim.x, ++item_ctr) {
             const FaItem it = prm.items[w];
             const Seq s = seq_of(prm, it.b);
-            if (lane == 0) ok = wait_bar(KV_FULL, item_ctr & 1, abort_flag, prm.err, 23);
-            if (lane == 0 && ok) ok = wait_bar(ACC_EMPTY, (item_ctr & 1) ^ 1, abort_flag, prm.err, 24);
+            if (lane == 0) ok = WAIT(KV_FULL, item_ctr & 1, 23);
+            if (lane == 0 && ok) ok = WAIT(ACC_EMPTY, (item_ctr & 1) ^ 1, 24);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
@@ -214,9 +219,9 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                     const int x = pair_ctr & 1;
                     const uint32_t sQ = sbase + kOffQ + x * 65536, sO = sbase + kOffO + x * 65536;
                     if (lane == 0) {
-                        ok = wait_bar(QDO_FULL(x), (pair_ctr >> 1) & 1, abort_flag, prm.err, 25);
+                        ok = WAIT(QDO_FULL(x), (pair_ctr >> 1) & 1, 25);
                         // S^T overwrites P of the previous pair: its gradient MMAs must have completed
-                        if (ok && pair_ctr > 0) ok = wait_bar(PDS_FREE, (pair_ctr - 1) & 1, abort_flag, prm.err, 26);
+                        if (ok && pair_ctr > 0) ok = WAIT(PDS_FREE, (pair_ctr - 1) & 1, 26);
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
@@ -227,7 +232,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                             mma(T_S, sdesc(sK + off, 16, 1024), sdesc(sQ + off, 16, 1024), ID_S, ks > 0);
                         }
                         // dP^T overwrites the previous pair's dQ^T once the flush has read it
-                        ok = wait_bar(DQ_FREE, (pair_ctr & 1) ^ 1, abort_flag, prm.err, 33);
+                        ok = WAIT(DQ_FREE, (pair_ctr & 1) ^ 1, 33);
                         if (ok) {
                             tc_fence_after();
                             for (int ks = 0; ks < 8; ++ks) {
@@ -235,7 +240,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                                 mma(T_DP, sdesc(sV + off, 16, 1024), sdesc(sO + off, 16, 1024), ID_S, ks > 0);
                             }
                             mma_commit(SDP_FULL);
-                            ok = wait_bar(PDS_FULL, pair_ctr & 1, abort_flag, prm.err, 27);
+                            ok = WAIT(PDS_FULL, pair_ctr & 1, 27);
                         }
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -323,9 +328,10 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                         hi64 = hi64 > kBlk ? kBlk : hi64;
                         const int lo = (int)lo64;
                         const uint32_t span = key_ok && hi64 > lo64 ? (uint32_t)(hi64 - lo64) : 0u;
-                        ok = wait_bar(CST_FULL(x), use & 1, abort_flag, prm.err, 32);
-                        if (ok) ok = wait_bar(SDP_FULL, pair_ctr & 1, abort_flag, prm.err, 28);
-                        if (ok && pair_ctr > 0) ok = wait_bar(PDS_FREE, (pair_ctr - 1) & 1, abort_flag, prm.err, 29);
+                        ok = WAIT(CST_FULL(x), use & 1, 32);
+                        if (ok) ok = WAIT(SDP_FULL, pair_ctr & 1, 28);
+                        if (ok && pair_ctr > 0) ok = WAIT(PDS_FREE, (pair_ctr - 1) & 1, 29);
+                        ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
                         if (!ok) break;
                         tc_fence_after();
 #pragma unroll 1
@@ -373,7 +379,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                         mbar_arrive(PDS_FULL);
                     }
                     if (do_flush) {
-                        ok = wait_bar(DQ_FULL, pair_ctr & 1, abort_flag, prm.err, 31);
+                        ok = __all_sync(0xffffffffu, WAIT(DQ_FULL, pair_ctr & 1, 31));
                         if (!ok) break;
                         tc_fence_after();
                         const int dim = j;
@@ -408,7 +414,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
             if (!ok) break;
             if (!do_out) continue;
             // dK / dV rows of this key block (zero when no query sees the block)
-            ok = wait_bar(ACC_FULL, item_ctr & 1, abort_flag, prm.err, 30);
+            ok = __all_sync(0xffffffffu, WAIT(ACC_FULL, item_ctr & 1, 30));
             if (!ok) break;
             tc_fence_after();
             const int64_t orow = ((s.ks + jl) * prm.Nkv + it.hk) * kFaD;
@@ -498,6 +504,7 @@ cudaError_t launch_fa_t(const FaFusedArgs& a, cudaStream_t st) {
     p.Nkv = (int)a.Nkv;
     p.mode = a.mode;
     p.scale = a.scale;
+    p.wait_ns = wait_limit_ns();
     const int64_t rows = a.T1 * a.Nq;
     if (rows > 0)
         fa_rowsum_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>((const T*)a.dy, (const T*)a.o, rows,

@@ -15,6 +15,7 @@ using namespace sfa;
 namespace {
 
 thread_local std::string g_last_error;
+thread_local uint64_t g_wait_ns = 0;  // 0: the default limit
 thread_local cudaEvent_t g_ev_before = nullptr, g_ev_after = nullptr;
 
 // Records the timing-hook events (if set) around the main kernel launch.
@@ -110,11 +111,31 @@ SeqDesc seq_desc(const sfa_shape* s, const Sizes& z, const int32_t* sq, const in
 
 void sfa::set_last_error(const char* msg) { g_last_error = msg; }
 
+uint64_t sfa::wait_limit_ns() { return g_wait_ns ? g_wait_ns : 4000000000ull; }
+
 extern "C" {
 
 const char* sfa_version(void) { return "0.1.0"; }
 
 const char* sfa_last_error_string(void) { return g_last_error.c_str(); }
+
+sfa_status sfa_set_wait_limit(uint64_t limit_ns) {
+    g_wait_ns = limit_ns;
+    return SFA_OK;
+}
+
+sfa_status sfa_workspace_status(const void* workspace, sfa_stream_t stream, int32_t* site_out) {
+    g_last_error.clear();
+    if (!workspace) return fail(SFA_ERR_NULLPTR, "workspace is NULL");
+    SFA_CUDA(cudaStreamSynchronize((cudaStream_t)stream), "synchronize stream");
+    int32_t word = 0;
+    SFA_CUDA(cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost), "read error word");
+    if (site_out) *site_out = word;
+    if (word != 0)
+        return fail(SFA_ERR_TIMEOUT, "a device-side wait exceeded its limit (wait site %d); the outputs of that call "
+                    "are invalid", word);
+    return SFA_OK;
+}
 
 sfa_status sfa_set_kernel_events(void* event_before, void* event_after) {
     g_ev_before = (cudaEvent_t)event_before;
@@ -200,6 +221,7 @@ sfa_status grad_impl(const void* query, const void* key, const void* value, cons
     a.dtype = shape->dtype; a.rowlist = (int32_t*)(w + ws.rowlist); a.rowcap = shape->topk * sparse_block_size;
     a.row_begin = row_begin; a.row_end = row_end;
 
+    SFA_CUDA(cudaMemsetAsync(w + ws.ctrl, 0, 256, s), "zero control word");
     if (own_acc)
         SFA_CUDA(cudaMemsetAsync(a.dkv_acc, 0, (size_t)z.T2 * kAccW * (det ? 8 : 4), s), "zero dK/dV accumulator");
     SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, (int32_t*)a.blocks, (int32_t*)a.nblk,
@@ -327,6 +349,7 @@ sfa_status sfa_fwd(const void* query, const void* key, const void* value, const 
     int32_t* blocks = (int32_t*)(w + ws.blocks);
     int32_t* nblk = (int32_t*)(w + ws.nblk);
     int32_t* nrows = (int32_t*)(w + ws.nrows);
+    SFA_CUDA(cudaMemsetAsync(w + ws.ctrl, 0, 256, s), "zero control word");
     a.blocks = blocks; a.nblk = nblk;
     a.out = out; a.smax = softmax_max; a.ssum = softmax_sum;
     SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, blocks, nblk, nrows, s), "index compaction");
@@ -418,7 +441,10 @@ static sfa_status check_cu(const int64_t* cu, int64_t B, int64_t T, const char* 
     return SFA_OK;
 }
 
-static size_t fa_cu_bytes(int64_t B) { return 2 * align256((size_t)B * 8); }
+// FA workspaces start with the 256-byte control area (device error word), then the
+// two cumulative-length arrays
+constexpr size_t kCtrl = 256;
+static size_t fa_cu_bytes(int64_t B) { return kCtrl + 2 * align256((size_t)B * 8); }
 
 // Workspace of the tensor-core dense backward (head dim 128): cumulative lengths,
 // work list, rowsum(dY o O), dQ accumulator, control word.
@@ -431,7 +457,7 @@ static FaFusedWs fa_fused_ws(const fa_shape* s, bool det) {
     w.items = o;  o = align256(o + fa_fused_max_items(s->B, s->T2, s->Nkv) * 16);
     w.rowsum = o; o = align256(o + (size_t)s->T1 * s->Nq * 4);
     w.dq = o;     o = align256(o + (size_t)s->T1 * s->Nq * s->D * (det ? 8 : 4));
-    w.ctrl = o;   o = align256(o + 256);
+    w.ctrl = 0;
     w.total = o;
     return w;
 }
@@ -477,9 +503,10 @@ sfa_status fa_grad(const void* q, const void* k, const void* v, const void* dy, 
     if (workspace_bytes < need) return fail(SFA_ERR_WORKSPACE, "workspace %zu < %zu", workspace_bytes, need);
     cudaStream_t s = (cudaStream_t)stream;
     char* w = (char*)workspace;
-    int64_t* cuq = (int64_t*)w;
-    int64_t* cukv = (int64_t*)(w + align256((size_t)shape->B * 8));
+    int64_t* cuq = (int64_t*)(w + kCtrl);
+    int64_t* cukv = (int64_t*)(w + kCtrl + align256((size_t)shape->B * 8));
     void* acc = w + fa_cu_bytes(shape->B);
+    SFA_CUDA(cudaMemsetAsync(w, 0, kCtrl, s), "zero control word");
     SFA_CUDA(cudaMemcpyAsync(cuq, actual_seq_qlen, shape->B * 8, cudaMemcpyHostToDevice, s), "copy seqlens");
     SFA_CUDA(cudaMemcpyAsync(cukv, actual_seq_kvlen, shape->B * 8, cudaMemcpyHostToDevice, s), "copy seqlens");
     if (fused) {
@@ -540,8 +567,9 @@ sfa_status fa_fwd(const void* q, const void* k, const void* v, const int64_t* ac
     if (workspace_bytes < need) return fail(SFA_ERR_WORKSPACE, "workspace %zu < %zu", workspace_bytes, need);
     cudaStream_t s = (cudaStream_t)stream;
     char* w = (char*)workspace;
-    int64_t* cuq = (int64_t*)w;
-    int64_t* cukv = (int64_t*)(w + align256((size_t)shape->B * 8));
+    int64_t* cuq = (int64_t*)(w + kCtrl);
+    int64_t* cukv = (int64_t*)(w + kCtrl + align256((size_t)shape->B * 8));
+    SFA_CUDA(cudaMemsetAsync(w, 0, kCtrl, s), "zero control word");
     SFA_CUDA(cudaMemcpyAsync(cuq, actual_seq_qlen, shape->B * 8, cudaMemcpyHostToDevice, s), "copy seqlens");
     SFA_CUDA(cudaMemcpyAsync(cukv, actual_seq_kvlen, shape->B * 8, cudaMemcpyHostToDevice, s), "copy seqlens");
     FaArgs a;

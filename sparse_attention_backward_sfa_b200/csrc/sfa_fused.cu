@@ -80,6 +80,7 @@ struct FusedParams {
     int64_t cap;
     float scale;
     int det;
+    uint64_t wait_ns;        // limit of every mbarrier wait (error word + clean exit past it)
 };
 
 // Item i of a tile's load schedule: kind (0 key chunk, 1 q chunk, 2 dO chunk) and chunk c.
@@ -93,6 +94,22 @@ __device__ __forceinline__ void item_of(int i, int& kind, int& c) {
     if (i < 4) { kind = 2; c = i; return; }
     if (i < 9) { kind = 1; c = i - 4; return; }
     kind = 0; c = i - 9;
+}
+
+// Named barrier 1 over the 128 softmax threads that also ANDs a flag across them:
+// a thread that gave up waiting takes the others with it, so none of them is
+// left at a later barrier of this group.
+__device__ __forceinline__ bool softmax_all(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
 }
 
 // Reductions of one 32-column chunk of a staged gradient block held by this
@@ -205,6 +222,10 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
     const uint32_t DONE = bar0 + 8u * (2 * C::kSlots + 11);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    // bounded mbarrier wait: past prm.wait_ns it records `code` in the error word and every role exits
+    auto WAIT = [&](uint32_t bar, uint32_t parity, int code) {
+        return wait_bar(bar, parity, abort_flag, prm.err, code, prm.wait_ns);
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kSlots; ++s) {
@@ -254,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
             const int ntiles = (n + kKeys - 1) / kKeys;
             for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
                 const int rb = tile_ctr & 1;
-                if (lane == 0) ok = wait_bar(ROWS_EMPTY(rb), ((tile_ctr >> 1) & 1) ^ 1, abort_flag, prm.err, 1);
+                if (lane == 0) ok = WAIT(ROWS_EMPTY(rb), ((tile_ctr >> 1) & 1) ^ 1, 1);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 int32_t* rid = rowids + rb * kKeys;
@@ -272,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 for (int it = 0; it < 28 && ok; ++it) {
                     int kind, c;
                     item_of(it, kind, c);
-                    if (lane == 0) ok = wait_bar(EMPTY(slot), sphase ^ 1, abort_flag, prm.err, 2);
+                    if (lane == 0) ok = WAIT(EMPTY(slot), sphase ^ 1, 2);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     const uint32_t dst = sbase + slot * kSlotBytes;
@@ -333,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 for (int it = 0; it < 14 && ok; ++it) {
                     int kind, c;
                     item_of(it, kind, c);
-                    if (lane == 0) ok = wait_bar(FULL(slot), sphase, abort_flag, prm.err, 3);
+                    if (lane == 0) ok = WAIT(FULL(slot), sphase, 3);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     tc_fence_after();
@@ -358,14 +379,14 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 if (!ok) break;
                 if (lane == 0) mma_commit(SDP_FULL);
                 // ---- gradient blocks ----
-                if (lane == 0) ok = wait_bar(PDS_FULL, tile_ctr & 1, abort_flag, prm.err, 4);
+                if (lane == 0) ok = WAIT(PDS_FULL, tile_ctr & 1, 4);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after();
                 for (int bi = 0; bi < 14 && ok; ++bi, ++blk_ctr) {
                     const int stg = blk_ctr & 1;
-                    if (lane == 0) ok = wait_bar(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, abort_flag, prm.err, 5);
-                    if (lane == 0 && ok) ok = wait_bar(FULL(slot), sphase, abort_flag, prm.err, 6);
+                    if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 5);
+                    if (lane == 0 && ok) ok = WAIT(FULL(slot), sphase, 6);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     tc_fence_after();
@@ -428,8 +449,9 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
             for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
                 // padding keys of the last tile get P = dS = 0 (their S is finite: a real gathered row)
                 const float vmul = tile * kKeys + j < n ? 1.f : 0.f;
-                ok = wait_bar(SDP_FULL, tile_ctr & 1, abort_flag, prm.err, 8);
-                if (ok && tile_ctr > 0) ok = wait_bar(PDS_FREE, (tile_ctr - 1) & 1, abort_flag, prm.err, 9);
+                ok = WAIT(SDP_FULL, tile_ctr & 1, 8);
+                if (ok && tile_ctr > 0) ok = WAIT(PDS_FREE, (tile_ctr - 1) & 1, 9);
+                ok = softmax_all(ok);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -501,13 +523,13 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 const int dqmode = ntiles == 1 ? DQ_SINGLE
                                    : (tile == 0 ? DQ_FIRST : (tile == ntiles - 1 ? DQ_LAST : DQ_MID));
                 const int rb = tile_ctr & 1;
-                ok = wait_bar(ROWS_FULL(rb), (tile_ctr >> 1) & 1, abort_flag, prm.err, 10);
+                ok = __all_sync(0xffffffffu, WAIT(ROWS_FULL(rb), (tile_ctr >> 1) & 1, 10));
                 if (!ok) break;
                 const int32_t* rid = rowids + rb * kKeys;
                 const int nvalid = min(kKeys, n - tile * kKeys);
                 for (int bi = 0; bi < 14 && ok; ++bi, ++blk_ctr) {
                     const int stg = blk_ctr & 1;
-                    ok = wait_bar(STG_FULL(stg), (blk_ctr >> 1) & 1, abort_flag, prm.err, 11);
+                    ok = __all_sync(0xffffffffu, WAIT(STG_FULL(stg), (blk_ctr >> 1) & 1, 11));
                     if (!ok) break;
                     tc_fence_after();
                     // which output block and which dims this lane quarter holds
@@ -575,6 +597,7 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
     p.cap = a.rowcap;
     p.scale = a.scale;
     p.det = DET ? 1 : 0;
+    p.wait_ns = wait_limit_ns();
 
     auto kern = sfa_bwd_fused_kernel<T, N1, DET>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<N1>::kSmem);

@@ -63,6 +63,7 @@ struct FwdParams {
     int64_t cap;
     float scale;
     int blk16;
+    uint64_t wait_ns;  // limit of every mbarrier wait
 };
 
 // Chunk order of a pass: pass 0 any order; pass 1 / 2 put the two value chunks of
@@ -96,6 +97,10 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
     const uint32_t DONE = bar0 + 8u * (2 * kSlots + 8);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    // bounded mbarrier wait: past prm.wait_ns it records `code` in the error word and every role exits
+    auto WAIT = [&](uint32_t bar, uint32_t parity, int code) {
+        return wait_bar(bar, parity, abort_flag, prm.err, code, prm.wait_ns);
+    };
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSlots; ++s) {
             mbar_init(FULL(s), 1);
@@ -157,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
                     for (int i = 0; i < 10 && ok; ++i) {
                         const int c = chunk_of(pass, i >> 1);
                         const bool is_key = (i & 1) == 0;
-                        if (lane == 0) ok = wait_bar(EMPTY(slot), sphase ^ 1, abort_flag, prm.err, 41);
+                        if (lane == 0) ok = WAIT(EMPTY(slot), sphase ^ 1, 41);
                         ok = __shfl_sync(0xffffffffu, ok, 0);
                         if (!ok) break;
                         const uint32_t dst = sbase + slot * kSlotBytes;
@@ -207,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
         bool ok = true;
         auto wait_full = [&]() -> bool {
             bool r = true;
-            if (lane == 0) r = wait_bar(FULL(slot), sphase, abort_flag, prm.err, 42);
+            if (lane == 0) r = WAIT(FULL(slot), sphase, 42);
             r = __shfl_sync(0xffffffffu, r, 0);
             if (r) tc_fence_after();
             return r;
@@ -220,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
         auto issue_s = [&](int pass, uint32_t (&vslot)[2]) -> bool {
             const int b = s_ctr & 1;
             bool r = true;
-            if (lane == 0) r = wait_bar(S_FREE(b), ((s_ctr >> 1) & 1) ^ 1, abort_flag, prm.err, 43);
+            if (lane == 0) r = WAIT(S_FREE(b), ((s_ctr >> 1) & 1) ^ 1, 43);
             r = __shfl_sync(0xffffffffu, r, 0);
             if (!r) return false;
             tc_fence_after();
@@ -254,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
         // out half += P . V of one tile (P from the softmax warps; V = the held key chunks)
         auto issue_o = [&](bool first_tile, const uint32_t (&vslot)[2]) -> bool {
             bool r = true;
-            if (lane == 0) r = wait_bar(P_FULL, p_ctr & 1, abort_flag, prm.err, 44);
+            if (lane == 0) r = WAIT(P_FULL, p_ctr & 1, 44);
             r = __shfl_sync(0xffffffffu, r, 0);
             if (!r) return false;
             tc_fence_after();
@@ -287,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
                     continue;
                 }
                 // the previous output half has been written out
-                if (lane == 0) ok = wait_bar(O_EMPTY, (o_ctr & 1) ^ 1, abort_flag, prm.err, 45);
+                if (lane == 0) ok = WAIT(O_EMPTY, (o_ctr & 1) ^ 1, 45);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after();
@@ -344,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
             float m2 = -INFINITY, l = 0.f;  // m2 = max * log2e
             for (int tile = 0; tile < ntiles && ok; ++tile, ++s_ctr) {
                 const int b = s_ctr & 1;
-                ok = wait_bar(S_FULL(b), (s_ctr >> 1) & 1, abort_flag, prm.err, 46);
+                ok = __all_sync(0xffffffffu, WAIT(S_FULL(b), (s_ctr >> 1) & 1, 46));
                 if (!ok) break;
                 tc_fence_after();
                 uint32_t mk[4];
@@ -385,9 +390,10 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
             for (int pass = 1; pass < 3 && ok; ++pass, ++o_ctr) {
                 for (int tile = 0; tile < ntiles && ok; ++tile, ++s_ctr, ++p_ctr) {
                     const int b = s_ctr & 1;
-                    ok = wait_bar(S_FULL(b), (s_ctr >> 1) & 1, abort_flag, prm.err, 47);
+                    ok = WAIT(S_FULL(b), (s_ctr >> 1) & 1, 47);
                     // P of the previous tile has been read by its output MMA
-                    if (ok) ok = wait_bar(P_FREE, (p_ctr & 1) ^ 1, abort_flag, prm.err, 48);
+                    if (ok) ok = WAIT(P_FREE, (p_ctr & 1) ^ 1, 48);
+                    ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
                     if (!ok) break;
                     tc_fence_after();
                     uint32_t mk[4];
@@ -420,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
                     mbar_arrive(P_FULL);
                 }
                 if (!ok) break;
-                ok = wait_bar(O_FULL, o_ctr & 1, abort_flag, prm.err, 49);
+                ok = __all_sync(0xffffffffu, WAIT(O_FULL, o_ctr & 1, 49));
                 if (!ok) break;
                 tc_fence_after();
                 T* o = reinterpret_cast<T*>(prm.out) + row * kD + 256 * (pass - 1);
@@ -473,6 +479,7 @@ cudaError_t launch_t(const FwdFusedArgs& a, cudaStream_t st) {
     p.cap = a.rowcap;
     p.scale = a.scale;
     p.blk16 = a.blk16;
+    p.wait_ns = wait_limit_ns();
     auto kern = sfa_fwd_fused_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;

@@ -115,7 +115,7 @@ struct GradWs {
     size_t order;   // [T1] int32 work order (longest first)
     size_t rowsum;  // [T1][N1] fp32 FlashSoftmaxGrad
     size_t rowlist; // [T1][topk*bs] int32 gathered key rows, fused path only
-    size_t ctrl;    // 256 B of counters / flags
+    size_t ctrl;    // 256 B of counters / flags (offset 0: the device error word)
     size_t total;
 };
 
@@ -126,6 +126,7 @@ constexpr int kMaxFusedGrid = 256;  // persistent CTAs of the fused kernel (one 
 inline GradWs grad_ws_layout(int64_t T1, int64_t T2, int64_t N1, int64_t topk, int64_t bs, bool det, bool fused) {
     GradWs w;
     size_t o = 0;
+    w.ctrl = o;   o = 256;  // error word first: sfa_workspace_status reads offset 0
     w.dkv = o;    o = align256(o + (size_t)T2 * kAccW * (det ? 8 : 4));
     w.dq = o;     o = align256(o + (fused ? (size_t)kMaxFusedGrid * N1 * kDK * 4 : 0));
     w.blocks = o; o = align256(o + (size_t)T1 * topk * 4);
@@ -134,7 +135,6 @@ inline GradWs grad_ws_layout(int64_t T1, int64_t T2, int64_t N1, int64_t topk, i
     w.order = o;  o = align256(o + (size_t)T1 * 4);
     w.rowsum = o; o = align256(o + (size_t)T1 * N1 * 4);
     w.rowlist = o; o = align256(o + (fused ? (size_t)T1 * topk * bs * 4 : 0));
-    w.ctrl = o;   o = align256(o + 256);
     w.total = o;
     return w;
 }
@@ -148,13 +148,13 @@ inline FwdWs fwd_ws_layout(int64_t T1, int64_t N1, int64_t topk, int64_t bs) {
     FwdWs w;
     const bool fused = N1 == 128;
     size_t o = 0;
+    w.ctrl = o;    o = 256;  // error word first
     w.blocks = o;  o = align256(o + (size_t)T1 * topk * 4);
     w.nblk = o;    o = align256(o + (size_t)T1 * 4);
     w.nrows = o;   o = align256(o + (size_t)T1 * 4);
     w.order = o;   o = align256(o + (fused ? (size_t)T1 * 4 : 0));
     w.rowlist = fused ? o : 0; o = align256(o + (fused ? (size_t)T1 * topk * bs * 4 : 0));
     w.nslots = o;  o = align256(o + (fused ? (size_t)T1 * 4 : 0));
-    w.ctrl = o;    o = align256(o + 256);
     w.total = o;
     return w;
 }
@@ -246,6 +246,9 @@ inline size_t fa_fused_max_items(int64_t B, int64_t T2, int64_t Nkv) { return (s
 cudaError_t launch_fa_bwd_fused(int dtype, const FaFusedArgs& a, cudaStream_t st);
 // Sets the message returned by sfa_last_error_string() on the calling thread.
 void set_last_error(const char* msg);
+// Limit of every device-side mbarrier wait of the fused kernels launched from the
+// calling thread (sfa_set_wait_limit; 4 s by default).
+uint64_t wait_limit_ns();
 cudaError_t launch_fa_fwd(int dtype, const FaArgs& a, cudaStream_t st);
 
 }  // namespace sfa

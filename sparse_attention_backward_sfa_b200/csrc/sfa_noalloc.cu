@@ -116,6 +116,8 @@ sfa_status sfa_grad_noalloc(const void* query, const void* key, const void* valu
 
     cudaError_t e;
     // the accumulator must start at zero; the rest of the scratch is fully rewritten
+    if ((e = cudaMemsetAsync(w + ws.ctrl, 0, 256, s)) != cudaSuccess)
+        return nfail(SFA_ERR_CUDA, "clear scratch: %s", cudaGetErrorString(e));
     if ((e = cudaMemsetAsync(a.dkv_acc, 0, (size_t)T2 * kAccW * (det ? 8 : 4), s)) != cudaSuccess)
         return nfail(SFA_ERR_CUDA, "clear scratch: %s", cudaGetErrorString(e));
     if ((e = launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, (int32_t*)a.blocks, (int32_t*)a.nblk,

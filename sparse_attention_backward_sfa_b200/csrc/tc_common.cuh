@@ -38,16 +38,17 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
-// Bounded wait: gives up after ~4 s (or as soon as another role aborted),
+// Bounded wait: gives up after `limit_ns` (or as soon as another role aborted),
 // recording `code` in the device error word.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err, int code) {
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err, int code,
+                                      uint64_t limit_ns) {
     if (mbar_try(bar, parity)) return true;
     uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try(bar, parity)) return true;
-        if ((it & 63) == 0) {
+        if ((it & 63) == 1) {  // from the first retry on: try_wait itself suspends for a while
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > 4000000000ull) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort_flag = 1;
                 atomicCAS(err, 0, code);
                 return false;

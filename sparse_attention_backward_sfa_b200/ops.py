@@ -171,7 +171,8 @@ def sfa_dkv_finalize(dkv_accum, query, key, query_rope, sparse_indices, *, layou
 
 
 def sfa_fwd(query, key, value, sparse_indices, query_rope, key_rope, *, scale: float, sparse_block_size: int,
-            layout: str, sparse_mode: int, actual_seq_lengths_q=None, actual_seq_lengths_kv=None, stream=None):
+            layout: str, sparse_mode: int, actual_seq_lengths_q=None, actual_seq_lengths_kv=None, workspace=None,
+            stream=None):
     """Forward of top-k sparse attention; returns (out, softmaxMax, softmaxSum)."""
     lib = N.load()
     dt = query.dtype
@@ -183,7 +184,9 @@ def sfa_fwd(query, key, value, sparse_indices, query_rope, key_rope, *, scale: f
     skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
     n = ctypes.c_size_t()
     N.check(lib.sfa_fwd_workspace_size(ctypes.byref(shape), sparse_block_size, sparse_mode, ctypes.byref(n)))
-    ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=query.device)
+    ws = workspace
+    if ws is None or ws.numel() < n.value:
+        ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=query.device)
     out = torch.empty_like(query)
     stat_shape = query.shape[:-1]
     smax = torch.empty(stat_shape, dtype=torch.float32, device=query.device)
@@ -276,3 +279,20 @@ def fa_fwd(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, scale: float, sparse_mode: i
                        ws.numel(), _stream(stream), _p(out), _p(smax), _p(ssum)))
     del aq, akv
     return out, smax, ssum
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Waits for `stream` and returns the wait-site code the last call left in the workspace's
+    error word: 0 when every device-side wait was satisfied, else the site that gave up."""
+    lib = N.load()
+    site = ctypes.c_int32(0)
+    st = lib.sfa_workspace_status(_p(workspace), _stream(stream), ctypes.byref(site))
+    if st not in (N.SFA_OK, N.SFA_ERR_TIMEOUT):
+        N.check(st)
+    return int(site.value)
+
+
+def set_wait_limit(limit_ns: int) -> None:
+    """Limit of every device-side wait of the fused kernels launched afterwards from this
+    thread (0: the default 4 s)."""
+    N.check(N.load().sfa_set_wait_limit(int(limit_ns)))

@@ -151,8 +151,9 @@ class DevFA:
                                                   scale=fp.scale, sparse_mode=fp.sparse_mode)
         return self.out, self.smax, self.ssum
 
-    def grad_gpu(self, deterministic=False):
+    def grad_gpu(self, deterministic=False, **extra):
         import sparse_attention_backward_sfa_b200 as S
         fp = self.fp
         return S.fa_grad(self.q, self.k, self.v, self.dy, self.smax, self.ssum, self.out, fp.cu_seqlens_q,
-                         fp.cu_seqlens_kv, scale=fp.scale, sparse_mode=fp.sparse_mode, deterministic=deterministic)
+                         fp.cu_seqlens_kv, scale=fp.scale, sparse_mode=fp.sparse_mode, deterministic=deterministic,
+                         **extra)
