@@ -231,6 +231,9 @@ sfa_status grad_impl(const void* query, const void* key, const void* value, cons
         SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, row_begin, row_end, shape->N1, (float*)a.rowsum, s),
                  "rowsum(dO*O)");
         SFA_CUDA(launch_order(a.nrows, row_begin, row_end, (int32_t*)a.order, a.ctrl, s), "work order");
+        // block-sparse lists sorted: consecutive selected blocks become contiguous key tiles
+        if (a.bs > 1 && a.topk <= kSortMaxTopk)
+            SFA_CUDA(launch_sort_blocks((int32_t*)a.blocks, a.nblk, a.topk, row_begin, row_end, s), "block sort");
         SFA_CUDA(launch_expand(a.blocks, a.nblk, a.sd, a.topk, a.bs, a.mode, a.rowcap, (int32_t*)a.rowlist, s),
                  "key row expansion");
         {
@@ -361,6 +364,9 @@ sfa_status sfa_fwd(const void* query, const void* key, const void* value, const 
         f.out = out; f.smax = softmax_max; f.ssum = softmax_sum; f.err = (int*)(w + ws.ctrl);
         f.T1 = z.T1; f.T2 = z.T2; f.rowcap = shape->topk * sparse_block_size; f.scale = scale; f.dtype = shape->dtype;
         SFA_CUDA(launch_order(nrows, 0, z.T1, (int32_t*)f.order, (int32_t*)(w + ws.ctrl), s), "work order");
+        // block-sparse lists sorted: consecutive selected blocks become contiguous key tiles
+        if (a.bs > 1 && a.topk <= kSortMaxTopk)
+            SFA_CUDA(launch_sort_blocks(blocks, nblk, a.topk, 0, z.T1, s), "block sort");
         f.blk16 = a.bs % 16 == 0 ? 1 : 0;
         if (f.blk16) {  // runs of 16 contiguous key rows: 16-row 2-D tile loads instead of row gathers
             f.nrows = (int32_t*)(w + ws.nslots);

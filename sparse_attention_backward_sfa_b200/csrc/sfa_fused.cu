@@ -63,7 +63,8 @@ template <int N1> struct Cfg {
 };
 
 struct FusedParams {
-    CUtensorMap mapQ, mapQr, mapO, mapK, mapKr;  // dO shares mapO
+    CUtensorMap mapQ, mapQr, mapO, mapK, mapKr;  // dO shares mapO; key maps: 1-row boxes (gather4)
+    CUtensorMap mapK128, mapKr128;                // key maps with 128-row boxes (contiguous tiles)
     const int32_t* rowlist;  // [T1][cap] global key rows of each query row
     const int32_t* nrows;    // [T1]
     const int32_t* order;    // [T1] work order
@@ -280,14 +281,20 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 if (!ok) break;
                 int32_t* rid = rowids + rb * kKeys;
                 const int first = rl[0];
-                // lane L owns key rows 4L..4L+3 of the tile (one gather4 per 64-dim half)
+                const int run0 = rl[tile * kKeys];
+                // lane L owns key rows 4L..4L+3 of the tile (one gather4 per 64-dim half); a tile
+                // whose rows are run0, run0+1, ... is loaded as one 128-row 2-D tile instead (its
+                // slots past the row's end then hold rows run0+s, masked like any padding key)
                 int32_t my[4];
+                bool contig = true;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int s = tile * kKeys + 4 * lane + e;
                     my[e] = s < n ? rl[s] : first;
+                    if (s < n && my[e] != run0 + 4 * lane + e) contig = false;
                     rid[4 * lane + e] = my[e];
                 }
+                contig = __all_sync(0xffffffffu, contig);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ROWS_FULL(rb));
                 for (int it = 0; it < 28 && ok; ++it) {
@@ -303,7 +310,13 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                         mbar_expect_tx(FULL(slot), halves * rows * 128u);
                     }
                     __syncwarp();
-                    if (kind == 0) {
+                    if (kind == 0 && contig) {
+                        if (lane == 0) {
+                            const CUtensorMap* map = c < 4 ? &prm.mapK128 : &prm.mapKr128;
+                            for (int h = 0; h < halves; ++h)
+                                tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, run0, FULL(slot));
+                        }
+                    } else if (kind == 0) {
                         // key rows: every lane gathers its own four rows, in parallel
                         const CUtensorMap* map = c < 4 ? &prm.mapK : &prm.mapKr;
                         for (int h = 0; h < halves; ++h)
@@ -447,8 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
             asm volatile("bar.sync 1, 128;" ::: "memory");
             const int ntiles = (n + kKeys - 1) / kKeys;
             for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
-                // padding keys of the last tile get P = dS = 0 (their S is finite: a real gathered row)
-                const float vmul = tile * kKeys + j < n ? 1.f : 0.f;
+                // padding keys of the last tile get P = dS = 0 (selected, not multiplied: a padding
+                // slot of a 2-D tile holds an arbitrary row whose score may exceed the row max)
+                const bool kv = tile * kKeys + j < n;
                 ok = WAIT(SDP_FULL, tile_ctr & 1, 8);
                 if (ok && tile_ctr > 0) ok = WAIT(PDS_FREE, (tile_ctr - 1) & 1, 9);
                 ok = softmax_all(ok);
@@ -474,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const int e = 4 * g + k;
-                            pv[k] = ex2_approx(fmaf(s[e], c1, -mm[k])) * (ll[k] * vmul);
+                            pv[k] = kv ? ex2_approx(fmaf(s[e], c1, -mm[k])) * ll[k] : 0.f;
                             dv[k] = pv[k] * (dp[e] - dd[k]) * scale;
                         }
                         pw[2 * g] = pack2<T>(pv[0], pv[1]);
@@ -579,7 +593,9 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
         !make_map(&p.mapQr, a.qr, a.dtype, kDr, (uint64_t)T1 * N1, kDr, N1) ||
         !make_map(&p.mapO, a.dout, a.dtype, kD, (uint64_t)T1 * N1, kD, N1) ||
         !make_map(&p.mapK, a.k, a.dtype, kD, (uint64_t)T2, kD, 1) ||
-        !make_map(&p.mapKr, a.kr, a.dtype, kDr, (uint64_t)T2, kDr, 1))
+        !make_map(&p.mapKr, a.kr, a.dtype, kDr, (uint64_t)T2, kDr, 1) ||
+        !make_map(&p.mapK128, a.k, a.dtype, kD, (uint64_t)T2, kD, kKeys) ||
+        !make_map(&p.mapKr128, a.kr, a.dtype, kDr, (uint64_t)T2, kDr, kKeys))
         return cudaErrorInvalidValue;
     p.rowlist = a.rowlist;
     p.nrows = a.nrows;

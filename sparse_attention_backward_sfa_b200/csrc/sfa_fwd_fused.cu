@@ -51,7 +51,8 @@ constexpr int kSmem = kOffMisc + 16;
 
 struct FwdParams {
     CUtensorMap mapQ, mapQr, mapK, mapKr;
-    CUtensorMap mapK16, mapKr16;  // 16-row boxes (block-aligned row lists)
+    CUtensorMap mapK16, mapKr16;    // 16-row boxes (block-aligned row lists)
+    CUtensorMap mapK128, mapKr128;  // 128-row boxes (tiles of consecutive key rows)
     const int32_t* rowlist;  // [T1][cap] global key rows of each query row
     const int32_t* nrows;    // [T1]
     const int32_t* order;    // [T1] work order
@@ -159,6 +160,16 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
                         const int s = tile * kKeys + 16 * (lane & 7);
                         gfirst = s < n ? rl[s] & 0x7fffffff : first;
                     }
+                    // a tile whose slots hold rows run0, run0+1, ... (padding flags aside) is one
+                    // 128-row 2-D tile; its slots past the list then hold rows run0+s, masked
+                    const int run0 = rl[tile * kKeys] & 0x7fffffff;
+                    bool contig = true;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int s = tile * kKeys + 4 * lane + e;
+                        if (s < n && my[e] != run0 + 4 * lane + e) contig = false;
+                    }
+                    contig = __all_sync(0xffffffffu, contig);
                     for (int i = 0; i < 10 && ok; ++i) {
                         const int c = chunk_of(pass, i >> 1);
                         const bool is_key = (i & 1) == 0;
@@ -169,7 +180,13 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
                         const int halves = c < 4 ? 2 : 1;
                         if (lane == 0) mbar_expect_tx(FULL(slot), halves * 128u * 128u);
                         __syncwarp();
-                        if (is_key && prm.blk16) {
+                        if (is_key && contig) {
+                            if (lane == 0) {
+                                const CUtensorMap* map = c < 4 ? &prm.mapK128 : &prm.mapKr128;
+                                for (int h = 0; h < halves; ++h)
+                                    tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, run0, FULL(slot));
+                            }
+                        } else if (is_key && prm.blk16) {
                             const int h = lane >> 3;
                             if (lane < 8 * halves)
                                 tma_load_2d(dst + h * kHalf + (lane & 7) * 2048, c < 4 ? &prm.mapK16 : &prm.mapKr16,
@@ -466,7 +483,9 @@ cudaError_t launch_t(const FwdFusedArgs& a, cudaStream_t st) {
         !make_map(&p.mapK, a.k, a.dtype, kD, (uint64_t)T2, kD, 1) ||
         !make_map(&p.mapKr, a.kr, a.dtype, kDr, (uint64_t)T2, kDr, 1) ||
         !make_map(&p.mapK16, a.k, a.dtype, kD, (uint64_t)T2, kD, 16) ||
-        !make_map(&p.mapKr16, a.kr, a.dtype, kDr, (uint64_t)T2, kDr, 16))
+        !make_map(&p.mapKr16, a.kr, a.dtype, kDr, (uint64_t)T2, kDr, 16) ||
+        !make_map(&p.mapK128, a.k, a.dtype, kD, (uint64_t)T2, kD, kKeys) ||
+        !make_map(&p.mapKr128, a.kr, a.dtype, kDr, (uint64_t)T2, kDr, kKeys))
         return cudaErrorInvalidValue;
     p.rowlist = a.rowlist;
     p.nrows = a.nrows;

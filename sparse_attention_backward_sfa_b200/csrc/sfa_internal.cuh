@@ -170,6 +170,11 @@ cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t 
 // work order of the fused kernel over query rows [row_begin, row_end) (row_end - row_begin entries)
 cudaError_t launch_order(const int32_t* nrows, int64_t row_begin, int64_t row_end, int32_t* order, int32_t* ctrl,
                          cudaStream_t st);
+// Sorts the kept block indices of rows [row_begin, row_end) ascending, in place
+// (topk <= kSortMaxTopk: the row is sorted in shared memory).
+constexpr int64_t kSortMaxTopk = 4096;
+cudaError_t launch_sort_blocks(int32_t* blocks, const int32_t* nblk, int64_t topk, int64_t row_begin, int64_t row_end,
+                               cudaStream_t st);
 cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs, int mode,
                           int64_t cap, int32_t* rowlist, cudaStream_t st);
 // block-aligned key-row lists for sparse_block_size % 16 == 0 (invalid slots: bit 31 set)

@@ -173,6 +173,50 @@ cudaError_t launch_expand_blocks(const int32_t* blocks, const int32_t* nblk, con
     return cudaGetLastError();
 }
 
+// Sorts each query row's kept block indices ascending (rows [row_begin, row_end)).
+// The sum over a row's keys does not depend on their order; sorted, the
+// expanded key rows form runs of consecutive rows, and a tile of 128 of them is
+// loaded as one 2-D tile instead of 32 four-row gathers.  One CTA per row, a
+// bitonic network over the next power of two >= the row's count in shared memory
+// (padding sorts last).
+__global__ void sort_blocks_kernel(int32_t* __restrict__ blocks, const int32_t* __restrict__ nblk, int64_t topk,
+                                   int64_t row_begin) {
+    extern __shared__ int32_t v[];
+    const int64_t t = row_begin + blockIdx.x;
+    const int n = nblk[t];
+    if (n <= 1) return;  // uniform over the CTA
+    int p = 1;
+    while (p < n) p <<= 1;
+    int32_t* row = blocks + t * topk;
+    for (int i = threadIdx.x; i < p; i += blockDim.x) v[i] = i < n ? row[i] : 0x7fffffff;
+    __syncthreads();
+    for (int k = 2; k <= p; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < p; i += blockDim.x) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const int32_t a = v[i], b = v[l];
+                    if ((a > b) == ((i & k) == 0)) {
+                        v[i] = b;
+                        v[l] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = threadIdx.x; i < n; i += blockDim.x) row[i] = v[i];
+}
+
+cudaError_t launch_sort_blocks(int32_t* blocks, const int32_t* nblk, int64_t topk, int64_t row_begin, int64_t row_end,
+                               cudaStream_t st) {
+    if (row_end <= row_begin || topk <= 1) return cudaGetLastError();
+    int p = 1;
+    while (p < topk) p <<= 1;
+    sort_blocks_kernel<<<(unsigned)(row_end - row_begin), 256, (size_t)p * 4, st>>>(blocks, nblk, topk, row_begin);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs, int mode,
                           int64_t cap, int32_t* rowlist, cudaStream_t st) {
     const int warps = 8;

@@ -41,6 +41,14 @@ FUSED = {
                                  index_mode="messy", seqlens_q=[5, 4], seqlens_kv=[300, 37]),
     "n64_tnd_bs32_causal": dict(layout="TND", seqlens_q=[40, 9], seqlens_kv=[200, 70], N1=64, topk=8, block_size=32,
                                 sparse_mode=3, index_mode="causal"),
+    # every causal block selected (random order, sorted before expansion): rows of up to three
+    # contiguous 128-key tiles with a ragged tail; the last sequence's tail tiles reach past the end
+    # of the key tensor (601 rows), where the 2-D tile reads zeros
+    "n128_tnd_bs16_all_blocks": dict(layout="TND", seqlens_q=[300, 45], seqlens_kv=[300, 301], N1=128, topk=40,
+                                     block_size=16, sparse_mode=3, index_mode="causal"),
+    # topk below the causal block count for later rows: contiguous and gathered tiles mixed
+    "n64_tnd_bs16_mixed_tiles": dict(layout="TND", seqlens_q=[200], seqlens_kv=[200], N1=64, topk=9, block_size=16,
+                                     sparse_mode=3, index_mode="causal"),
 }
 
 
@@ -100,6 +108,10 @@ FWD = {
     "n128_bsnd_bs16_messy": FUSED["n128_bsnd_bs16_messy"],
     "n128_tnd_bs32_causal": dict(layout="TND", seqlens_q=[40, 9], seqlens_kv=[200, 70], N1=128, topk=8, block_size=32,
                                  sparse_mode=3, index_mode="causal"),
+    # contiguous 128-key tiles (all causal blocks selected), tails past the end of the key tensor
+    "n128_tnd_bs16_all_blocks": FUSED["n128_tnd_bs16_all_blocks"],
+    # contiguous and 16-row-tile key loads mixed in one row
+    "n128_tnd_bs16_mixed_tiles": dict(FUSED["n64_tnd_bs16_mixed_tiles"], N1=128),
 }
 
 
