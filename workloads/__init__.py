@@ -17,4 +17,8 @@ from .gen import (  # noqa: F401
     FAProblem,
     tiny_problem,
     subproblem,
+    IndexerProblem,
+    INDEXER_WORKLOAD,
+    indexer_problem,
+    make_device_indexer_problem,
 )

@@ -375,3 +375,95 @@ def _row_rank(tensor: torch.Tensor, flat_rows: int) -> int:
         if lead == flat_rows:
             return tensor.dim() - r
     raise ValueError("row count does not match a leading product of the shape")
+
+
+# ---------------------------------------------------------------------------
+# Dense lightning-indexer gradient with KL loss: inputs
+# ---------------------------------------------------------------------------
+INDEXER_WORKLOAD = "indexer_kl_tnd_2048-4096-4096-6144_n128_g64_d128_causal"
+
+
+@dataclass
+class IndexerProblem:
+    """Inputs of the dense lightning-indexer gradient (flattened like Problem):
+    q [T1, N1, D], q_rope [T1, N1, Dr], k [T2, D], k_rope [T2, Dr] (the main
+    attention, one key head), q_index [T1, G, Di], k_index [T2, Di] (one indexer
+    key head), weights [T1, G].  The softmax statistics of both distributions are
+    not made here: the caller derives them (oracle or GPU forward)."""
+
+    name: str
+    layout: str
+    B: int
+    S1: int
+    S2: int
+    T1: int
+    T2: int
+    N1: int
+    G: int
+    Di: int
+    D: int
+    Dr: int
+    sparse_mode: int
+    scale: float
+    seqlens_q: Optional[np.ndarray]  # BSND: per-batch lengths or None; TND: cumulative ends
+    seqlens_kv: Optional[np.ndarray]
+    q: np.ndarray
+    q_rope: np.ndarray
+    k: np.ndarray
+    k_rope: np.ndarray
+    q_index: np.ndarray
+    k_index: np.ndarray
+    weights: np.ndarray
+    meta: Dict = field(default_factory=dict)
+
+
+def indexer_problem(seed: int, layout: str = "TND", B: int = 1, S1: int = 0, S2: int = 0, seqlens_q=None,
+                    seqlens_kv=None, N1: int = 4, G: int = 4, Di: int = 8, D: int = 8, Dr: int = 4,
+                    sparse_mode: int = 3, scale: Optional[float] = None, round_bf16: bool = True) -> IndexerProblem:
+    """Small or medium indexer-gradient problem.  q / k / q_rope / k_rope /
+    q_index / k_index are N(0, 1); weights are N(0, 1) / sqrt(G); all rounded to
+    bf16 unless round_bf16 is False.  For TND, seqlens_q/kv are per-sequence
+    lengths here and are returned cumulative (int64)."""
+    rng = np.random.default_rng(seed)
+    if layout == "TND":
+        lq = np.asarray(seqlens_q, np.int64)
+        lk = np.asarray(seqlens_kv if seqlens_kv is not None else seqlens_q, np.int64)
+        B = len(lq)
+        T1, T2 = int(lq.sum()), int(lk.sum())
+        sq, skv = np.cumsum(lq).astype(np.int64), np.cumsum(lk).astype(np.int64)
+        S1 = S2 = 0
+    else:
+        T1, T2 = B * S1, B * S2
+        sq = None if seqlens_q is None else np.asarray(seqlens_q, np.int64)
+        skv = None if seqlens_kv is None else np.asarray(seqlens_kv, np.int64)
+    rnd = bf16_round if round_bf16 else (lambda a: a.astype(np.float64))
+    q = rnd(rng.standard_normal((T1, N1, D)))
+    qr = rnd(rng.standard_normal((T1, N1, Dr)))
+    k = rnd(rng.standard_normal((T2, D)))
+    kr = rnd(rng.standard_normal((T2, Dr)))
+    qi = rnd(rng.standard_normal((T1, G, Di)))
+    ki = rnd(rng.standard_normal((T2, Di)))
+    w = rnd(rng.standard_normal((T1, G)) / math.sqrt(G))
+    sc = 1.0 / math.sqrt(D + Dr) if scale is None else scale
+    return IndexerProblem(f"indexer{seed}", layout, B, S1, S2, T1, T2, N1, G, Di, D, Dr, sparse_mode, sc, sq, skv,
+                          q, qr, k, kr, qi, ki, w, meta={"seed": seed})
+
+
+def make_device_indexer_problem(device="cuda", seed: int = 3000, seqs=(2048, 4096, 4096, 6144), N1: int = 128,
+                                G: int = 64, Di: int = 128) -> IndexerProblem:
+    """The indexer-gradient benchmark workload generated on the device (torch
+    bf16 tensors in the library's TND layouts: q [T1,N1,512], key [T2,1,512],
+    q_index [T1,G,Di], k_index [T2,1,Di], weights [T1,G]); causal (mode 3)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    D, Dr = 512, 64
+    lens = [int(x) for x in seqs]
+    T = int(sum(lens))
+    cu = torch.tensor(np.cumsum(lens), dtype=torch.int64, device=device)
+
+    def rnd(*shape, s=1.0):
+        return (torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * s).to(torch.bfloat16)
+
+    return IndexerProblem(INDEXER_WORKLOAD, "TND", len(lens), 0, 0, T, T, N1, G, Di, D, Dr, 3, _scale(D, Dr), cu, cu,
+                          rnd(T, N1, D), rnd(T, N1, Dr), rnd(T, 1, D), rnd(T, 1, Dr), rnd(T, G, Di), rnd(T, 1, Di),
+                          rnd(T, G, s=1.0 / math.sqrt(G)), meta={"seed": seed, "device": True})
