@@ -1,6 +1,7 @@
 /*
- * sfa.h - C ABI of libsfa: top-k sparse attention backward (SparseFlashAttentionGrad)
- * and the dense varlen FlashAttention backward (FlashAttentionUnpaddingScoreGrad)
+ * sfa.h - C ABI of libsfa: top-k sparse attention backward (SparseFlashAttentionGrad),
+ * the dense varlen FlashAttention backward (FlashAttentionUnpaddingScoreGrad) and
+ * the dense lightning-indexer gradient with KL loss (DenseLightningIndexerGradKLLoss)
  * for NVIDIA B200 (sm_100a).
  *
  * Conventions shared by every entry point
@@ -304,12 +305,69 @@ sfa_status fa_fwd(const void *q, const void *k, const void *v, const int64_t *ac
                   float *softmax_sum);
 
 /* ------------------------------------------------------------------------- */
+/* Dense lightning-indexer gradient with KL loss (DenseLightningIndexerGradKLLoss) */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Problem sizes of an indexer-gradient call.
+ *   layout  SFA_LAYOUT_BSND: query [B,S1,N1,D], queryRope [B,S1,N1,Dr], key [B,S2,1,D],
+ *                            keyRope [B,S2,1,Dr], queryIndex [B,S1,G,Di], keyIndex
+ *                            [B,S2,1,Di], weights [B,S1,G], softmaxMax/Sum [B,S1,N1],
+ *                            softmaxMaxIndex/SumIndex [B,S1]; T1/T2 ignored.
+ *           SFA_LAYOUT_TND:  the same with [T1,...] / [T2,...] leading dims; S1/S2 ignored.
+ *   Supported: D = 512, Dr = 64 (the main attention's MLA shape, one key head),
+ *   N1 in {64, 128}, G = 64, Di = 128 (one indexer key head), B in [1, 256].
+ */
+typedef struct lig_shape {
+    int32_t layout;
+    int32_t dtype;  /* SFA_DTYPE_BF16 | SFA_DTYPE_FP16 for every 16-bit tensor */
+    int64_t B;
+    int64_t S1, S2;
+    int64_t T1, T2;
+    int64_t N1;     /* main-attention query heads */
+    int64_t D, Dr;
+    int64_t G;      /* indexer query heads */
+    int64_t Di;     /* indexer head dim */
+} lig_shape;
+
+sfa_status lig_kl_grad_workspace_size(const lig_shape *shape, int64_t sparse_mode, size_t *workspace_bytes);
+
+/*
+ * DenseLightningIndexerGradKLLoss README (功能说明, formulas 1-4; 参数说明 for the
+ * argument list).  Per query token t and every key row j it sees (sparse_mode 0:
+ * its whole batch / sequence; 3: j <= pos + S2_b - S1_b):
+ *   I_tj  = sum_g W[t,g] ReLU(queryIndex[t,g] . keyIndex[j])
+ *   p_tj  = (1/N1) sum_h exp(scale * Q~[t,h].K~[j] - softmaxMax[t,h]) / softmaxSum[t,h]
+ *           (Q~ = query || queryRope, K~ = key || keyRope; a softmaxSum of 0 gives 0)
+ *   sI_tj = exp(I_tj - softmaxMaxIndex[t]) / softmaxSumIndex[t]
+ *   loss  = sum_t sum_j p_tj (log p_tj - log sI_tj)          (0 where p = 0)
+ *   dI    = sI - p;  dWeights[t,g] = sum_j dI_tj ReLU(S_tgj)   (S = queryIndex . keyIndex)
+ *   dQueryIndex[t,g] = sum_j dI_tj W[t,g] [S_tgj > 0] keyIndex[j]
+ *   dKeyIndex[j]     = sum_{t,g} dI_tj W[t,g] [S_tgj > 0] queryIndex[t,g]
+ * Statistics are used as given (they are the forward's outputs).  A token with no
+ * visible key (BSND padding rows included) gets zero dQueryIndex / dWeights rows.
+ *   actual_seq_lengths_query / _key: DEVICE int64 [B] (the page's INT64 tensors):
+ *     BSND per-batch valid lengths (NULL = S1 / S2), TND cumulative end offsets
+ *     (required).  pre_tokens / next_tokens are ignored (modes 0 and 3 only).
+ *   Outputs: d_query_index [.., G, Di], d_key_index [.., 1, Di], d_weights [.., G]
+ *     (16-bit), loss: one fp32 (device).  dKeyIndex is summed with fp32 atomics
+ *     (run-to-run differences in the last bits); loss is a fixed-order sum.
+ */
+sfa_status lig_kl_grad(const void *query, const void *key, const void *query_index, const void *key_index,
+                       const void *weights, const float *softmax_max, const float *softmax_sum,
+                       const float *softmax_max_index, const float *softmax_sum_index, const void *query_rope,
+                       const void *key_rope, const int64_t *actual_seq_lengths_query,
+                       const int64_t *actual_seq_lengths_key, double scale, int64_t sparse_mode, int64_t pre_tokens,
+                       int64_t next_tokens, const lig_shape *shape, void *workspace, size_t workspace_bytes,
+                       sfa_stream_t stream, void *d_query_index, void *d_key_index, void *d_weights, float *loss);
+
+/* ------------------------------------------------------------------------- */
 /* Diagnostics                                                                */
 /* ------------------------------------------------------------------------- */
 
 /*
  * Timing hook for benchmarks: the next sfa_grad / sfa_grad_rows / sfa_fwd /
- * fa_grad call on the calling thread records `event_before` immediately before
+ * fa_grad / lig_kl_grad call on the calling thread records `event_before` immediately before
  * and `event_after` immediately after launching its main kernel (the fused
  * tensor-core kernel or the CUDA-core kernel), on that call's stream.  Both are cudaEvent_t
  * handles created by the caller; NULL clears the hook.  Consumed by one call.
@@ -320,7 +378,8 @@ sfa_status sfa_set_kernel_events(void *event_before, void *event_after);
  * Failure detection.  Every wait of the fused kernels on an mbarrier (a load, an
  * MMA or another warp role) is bounded: past the limit the kernel writes a
  * non-zero wait-site code into its workspace's error word (the first 4 bytes of
- * the workspace of sfa_grad / sfa_grad_rows / sfa_fwd / fa_grad / fa_fwd, zeroed
+ * the workspace of sfa_grad / sfa_grad_rows / sfa_fwd / fa_grad / fa_fwd /
+ * lig_kl_grad, zeroed
  * at the start of each such call), stops issuing work, drains what it issued,
  * frees its tensor memory and exits; the CUDA context stays usable.  (The pages
  * name only an AI Core "timeout or trap" error for oversized problems, 约束说明 of

@@ -35,6 +35,13 @@ class FaShape(ctypes.Structure):
                 ("D", ctypes.c_int64)]
 
 
+class LigShape(ctypes.Structure):
+    _fields_ = [("layout", ctypes.c_int32), ("dtype", ctypes.c_int32), ("B", ctypes.c_int64),
+                ("S1", ctypes.c_int64), ("S2", ctypes.c_int64), ("T1", ctypes.c_int64), ("T2", ctypes.c_int64),
+                ("N1", ctypes.c_int64), ("D", ctypes.c_int64), ("Dr", ctypes.c_int64), ("G", ctypes.c_int64),
+                ("Di", ctypes.c_int64)]
+
+
 class SfaError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(f"{status}: {msg}")
@@ -50,6 +57,7 @@ _SZ = ctypes.c_size_t
 _PSZ = ctypes.POINTER(ctypes.c_size_t)
 _PSH = ctypes.POINTER(SfaShape)
 _PFA = ctypes.POINTER(FaShape)
+_PLG = ctypes.POINTER(LigShape)
 
 SIGNATURES = {
     "sfa_grad_workspace_size": [_PSH, _I64, _I64, _I32, _PSZ],
@@ -73,6 +81,9 @@ SIGNATURES = {
     "sfa_dkv_finalize": [_V, _PSH, _I32, _V, _V, _V, _V],
     "sfa_grad_noalloc": [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _F, _I64, _I64, _I64, _I64, _I32, _PSH, _V,
                          _V, _V, _V, _V, _V],
+    "lig_kl_grad_workspace_size": [_PLG, _I64, _PSZ],
+    "lig_kl_grad": [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _Dbl, _I64, _I64, _I64, _PLG, _V, _SZ, _V,
+                    _V, _V, _V, _V],
     "sfa_status_string": [_I32],
     "sfa_last_error_string": [],
     "sfa_version": [],

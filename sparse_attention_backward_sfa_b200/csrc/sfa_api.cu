@@ -589,3 +589,135 @@ sfa_status fa_fwd(const void* q, const void* k, const void* v, const int64_t* ac
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Dense lightning-indexer gradient with KL loss
+// ---------------------------------------------------------------------------
+namespace {
+
+struct LigWs {
+    size_t ctrl, sq, skv, nkeys, kvrow, order, loss, dki, total;
+};
+
+LigWs lig_ws_layout(const lig_shape* s) {
+    LigWs w;
+    size_t o = 0;
+    w.ctrl = o;  o += 256;
+    w.sq = o;    o = align256(o + (size_t)s->B * 4);
+    w.skv = o;   o = align256(o + (size_t)s->B * 4);
+    w.nkeys = o; o = align256(o + (size_t)s->T1 * 4);
+    w.kvrow = o; o = align256(o + (size_t)s->T1 * 4);
+    w.order = o; o = align256(o + (size_t)s->T1 * 4);
+    w.loss = o;  o = align256(o + (size_t)s->T1 * 4);
+    w.dki = o;   o = align256(o + (size_t)s->T2 * s->Di * 4);
+    w.total = o;
+    return w;
+}
+
+// Validates a lig_shape (filling T1 / T2 for BSND) into `z`.
+sfa_status check_lig(const lig_shape* in, int64_t sparse_mode, lig_shape* z) {
+    if (!in) return fail(SFA_ERR_NULLPTR, "shape is NULL");
+    *z = *in;
+    if (z->layout != SFA_LAYOUT_BSND && z->layout != SFA_LAYOUT_TND)
+        return fail(SFA_ERR_INVALID, "layout %d", (int)z->layout);
+    if (z->dtype != SFA_DTYPE_BF16 && z->dtype != SFA_DTYPE_FP16) return fail(SFA_ERR_INVALID, "dtype %d", (int)z->dtype);
+    if (z->D != kD || z->Dr != kDr) return fail(SFA_ERR_INVALID, "D=%lld Dr=%lld: only 512 / 64", (long long)z->D,
+                                                (long long)z->Dr);
+    if (z->N1 != 64 && z->N1 != 128) return fail(SFA_ERR_INVALID, "N1=%lld: 64 or 128", (long long)z->N1);
+    if (z->G != kLigG || z->Di != kLigDi)
+        return fail(SFA_ERR_INVALID, "G=%lld Di=%lld: only %d / %d", (long long)z->G, (long long)z->Di, kLigG, kLigDi);
+    if (z->B < 1 || z->B > 256) return fail(SFA_ERR_INVALID, "B=%lld outside [1,256]", (long long)z->B);
+    if (sparse_mode != 0 && sparse_mode != 3) return fail(SFA_ERR_INVALID, "sparse_mode %lld", (long long)sparse_mode);
+    if (z->layout == SFA_LAYOUT_BSND) {
+        if (z->S1 < 1 || z->S2 < 1 || z->S1 > (1 << 17) || z->S2 > (1 << 17))
+            return fail(SFA_ERR_INVALID, "S1=%lld S2=%lld outside [1,128K]", (long long)z->S1, (long long)z->S2);
+        z->T1 = z->B * z->S1;
+        z->T2 = z->B * z->S2;
+    } else if (z->T1 < 1 || z->T2 < 1) {
+        return fail(SFA_ERR_INVALID, "T1=%lld T2=%lld", (long long)z->T1, (long long)z->T2);
+    }
+    if (z->T1 * (int64_t)kLigG >= ((int64_t)1 << 31) || z->T1 * z->N1 >= ((int64_t)1 << 31) ||
+        z->T2 >= ((int64_t)1 << 31))
+        return fail(SFA_ERR_INVALID, "T1=%lld T2=%lld too large", (long long)z->T1, (long long)z->T2);
+    return SFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sfa_status lig_kl_grad_workspace_size(const lig_shape* shape, int64_t sparse_mode, size_t* workspace_bytes) {
+    g_last_error.clear();
+    if (!workspace_bytes) return fail(SFA_ERR_NULLPTR, "workspace_bytes is NULL");
+    lig_shape z;
+    sfa_status st = check_lig(shape, sparse_mode, &z);
+    if (st != SFA_OK) return st;
+    *workspace_bytes = lig_ws_layout(&z).total;
+    return SFA_OK;
+}
+
+sfa_status lig_kl_grad(const void* query, const void* key, const void* query_index, const void* key_index,
+                       const void* weights, const float* softmax_max, const float* softmax_sum,
+                       const float* softmax_max_index, const float* softmax_sum_index, const void* query_rope,
+                       const void* key_rope, const int64_t* actual_seq_lengths_query,
+                       const int64_t* actual_seq_lengths_key, double scale, int64_t sparse_mode, int64_t pre_tokens,
+                       int64_t next_tokens, const lig_shape* shape, void* workspace, size_t workspace_bytes,
+                       sfa_stream_t stream, void* d_query_index, void* d_key_index, void* d_weights, float* loss) {
+    (void)pre_tokens;
+    (void)next_tokens;
+    g_last_error.clear();
+    lig_shape z;
+    sfa_status st = check_lig(shape, sparse_mode, &z);
+    if (st != SFA_OK) return st;
+    if (!query || !key || !query_index || !key_index || !weights || !softmax_max || !softmax_sum ||
+        !softmax_max_index || !softmax_sum_index || !query_rope || !key_rope || !workspace || !d_query_index ||
+        !d_key_index || !d_weights || !loss)
+        return fail(SFA_ERR_NULLPTR, "a required pointer is NULL");
+    if (z.layout == SFA_LAYOUT_TND && (!actual_seq_lengths_query || !actual_seq_lengths_key))
+        return fail(SFA_ERR_NULLPTR, "TND needs actual_seq_lengths_query and actual_seq_lengths_key");
+    if (!(scale == scale) || scale > 1e30 || scale < -1e30) return fail(SFA_ERR_INVALID, "scale is not finite");
+    const void* tma_ptrs[] = {query, key, query_index, key_index, query_rope, key_rope};
+    for (const void* ptr : tma_ptrs)
+        if (((uintptr_t)ptr & 15u) != 0) return fail(SFA_ERR_INVALID, "16-bit tensors must be 16-byte aligned");
+    if (((uintptr_t)workspace & 255u) != 0) return fail(SFA_ERR_INVALID, "workspace not 256-byte aligned");
+    const LigWs ws = lig_ws_layout(&z);
+    if (workspace_bytes < ws.total)
+        return fail(SFA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, ws.total);
+    cudaStream_t s = (cudaStream_t)stream;
+    char* w = (char*)workspace;
+
+    sfa_shape ss;
+    memset(&ss, 0, sizeof ss);
+    ss.layout = z.layout; ss.dtype = z.dtype; ss.B = z.B; ss.S1 = z.S1; ss.S2 = z.S2;
+    Sizes sz;
+    sz.T1 = z.T1;
+    sz.T2 = z.T2;
+    const SeqDesc sd = seq_desc(&ss, sz, nullptr, nullptr);
+
+    LigArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = query; a.qr = query_rope; a.k = key; a.kr = key_rope; a.qi = query_index; a.ki = key_index;
+    a.weights = weights; a.smax = softmax_max; a.ssum = softmax_sum; a.smax_i = softmax_max_index;
+    a.ssum_i = softmax_sum_index;
+    a.nkeys = (int32_t*)(w + ws.nkeys); a.kvrow = (int32_t*)(w + ws.kvrow); a.order = (int32_t*)(w + ws.order);
+    a.dki_acc = (float*)(w + ws.dki); a.loss_rows = (float*)(w + ws.loss);
+    a.dqi = d_query_index; a.dw = d_weights; a.err = (int*)(w + ws.ctrl);
+    a.T1 = z.T1; a.T2 = z.T2; a.N1 = z.N1; a.scale = (float)scale; a.dtype = z.dtype;
+
+    SFA_CUDA(cudaMemsetAsync(w + ws.ctrl, 0, 256, s), "zero control word");
+    SFA_CUDA(cudaMemsetAsync(a.dki_acc, 0, (size_t)z.T2 * z.Di * 4, s), "zero dKeyIndex accumulator");
+    SFA_CUDA(launch_lig_prep(sd, (int)sparse_mode, actual_seq_lengths_query, actual_seq_lengths_key,
+                             (int32_t*)(w + ws.sq), (int32_t*)(w + ws.skv), (int32_t*)a.nkeys, (int32_t*)a.kvrow, s),
+             "row bookkeeping");
+    SFA_CUDA(launch_order(a.nkeys, 0, z.T1, (int32_t*)a.order, a.err, s), "work order");
+    {
+        KernelEvents ev(s);
+        SFA_CUDA(launch_lig_fused(a, s), "fused indexer gradient");
+    }
+    SFA_CUDA(launch_lig_finish(z.dtype, a.dki_acc, z.T2, d_key_index, a.loss_rows, z.T1, loss, s),
+             "dKeyIndex cast and loss sum");
+    return SFA_OK;
+}
+
+}  // extern "C"
+

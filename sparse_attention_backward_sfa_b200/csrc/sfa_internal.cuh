@@ -250,6 +250,31 @@ size_t fa_fused_items(const int64_t* cu_q, const int64_t* cu_kv, int64_t B, int6
 inline size_t fa_fused_max_items(int64_t B, int64_t T2, int64_t Nkv) { return (size_t)Nkv * (T2 / 128 + B + 1); }
 cudaError_t launch_fa_bwd_fused(int dtype, const FaFusedArgs& a, cudaStream_t st);
 // Sets the message returned by sfa_last_error_string() on the calling thread.
+// ---------------------------------------------------------------------------
+// Dense lightning-indexer gradient with KL loss (DenseLightningIndexerGradKLLoss)
+constexpr int kLigG = 64;    // indexer query heads the fused kernel supports
+constexpr int kLigDi = 128;  // indexer head dim the fused kernel supports
+struct LigArgs {
+    const void *q, *qr, *k, *kr, *qi, *ki, *weights;
+    const float *smax, *ssum, *smax_i, *ssum_i;
+    const int32_t *nkeys, *kvrow, *order;
+    float* dki_acc;   // [T2][Di] fp32, zeroed by the caller
+    float* loss_rows; // [T1]
+    void *dqi, *dw;
+    int* err;
+    int64_t T1, T2, N1;
+    float scale;
+    int dtype;
+};
+// Row bookkeeping: int64 sequence lengths (null for BSND full lengths) copied to
+// int32, then per query row its visible key count and first key row.
+cudaError_t launch_lig_prep(const SeqDesc& sd, int mode, const int64_t* sq64, const int64_t* skv64, int32_t* sq32,
+                            int32_t* skv32, int32_t* nkeys, int32_t* kvrow, cudaStream_t st);
+cudaError_t launch_lig_fused(const LigArgs& a, cudaStream_t st);
+// dKeyIndex from the fp32 accumulator, and the loss as the fixed-order sum of the rows' losses.
+cudaError_t launch_lig_finish(int dtype, const float* dki_acc, int64_t T2, void* dki, const float* loss_rows,
+                              int64_t T1, float* loss, cudaStream_t st);
+
 void set_last_error(const char* msg);
 // Limit of every device-side mbarrier wait of the fused kernels launched from the
 // calling thread (sfa_set_wait_limit; 4 s by default).

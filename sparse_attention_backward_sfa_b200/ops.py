@@ -281,6 +281,73 @@ def fa_fwd(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, scale: float, sparse_mode: i
     return out, smax, ssum
 
 
+def lig_shape(query: torch.Tensor, key: torch.Tensor, query_index: torch.Tensor, key_index: torch.Tensor,
+              layout: str, actual_seq_lengths_query=None) -> N.LigShape:
+    """Sizes of a dense lightning-indexer gradient call from its tensors."""
+    s = N.LigShape()
+    _need(query.dtype in _DT, "query must be bf16 or fp16")
+    s.dtype = _DT[query.dtype]
+    if layout == "BSND":
+        _need(query.dim() == 4 and key.dim() == 4, "BSND tensors are 4-D")
+        s.layout = N.LAYOUT_BSND
+        s.B, s.S1, s.N1, s.D = query.shape
+        _, s.S2, _, _ = key.shape
+        s.T1, s.T2 = s.B * s.S1, s.B * s.S2
+        _, _, s.G, s.Di = query_index.shape
+    elif layout == "TND":
+        _need(query.dim() == 3 and key.dim() == 3, "TND tensors are 3-D")
+        s.layout = N.LAYOUT_TND
+        s.T1, s.N1, s.D = query.shape
+        s.T2 = key.shape[0]
+        s.S1 = s.S2 = 0
+        _need(actual_seq_lengths_query is not None, "TND needs actual sequence lengths")
+        s.B = actual_seq_lengths_query.numel()
+        _, s.G, s.Di = query_index.shape
+    else:
+        raise ValueError(f"layout {layout!r}")
+    s.Dr = 64
+    return s
+
+
+def lig_kl_grad_workspace_size(shape: N.LigShape, sparse_mode: int) -> int:
+    n = ctypes.c_size_t()
+    N.check(N.load().lig_kl_grad_workspace_size(ctypes.byref(shape), int(sparse_mode), ctypes.byref(n)))
+    return n.value
+
+
+def lig_kl_grad(query, key, query_index, key_index, weights, softmax_max, softmax_sum, softmax_max_index,
+                softmax_sum_index, query_rope, key_rope, *, scale: float, layout: str, sparse_mode: int,
+                actual_seq_lengths_query=None, actual_seq_lengths_key=None, pre_tokens: int = 65536,
+                next_tokens: int = 65536, workspace=None, outputs=None, stream=None):
+    """Dense lightning-indexer gradient with KL loss (lig_kl_grad in include/sfa.h).
+    Returns (dQueryIndex, dKeyIndex, dWeights, loss) with loss a 1-element fp32 CUDA tensor."""
+    lib = N.load()
+    for name, t in (("query", query), ("key", key), ("query_index", query_index), ("key_index", key_index),
+                    ("weights", weights), ("query_rope", query_rope), ("key_rope", key_rope)):
+        _check16(name, t, query.dtype)
+    for name, t in (("softmax_max", softmax_max), ("softmax_sum", softmax_sum),
+                    ("softmax_max_index", softmax_max_index), ("softmax_sum_index", softmax_sum_index)):
+        _need(t.is_cuda and t.is_contiguous() and t.dtype == torch.float32, f"{name}: contiguous fp32 CUDA tensor")
+    for name, t in (("actual_seq_lengths_query", actual_seq_lengths_query),
+                    ("actual_seq_lengths_key", actual_seq_lengths_key)):
+        _need(t is None or (t.is_cuda and t.dtype == torch.int64 and t.is_contiguous()),
+              f"{name}: int64 CUDA tensor")
+    shape = lig_shape(query, key, query_index, key_index, layout, actual_seq_lengths_query)
+    need = lig_kl_grad_workspace_size(shape, sparse_mode)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=query.device)
+    if outputs is None:
+        outputs = (torch.empty_like(query_index), torch.empty_like(key_index), torch.empty_like(weights),
+                   torch.empty(1, dtype=torch.float32, device=query.device))
+    dqi, dki, dw, loss = outputs
+    N.check(lib.lig_kl_grad(_p(query), _p(key), _p(query_index), _p(key_index), _p(weights), _p(softmax_max),
+                            _p(softmax_sum), _p(softmax_max_index), _p(softmax_sum_index), _p(query_rope),
+                            _p(key_rope), _p(actual_seq_lengths_query), _p(actual_seq_lengths_key), float(scale),
+                            int(sparse_mode), int(pre_tokens), int(next_tokens), ctypes.byref(shape), _p(workspace),
+                            workspace.numel(), _stream(stream), _p(dqi), _p(dki), _p(dw), _p(loss)))
+    return dqi, dki, dw, loss
+
+
 def workspace_status(workspace: torch.Tensor, stream=None) -> int:
     """Waits for `stream` and returns the wait-site code the last call left in the workspace's
     error word: 0 when every device-side wait was satisfied, else the site that gave up."""

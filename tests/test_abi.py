@@ -138,3 +138,45 @@ def test_fa_host_errors(lib):
     st = lib.fa_grad(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ok, ok, 0.08, 1.0, 0, 0, 8, 3, 0, ctypes.byref(s),
                      FAKE, 1 << 40, None, FAKE, FAKE, FAKE)
     assert st == N.SFA_ERR_INVALID  # head_num != Nq
+
+
+def _lig_shape(**kw):
+    s = N.LigShape()
+    d = dict(layout=0, dtype=0, B=1, S1=64, S2=256, T1=0, T2=0, N1=128, D=512, Dr=64, G=64, Di=128)
+    d.update(kw)
+    for k, v in d.items():
+        setattr(s, k, v)
+    return s
+
+
+@pytest.mark.parametrize("kw,mode,code", [
+    ({}, 3, N.SFA_OK),
+    ({}, 0, N.SFA_OK),
+    (dict(N1=64), 3, N.SFA_OK),
+    (dict(layout=1, T1=300, T2=300, B=2), 3, N.SFA_OK),
+    ({}, 1, N.SFA_ERR_INVALID),
+    (dict(N1=32), 3, N.SFA_ERR_INVALID),
+    (dict(G=32), 3, N.SFA_ERR_INVALID),
+    (dict(Di=64), 3, N.SFA_ERR_INVALID),
+    (dict(D=256), 3, N.SFA_ERR_INVALID),
+    (dict(B=0), 3, N.SFA_ERR_INVALID),
+    (dict(layout=2), 3, N.SFA_ERR_INVALID),
+    (dict(dtype=2), 3, N.SFA_ERR_INVALID),
+    (dict(layout=1, T1=0, T2=10, B=1), 3, N.SFA_ERR_INVALID),
+])
+def test_lig_workspace_size_validation(lib, kw, mode, code):
+    n = ctypes.c_size_t(0)
+    sh = _lig_shape(**kw)
+    assert lib.lig_kl_grad_workspace_size(ctypes.byref(sh), mode, ctypes.byref(n)) == code
+    if code == N.SFA_OK:
+        T2 = sh.T2 if sh.layout == 1 else sh.B * sh.S2
+        assert n.value >= T2 * 128 * 4  # holds the fp32 dKeyIndex accumulator
+
+
+def test_lig_rejects_null_pointers_before_launch(lib):
+    sh = _lig_shape()
+    n = ctypes.c_size_t(0)
+    assert lib.lig_kl_grad_workspace_size(ctypes.byref(sh), 3, ctypes.byref(n)) == N.SFA_OK
+    args = [None] * 13 + [0.05, 3, 0, 0, ctypes.byref(sh), None, n.value, None] + [None] * 4
+    assert lib.lig_kl_grad(*args) == N.SFA_ERR_NULLPTR
+    assert lib.lig_kl_grad_workspace_size(None, 3, ctypes.byref(n)) == N.SFA_ERR_NULLPTR
