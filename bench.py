@@ -46,6 +46,7 @@ PROFILE_SUMMARIES = {
     4: ("sfa_bwd_fused_kernel_workload4.md", ("sfa_fused.cu", "tc_common.cuh")),
     2: ("fa_bwd_fused_kernel_workload2.md", ("fa_fused.cu", "tc_common.cuh")),
     "fwd4": ("sfa_fwd_fused_kernel_workload4.md", ("sfa_fwd_fused.cu", "tc_common.cuh")),
+    "lig": ("lig_fused_kernel_indexer.md", ("lig_fused.cu", "tc_common.cuh")),
 }
 
 
@@ -367,6 +368,146 @@ def run_fwd(args, local_rank):
             "gpu_launches": (4 if p.N1 == 128 else 2) * args.steps, "clocks": clk.summary()}
 
 
+def indexer_flop_per_pair(N1: int, G: int, Di: int) -> int:
+    """Algorithmic FLOP of the indexer gradient per visible (query row, key) pair:
+    the main scores (2*N1*576) and the indexer's three contractions (scores, dq~I, dK~I)."""
+    return 2 * N1 * 576 + 6 * G * Di
+
+
+def indexer_inputs(dev, seqs=None):
+    """The indexer-gradient workload with consistent statistics: the main attention's
+    from sfa_fwd over every causal block, the indexer's max / sum of exp(I - max) over
+    the visible keys computed with torch in row chunks (input preparation)."""
+    import torch
+    import sparse_attention_backward_sfa_b200 as S
+    from workloads import make_device_indexer_problem
+    p = make_device_indexer_problem(device=dev, **({"seqs": seqs} if seqs else {}))
+    lens = np.diff(np.concatenate([[0], p.seqlens_q.cpu().numpy()])).astype(np.int64)
+    bs = 16
+    nb = int(-(-lens.max() // bs))
+    cu32 = p.seqlens_q.to(torch.int32)
+    idx = torch.arange(nb, dtype=torch.int32, device=dev).repeat(p.T1, 1).reshape(p.T1, 1, nb).contiguous()
+    _, smax, ssum = S.sfa_fwd(p.q, p.k, p.k, idx, p.q_rope, p.k_rope, scale=p.scale, sparse_block_size=bs,
+                              layout="TND", sparse_mode=3, actual_seq_lengths_q=cu32, actual_seq_lengths_kv=cu32)
+    del idx
+    mi = torch.zeros(p.T1, dtype=torch.float32, device=dev)
+    li = torch.zeros(p.T1, dtype=torch.float32, device=dev)
+    ki = p.k_index.reshape(p.T2, p.Di).float()
+    start = 0
+    for L in lens.tolist():
+        kseq = ki[start:start + L]
+        for r0 in range(0, L, 256):
+            r1 = min(L, r0 + 256)
+            qi = p.q_index[start + r0:start + r1].float()                      # [r, G, Di]
+            w = p.weights[start + r0:start + r1].float()                       # [r, G]
+            I = torch.einsum("rg,rgj->rj", w, torch.relu(torch.einsum("rgd,jd->rgj", qi, kseq)))
+            pos = torch.arange(r0, r1, device=dev)[:, None]
+            I = I.masked_fill(torch.arange(L, device=dev)[None, :] > pos, float("-inf"))
+            m = I.max(dim=1).values
+            mi[start + r0:start + r1] = m
+            li[start + r0:start + r1] = torch.exp(I - m[:, None]).sum(dim=1)
+        start += L
+    return p, lens, smax, ssum, mi, li
+
+
+def run_indexer(args, local_rank):
+    """The dense lightning-indexer gradient with KL loss (lig_kl_grad), one GPU, TND
+    sequences {2048, 4096, 4096, 6144}, N1 = 128, G = 64, Di = 128, causal."""
+    import torch
+    import sparse_attention_backward_sfa_b200 as S
+    from sparse_attention_backward_sfa_b200 import _native as N
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lib = N.load()
+    p, lens, smax, ssum, mi, li = indexer_inputs(dev, SEQS if args.seqs else None)
+    pairs = int(sum(int(L) * (int(L) + 1) // 2 for L in lens))
+    flop = pairs * indexer_flop_per_pair(p.N1, p.G, p.Di)
+    shape = S.lig_shape(p.q, p.k, p.q_index, p.k_index, "TND", p.seqlens_q)
+    ws = torch.empty(S.lig_kl_grad_workspace_size(shape, 3), dtype=torch.uint8, device=dev)
+    outs = (torch.empty_like(p.q_index), torch.empty_like(p.k_index), torch.empty_like(p.weights),
+            torch.empty(1, dtype=torch.float32, device=dev))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            N.check(lib.sfa_set_kernel_events(ctypes_ptr(ev[0]), ctypes_ptr(ev[1])))
+        S.lig_kl_grad(p.q, p.k, p.q_index, p.k_index, p.weights, smax, ssum, mi, li, p.q_rope, p.k_rope,
+                      scale=p.scale, layout="TND", sparse_mode=3, actual_seq_lengths_query=p.seqlens_q,
+                      actual_seq_lengths_key=p.seqlens_kv, workspace=ws, outputs=outs)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        a.record(stream)
+        b.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms_step = t0.elapsed_time(t1) / args.steps
+    kern = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    err = int(ws[:4].view(torch.int32).item())
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    cpu = None
+    if not args.no_cpu_baseline:
+        cpu = indexer_cpu_baseline(p, lens, smax, ssum, mi, li, args.cpu_budget)
+    from workloads import INDEXER_WORKLOAD
+    return {"metric": "lightning-indexer KL-loss backward TFLOP/s (bf16, 2*N1*576 + 6*G*Di FLOP per visible pair)",
+            "value": flop / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": INDEXER_WORKLOAD if not args.seqs else f"indexer_kl_tnd_{args.seqs}",
+                       "N1": p.N1, "G": p.G, "Di": p.Di, "visible_pairs": pairs,
+                       "l2": "inputs larger than L2 (q 2.4 GB per step)"},
+            "roofline": {"bound": "tensor", "achieved": flop / (kern * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                         "frac": flop / (kern * 1e-3) / 1e12 / peak, "kernel": "lig_fused_kernel", "kernel_ms": kern,
+                         "peak_source": src,
+                         "traffic": recorded_traffic("lig") if not args.seqs else None},
+            "cpu_baseline": cpu, "gpu_launches": 7 * args.steps, "clocks": clk.summary(),
+            "device_error_word": err}
+
+
+def indexer_cpu_baseline(p, lens, smax, ssum, mi, li, budget_s: float):
+    """The indexer oracle (fp64 numpy, as it stands) on a bounded sample of query rows."""
+    import torch
+    from oracle import indexer_kl_oracle as O
+    from workloads import RowView
+    rng = np.random.default_rng(54321)
+    T1 = p.T1
+    k = p.k.reshape(p.T2, p.D).float().cpu().numpy()
+    kr = p.k_rope.reshape(p.T2, p.Dr).float().cpu().numpy()
+    ki = p.k_index.reshape(p.T2, p.Di).float().cpu().numpy()
+    sq = p.seqlens_q.cpu().numpy()
+    starts = np.concatenate([[0], sq[:-1]])
+    per_pair = indexer_flop_per_pair(p.N1, p.G, p.Di)
+    done, elapsed, flop, n = 0, 0.0, 0, 2
+    while elapsed < budget_s and done < T1:
+        toks = np.sort(rng.choice(T1, size=n, replace=False))
+        views = [RowView(x, toks, T1) for x in (p.q, p.q_rope, p.q_index, p.weights, smax, ssum, mi.reshape(T1, 1),
+                                                li.reshape(T1, 1))]
+        qv, qrv, qiv, wv, mv, lv, miv, liv = views
+        c0 = time.perf_counter()
+        O.indexer_kl_grad(qv, k, qiv, ki, wv, mv, lv, miv, liv, qrv, kr, p.scale, "TND", p.B, 0, 0, sq, sq, 3,
+                          tokens=toks)
+        elapsed += time.perf_counter() - c0
+        for t in toks:
+            b = int(np.searchsorted(sq, t, side="right"))
+            flop += (int(t) - int(starts[b]) + 1) * per_pair
+        done += n
+        n = min(2 * n, 64)
+    return {"value": flop / elapsed / 1e12 if elapsed > 0 else 0.0, "unit": "TFLOP/s",
+            "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"{done} query rows of the indexer workload (fp64 numpy oracle, {elapsed:.1f} s)"}
+
+
 def run_fa(args, rank, world, local_rank):
     """Workload 2: dense varlen FA backward (TND, causal); 1280 FLOP per valid
     (query row, head, key) triple."""
@@ -484,6 +625,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--fwd", action="store_true",
                     help="time the forward (sfa_fwd: out + softmax statistics) instead of the backward")
+    ap.add_argument("--indexer", action="store_true",
+                    help="time the dense lightning-indexer gradient with KL loss (lig_kl_grad)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqs", default=None,
                     help="comma-separated sequence lengths replacing workload 4's (smaller profiling case)")
@@ -527,6 +670,11 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    if args.indexer:
+        if world > 1:
+            raise SystemExit("--indexer: one GPU")
+        print(json.dumps(run_indexer(args, local_rank)), flush=True)
+        return
     if args.fwd:
         if world > 1 or args.workload == 2:
             raise SystemExit("--fwd: one GPU, sparse workloads (3, 4, 5)")

@@ -111,8 +111,8 @@ def indexer_kl_grad(q, k, q_index, k_index, weights, softmax_max, softmax_sum, s
     """
     T1 = len(q)
     T2 = len(k)
-    G, Di = np.asarray(q_index[0]).shape
     sel = None if tokens is None else set(int(t) for t in tokens)
+    G, Di = np.asarray(q_index[0 if sel is None else min(sel)]).shape
     kt_all = np.concatenate([np.asarray(k, dtype), np.asarray(k_rope, dtype)], axis=1)  # [T2, D + Dr]
     ki_all = np.asarray(k_index, dtype)
     dq_index = np.zeros((T1, G, Di), dtype)
@@ -137,8 +137,8 @@ def indexer_kl_grad(q, k, q_index, k_index, weights, softmax_max, softmax_sum, s
             p = prob.sum(axis=0) / N1                                             # [n]
             # indexer distribution with the given statistics
             s, i = indexer_scores(q_index, k_index, weights, t, sp.kv_start, n, dtype)
-            mi = float(softmax_max_index[t])
-            li = float(softmax_sum_index[t])
+            mi = float(np.asarray(softmax_max_index[t]).reshape(-1)[0])
+            li = float(np.asarray(softmax_sum_index[t]).reshape(-1)[0])
             log_si = (i - mi) - np.log(li) if li > 0 else np.full(n, -np.inf)
             si = np.exp(log_si)
             # KL(p || softmax(I)) with 0 log 0 = 0
