@@ -18,10 +18,10 @@
 //    key head each); keys are consecutive rows, so every operand chunk is a 2-D
 //    TMA tile (128 key rows, or the row's N1 / G head rows) of 128 (64 for the
 //    rope) dims, held as two 128-byte-row SW128 halves 16 KB apart in a ring of
-//    32 KB slots.  Per tile the producer loads K0 Q0 .. K4 Q4 (S~^T) then K~I and
-//    q~I; the last two stay in their slots until the gradient MMAs have read them
-//    (the next tile's first four loads use the other slots, so the ring cannot
-//    dead-lock).
+//    32 KB slots that carries K0 Q0 .. K4 Q4 (S~^T) and is released chunk by chunk
+//    as the S~^T MMAs read it, so it prefetches the next tile while the compute
+//    warps work; the K~I tile (double-buffered) and the row's q~I have buffers of
+//    their own, held until the gradient MMAs have read them.
 //  * TMEM (512 columns): S~^T [0,N1), SI^T [128,192), dq~I^T [256,320) (kept
 //    over the row's tiles), dK~I^T [384,512).  TMEM lane = key while the scores
 //    are read (each thread owns one key: the head sums stay in registers) and
@@ -48,18 +48,21 @@ namespace {
 using namespace tc;
 
 constexpr int kThreads = 192;
-constexpr int kSlots = 6;
+constexpr int kSlots = 4;
 constexpr int kSlotBytes = 32768;
 constexpr int kHalf = 16384;
 constexpr int kKeys = 128;
-constexpr int kOffDS = kSlots * kSlotBytes;   // dS [128 keys x 64 heads] 16-bit, one SW128 block
+constexpr int kOffKI = kSlots * kSlotBytes;   // K~I tiles, double-buffered [2][128 keys x Di]
+constexpr int kOffQI = kOffKI + 2 * kSlotBytes;  // q~I of the row [G heads x Di]: two 8 KB SW128 halves
+constexpr int kQIHalf = 8192;
+constexpr int kOffDS = kOffQI + 16384;        // dS [128 keys x 64 heads] 16-bit, one SW128 block
 constexpr int kOffConst = kOffDS + 16384;     // float constants, see below
 // constants: [0,128) max*log2e, [128,256) 1/sum of the main heads, [256,320) W,
 // [320,576) dW partials [4 warps][64], [576,580) loss partials, [580] maxI*log2e,
 // [581] 1/sumI, [582] log(sumI), [583] maxI
 constexpr int kNumConst = 584;
 constexpr int kOffBar = kOffConst + kNumConst * 4;
-constexpr int kNumBars = 2 * kSlots + 8;
+constexpr int kNumBars = 2 * kSlots + 14;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmem = kOffMisc + 16;
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
@@ -150,6 +153,10 @@ __global__ void __launch_bounds__(kThreads, 1) lig_fused_kernel(const __grid_con
     const uint32_t DQI_FULL = bar0 + 8u * (2 * kSlots + 5);
     const uint32_t DQI_FREE = bar0 + 8u * (2 * kSlots + 6);
     const uint32_t DONE = bar0 + 8u * (2 * kSlots + 7);
+    auto KI_FULL = [&](int b) { return bar0 + 8u * (2 * kSlots + 8 + b); };
+    auto KI_EMPTY = [&](int b) { return bar0 + 8u * (2 * kSlots + 10 + b); };
+    const uint32_t QI_FULL = bar0 + 8u * (2 * kSlots + 12);
+    const uint32_t QI_EMPTY = bar0 + 8u * (2 * kSlots + 13);
     float* cst = reinterpret_cast<float*>(smem + kOffConst);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
@@ -171,6 +178,12 @@ __global__ void __launch_bounds__(kThreads, 1) lig_fused_kernel(const __grid_con
         mbar_init(DQI_FULL, 1);
         mbar_init(DQI_FREE, 128);
         mbar_init(DONE, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(KI_FULL(b), 1);
+            mbar_init(KI_EMPTY(b), 1);
+        }
+        mbar_init(QI_FULL, 1);
+        mbar_init(QI_EMPTY, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -188,49 +201,67 @@ __global__ void __launch_bounds__(kThreads, 1) lig_fused_kernel(const __grid_con
 
     if (warp == 4) {
         // =================== TMA producer ===================
+        // per tile: the K~I tile into its double buffer, then K0 Q0 .. K4 Q4 through the ring;
+        // the row's q~I after its first tile's chunks (it is first read by that tile's SI MMA)
         int slot = 0;
         uint32_t sphase = 0;
+        int tile_ctr = 0, row_ctr = 0;
         bool ok = true;
         uint32_t issued_mask = 0;
+        int ki_loads = 0, qi_loads = 0;  // loads issued into the K~I buffers / the q~I buffer
         for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
             const int t = prm.order[w];
             const int n = prm.nkeys[t];
             if (n <= 0) continue;
             const int kv0 = prm.kvrow[t];
             const int ntiles = (n + kKeys - 1) / kKeys;
-            for (int tile = 0; tile < ntiles && ok; ++tile) {
+            for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
                 const int krow = kv0 + tile * kKeys;
-                for (int it = 0; it < 12 && ok; ++it) {
+                const int kb = tile_ctr & 1;
+                if (lane == 0) ok = WAIT(KI_EMPTY(kb), ((tile_ctr >> 1) & 1) ^ 1, 60);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (lane == 0) {
+                    const uint32_t dst = sbase + kOffKI + kb * kSlotBytes;
+                    mbar_expect_tx(KI_FULL(kb), 2 * kKeys * 128u);
+                    for (int h = 0; h < 2; ++h) tma_load_2d(dst + h * kHalf, &prm.mapKI, h * 64, krow, KI_FULL(kb));
+                }
+                ++ki_loads;
+                for (int it = 0; it < 10 && ok; ++it) {  // K0 Q0 K1 Q1 ... K4 Q4 (chunk 4 = the 64 rope dims)
                     if (lane == 0) ok = WAIT(EMPTY(slot), sphase ^ 1, 61);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     if (lane == 0) {
                         const uint32_t dst = sbase + slot * kSlotBytes;
-                        if (it < 10) {  // K0 Q0 K1 Q1 ... K4 Q4 (chunk 4 = the 64 rope dims)
-                            const int c = it >> 1;
-                            const int halves = c < 4 ? 2 : 1;
-                            const bool is_q = it & 1;
-                            mbar_expect_tx(FULL(slot), halves * (is_q ? N1 : kKeys) * 128u);
-                            for (int h = 0; h < halves; ++h) {
-                                const int col = c < 4 ? c * 128 + h * 64 : 0;
-                                if (is_q)
-                                    tma_load_2d(dst + h * kHalf, c < 4 ? &prm.mapQ : &prm.mapQr, col, t * N1, FULL(slot));
-                                else
-                                    tma_load_2d(dst + h * kHalf, c < 4 ? &prm.mapK : &prm.mapKr, col, krow, FULL(slot));
-                            }
-                        } else if (it == 10) {  // K~I tile [128 keys x Di]
-                            mbar_expect_tx(FULL(slot), 2 * kKeys * 128u);
-                            for (int h = 0; h < 2; ++h) tma_load_2d(dst + h * kHalf, &prm.mapKI, h * 64, krow, FULL(slot));
-                        } else {  // q~I of the row [G heads x Di]
-                            mbar_expect_tx(FULL(slot), 2 * kG * 128u);
-                            for (int h = 0; h < 2; ++h) tma_load_2d(dst + h * kHalf, &prm.mapQI, h * 64, t * kG, FULL(slot));
+                        const int c = it >> 1;
+                        const int halves = c < 4 ? 2 : 1;
+                        const bool is_q = it & 1;
+                        mbar_expect_tx(FULL(slot), halves * (is_q ? N1 : kKeys) * 128u);
+                        for (int h = 0; h < halves; ++h) {
+                            const int col = c < 4 ? c * 128 + h * 64 : 0;
+                            if (is_q)
+                                tma_load_2d(dst + h * kHalf, c < 4 ? &prm.mapQ : &prm.mapQr, col, t * N1, FULL(slot));
+                            else
+                                tma_load_2d(dst + h * kHalf, c < 4 ? &prm.mapK : &prm.mapKr, col, krow, FULL(slot));
                         }
                         issued_mask |= 1u << slot;
                     }
                     __syncwarp();
                     if (++slot == kSlots) { slot = 0; sphase ^= 1; }
                 }
+                if (ok && tile == 0) {
+                    // the previous row's last gradient MMAs have read its q~I
+                    if (lane == 0) ok = WAIT(QI_EMPTY, (row_ctr & 1) ^ 1, 59);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (ok && lane == 0) {
+                        mbar_expect_tx(QI_FULL, 2 * kG * 128u);
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_2d(sbase + kOffQI + h * kQIHalf, &prm.mapQI, h * 64, t * kG, QI_FULL);
+                    }
+                    if (ok) ++qi_loads;
+                }
             }
+            ++row_ctr;
         }
         if (lane == 0) {  // drain: every issued load must land before the CTA exits
             for (int k = 0; k < kSlots; ++k) {
@@ -240,6 +271,20 @@ __global__ void __launch_bounds__(kThreads, 1) lig_fused_kernel(const __grid_con
                     uint64_t t0 = globaltimer();
                     while (!mbar_try(FULL(s), ph) && globaltimer() - t0 < 1000000000ull) {
                     }
+                }
+            }
+            // the last load into each K~I buffer and the last q~I load
+            for (int k = 1; k <= 2; ++k) {
+                const int c = ki_loads - k;
+                if (c >= 0) {
+                    uint64_t t0 = globaltimer();
+                    while (!mbar_try(KI_FULL(c & 1), (c >> 1) & 1) && globaltimer() - t0 < 1000000000ull) {
+                    }
+                }
+            }
+            if (qi_loads > 0) {
+                uint64_t t0 = globaltimer();
+                while (!mbar_try(QI_FULL, (qi_loads - 1) & 1) && globaltimer() - t0 < 1000000000ull) {
                 }
             }
         }
@@ -294,21 +339,20 @@ __global__ void __launch_bounds__(kThreads, 1) lig_fused_kernel(const __grid_con
                     advance();
                 }
                 if (!ok) break;
-                // ---- SI^T; K~I and q~I stay in their slots for the gradients ----
-                ok = wait_full(64);
+                // ---- SI^T from this tile's K~I buffer and the row's q~I ----
+                const int kb = tile_ctr & 1;
+                const uint32_t ski = sbase + kOffKI + kb * kSlotBytes;
+                const uint32_t sqi = sbase + kOffQI;
+                if (lane == 0) ok = WAIT(KI_FULL(kb), (tile_ctr >> 1) & 1, 64);
+                if (lane == 0 && ok && tile == 0) ok = WAIT(QI_FULL, row_ctr & 1, 65);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
-                const uint32_t ski = sbase + slot * kSlotBytes;
-                const int kislot = slot;
-                advance();
-                ok = wait_full(65);
-                if (!ok) break;
-                const uint32_t sqi = sbase + slot * kSlotBytes;
-                const int qislot = slot;
-                advance();
+                tc_fence_after();
                 if (lane == 0) {
                     for (int ks = 0; ks < kDi / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-                        mma(T_SI, sdesc(ski + off, 16, 1024), sdesc(sqi + off, 16, 1024), ID_SI, ks > 0 ? 1u : 0u);
+                        const uint32_t oa = (ks >> 2) * kHalf + (ks & 3) * 32;
+                        const uint32_t ob = (ks >> 2) * kQIHalf + (ks & 3) * 32;
+                        mma(T_SI, sdesc(ski + oa, 16, 1024), sdesc(sqi + ob, 16, 1024), ID_SI, ks > 0 ? 1u : 0u);
                     }
                     mma_commit(S_FULL);
                 }
@@ -328,13 +372,15 @@ __global__ void __launch_bounds__(kThreads, 1) lig_fused_kernel(const __grid_con
                             (tile > 0 || ks > 0) ? 1u : 0u);
                     // dK~I^T [Di x keys] = q~I^T . dS (K = G heads, 16 per step)
                     for (int ks = 0; ks < kG / 16; ++ks)
-                        mma(T_DKI, sdesc(sqi + ks * 2048, kHalf, 1024), sdesc(sDS + ks * 32, 16, 1024), ID_DK,
+                        mma(T_DKI, sdesc(sqi + ks * 2048, kQIHalf, 1024), sdesc(sDS + ks * 32, 16, 1024), ID_DK,
                             ks > 0 ? 1u : 0u);
                     mma_commit(DKI_FULL);
                     mma_commit(DS_FREE);
-                    mma_commit(EMPTY(kislot));
-                    mma_commit(EMPTY(qislot));
-                    if (tile == ntiles - 1) mma_commit(DQI_FULL);
+                    mma_commit(KI_EMPTY(kb));
+                    if (tile == ntiles - 1) {
+                        mma_commit(DQI_FULL);
+                        mma_commit(QI_EMPTY);
+                    }
                 }
                 __syncwarp();
             }
