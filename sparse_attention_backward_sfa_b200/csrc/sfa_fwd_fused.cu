@@ -8,15 +8,18 @@
 //   softmaxSum = sum_j exp(scale * Q~.K~_j - softmaxMax)
 //   out        = sum_j exp(scale * Q~.K~_j - softmaxMax) / softmaxSum * V_j
 //
-// Work item = one query row.  Three passes over its 128-key tiles reuse the same
+// Work item = one query row.  Two passes over its 128-key tiles reuse the same
 // S = Q~.K~^T MMA ([128 heads x 128 keys], K = 576, TMEM lane = head):
-//   pass 0: the row statistics (per-thread running max, then sum);
-//   pass 1 / 2: P = exp2(S*scale*log2e - (max*log2e + log2 sum)) to shared
-//   memory (16-bit, SW128), then out[:, 256h, 256h+256) += P . V in TMEM, where
-//   V's two 128-dim chunks are the key chunks the S MMA just read.
-// Recomputing S (3x 19 MFLOP per tile against 17 MFLOP of P.V) keeps the 512-dim
-// fp32 output half (256 TMEM columns) and two S buffers within TMEM and needs no
-// rescaling of the accumulated output.
+//   pass 1: a per-head running max m_run; P = exp2(S*scale*log2e - m_used) to shared
+//   memory (16-bit, SW128) and out[:, 0, 256) += P . V in TMEM, where m_used follows
+//   m_run lazily: only when m_run exceeds it by more than 8 (log2 units) are the
+//   accumulated half and the running sum rescaled, so P stays below 2^8; the half is
+//   divided by the sum when written out, and the statistics are taken relative to the
+//   true max;
+//   pass 2: P = exp2(S*scale*log2e - (m_used + log2 sum)), out[:, 256, 512) += P . V.
+// V's two 128-dim chunks are the key chunks the S MMA just read.  Recomputing S once
+// (2x 19 MFLOP per tile against 17 MFLOP of P.V) keeps the 512-dim fp32 output half
+// (256 TMEM columns) and two S buffers within TMEM.
 // Key rows arrive by TMA tile::gather4, or, when the row lists are block-aligned
 // runs of 16 contiguous rows (block size a multiple of 16; padding slots flagged
 // with bit 31), as one 16-row 2-D tile per run (~2.7x the gather rate on B200).
@@ -43,6 +46,7 @@ constexpr int kSlots = 6;
 constexpr int kSlotBytes = 32768;
 constexpr int kHalf = 16384;
 constexpr int kKeys = 128;
+constexpr float kLazy = 8.f;  // log2 headroom of P before the output half is rescaled
 constexpr int kOffP = kSlots * kSlotBytes;       // P [128 heads x 128 keys] 16-bit, two SW128 halves
 constexpr int kOffBar = kOffP + 32768;
 constexpr int kNumBars = 2 * kSlots + 11;
@@ -145,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
             const int32_t* rl = prm.rowlist + (int64_t)t * prm.cap;
             const int ntiles = (n + kKeys - 1) / kKeys;
             const int first = rl[0] & 0x7fffffff;
-            for (int pass = 0; pass < 3 && ok; ++pass) {
+            for (int pass = 1; pass < 3 && ok; ++pass) {
                 for (int tile = 0; tile < ntiles && ok; ++tile) {
                     int32_t my[4];  // lane L gathers key rows 4L..4L+3 of the tile
 #pragma unroll
@@ -302,12 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
             const int n = prm.nrows[t];
             if (n <= 0) continue;
             const int ntiles = (n + kKeys - 1) / kKeys;
-            for (int pass = 0; pass < 3 && ok; ++pass) {
-                if (pass == 0) {
-                    uint32_t vs[2];
-                    for (int tile = 0; tile < ntiles && ok; ++tile) ok = issue_s(0, vs);
-                    continue;
-                }
+            for (int pass = 1; pass < 3 && ok; ++pass) {
                 // the previous output half has been written out
                 if (lane == 0) ok = WAIT(O_EMPTY, (o_ctr & 1) ^ 1, 45);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -362,70 +361,75 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
                     mk[k] = __ballot_sync(0xffffffffu, s < n && rl[s] >= 0);
                 }
             };
-            // ---- pass 0: running max of the scaled scores, then the sum (in log2 units) ----
-            float m2 = -INFINITY, l = 0.f;  // m2 = max * log2e
-            for (int tile = 0; tile < ntiles && ok; ++tile, ++s_ctr) {
-                const int b = s_ctr & 1;
-                ok = __all_sync(0xffffffffu, WAIT(S_FULL(b), (s_ctr >> 1) & 1, 46));
-                if (!ok) break;
-                tc_fence_after();
-                uint32_t mk[4];
-                tile_mask(tile, mk);
-                float tmax = -INFINITY;
-#pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    float s[32];
-                    tmem_ld32(T_S(b) + lane_base + cc * 32, s);
-                    tmem_wait_ld();
-                    const uint32_t mw = cc == 0 ? mk[0] : cc == 1 ? mk[1] : cc == 2 ? mk[2] : mk[3];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if ((mw >> e) & 1u) tmax = fmaxf(tmax, s[e]);
-                }
-                const float mn = fmaxf(m2, tmax * c1);
-                float sum = 0.f;
-#pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    float s[32];
-                    tmem_ld32(T_S(b) + lane_base + cc * 32, s);
-                    tmem_wait_ld();
-                    const uint32_t mw = cc == 0 ? mk[0] : cc == 1 ? mk[1] : cc == 2 ? mk[2] : mk[3];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if ((mw >> e) & 1u) sum += ex2_approx(fmaf(s[e], c1, -mn));
-                }
-                l = l * ex2_approx(m2 - mn) + sum;  // ex2(-inf) = 0 on the first tile
-                m2 = mn;
-                tc_fence_before();
-                mbar_arrive(S_FREE(b));
-            }
-            if (!ok) break;
-            prm.smax[row] = m2 * 0.6931471805599453f;  // back to natural-log units: max of scale * Q~.K~
-            prm.ssum[row] = l;
-            const float mc = m2 + log2f(l);  // P = exp2(S*c1 - mc) = exp(scaled - max) / sum
-            // ---- passes 1 / 2: P to shared memory, out half = P . V ----
+            // pass 1: output half 0 with a running max (lazy rescaling); pass 2: half 1 with the
+            // final statistics.  m_run = max * log2e so far; P is taken relative to m_used, which
+            // moves up (rescaling the accumulated half and the sum) only when m_run exceeds it by
+            // more than kLazy, so P stays below 2^kLazy.
+            float m_run = -INFINITY, m_used = -INFINITY, l = 0.f, mc = 0.f;
             for (int pass = 1; pass < 3 && ok; ++pass, ++o_ctr) {
                 for (int tile = 0; tile < ntiles && ok; ++tile, ++s_ctr, ++p_ctr) {
                     const int b = s_ctr & 1;
                     ok = WAIT(S_FULL(b), (s_ctr >> 1) & 1, 47);
-                    // P of the previous tile has been read by its output MMA
+                    // P of the previous tile has been read by its output MMA (the half is stable)
                     if (ok) ok = WAIT(P_FREE, (p_ctr & 1) ^ 1, 48);
                     ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
                     if (!ok) break;
                     tc_fence_after();
                     uint32_t mk[4];
                     tile_mask(tile, mk);
+                    float msub = mc;  // pass 2: P = exp2(S*c1 - (m_used + log2 l)), normalised
+                    if (pass == 1) {
+                        float tmax = -INFINITY;
+#pragma unroll 1
+                        for (int cc = 0; cc < 4; ++cc) {
+                            float sv[32];
+                            tmem_ld32(T_S(b) + lane_base + cc * 32, sv);
+                            tmem_wait_ld();
+                            const uint32_t mw = cc == 0 ? mk[0] : cc == 1 ? mk[1] : cc == 2 ? mk[2] : mk[3];
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if ((mw >> e) & 1u) tmax = fmaxf(tmax, sv[e]);
+                        }
+                        m_run = fmaxf(m_run, tmax * c1);
+                        // the decision is per head (thread); the TMEM loads / stores below are
+                        // warp-collective, so a warp rescales when any of its heads needs it and
+                        // the other heads apply a factor of 1
+                        const bool need = m_run > m_used + kLazy;
+                        const float f = need ? ex2_approx(m_used - m_run) : 1.f;  // 0 on the first tile
+                        if (tile > 0 && __any_sync(0xffffffffu, need)) {
+                            // rescale the accumulated output half (TMEM lane = head)
+#pragma unroll 1
+                            for (int cc = 0; cc < 8; ++cc) {
+                                float v[32];
+                                tmem_ld32(T_O + lane_base + cc * 32, v);
+                                tmem_wait_ld();
+                                uint32_t r[32];
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(v[e] * f);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) tmem_st8(T_O + lane_base + cc * 32 + 8 * q, r + 8 * q);
+                            }
+                            tmem_wait_st();
+                        }
+                        if (need) {
+                            l *= f;
+                            m_used = m_run;
+                        }
+                        msub = m_used;
+                    }
+                    float psum = 0.f;
 #pragma unroll 1
                     for (int cc = 0; cc < 4; ++cc) {
-                        float s[32];
-                        tmem_ld32(T_S(b) + lane_base + cc * 32, s);
+                        float sv[32];
+                        tmem_ld32(T_S(b) + lane_base + cc * 32, sv);
                         tmem_wait_ld();
                         uint32_t pw[16];
                         const uint32_t mw = cc == 0 ? mk[0] : cc == 1 ? mk[1] : cc == 2 ? mk[2] : mk[3];
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
-                            const float p0 = (mw >> e) & 1u ? ex2_approx(fmaf(s[e], c1, -mc)) : 0.f;
-                            const float p1 = (mw >> (e + 1)) & 1u ? ex2_approx(fmaf(s[e + 1], c1, -mc)) : 0.f;
+                            const float p0 = (mw >> e) & 1u ? ex2_approx(fmaf(sv[e], c1, -msub)) : 0.f;
+                            const float p1 = (mw >> (e + 1)) & 1u ? ex2_approx(fmaf(sv[e + 1], c1, -msub)) : 0.f;
+                            psum += p0 + p1;
                             pw[e >> 1] = pack2<T>(p0, p1);
                         }
                         // keys [32cc, 32cc+32) of head row h: SW128 half cc/2, 16-byte units 4(cc%2)..+4
@@ -437,16 +441,24 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
                                 make_uint4(pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
                         }
                     }
+                    if (pass == 1) l += psum;
                     fence_view_async_shared();
                     tc_fence_before();
                     mbar_arrive(S_FREE(b));
                     mbar_arrive(P_FULL);
+                }
+                if (pass == 1 && ok) {
+                    // statistics relative to the true max (natural-log units for softmaxMax)
+                    prm.smax[row] = m_run * 0.6931471805599453f;
+                    prm.ssum[row] = l * ex2_approx(m_used - m_run);
+                    mc = m_used + log2f(l);
                 }
                 if (!ok) break;
                 ok = __all_sync(0xffffffffu, WAIT(O_FULL, o_ctr & 1, 49));
                 if (!ok) break;
                 tc_fence_after();
                 T* o = reinterpret_cast<T*>(prm.out) + row * kD + 256 * (pass - 1);
+                const float inv = pass == 1 ? 1.f / l : 1.f;  // half 0 holds P relative to m_used, unnormalised
 #pragma unroll 1
                 for (int cc = 0; cc < 8; ++cc) {
                     float v[32];
@@ -454,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_fwd_fused_kernel(const __grid
                     tmem_wait_ld();
                     uint32_t wv[16];
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) wv[e >> 1] = pack2<T>(v[e], v[e + 1]);
+                    for (int e = 0; e < 32; e += 2) wv[e >> 1] = pack2<T>(v[e] * inv, v[e + 1] * inv);
                     uint4* d4 = reinterpret_cast<uint4*>(o + cc * 32);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) d4[u] = make_uint4(wv[4 * u], wv[4 * u + 1], wv[4 * u + 2], wv[4 * u + 3]);

@@ -129,6 +129,39 @@ def test_fused_fwd_parity(case):
     np.testing.assert_allclose(gl, rl, rtol=2e-5, atol=1e-6)
 
 
+def test_fused_fwd_running_max_rescale():
+    """Key norms that grow with the key index (rows sorted ascending): the running max of
+    later tiles exceeds the first tiles' by more than the lazy-rescaling headroom, so the
+    accumulated output half and the sum are rescaled during the first output pass."""
+    from parity import assert_close, oracle_forward
+    from workloads import bf16_round
+    p = tiny(111, layout="TND", seqlens_q=[300, 40], seqlens_kv=[300, 500], N1=128, topk=40, block_size=16,
+             sparse_mode=3, index_mode="causal")
+    f = (1.0 + 8.0 * np.arange(p.T2) / p.T2)[:, None]
+    p.k = bf16_round(p.k * f)
+    p.k_rope = bf16_round(p.k_rope * f)
+    # precondition: for many (row, head) pairs the max over all keys exceeds the first 128-key
+    # tile's (keys in ascending order) by more than 8 in log2 units
+    from oracle.sfa_oracle import make_spans, selected_rows
+    kt = np.concatenate([p.k, p.k_rope], 1)
+    moved = 0
+    for sp in make_spans(p.layout, p.B, p.S1, p.S2, p.seqlens_q, p.seqlens_kv):
+        for pos in range(sp.q_len):
+            t = sp.q_start + pos
+            rows = sorted(selected_rows(p.indices[t], p.block_size, pos, sp.q_len, sp.kv_len, p.sparse_mode))
+            if len(rows) > 128:
+                sc = np.concatenate([p.q[t], p.q_rope[t]], 1) @ kt[sp.kv_start + np.array(rows)].T
+                moved += int(((sc.max(1) - sc[:, :128].max(1)) * p.scale / np.log(2) > 8).sum())
+    assert moved > 1000
+    dp = DevProblem(p)
+    dp.forward_gpu()
+    ro, rm, rl = oracle_forward(p)
+    go, gm, gl = dp.host_fwd_inputs()
+    assert_close("out", go, ro)
+    np.testing.assert_allclose(gm, rm, rtol=2e-5, atol=2e-5)
+    np.testing.assert_allclose(gl, rl, rtol=2e-5, atol=1e-6)
+
+
 def test_fused_fwd_fp16():
     from parity import assert_close, oracle_forward
     p = tiny(109, **FWD["n128_tnd_bs16_causal"])
