@@ -84,17 +84,35 @@ struct FusedParams {
     uint64_t wait_ns;        // limit of every mbarrier wait (error word + clean exit past it)
 };
 
-// Item i of a tile's load schedule: kind (0 key chunk, 1 q chunk, 2 dO chunk) and chunk c.
+// Load schedule of a tile (kind 0 key chunk, 1 q chunk, 2 dO chunk; chunk c):
+//   S / dP phase, items 0..13: K0 Q0 O0 K1 Q1 O1 K2 Q2 O2 K3 Q3 O3 K4 Q4.  The last five
+//   (K3 Q3 O3 K4 Q4) stay in their slots and feed the first five gradient blocks.
+//   gradient loads, items 14..22: O0 O1 O2 (dV), Q0 Q1 Q2 (dK), K0 K1 K2 (dQ).
+constexpr int kItems = 23;
+constexpr int kHeldFirst = 9;  // items 9..13 are held for the gradient phase
 __device__ __forceinline__ void item_of(int i, int& kind, int& c) {
-    if (i < 14) {  // S / dP phase: K0 Q0 O0 K1 Q1 O1 ... K3 Q3 O3 K4 Q4
+    if (i < 14) {
         c = i / 3;
         kind = i - 3 * c;
         return;
     }
-    i -= 14;       // gradient phase: O0..O3 (dV), Q0..Q4 (dK), K0..K4 (dQ)
-    if (i < 4) { kind = 2; c = i; return; }
-    if (i < 9) { kind = 1; c = i - 4; return; }
-    kind = 0; c = i - 9;
+    i -= 14;
+    kind = 2 - i / 3;
+    c = i % 3;
+}
+// Gradient block bi of a tile: output kind (2 dV, 1 dK~, 0 dQ~, the same as the kind of
+// the chunk it reads as A) and block b.  Blocks 0..4 read the held chunks K3 Q3 O3 K4 Q4
+// in their ring order; blocks 5..13 read the gradient loads in order.
+__device__ __forceinline__ void block_of(int bi, int& kind, int& b) {
+    if (bi < 5) {
+        const int held = kHeldFirst + bi;
+        b = held / 3;
+        kind = held - 3 * b;
+        return;
+    }
+    bi -= 5;
+    kind = 2 - bi / 3;
+    b = bi % 3;
 }
 
 // Named barrier 1 over the 128 softmax threads that also ANDs a flag across them:
@@ -297,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 contig = __all_sync(0xffffffffu, contig);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ROWS_FULL(rb));
-                for (int it = 0; it < 28 && ok; ++it) {
+                for (int it = 0; it < kItems && ok; ++it) {
                     int kind, c;
                     item_of(it, kind, c);
                     if (lane == 0) ok = WAIT(EMPTY(slot), sphase ^ 1, 2);
@@ -364,6 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
             for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
                 // ---- S^T and dP^T over the 5 / 4 chunks ----
                 uint32_t slotK = 0;
+                int hold0 = 0;  // slot of K3, the first held item (the five held items are consecutive in the ring)
                 for (int it = 0; it < 14 && ok; ++it) {
                     int kind, c;
                     item_of(it, kind, c);
@@ -373,6 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                     tc_fence_after();
                     const uint32_t sa = sbase + slot * kSlotBytes;
                     if (kind == 0) slotK = sa;
+                    if (it == kHeldFirst) hold0 = slot;
                     if (lane == 0 && kind != 0) {
                         const uint32_t dst = kind == 1 ? T_S : T_DP;
                         const int ksteps = c < 4 ? 8 : 4;
@@ -382,9 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                             const uint64_t b = sdesc(sa + off, 16, 1024);
                             mma(dst, a, b, ID_S, (c > 0 || ks > 0) ? 1u : 0u);
                         }
-                        // a slot is released once the MMAs that read it have completed
-                        mma_commit(EMPTY(slot));
-                        if (kind == 2 || c == 4) mma_commit(EMPTY((slotK - sbase) / kSlotBytes));
+                        // a slot is released once the MMAs that read it have completed, unless it
+                        // is held for a gradient block (K3 Q3 O3 K4 Q4)
+                        if (it < kHeldFirst) mma_commit(EMPTY(slot));
+                        if ((kind == 2 || c == 4) && c < 3) mma_commit(EMPTY((slotK - sbase) / kSlotBytes));
                     }
                     __syncwarp();
                     if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
@@ -398,17 +419,21 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 tc_fence_after();
                 for (int bi = 0; bi < 14 && ok; ++bi, ++blk_ctr) {
                     const int stg = blk_ctr & 1;
+                    int kind, b;
+                    block_of(bi, kind, b);
+                    const bool held = bi < 5;  // its chunk was loaded (and waited for) in the S / dP phase
                     if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 5);
-                    if (lane == 0 && ok) ok = WAIT(FULL(slot), sphase, 6);
+                    if (lane == 0 && ok && !held) ok = WAIT(FULL(slot), sphase, 6);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t sa = sbase + slot * kSlotBytes;
+                    const int cslot = held ? (hold0 + bi) % C::kSlots : slot;
+                    const uint32_t sa = sbase + cslot * kSlotBytes;
                     if (lane == 0) {
                         const uint32_t dst = T_STG(stg);
-                        if (bi < 9) {
+                        if (kind != 0) {
                             // dV^T (A = dO chunk) or dK~^T (A = q chunk): [128 dims x 128 keys], K = heads
-                            const uint32_t bsrc = bi < 4 ? sP : sDS;
+                            const uint32_t bsrc = kind == 2 ? sP : sDS;
                             for (int ks = 0; ks < N1 / 16; ++ks) {
                                 const uint64_t a = sdesc(sa + ks * 2048, kHalf, 1024);
                                 const uint64_t b = sdesc(bsrc + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
@@ -422,11 +447,11 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                                 mma(dst, a, b, ID_Q, ks > 0 ? 1u : 0u);
                             }
                         }
-                        mma_commit(EMPTY(slot));
+                        mma_commit(EMPTY(cslot));
                         mma_commit(STG_FULL(stg));
                     }
                     __syncwarp();
-                    if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+                    if (!held && ++slot == C::kSlots) { slot = 0; sphase ^= 1; }
                 }
                 if (lane == 0 && ok) mma_commit(PDS_FREE);
             }
@@ -548,9 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                     tc_fence_after();
                     // which output block and which dims this lane quarter holds
                     int kind, b;
-                    if (bi < 4) { kind = 2; b = bi; }
-                    else if (bi < 9) { kind = 1; b = bi - 4; }
-                    else { kind = 0; b = bi - 9; }
+                    block_of(bi, kind, b);
                     const bool active = b < 4 || q < 2;  // rope blocks: 64 valid dims
                     const int dim = (b < 4 ? b * 128 : kD) + q * 32 + lane;
                     if (active) {
