@@ -53,13 +53,12 @@ def device_args(p, dtype=torch.bfloat16):
         lead_q, lead_k = (p.B, p.S1), (p.B, p.S2)
     else:
         lead_q, lead_k = (p.T1,), (p.T2,)
-    one = (1,) if p.layout == "BSND" else (1,)
     q = t(p.q, lead_q + (p.N1, p.D))
     qr = t(p.q_rope, lead_q + (p.N1, p.Dr))
-    k = t(p.k, lead_k + one + (p.D,))
-    kr = t(p.k_rope, lead_k + one + (p.Dr,))
+    k = t(p.k, lead_k + (1, p.D))          # one key head
+    kr = t(p.k_rope, lead_k + (1, p.Dr))
     qi = t(p.q_index, lead_q + (p.G, p.Di))
-    ki = t(p.k_index, lead_k + one + (p.Di,))
+    ki = t(p.k_index, lead_k + (1, p.Di))
     w = t(p.weights, lead_q + (p.G,))
     sq = None if p.seqlens_q is None else torch.tensor(p.seqlens_q, dtype=torch.int64, device=dev)
     skv = None if p.seqlens_kv is None else torch.tensor(p.seqlens_kv, dtype=torch.int64, device=dev)
