@@ -87,7 +87,9 @@ struct FusedParams {
 // Load schedule of a tile (kind 0 key chunk, 1 q chunk, 2 dO chunk; chunk c):
 //   S / dP phase, items 0..13: K0 Q0 O0 K1 Q1 O1 K2 Q2 O2 K3 Q3 O3 K4 Q4.  The last five
 //   (K3 Q3 O3 K4 Q4) stay in their slots and feed the first five gradient blocks.
-//   gradient loads, items 14..22: O0 O1 O2 (dV), Q0 Q1 Q2 (dK), K0 K1 K2 (dQ).
+//   gradient loads, items 14..22: K0 K1 K2 (dQ), Q0 Q1 Q2 (dK), O0 O1 O2 (dV): the 64-bit dK / dV
+//   blocks come last, so the flush of the final two (the largest) overlaps the next tile's
+//   S / dP loads and MMAs.
 constexpr int kItems = 23;
 constexpr int kHeldFirst = 9;  // items 9..13 are held for the gradient phase
 __device__ __forceinline__ void item_of(int i, int& kind, int& c) {
@@ -97,7 +99,7 @@ __device__ __forceinline__ void item_of(int i, int& kind, int& c) {
         return;
     }
     i -= 14;
-    kind = 2 - i / 3;
+    kind = i / 3;
     c = i % 3;
 }
 // Gradient block bi of a tile: output kind (2 dV, 1 dK~, 0 dQ~, the same as the kind of
@@ -111,7 +113,7 @@ __device__ __forceinline__ void block_of(int bi, int& kind, int& b) {
         return;
     }
     bi -= 5;
-    kind = 2 - bi / 3;
+    kind = bi / 3;
     b = bi % 3;
 }
 
