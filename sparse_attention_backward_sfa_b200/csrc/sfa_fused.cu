@@ -84,37 +84,24 @@ struct FusedParams {
     uint64_t wait_ns;        // limit of every mbarrier wait (error word + clean exit past it)
 };
 
-// Load schedule of a tile (kind 0 key chunk, 1 q chunk, 2 dO chunk; chunk c):
-//   S / dP phase, items 0..13: K0 Q0 O0 K1 Q1 O1 K2 Q2 O2 K3 Q3 O3 K4 Q4.  The last five
-//   (K3 Q3 O3 K4 Q4) stay in their slots and feed the first five gradient blocks.
-//   gradient loads, items 14..22: K0 K1 K2 (dQ), Q0 Q1 Q2 (dK), O0 O1 O2 (dV): the 64-bit dK / dV
-//   blocks come last, so the flush of the final two (the largest) overlaps the next tile's
-//   S / dP loads and MMAs.
-constexpr int kItems = 23;
-constexpr int kHeldFirst = 9;  // items 9..13 are held for the gradient phase
-__device__ __forceinline__ void item_of(int i, int& kind, int& c) {
-    if (i < 14) {
-        c = i / 3;
-        kind = i - 3 * c;
-        return;
-    }
-    i -= 14;
-    kind = i / 3;
-    c = i % 3;
+// Schedule of a tile's loads and MMAs (kind 0 key chunk, 1 q chunk, 2 dO chunk; chunk c):
+//   S / dP items j = 0..13: K0 Q0 O0 K1 Q1 O1 K2 Q2 O2 K3 Q3 O3 K4 Q4;
+//   gradient blocks k = 0..13: dQ~ 0..4 (A = key chunk k), dK~ 0..4 (A = q chunk), dV 0..3
+//   (A = dO chunk), each loading its own chunk; the output kind equals the chunk's kind.
+// Software pipeline: after gradient block k >= kInterleave of tile i come the S / dP items
+// 2(k - kInterleave) and 2(k - kInterleave) + 1 of tile i + 1, so the next tile's S^T / dP^T
+// loads and MMAs run while this tile's reduction flush (the SM's reduction path is the bound
+// of the gradient phase) continues; the first tile's S / dP items come first.
+constexpr int kInterleave = 7;
+__device__ __forceinline__ void sdp_item(int j, int& kind, int& c) {
+    c = j / 3;
+    kind = j - 3 * c;
 }
-// Gradient block bi of a tile: output kind (2 dV, 1 dK~, 0 dQ~, the same as the kind of
-// the chunk it reads as A) and block b.  Blocks 0..4 read the held chunks K3 Q3 O3 K4 Q4
-// in their ring order; blocks 5..13 read the gradient loads in order.
-__device__ __forceinline__ void block_of(int bi, int& kind, int& b) {
-    if (bi < 5) {
-        const int held = kHeldFirst + bi;
-        b = held / 3;
-        kind = held - 3 * b;
-        return;
-    }
-    bi -= 5;
-    kind = bi / 3;
-    b = bi % 3;
+__device__ __forceinline__ void block_of(int k, int& kind, int& b) {
+    if (k < 5) { kind = 0; b = k; return; }
+    if (k < 10) { kind = 1; b = k - 5; return; }
+    kind = 2;
+    b = k - 10;
 }
 
 // Named barrier 1 over the 128 softmax threads that also ANDs a flag across them:
@@ -285,72 +272,115 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
         // =================== TMA producer ===================
         int slot = 0;
         uint32_t sphase = 0;
-        int tile_ctr = 0;
+        int tile_ctr = 0;  // tiles whose row ids have been staged
         bool ok = true;
         uint32_t issued_mask = 0;  // slots that have received loads
-        for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
-            const int t = prm.order[w];
-            const int n = prm.nrows[t];
-            if (n <= 0) continue;
-            const int32_t* rl = prm.rowlist + (int64_t)t * prm.cap;
-            const int ntiles = (n + kKeys - 1) / kKeys;
-            for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
+        // the CTA's tiles in order: row w (stepping by gridDim.x, rows without keys skipped), tile
+        struct Tile {
+            int t, n, tile, first, run0;
+            bool contig;
+            int32_t my[4];
+            const int32_t* rl;
+        };
+        int w_next = blockIdx.x, tile_next = 0;
+        // advances to the next tile of the CTA and stages its key row ids (for the flush warps);
+        // returns false at the end of the work
+        auto next_tile = [&](Tile& x) -> bool {
+            while (w_next < nwork) {
+                const int t = prm.order[w_next];
+                const int n = prm.nrows[t];
+                if (tile_next * kKeys >= n) {  // row done (or without keys): next row
+                    w_next += gridDim.x;
+                    tile_next = 0;
+                    continue;
+                }
+                x.t = t;
+                x.n = n;
+                x.tile = tile_next++;
+                x.rl = prm.rowlist + (int64_t)t * prm.cap;
                 const int rb = tile_ctr & 1;
                 if (lane == 0) ok = WAIT(ROWS_EMPTY(rb), ((tile_ctr >> 1) & 1) ^ 1, 1);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
+                if (!ok) return false;
                 int32_t* rid = rowids + rb * kKeys;
-                const int first = rl[0];
-                const int run0 = rl[tile * kKeys];
+                x.first = x.rl[0];
+                x.run0 = x.rl[x.tile * kKeys];
                 // lane L owns key rows 4L..4L+3 of the tile (one gather4 per 64-dim half); a tile
                 // whose rows are run0, run0+1, ... is loaded as one 128-row 2-D tile instead (its
                 // slots past the row's end then hold rows run0+s, masked like any padding key)
-                int32_t my[4];
                 bool contig = true;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int s = tile * kKeys + 4 * lane + e;
-                    my[e] = s < n ? rl[s] : first;
-                    if (s < n && my[e] != run0 + 4 * lane + e) contig = false;
-                    rid[4 * lane + e] = my[e];
+                    const int s = x.tile * kKeys + 4 * lane + e;
+                    x.my[e] = s < n ? x.rl[s] : x.first;
+                    if (s < n && x.my[e] != x.run0 + 4 * lane + e) contig = false;
+                    rid[4 * lane + e] = x.my[e];
                 }
-                contig = __all_sync(0xffffffffu, contig);
+                x.contig = __all_sync(0xffffffffu, contig);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ROWS_FULL(rb));
-                for (int it = 0; it < kItems && ok; ++it) {
-                    int kind, c;
-                    item_of(it, kind, c);
-                    if (lane == 0) ok = WAIT(EMPTY(slot), sphase ^ 1, 2);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    const uint32_t dst = sbase + slot * kSlotBytes;
-                    const int halves = c < 4 ? 2 : 1;
-                    if (lane == 0) {
-                        const uint32_t rows = kind == 0 ? kKeys : N1;
-                        mbar_expect_tx(FULL(slot), halves * rows * 128u);
+                ++tile_ctr;
+                return true;
+            }
+            return false;
+        };
+        // one chunk of tile x into the next ring slot
+        auto load = [&](const Tile& x, int kind, int c) -> bool {
+            if (lane == 0) ok = WAIT(EMPTY(slot), sphase ^ 1, 2);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) return false;
+            const uint32_t dst = sbase + slot * kSlotBytes;
+            const int halves = c < 4 ? 2 : 1;
+            if (lane == 0) {
+                const uint32_t rows = kind == 0 ? kKeys : N1;
+                mbar_expect_tx(FULL(slot), halves * rows * 128u);
+            }
+            __syncwarp();
+            if (kind == 0 && x.contig) {
+                if (lane == 0) {
+                    const CUtensorMap* map = c < 4 ? &prm.mapK128 : &prm.mapKr128;
+                    for (int h = 0; h < halves; ++h)
+                        tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, x.run0, FULL(slot));
+                }
+            } else if (kind == 0) {
+                // key rows: every lane gathers its own four rows, in parallel
+                const CUtensorMap* map = c < 4 ? &prm.mapK : &prm.mapKr;
+                for (int h = 0; h < halves; ++h)
+                    tma_gather4(dst + h * kHalf + lane * 512, map, c < 4 ? c * 128 + h * 64 : 0, x.my[0], x.my[1],
+                                x.my[2], x.my[3], FULL(slot));
+            } else if (lane == 0) {
+                const CUtensorMap* map = kind == 1 ? (c < 4 ? &prm.mapQ : &prm.mapQr) : &prm.mapO;
+                for (int h = 0; h < halves; ++h)
+                    tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, x.t * N1, FULL(slot));
+            }
+            if (lane == 0) issued_mask |= 1u << slot;
+            if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+            return true;
+        };
+        Tile cur, nxt;
+        bool have = next_tile(cur);
+        for (int j = 0; j < 14 && have && ok; ++j) {  // the first tile's S / dP items
+            int kind, c;
+            sdp_item(j, kind, c);
+            ok = load(cur, kind, c);
+        }
+        while (have && ok) {
+            bool have_next = false;
+            for (int k = 0; k < 14 && ok; ++k) {
+                int kind, b;
+                block_of(k, kind, b);
+                ok = load(cur, kind, b);
+                if (ok && k == kInterleave) have_next = next_tile(nxt);
+                if (ok && have_next && k >= kInterleave) {
+                    for (int q = 0; q < 2 && ok; ++q) {
+                        int kd, c;
+                        sdp_item(2 * (k - kInterleave) + q, kd, c);
+                        ok = load(nxt, kd, c);
                     }
-                    __syncwarp();
-                    if (kind == 0 && contig) {
-                        if (lane == 0) {
-                            const CUtensorMap* map = c < 4 ? &prm.mapK128 : &prm.mapKr128;
-                            for (int h = 0; h < halves; ++h)
-                                tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, run0, FULL(slot));
-                        }
-                    } else if (kind == 0) {
-                        // key rows: every lane gathers its own four rows, in parallel
-                        const CUtensorMap* map = c < 4 ? &prm.mapK : &prm.mapKr;
-                        for (int h = 0; h < halves; ++h)
-                            tma_gather4(dst + h * kHalf + lane * 512, map, c < 4 ? c * 128 + h * 64 : 0, my[0], my[1],
-                                        my[2], my[3], FULL(slot));
-                    } else if (lane == 0) {
-                        const CUtensorMap* map = kind == 1 ? (c < 4 ? &prm.mapQ : &prm.mapQr) : &prm.mapO;
-                        for (int h = 0; h < halves; ++h)
-                            tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, t * N1, FULL(slot));
-                    }
-                    if (lane == 0) issued_mask |= 1u << slot;
-                    if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
                 }
             }
+            cur = nxt;
+            have = have_next;
         }
         // drain: every issued load must land before the CTA can exit
         if (lane == 0) {
@@ -376,87 +406,103 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
         int tile_ctr = 0;
         int blk_ctr = 0;
         bool ok = true;
-        for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
-            const int t = prm.order[w];
-            const int n = prm.nrows[t];
-            if (n <= 0) continue;
-            const int ntiles = (n + kKeys - 1) / kKeys;
-            for (int tile = 0; tile < ntiles && ok; ++tile, ++tile_ctr) {
-                // ---- S^T and dP^T over the 5 / 4 chunks ----
-                uint32_t slotK = 0;
-                int hold0 = 0;  // slot of K3, the first held item (the five held items are consecutive in the ring)
-                for (int it = 0; it < 14 && ok; ++it) {
-                    int kind, c;
-                    item_of(it, kind, c);
-                    if (lane == 0) ok = WAIT(FULL(slot), sphase, 3);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t sa = sbase + slot * kSlotBytes;
-                    if (kind == 0) slotK = sa;
-                    if (it == kHeldFirst) hold0 = slot;
-                    if (lane == 0 && kind != 0) {
-                        const uint32_t dst = kind == 1 ? T_S : T_DP;
-                        const int ksteps = c < 4 ? 8 : 4;
-                        for (int ks = 0; ks < ksteps; ++ks) {
-                            const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-                            const uint64_t a = sdesc(slotK + off, 16, 1024);
-                            const uint64_t b = sdesc(sa + off, 16, 1024);
-                            mma(dst, a, b, ID_S, (c > 0 || ks > 0) ? 1u : 0u);
-                        }
-                        // a slot is released once the MMAs that read it have completed, unless it
-                        // is held for a gradient block (K3 Q3 O3 K4 Q4)
-                        if (it < kHeldFirst) mma_commit(EMPTY(slot));
-                        if ((kind == 2 || c == 4) && c < 3) mma_commit(EMPTY((slotK - sbase) / kSlotBytes));
-                    }
-                    __syncwarp();
-                    if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+        uint32_t slotK = 0;  // key chunk of the S / dP item pair in progress
+        auto wait_full = [&](int code) -> bool {
+            bool r = true;
+            if (lane == 0) r = WAIT(FULL(slot), sphase, code);
+            r = __shfl_sync(0xffffffffu, r, 0);
+            if (r) tc_fence_after();
+            return r;
+        };
+        // S / dP item j of a tile (S^T, dP^T accumulate into their TMEM columns)
+        auto sdp = [&](int j) -> bool {
+            int kind, c;
+            sdp_item(j, kind, c);
+            if (!wait_full(3)) return false;
+            const uint32_t sa = sbase + slot * kSlotBytes;
+            if (kind == 0) slotK = sa;
+            if (lane == 0 && kind != 0) {
+                const uint32_t dst = kind == 1 ? T_S : T_DP;
+                const int ksteps = c < 4 ? 8 : 4;
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                    mma(dst, sdesc(slotK + off, 16, 1024), sdesc(sa + off, 16, 1024), ID_S, (c > 0 || ks > 0) ? 1u : 0u);
                 }
-                if (!ok) break;
-                if (lane == 0) mma_commit(SDP_FULL);
-                // ---- gradient blocks ----
-                if (lane == 0) ok = WAIT(PDS_FULL, tile_ctr & 1, 4);
+                // a slot is released once the MMAs that read it have completed
+                mma_commit(EMPTY(slot));
+                if (kind == 2 || c == 4) mma_commit(EMPTY((slotK - sbase) / kSlotBytes));
+                if (j == 13) mma_commit(SDP_FULL);
+            }
+            __syncwarp();
+            if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+            return true;
+        };
+        // the CTA's tile count per row, in the producer's order
+        int w_next = blockIdx.x, tile_next = 0;
+        auto next_tile = [&]() -> bool {
+            while (w_next < nwork) {
+                const int n = prm.nrows[prm.order[w_next]];
+                if (tile_next * kKeys >= n) {
+                    w_next += gridDim.x;
+                    tile_next = 0;
+                    continue;
+                }
+                ++tile_next;
+                return true;
+            }
+            return false;
+        };
+        bool have = next_tile();
+        for (int j = 0; j < 14 && have && ok; ++j) ok = sdp(j);  // the first tile's S / dP
+        while (have && ok) {
+            // ---- gradient blocks of this tile, the next tile's S / dP interleaved ----
+            if (lane == 0) ok = WAIT(PDS_FULL, tile_ctr & 1, 4);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            bool have_next = false;
+            for (int k = 0; k < 14 && ok; ++k, ++blk_ctr) {
+                const int stg = blk_ctr & 1;
+                int kind, b;
+                block_of(k, kind, b);
+                if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 5);
+                if (lane == 0 && ok) ok = WAIT(FULL(slot), sphase, 6);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after();
-                for (int bi = 0; bi < 14 && ok; ++bi, ++blk_ctr) {
-                    const int stg = blk_ctr & 1;
-                    int kind, b;
-                    block_of(bi, kind, b);
-                    const bool held = bi < 5;  // its chunk was loaded (and waited for) in the S / dP phase
-                    if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 5);
-                    if (lane == 0 && ok && !held) ok = WAIT(FULL(slot), sphase, 6);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const int cslot = held ? (hold0 + bi) % C::kSlots : slot;
-                    const uint32_t sa = sbase + cslot * kSlotBytes;
-                    if (lane == 0) {
-                        const uint32_t dst = T_STG(stg);
-                        if (kind != 0) {
-                            // dV^T (A = dO chunk) or dK~^T (A = q chunk): [128 dims x 128 keys], K = heads
-                            const uint32_t bsrc = kind == 2 ? sP : sDS;
-                            for (int ks = 0; ks < N1 / 16; ++ks) {
-                                const uint64_t a = sdesc(sa + ks * 2048, kHalf, 1024);
-                                const uint64_t b = sdesc(bsrc + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
-                                mma(dst, a, b, ID_G, ks > 0 ? 1u : 0u);
-                            }
-                        } else {
-                            // dQ~^T: A = key chunk [128 dims x 128 keys] (MN), B = dS [heads x keys] (MN)
-                            for (int ks = 0; ks < kKeys / 16; ++ks) {
-                                const uint64_t a = sdesc(sa + ks * 2048, kHalf, 1024);
-                                const uint64_t b = sdesc(sDS + ks * 2048, kHalf, 1024);
-                                mma(dst, a, b, ID_Q, ks > 0 ? 1u : 0u);
-                            }
+                const uint32_t sa = sbase + slot * kSlotBytes;
+                if (lane == 0) {
+                    const uint32_t dst = T_STG(stg);
+                    if (kind != 0) {
+                        // dV^T (A = dO chunk) or dK~^T (A = q chunk): [128 dims x 128 keys], K = heads
+                        const uint32_t bsrc = kind == 2 ? sP : sDS;
+                        for (int ks = 0; ks < N1 / 16; ++ks) {
+                            const uint64_t a = sdesc(sa + ks * 2048, kHalf, 1024);
+                            const uint64_t bd = sdesc(bsrc + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
+                            mma(dst, a, bd, ID_G, ks > 0 ? 1u : 0u);
                         }
-                        mma_commit(EMPTY(cslot));
-                        mma_commit(STG_FULL(stg));
+                    } else {
+                        // dQ~^T: A = key chunk [128 dims x 128 keys] (MN), B = dS [heads x keys] (MN)
+                        for (int ks = 0; ks < kKeys / 16; ++ks) {
+                            const uint64_t a = sdesc(sa + ks * 2048, kHalf, 1024);
+                            const uint64_t bd = sdesc(sDS + ks * 2048, kHalf, 1024);
+                            mma(dst, a, bd, ID_Q, ks > 0 ? 1u : 0u);
+                        }
                     }
-                    __syncwarp();
-                    if (!held && ++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+                    mma_commit(EMPTY(slot));
+                    mma_commit(STG_FULL(stg));
+                    if (k == 13) mma_commit(PDS_FREE);
                 }
-                if (lane == 0 && ok) mma_commit(PDS_FREE);
+                __syncwarp();
+                if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+                // the next tile's S^T / dP^T overwrite this tile's: the softmax warps have read
+                // them (PDS_FULL above), and P / dS stay in shared memory until PDS_FREE
+                if (k == kInterleave) have_next = next_tile();
+                if (have_next && k >= kInterleave)
+                    for (int q = 0; q < 2 && ok; ++q) ok = sdp(2 * (k - kInterleave) + q);
             }
+            ++tile_ctr;
+            have = have_next;
         }
         if (lane == 0) {
             mma_commit(DONE);
