@@ -352,6 +352,8 @@ sfa_status lig_kl_grad_workspace_size(const lig_shape *shape, int64_t sparse_mod
  *   Outputs: d_query_index [.., G, Di], d_key_index [.., 1, Di], d_weights [.., G]
  *     (16-bit), loss: one fp32 (device).  dKeyIndex is summed with fp32 atomics
  *     (run-to-run differences in the last bits); loss is a fixed-order sum.
+ *   The 16-bit inputs must be 16-byte aligned (they are read by TMA) and the
+ *   workspace 256-byte aligned (SFA_ERR_INVALID otherwise).
  */
 sfa_status lig_kl_grad(const void *query, const void *key, const void *query_index, const void *key_index,
                        const void *weights, const float *softmax_max, const float *softmax_sum,

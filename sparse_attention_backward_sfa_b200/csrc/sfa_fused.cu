@@ -19,8 +19,12 @@
 //  * Every operand is a "chunk" of 128 dims (64 for the rope) held as two
 //    128-byte-row SW128 halves 16 KB apart; the same bytes serve as a K-major
 //    operand (S^T, dP^T) and as an MN-major one (gradients).  Chunks stream
-//    through a ring of 32 KB slots: key rows by TMA tile::gather4, the query
-//    row's q / qRope / dO by 2-D TMA tiles.
+//    through a ring of 32 KB slots: key rows by TMA tile::gather4 (or one
+//    128-row 2-D tile when the tile's rows are consecutive), the query row's
+//    q / qRope / dO by 2-D TMA tiles.
+//  * The producer and MMA warps run a cross-tile software pipeline: the next
+//    tile's S^T / dP^T items are interleaved into this tile's last gradient
+//    blocks, so the next scores are formed while this tile's reductions flush.
 //  * P and dS live in shared memory as bf16 [keys x heads] (SW128 halves of 64
 //    heads); S^T / dP^T and two 128-column staging accumulators live in TMEM
 //    (all 512 columns).
