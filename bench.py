@@ -365,7 +365,9 @@ def run_fwd(args, local_rank):
             "roofline": {"bound": "tensor", "achieved": flop / (kern * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
                          "frac": flop / (kern * 1e-3) / 1e12 / peak, "kernel_ms": kern,
                          "traffic": recorded_traffic("fwd4") if args.workload == 4 and not args.seqs else None},
-            "gpu_launches": (4 if p.N1 == 128 else 2) * args.steps, "clocks": clk.summary()}
+            # fused path: compact, order, block sort (block-sparse, topk <= 4096), expand, fused forward
+            "gpu_launches": ((4 + int(p.block_size > 1 and p.topk <= 4096)) if p.N1 == 128 else 2) * args.steps,
+            "clocks": clk.summary()}
 
 
 def indexer_flop_per_pair(N1: int, G: int, Di: int) -> int:
@@ -775,7 +777,8 @@ def main():
                          else None},
             "cpu_baseline": cpu,
             "e2e": r["e2e"],
-            "gpu_launches": 6 * args.steps,  # compact, rowsum, order, expand, fused backward, cast
+            # compact, rowsum, order, block sort (block-sparse lists of topk <= 4096), expand, fused, cast
+            "gpu_launches": (6 + int(p.block_size > 1 and p.topk <= 4096)) * args.steps,
             "clocks": r["clocks"],
             "device_error_word": r["err_word"],
         }
