@@ -261,6 +261,33 @@ def test_fa_oracle_sdpa_causal_square():
         st = int(e)
 
 
+def test_fa_oracle_sdpa_lower_right_causal_nonsquare():
+    """sparseMode 3 with fewer queries than keys is aligned at the bottom-right corner: the
+    library's lower-right causal bias (torch.nn.attention.bias.causal_lower_right) in SDPA,
+    fp64 autograd, gives the same outputs and gradients."""
+    from torch.nn.attention.bias import causal_lower_right
+    fp = make_fa_problem(seed=10, lens=(5, 3), kv_lens=(9, 7), N=2, Nkv=2, D=8, sparse_mode=3)
+    q, k, v, dy = (a.astype(np.float64) for a in (fp.q, fp.k, fp.v, fp.dy))
+    out, m, l = O.fa_forward(q, k, v, fp.cu_seqlens_q, fp.cu_seqlens_kv, fp.scale, 3)
+    dq, dk, dv = O.fa_backward(q, k, v, dy, m, l, out, fp.cu_seqlens_q, fp.cu_seqlens_kv, fp.scale, 3)
+    sq = sk = 0
+    for eq, ek in zip(fp.cu_seqlens_q, fp.cu_seqlens_kv):
+        qs, ks = slice(sq, int(eq)), slice(sk, int(ek))
+        Lq, Lk = int(eq) - sq, int(ek) - sk
+        Q = torch.tensor(q[qs]).transpose(0, 1).requires_grad_(True)
+        K = torch.tensor(k[ks]).transpose(0, 1).requires_grad_(True)
+        V = torch.tensor(v[ks]).transpose(0, 1).requires_grad_(True)
+        mask = causal_lower_right(Lq, Lk)
+        y = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None], attn_mask=mask,
+                                                             scale=fp.scale)[0]
+        (y * torch.tensor(dy[qs]).transpose(0, 1)).sum().backward()
+        np.testing.assert_allclose(y.detach().transpose(0, 1).numpy(), out[qs], atol=1e-12)
+        np.testing.assert_allclose(Q.grad.transpose(0, 1).numpy(), dq[qs], atol=1e-11)
+        np.testing.assert_allclose(K.grad.transpose(0, 1).numpy(), dk[ks], atol=1e-11)
+        np.testing.assert_allclose(V.grad.transpose(0, 1).numpy(), dv[ks], atol=1e-11)
+        sq, sk = int(eq), int(ek)
+
+
 def test_page2_worked_example_all_ones():
     g = json.load(open(os.path.join(GOLD, "fa_grad_allones.json")))
     T, N, D = g["T"], g["N"], g["D"]

@@ -62,6 +62,31 @@ def test_sfa_oracle_mistake_is_caught(name, monkeypatch):
 
 
 # ---------------------------------------------------------------------------
+# dense FA oracle: finite differences with GQA and the bottom-right causal mask, torch SDPA
+# with is_causal, the page's all-ones worked example
+FA_MUTATIONS = {
+    "gqa_head_map": ("            hk = h // g\n", "            hk = h % Nkv\n"),
+    "dq_scale_dropped": ("dq[qs, h] = scale * (ds @ k[ks, hk])", "dq[qs, h] = ds @ k[ks, hk]"),
+    "dk_overwrites_heads": ("dk[ks, hk] += scale * (ds.T @ q[qs, h])", "dk[ks, hk] = scale * (ds.T @ q[qs, h])"),
+    "causal_top_left": ("return j <= i + (kv_len - q_len)", "return j <= i"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FA_MUTATIONS))
+def test_fa_oracle_mistake_is_caught(name, monkeypatch):
+    import test_oracle_pins as pins
+    mod = mutant(SFO, *FA_MUTATIONS[name])
+    monkeypatch.setattr(pins, "O", mod)
+    checks = [
+        (pins.test_fa_oracle_fd_gqa_bottom_right_causal,),
+        (pins.test_fa_oracle_sdpa_causal_square,),
+        (pins.test_fa_oracle_sdpa_lower_right_causal_nonsquare,),
+        (pins.test_page2_worked_example_all_ones,),
+    ]
+    assert any(fails(c[0], *c[1:]) for c in checks), f"planted mistake {name} passed every pin"
+
+
+# ---------------------------------------------------------------------------
 # indexer-gradient oracle: finite differences of the loss, torch autograd with kl_div
 IKO_MUTATIONS = {
     "target_not_normalised": ("p = prob.sum(axis=0) / N1", "p = prob.sum(axis=0) / (2 * N1)"),
@@ -96,5 +121,8 @@ def test_unmutated_oracles_pass_the_same_checks():
     import test_oracle_pins as spins
     assert not fails(spins.test_fd_gradients_bsnd, 1, 3, "causal")
     assert not fails(spins.test_sdpa_special_case_forward_and_backward)
+    assert not fails(spins.test_fa_oracle_fd_gqa_bottom_right_causal)
+    assert not fails(spins.test_fa_oracle_sdpa_causal_square)
+    assert not fails(spins.test_fa_oracle_sdpa_lower_right_causal_nonsquare)
     assert not fails(ipins.test_finite_differences, "tnd_causal")
     assert not fails(ipins.test_torch_autograd_special_case, "tnd_causal")
