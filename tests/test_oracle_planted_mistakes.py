@@ -44,6 +44,9 @@ SFA_MUTATIONS = {
     "dv_uses_ds": ("np.add.at(dv, g, p.T @ do)", "np.add.at(dv, g, (p * (dp - dp.mean())).T @ do)"),
     "causal_off_by_one": ("if sparse_mode == 3 and j > q_pos + kv_len - q_len:",
                           "if sparse_mode == 3 and j >= q_pos + kv_len - q_len:"),
+    "causal_top_left": ("if sparse_mode == 3 and j > q_pos + kv_len - q_len:",
+                        "if sparse_mode == 3 and j > q_pos:"),
+    "block_rows_not_cut_at_sequence_end": ("            if j >= kv_len:\n                break\n", ""),
 }
 
 
