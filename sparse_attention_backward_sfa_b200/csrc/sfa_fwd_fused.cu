@@ -22,7 +22,9 @@
 // (256 TMEM columns) and two S buffers within TMEM.
 // Key rows arrive by TMA tile::gather4, or, when the row lists are block-aligned
 // runs of 16 contiguous rows (block size a multiple of 16; padding slots flagged
-// with bit 31), as one 16-row 2-D tile per run (~2.7x the gather rate on B200).
+// with bit 31), as one 16-row 2-D tile per run (~2.7x the gather rate on B200), or,
+// when all 128 rows of a tile are consecutive (sorted block lists), as one 128-row
+// 2-D tile per 64-column half.
 // Warps: 0-3 softmax / output write-out (thread = head), 4 TMA producer, 5 MMA.
 // Every mbarrier wait is bounded; on timeout the kernel records an error word,
 // stops issuing, drains its loads and frees its TMEM.
