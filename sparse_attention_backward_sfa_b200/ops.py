@@ -282,8 +282,9 @@ def fa_fwd(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, scale: float, sparse_mode: i
 
 
 def lig_shape(query: torch.Tensor, key: torch.Tensor, query_index: torch.Tensor, key_index: torch.Tensor,
-              layout: str, actual_seq_lengths_query=None) -> N.LigShape:
-    """Sizes of a dense lightning-indexer gradient call from its tensors."""
+              layout: str, actual_seq_lengths_query=None, query_rope: Optional[torch.Tensor] = None) -> N.LigShape:
+    """Sizes of a dense lightning-indexer gradient call from its tensors (Dr from query_rope,
+    64 when it is not given)."""
     s = N.LigShape()
     _need(query.dtype in _DT, "query must be bf16 or fp16")
     s.dtype = _DT[query.dtype]
@@ -305,7 +306,7 @@ def lig_shape(query: torch.Tensor, key: torch.Tensor, query_index: torch.Tensor,
         _, s.G, s.Di = query_index.shape
     else:
         raise ValueError(f"layout {layout!r}")
-    s.Dr = 64
+    s.Dr = 64 if query_rope is None else query_rope.shape[-1]
     return s
 
 
@@ -332,7 +333,7 @@ def lig_kl_grad(query, key, query_index, key_index, weights, softmax_max, softma
                     ("actual_seq_lengths_key", actual_seq_lengths_key)):
         _need(t is None or (t.is_cuda and t.dtype == torch.int64 and t.is_contiguous()),
               f"{name}: int64 CUDA tensor")
-    shape = lig_shape(query, key, query_index, key_index, layout, actual_seq_lengths_query)
+    shape = lig_shape(query, key, query_index, key_index, layout, actual_seq_lengths_query, query_rope)
     need = lig_kl_grad_workspace_size(shape, sparse_mode)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=query.device)

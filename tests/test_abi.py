@@ -180,3 +180,19 @@ def test_lig_rejects_null_pointers_before_launch(lib):
     args = [None] * 13 + [0.05, 3, 0, 0, ctypes.byref(sh), None, n.value, None] + [None] * 4
     assert lib.lig_kl_grad(*args) == N.SFA_ERR_NULLPTR
     assert lib.lig_kl_grad_workspace_size(None, 3, ctypes.byref(n)) == N.SFA_ERR_NULLPTR
+
+
+def test_lig_shape_reads_rope_width_from_the_tensor(lib):
+    """The binding takes Dr from queryRope, so a wrong rope width reaches the library's check."""
+    import torch
+    from sparse_attention_backward_sfa_b200 import ops
+    q = torch.empty(10, 128, 512, dtype=torch.bfloat16)
+    k = torch.empty(10, 1, 512, dtype=torch.bfloat16)
+    qi = torch.empty(10, 64, 128, dtype=torch.bfloat16)
+    ki = torch.empty(10, 1, 128, dtype=torch.bfloat16)
+    sq = torch.tensor([10], dtype=torch.int64)
+    good = ops.lig_shape(q, k, qi, ki, "TND", sq, torch.empty(10, 128, 64, dtype=torch.bfloat16))
+    bad = ops.lig_shape(q, k, qi, ki, "TND", sq, torch.empty(10, 128, 32, dtype=torch.bfloat16))
+    n = ctypes.c_size_t(0)
+    assert lib.lig_kl_grad_workspace_size(ctypes.byref(good), 3, ctypes.byref(n)) == N.SFA_OK
+    assert lib.lig_kl_grad_workspace_size(ctypes.byref(bad), 3, ctypes.byref(n)) == N.SFA_ERR_INVALID
