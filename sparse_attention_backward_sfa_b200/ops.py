@@ -334,6 +334,14 @@ def lig_kl_grad(query, key, query_index, key_index, weights, softmax_max, softma
         _need(t is None or (t.is_cuda and t.dtype == torch.int64 and t.is_contiguous()),
               f"{name}: int64 CUDA tensor")
     shape = lig_shape(query, key, query_index, key_index, layout, actual_seq_lengths_query, query_rope)
+    # the library sees raw pointers: every tensor must hold exactly the elements its layout implies
+    T1, T2 = shape.T1, shape.T2
+    for name, t, n in (("key", key, T2 * shape.D), ("key_index", key_index, T2 * shape.Di),
+                       ("weights", weights, T1 * shape.G), ("query_rope", query_rope, T1 * shape.N1 * shape.Dr),
+                       ("key_rope", key_rope, T2 * shape.Dr), ("softmax_max", softmax_max, T1 * shape.N1),
+                       ("softmax_sum", softmax_sum, T1 * shape.N1), ("softmax_max_index", softmax_max_index, T1),
+                       ("softmax_sum_index", softmax_sum_index, T1)):
+        _need(t.numel() == n, f"{name}: {t.numel()} elements, expected {n}")
     need = lig_kl_grad_workspace_size(shape, sparse_mode)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=query.device)
