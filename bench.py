@@ -193,13 +193,18 @@ def run_ours(args, rank, world, local_rank):
             return
         dq, dk, dv, dqr, dkr = outs
         acc.zero_()
+        dmax = None
+        if p.deterministic:  # the fixed-point grid: max|dOut| over every rank's rows
+            dmax = S.dout_absmax(do, q, k, qr, idx, layout=p.layout, row_begin=rb, row_end=re_,
+                                 actual_seq_lengths_q=sq)
+            dist.all_reduce(dmax, op=dist.ReduceOp.MAX)
         S.sfa_grad_rows(q, k, k, idx, do, o, mx, sm, qr, kr, row_begin=rb, row_end=re_, dkv_accum=acc,
-                        deterministic=p.deterministic, workspace=ws, d_query=dq, d_query_rope=dqr, scale=p.scale,
-                        sparse_block_size=p.block_size, layout=p.layout, sparse_mode=p.sparse_mode,
-                        actual_seq_lengths_q=sq, actual_seq_lengths_kv=skv)
+                        deterministic=p.deterministic, dout_absmax=dmax, workspace=ws, d_query=dq,
+                        d_query_rope=dqr, scale=p.scale, sparse_block_size=p.block_size, layout=p.layout,
+                        sparse_mode=p.sparse_mode, actual_seq_lengths_q=sq, actual_seq_lengths_kv=skv)
         dist.all_reduce(acc, op=dist.ReduceOp.SUM)
-        S.sfa_dkv_finalize(acc, q, k, qr, idx, layout=p.layout, deterministic=p.deterministic,
-                           actual_seq_lengths_q=sq, outputs=(dk, dv, dkr))
+        S.sfa_dkv_finalize(acc, q, k, qr, idx, layout=p.layout, deterministic=p.deterministic, dout_absmax=dmax,
+                           scale=p.scale, actual_seq_lengths_q=sq, outputs=(dk, dv, dkr))
 
     def step(ev=None):
         if ev is not None:

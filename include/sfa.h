@@ -116,10 +116,22 @@ sfa_status sfa_grad_workspace_size(const sfa_shape *shape, int64_t sparse_block_
  *   scale                           scaleValue (applied in S, dQuery, dKey)
  *   pre_tokens, next_tokens         accepted and ignored (no effect for modes 0/3)
  *   deterministic                   0: fp32 atomic scatter (run-to-run order may
- *                                   differ); 1: bit-identical results run to run
- *                                   (64-bit fixed-point scatter, 32 fraction bits;
- *                                   every partial sum of a dKey/dValue element
- *                                   must stay below 2^31 in magnitude)
+ *                                   differ); 1: bit-identical results run to run:
+ *                                   the key-side sums are 64-bit fixed point on a
+ *                                   power-of-two grid chosen per call from
+ *                                   max|d_out|, T1*N1 and scale (dValue: 2^-e with
+ *                                   e = 54 - ceil(log2(T1*N1)) - E(max|d_out|);
+ *                                   dKey/dKeyRope: e = 42 - ceil(log2(T1*N1)) -
+ *                                   E(max|d_out|) - E(|scale|), E(x) the least k
+ *                                   with x <= 2^k).  Scaling d_out by 2^k scales
+ *                                   the results by exactly 2^k, so the precision
+ *                                   does not depend on the gradient's magnitude.
+ *                                   The grid leaves 2^8 of range for dValue over
+ *                                   the bound T1*N1*max|d_out| (which holds when
+ *                                   softmax_max/_sum are the forward's statistics,
+ *                                   so that every row's P sums to 1) and about 2^11
+ *                                   for dKey over unit-scale activations; inputs
+ *                                   outside that range may saturate.
  *   workspace, workspace_bytes      >= sfa_grad_workspace_size(); 256-byte aligned
  *   d_query, d_query_rope           [.., N1, D|Dr] 16-bit outputs; rows of BSND
  *                                   padding tokens (position >= S1_b) are zero
@@ -144,7 +156,7 @@ sfa_status sfa_grad(const void *query, const void *key, const void *value, const
  *
  * sfa_dkv_accum_size - bytes of the key-side accumulator: [T2][1088] (columns
  * dKey 0-511 | dKeyRope 512-575 | dValue 576-1087), fp32 when deterministic == 0,
- * int64 fixed point (value * 2^32, rounded) when 1.  Host only.
+ * int64 fixed point (the grid of sfa_grad's deterministic mode) when 1.  Host only.
  */
 sfa_status sfa_dkv_accum_size(const sfa_shape *shape, int32_t deterministic, size_t *accum_bytes);
 
@@ -161,6 +173,12 @@ sfa_status sfa_dkv_accum_size(const sfa_shape *shape, int32_t deterministic, siz
  *     (other GPUs) element-wise before sfa_dkv_finalize.  With deterministic == 1
  *     the accumulator is integer, so that element-wise addition is exact and
  *     order-independent and the final outputs are bit-identical to sfa_grad's.
+ *   - dout_absmax (device fp32, deterministic mode only; may be NULL otherwise):
+ *     max|d_out| over EVERY row whose contributions go into this accumulator (on
+ *     every GPU), which fixes the fixed-point grid: zero it, add each range with
+ *     sfa_dout_absmax and, across GPUs, combine the values with a max-reduction
+ *     before the first sfa_grad_rows call.  All calls on one accumulator (and
+ *     sfa_dkv_finalize) must see the same value and the same scale.
  *   - Enqueued on `stream`; nothing is allocated and nothing synchronizes.
  */
 sfa_status sfa_grad_rows(const void *query, const void *key, const void *value, const int32_t *sparse_indices,
@@ -169,16 +187,27 @@ sfa_status sfa_grad_rows(const void *query, const void *key, const void *value, 
                          const void *query_rope, const void *key_rope, float scale, int64_t sparse_block_size,
                          int64_t sparse_mode, int32_t deterministic, int64_t row_begin, int64_t row_end,
                          const sfa_shape *shape, void *workspace, size_t workspace_bytes, sfa_stream_t stream,
-                         void *dkv_accum, void *d_query, void *d_query_rope);
+                         void *dkv_accum, const float *dout_absmax, void *d_query, void *d_query_rope);
+
+/*
+ * sfa_dout_absmax - max-merges max|d_out| over query rows [row_begin, row_end)
+ * into *dout_absmax (device fp32, caller-zeroed before the first range).  The
+ * value sets the fixed-point grid of deterministic row ranges (sfa_grad_rows).
+ */
+sfa_status sfa_dout_absmax(const void *d_out, const sfa_shape *shape, int64_t row_begin, int64_t row_end,
+                           sfa_stream_t stream, float *dout_absmax);
 
 /*
  * sfa_dkv_finalize - casts a (summed) key-side accumulator into the 16-bit
  * d_key [.., N2, D], d_value [.., N2, D] and d_key_rope [.., N2, Dr] outputs
- * (round to nearest even; fixed point is divided by 2^32 first).  `shape` gives
- * T2 and the dtype; `deterministic` selects the accumulator format.
+ * (round to nearest even; fixed point is scaled back by its grid first).
+ * `shape` gives T1, N1, T2 and the dtype; `deterministic` selects the
+ * accumulator format; dout_absmax and scale must be the ones the accumulator
+ * was filled with (dout_absmax may be NULL when deterministic == 0).
  */
-sfa_status sfa_dkv_finalize(const void *dkv_accum, const sfa_shape *shape, int32_t deterministic, sfa_stream_t stream,
-                            void *d_key, void *d_value, void *d_key_rope);
+sfa_status sfa_dkv_finalize(const void *dkv_accum, const sfa_shape *shape, int32_t deterministic,
+                            const float *dout_absmax, float scale, sfa_stream_t stream, void *d_key, void *d_value,
+                            void *d_key_rope);
 
 /*
  * sfa_grad_noalloc - sfa_grad for callers that cannot allocate device memory.
@@ -197,8 +226,11 @@ sfa_status sfa_dkv_finalize(const void *dkv_accum, const sfa_shape *shape, int32
  *    T2 x 1088 x 4 bytes, or x 8 when deterministic, plus T1 x topk x 4 bytes of
  *    index tables) are rejected with SFA_ERR_WORKSPACE before any device work.
  *  - The first call on each device looks up the array's device address with
- *    cudaGetSymbolAddress (with that device current); make that first call
- *    before any stream capture on the device.
+ *    cudaGetSymbolAddress (with that device current) and keeps it for the life
+ *    of the process; make that first call before any stream capture on the
+ *    device.  Calls after a reset of the device (cudaDeviceReset, or the primary
+ *    context being torn down and re-created) are not supported: the kept address
+ *    belongs to the old context.
  *  - All calls on a device share the array, which keeps the previous call's
  *    contents (the accumulator is cleared on the call's stream).  Calls whose
  *    work overlaps on the GPU (other streams, other threads) race on it and
@@ -287,6 +319,10 @@ sfa_status fa_grad_workspace_size(const fa_shape *shape, int64_t sparse_mode, in
  *   cumulative end offsets (last = T1 / T2); copied into the workspace before
  *   the call returns.  keep_prob must be 1 (no dropout); pre/next_tokens are
  *   ignored for sparse_mode 0 / 3; head_num must equal Nq.
+ *   deterministic: 0 fp32 atomics; 1 bit-identical run to run, every atomically
+ *   summed gradient in 64-bit fixed point on the per-call grid of sfa_grad's
+ *   deterministic mode (max|dy|, T1 * Nq/Nkv and scale; dq: e = 42 - E(max|dy|)
+ *   - E(|scale|)).
  */
 sfa_status fa_grad(const void *q, const void *k, const void *v, const void *dy, const float *softmax_max,
                    const float *softmax_sum, const void *attention_in, const int64_t *actual_seq_qlen,

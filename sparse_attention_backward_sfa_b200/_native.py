@@ -77,8 +77,9 @@ SIGNATURES = {
     "sfa_set_wait_limit": [ctypes.c_uint64],
     "sfa_dkv_accum_size": [_PSH, _I32, _PSZ],
     "sfa_grad_rows": [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _F, _I64, _I64, _I32, _I64, _I64, _PSH, _V,
-                      _SZ, _V, _V, _V, _V],
-    "sfa_dkv_finalize": [_V, _PSH, _I32, _V, _V, _V, _V],
+                      _SZ, _V, _V, _V, _V, _V],
+    "sfa_dout_absmax": [_V, _PSH, _I64, _I64, _V, _V],
+    "sfa_dkv_finalize": [_V, _PSH, _I32, _V, _F, _V, _V, _V, _V],
     "sfa_grad_noalloc": [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _F, _I64, _I64, _I64, _I64, _I32, _PSH, _V,
                          _V, _V, _V, _V, _V],
     "lig_kl_grad_workspace_size": [_PLG, _I64, _PSZ],

@@ -63,6 +63,8 @@ struct FaParams {
     void* dk;             // [T2][Nkv][128]
     void* dv;
     int* err;
+    const float* dmax;    // deterministic mode: max|dY| that sets the dQ fixed-point grid
+    int64_t T1;
     int B, Nq, Nkv, mode;
     float scale;
     uint64_t wait_ns;  // limit of every mbarrier wait
@@ -285,6 +287,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
         const int j = quarter * 32 + lane;            // key (softmax / write-out) or dim (flush)
         const int cs = warp >> 2;                     // softmax: which half of the query columns
         const int hsel = (warp - 4) >> 2;             // flush: which half of the query columns
+        const float fmul_q = DET ? fix_mul(fix_exponents(*prm.dmax, prm.scale, prm.T1, prm.Nq / prm.Nkv).q) : 0.f;
         const float c1 = scale * 1.4426950408889634f;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         int item_ctr = 0, pair_ctr = 0;
@@ -398,7 +401,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                                 unsigned long long* d = reinterpret_cast<unsigned long long*>(prm.dq_acc) + base;
 #pragma unroll
                                 for (int e = 0; e < 32; ++e, d += step)
-                                    if (e < lim) atomicAdd(d, (unsigned long long)__float2ll_rn(v[e] * kFixScale));
+                                    if (e < lim) atomicAdd(d, fix_round(v[e], fmul_q));
                             } else {
                                 float* d = reinterpret_cast<float*>(prm.dq_acc) + base;
 #pragma unroll
@@ -470,10 +473,12 @@ __global__ void fa_rowsum_kernel(const T* __restrict__ dy, const T* __restrict__
 }
 
 template <typename T, bool DET>
-__global__ void fa_cast_dq_kernel(const void* __restrict__ acc, int64_t n, T* __restrict__ dq) {
+__global__ void fa_cast_dq_kernel(const void* __restrict__ acc, int64_t n, T* __restrict__ dq,
+                                  const float* __restrict__ dmax, float scale, int64_t T1, int64_t G) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
-    const float x = DET ? (float)((double)reinterpret_cast<const long long*>(acc)[i] * kFixInv)
+    const float x = DET ? (float)((double)reinterpret_cast<const long long*>(acc)[i] *
+                                  fix_inv(fix_exponents(*dmax, scale, T1, G).q))
                         : reinterpret_cast<const float*>(acc)[i];
     dq[i] = from_f<T>(x);
 }
@@ -499,6 +504,8 @@ cudaError_t launch_fa_t(const FaFusedArgs& a, cudaStream_t st) {
     p.dk = a.dk;
     p.dv = a.dv;
     p.err = a.err;
+    p.dmax = a.dout_absmax;
+    p.T1 = a.T1;
     p.B = (int)a.B;
     p.Nq = (int)a.Nq;
     p.Nkv = (int)a.Nkv;
@@ -520,7 +527,8 @@ cudaError_t launch_fa_t(const FaFusedArgs& a, cudaStream_t st) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t n = a.T1 * a.Nq * kFaD;
     if (n > 0)
-        fa_cast_dq_kernel<T, DET><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.dq_acc, n, (T*)a.dq);
+        fa_cast_dq_kernel<T, DET><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.dq_acc, n, (T*)a.dq, a.dout_absmax,
+                                                                            a.scale, a.T1, a.Nq / a.Nkv);
     return cudaGetLastError();
 }
 

@@ -50,9 +50,8 @@ __device__ __forceinline__ FaTok fa_tok(const FaArgs& a, int64_t t, int mode) {
 }
 
 template <bool DET>
-__device__ __forceinline__ void acc_add(void* acc, int64_t off, float x) {
-    if (DET) atomicAdd(reinterpret_cast<unsigned long long*>(acc) + off,
-                       (unsigned long long)__float2ll_rn(x * kFixScale));
+__device__ __forceinline__ void acc_add(void* acc, int64_t off, float x, float fmul) {
+    if (DET) atomicAdd(reinterpret_cast<unsigned long long*>(acc) + off, fix_round(x, fmul));
     else atomicAdd(reinterpret_cast<float*>(acc) + off, x);
 }
 
@@ -66,6 +65,12 @@ __global__ void __launch_bounds__(256) fa_bwd_kernel(FaArgs a) {
     const int hk = h / (int)(a.Nq / a.Nkv);
     const int D = (int)a.D;
     const FaTok ti = fa_tok(a, t, a.mode);
+    float fmul_k = 0.f, fmul_v = 0.f;  // fixed-point grids of dK and dV (deterministic mode)
+    if (DET) {
+        const FixExp fe = fix_exponents(*a.dout_absmax, a.scale, a.T1, a.Nq / a.Nkv);
+        fmul_k = fix_mul(fe.k);
+        fmul_v = fix_mul(fe.v);
+    }
     float dq[NC];
 #pragma unroll
     for (int c = 0; c < NC; ++c) dq[c] = 0.f;
@@ -110,8 +115,8 @@ __global__ void __launch_bounds__(256) fa_bwd_kernel(FaArgs a) {
                 const int d = c * 32 + lane;
                 dq[c] = fmaf(ds, kv[c], dq[c]);
                 if (d < D) {
-                    acc_add<DET>(a.dkv_acc, g + d, sds * qv[c]);
-                    acc_add<DET>(a.dkv_acc, kvD + g + d, p * dyv[c]);
+                    acc_add<DET>(a.dkv_acc, g + d, sds * qv[c], fmul_k);
+                    acc_add<DET>(a.dkv_acc, kvD + g + d, p * dyv[c], fmul_v);
                 }
             }
         }
@@ -125,12 +130,17 @@ __global__ void __launch_bounds__(256) fa_bwd_kernel(FaArgs a) {
 }
 
 template <typename T, bool DET>
-__global__ void fa_cast_kernel(const void* __restrict__ acc, int64_t n, T* __restrict__ dk, T* __restrict__ dv) {
+__global__ void fa_cast_kernel(const void* __restrict__ acc, int64_t n, T* __restrict__ dk, T* __restrict__ dv,
+                               const float* __restrict__ dmax, float scale, int64_t T1, int64_t G) {
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= 2 * n) return;
     float x;
-    if (DET) x = (float)((double)reinterpret_cast<const long long*>(acc)[i] * kFixInv);
-    else x = reinterpret_cast<const float*>(acc)[i];
+    if (DET) {
+        const FixExp fe = fix_exponents(*dmax, scale, T1, G);
+        x = (float)((double)reinterpret_cast<const long long*>(acc)[i] * fix_inv(i < n ? fe.k : fe.v));
+    } else {
+        x = reinterpret_cast<const float*>(acc)[i];
+    }
     if (i < n) dk[i] = from_f<T>(x);
     else dv[i - n] = from_f<T>(x);
 }
@@ -209,7 +219,9 @@ cudaError_t fa_bwd_dispatch(const FaArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const int64_t n = a.T2 * a.Nkv * a.D;
     if (n > 0)
-        fa_cast_kernel<T, DET><<<(unsigned)((2 * n + 255) / 256), 256, 0, st>>>(a.dkv_acc, n, (T*)a.dk, (T*)a.dv);
+        fa_cast_kernel<T, DET><<<(unsigned)((2 * n + 255) / 256), 256, 0, st>>>(a.dkv_acc, n, (T*)a.dk, (T*)a.dv,
+                                                                            a.dout_absmax, a.scale, a.T1,
+                                                                            a.Nq / a.Nkv);
     return cudaGetLastError();
 }
 

@@ -181,7 +181,8 @@ sfa_status grad_impl(const void* query, const void* key, const void* value, cons
                      const void* query_rope, const void* key_rope, float scale, int64_t sparse_block_size,
                      int64_t sparse_mode, int32_t deterministic, const sfa_shape* shape, void* workspace,
                      size_t workspace_bytes, sfa_stream_t stream, int64_t row_begin, int64_t row_end, void* acc,
-                     void* d_query, void* d_key, void* d_value, void* d_query_rope, void* d_key_rope) {
+                     const float* dout_absmax, void* d_query, void* d_key, void* d_value, void* d_query_rope,
+                     void* d_key_rope) {
     g_last_error.clear();
     Sizes z;
     sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
@@ -200,6 +201,8 @@ sfa_status grad_impl(const void* query, const void* key, const void* value, cons
     if (((uintptr_t)workspace & 255u) != 0) return fail(SFA_ERR_INVALID, "workspace not 256-byte aligned");
     if (!own_acc && ((uintptr_t)acc & 255u) != 0) return fail(SFA_ERR_INVALID, "dkv_accum not 256-byte aligned");
     const bool det = deterministic != 0;
+    if (det && !own_acc && !dout_absmax)
+        return fail(SFA_ERR_NULLPTR, "deterministic: dout_absmax (max|d_out| over every row of the accumulator) is NULL");
     const bool fused_shape = fused_supported(shape->N1);
     const GradWs ws = grad_ws_layout(z.T1, z.T2, shape->N1, shape->topk, sparse_block_size, det, fused_shape);
     if (workspace_bytes < ws.total)
@@ -220,16 +223,21 @@ sfa_status grad_impl(const void* query, const void* key, const void* value, cons
     a.dq = d_query; a.dqr = d_query_rope;
     a.dtype = shape->dtype; a.rowlist = (int32_t*)(w + ws.rowlist); a.rowcap = shape->topk * sparse_block_size;
     a.row_begin = row_begin; a.row_end = row_end;
+    // deterministic mode: the fixed-point grid follows max|dOut| (the workspace's own copy for a
+    // whole-problem call, computed below; the caller's for a row range)
+    float* own_dmax = (float*)(w + ws.ctrl + kCtrlDmax);
+    a.dout_absmax = own_acc ? own_dmax : dout_absmax;
 
     SFA_CUDA(cudaMemsetAsync(w + ws.ctrl, 0, 256, s), "zero control word");
     if (own_acc)
         SFA_CUDA(cudaMemsetAsync(a.dkv_acc, 0, (size_t)z.T2 * kAccW * (det ? 8 : 4), s), "zero dK/dV accumulator");
+    float* rowsum_dmax = own_acc && det ? own_dmax : nullptr;  // max|dO| taken by the rowsum pass
     SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, (int32_t*)a.blocks, (int32_t*)a.nblk,
                             (int32_t*)a.nrows, s), "index compaction");
     const bool fused = fused_shape && value == key;
     if (fused) {
-        SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, row_begin, row_end, shape->N1, (float*)a.rowsum, s),
-                 "rowsum(dO*O)");
+        SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, row_begin, row_end, shape->N1, (float*)a.rowsum, s,
+                               rowsum_dmax), "rowsum(dO*O)");
         SFA_CUDA(launch_order(a.nrows, row_begin, row_end, (int32_t*)a.order, a.ctrl, s), "work order");
         // block-sparse lists sorted: consecutive selected blocks become contiguous key tiles
         if (a.bs > 1 && a.topk <= kSortMaxTopk)
@@ -241,12 +249,14 @@ sfa_status grad_impl(const void* query, const void* key, const void* value, cons
             SFA_CUDA(launch_bwd_fused(shape->dtype, a, s), "fused backward");
         }
     } else {
+        if (rowsum_dmax)
+            SFA_CUDA(launch_absmax(shape->dtype, d_out, z.T1 * shape->N1 * kD, own_dmax, s), "max|dOut|");
         KernelEvents ev(s);
         SFA_CUDA(launch_bwd_generic(shape->dtype, a, s), "backward");
     }
     if (own_acc)
-        SFA_CUDA(launch_cast_dkv(shape->dtype, det, a.dkv_acc, z.T2, d_key, d_key_rope, d_value, s),
-                 "cast dKey/dValue");
+        SFA_CUDA(launch_cast_dkv(shape->dtype, det, a.dkv_acc, z.T2, d_key, d_key_rope, d_value, s, own_dmax, scale,
+                                 z.T1, shape->N1), "cast dKey/dValue");
     return SFA_OK;
 }
 
@@ -269,7 +279,7 @@ sfa_status sfa_grad(const void* query, const void* key, const void* value, const
     if (st != SFA_OK) return st;
     return grad_impl(query, key, value, sparse_indices, d_out, out, softmax_max, softmax_sum, actual_seq_lengths_q,
                      actual_seq_lengths_kv, query_rope, key_rope, scale, sparse_block_size, sparse_mode, deterministic,
-                     shape, workspace, workspace_bytes, stream, 0, z.T1, nullptr, d_query, d_key, d_value,
+                     shape, workspace, workspace_bytes, stream, 0, z.T1, nullptr, nullptr, d_query, d_key, d_value,
                      d_query_rope, d_key_rope);
 }
 
@@ -289,27 +299,46 @@ sfa_status sfa_grad_rows(const void* query, const void* key, const void* value, 
                          const void* query_rope, const void* key_rope, float scale, int64_t sparse_block_size,
                          int64_t sparse_mode, int32_t deterministic, int64_t row_begin, int64_t row_end,
                          const sfa_shape* shape, void* workspace, size_t workspace_bytes, sfa_stream_t stream,
-                         void* dkv_accum, void* d_query, void* d_query_rope) {
+                         void* dkv_accum, const float* dout_absmax, void* d_query, void* d_query_rope) {
     if (!dkv_accum) {
         g_last_error = "dkv_accum is NULL";
         return SFA_ERR_NULLPTR;
     }
     return grad_impl(query, key, value, sparse_indices, d_out, out, softmax_max, softmax_sum, actual_seq_lengths_q,
                      actual_seq_lengths_kv, query_rope, key_rope, scale, sparse_block_size, sparse_mode, deterministic,
-                     shape, workspace, workspace_bytes, stream, row_begin, row_end, dkv_accum, d_query, nullptr,
-                     nullptr, d_query_rope, nullptr);
+                     shape, workspace, workspace_bytes, stream, row_begin, row_end, dkv_accum, dout_absmax, d_query,
+                     nullptr, nullptr, d_query_rope, nullptr);
 }
 
-sfa_status sfa_dkv_finalize(const void* dkv_accum, const sfa_shape* shape, int32_t deterministic, sfa_stream_t stream,
-                            void* d_key, void* d_value, void* d_key_rope) {
+sfa_status sfa_dout_absmax(const void* d_out, const sfa_shape* shape, int64_t row_begin, int64_t row_end,
+                           sfa_stream_t stream, float* dout_absmax) {
+    g_last_error.clear();
+    Sizes z;
+    sfa_status st = check_shape(shape, 1, 0, &z);
+    if (st != SFA_OK) return st;
+    if (!d_out || !dout_absmax) return fail(SFA_ERR_NULLPTR, "a required pointer is NULL");
+    if (row_begin < 0 || row_end < row_begin || row_end > z.T1)
+        return fail(SFA_ERR_INVALID, "row range [%lld, %lld) outside [0, %lld]", (long long)row_begin,
+                    (long long)row_end, (long long)z.T1);
+    const int64_t per_row = shape->N1 * kD;
+    const char* base = (const char*)d_out + (size_t)row_begin * per_row * 2;
+    SFA_CUDA(launch_absmax(shape->dtype, base, (row_end - row_begin) * per_row, dout_absmax, (cudaStream_t)stream),
+             "max|dOut|");
+    return SFA_OK;
+}
+
+sfa_status sfa_dkv_finalize(const void* dkv_accum, const sfa_shape* shape, int32_t deterministic,
+                            const float* dout_absmax, float scale, sfa_stream_t stream, void* d_key, void* d_value,
+                            void* d_key_rope) {
     g_last_error.clear();
     Sizes z;
     sfa_status st = check_shape(shape, 1, 0, &z);
     if (st != SFA_OK) return st;
     if (!dkv_accum || !d_key || !d_value || !d_key_rope) return fail(SFA_ERR_NULLPTR, "a required pointer is NULL");
+    if (deterministic && !dout_absmax) return fail(SFA_ERR_NULLPTR, "deterministic: dout_absmax is NULL");
     if (((uintptr_t)dkv_accum & 255u) != 0) return fail(SFA_ERR_INVALID, "dkv_accum not 256-byte aligned");
     SFA_CUDA(launch_cast_dkv(shape->dtype, deterministic != 0, dkv_accum, z.T2, d_key, d_key_rope, d_value,
-                             (cudaStream_t)stream), "cast dKey/dValue");
+                             (cudaStream_t)stream, dout_absmax, scale, z.T1, shape->N1), "cast dKey/dValue");
     return SFA_OK;
 }
 
@@ -533,6 +562,10 @@ sfa_status fa_grad(const void* q, const void* k, const void* v, const void* dy, 
         f.Nkv = shape->Nkv; f.mode = (int)sparse_mode; f.scale = (float)scale; f.det = det; f.dtype = shape->dtype;
         f.items = w + fw.items; f.nitems = (int)nitems; f.rowsum = (float*)(w + fw.rowsum); f.dq_acc = w + fw.dq;
         f.err = (int*)(w + fw.ctrl); f.dq = dq; f.dk = dk; f.dv = dv;
+        f.dout_absmax = (const float*)(w + fw.ctrl + kCtrlDmax);
+        if (det)
+            SFA_CUDA(launch_absmax(shape->dtype, dy, shape->T1 * shape->Nq * shape->D, (float*)f.dout_absmax, s),
+                     "max|dY|");
         KernelEvents ev(s);
         SFA_CUDA(launch_fa_bwd_fused(shape->dtype, f, s), "fa backward (tensor cores)");
         return SFA_OK;
@@ -544,6 +577,10 @@ sfa_status fa_grad(const void* q, const void* k, const void* v, const void* dy, 
     a.cu_q = cuq; a.cu_kv = cukv; a.B = shape->B; a.T1 = shape->T1; a.T2 = shape->T2; a.Nq = shape->Nq;
     a.Nkv = shape->Nkv; a.D = shape->D; a.mode = (int)sparse_mode; a.scale = (float)scale; a.det = det;
     a.dkv_acc = acc; a.dq = dq; a.dk = dk; a.dv = dv;
+    a.dout_absmax = (const float*)(w + kCtrlDmax);
+    if (det)
+        SFA_CUDA(launch_absmax(shape->dtype, dy, shape->T1 * shape->Nq * shape->D, (float*)a.dout_absmax, s),
+                 "max|dY|");
     KernelEvents ev(s);
     SFA_CUDA(launch_fa_bwd(shape->dtype, a, s), "fa backward");
     return SFA_OK;

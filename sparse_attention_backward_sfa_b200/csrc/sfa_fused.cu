@@ -80,6 +80,7 @@ struct FusedParams {
     void* dq_out;            // dQuery [T1][N1][512]
     void* dqr_out;           // dQueryRope [T1][N1][64]
     int* err;                // device error word
+    const float* dmax;       // deterministic mode: max|dOut| that sets the fixed-point grid
     int64_t T1;
     int64_t nwork;           // entries of `order` (query rows processed by this launch)
     int64_t cap;
@@ -182,7 +183,7 @@ __device__ __forceinline__ void flush_dq(const float (&v)[32], int mode, int cc,
 
 template <bool DET, int N1>
 __device__ __forceinline__ void flush_chunk(const float (&v)[32], int kind, int cc, int t, int dim, const int32_t* rid,
-                                            int nvalid, const FusedParams& prm) {
+                                            int nvalid, const FusedParams& prm, float fmul) {
     const size_t col = kind == 2 ? kDK + dim : dim;
     const int32_t* r = rid + cc * 32;
     const int lim = nvalid - cc * 32;
@@ -192,7 +193,7 @@ __device__ __forceinline__ void flush_chunk(const float (&v)[32], int kind, int 
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
             const size_t off = (size_t)(uint32_t)r[e] * kAccW;
-            if (DET) atomicAdd(d64 + off, (unsigned long long)__float2ll_rn(v[e] * kFixScale));
+            if (DET) atomicAdd(d64 + off, fix_round(v[e], fmul));
             else atomicAdd(d32 + off, v[e]);
         }
     } else {
@@ -200,7 +201,7 @@ __device__ __forceinline__ void flush_chunk(const float (&v)[32], int kind, int 
         for (int e = 0; e < 32; ++e) {
             if (e < lim) {
                 const size_t off = (size_t)(uint32_t)r[e] * kAccW;
-                if (DET) atomicAdd(d64 + off, (unsigned long long)__float2ll_rn(v[e] * kFixScale));
+                if (DET) atomicAdd(d64 + off, fix_round(v[e], fmul));
                 else atomicAdd(d32 + off, v[e]);
             }
         }
@@ -598,6 +599,12 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
         int blk_ctr = 0;
         bool ok = true;
         const int ep = threadIdx.x - 128;  // 0..255 across the flush warps
+        float fmul_k = 0.f, fmul_v = 0.f;  // fixed-point grids of dK~ and dV (deterministic mode)
+        if (DET) {
+            const FixExp fe = fix_exponents(*prm.dmax, prm.scale, prm.T1, N1);
+            fmul_k = fix_mul(fe.k);
+            fmul_v = fix_mul(fe.v);
+        }
         for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
             const int t = prm.order[w];
             const int n = prm.nrows[t];
@@ -637,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                             tmem_ld32(T_STG(stg) + lane_base + cc * 32, v);
                             tmem_wait_ld();
                             if (kind == 0) flush_dq<T, N1>(v, dqmode, cc, t, dim, prm);
-                            else flush_chunk<DET, N1>(v, kind, cc, t, dim, rid, nvalid, prm);
+                            else flush_chunk<DET, N1>(v, kind, cc, t, dim, rid, nvalid, prm, kind == 2 ? fmul_v : fmul_k);
                         }
                     }
                     tc_fence_before();
@@ -683,6 +690,7 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
     p.dq_out = a.dq;
     p.dqr_out = a.dqr;
     p.err = a.ctrl;
+    p.dmax = a.dout_absmax;
     p.T1 = T1;
     p.nwork = a.row_end - a.row_begin;
     p.cap = a.rowcap;

@@ -25,10 +25,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 template <bool DET>
-__device__ __forceinline__ void scatter_add(void* acc, int64_t off, float x) {
+__device__ __forceinline__ void scatter_add(void* acc, int64_t off, float x, float fmul) {
     if (DET) {
-        long long q = __float2ll_rn(x * kFixScale);
-        atomicAdd(reinterpret_cast<unsigned long long*>(acc) + off, (unsigned long long)q);
+        atomicAdd(reinterpret_cast<unsigned long long*>(acc) + off, fix_round(x, fmul));
     } else {
         atomicAdd(reinterpret_cast<float*>(acc) + off, x);
     }
@@ -51,6 +50,12 @@ __global__ void __launch_bounds__(256) sfa_bwd_generic_kernel(GradArgs a) {
     float dq[kQC];
 #pragma unroll
     for (int c = 0; c < kQC; ++c) dq[c] = 0.f;
+    float fmul_k = 0.f, fmul_v = 0.f;  // fixed-point grids of dK~ and dV (deterministic mode)
+    if (DET) {
+        const FixExp fe = fix_exponents(*a.dout_absmax, a.scale, a.sd.T1, a.N1);
+        fmul_k = fix_mul(fe.k);
+        fmul_v = fix_mul(fe.v);
+    }
 
     if (ti.valid) {
         float qv[kQC], dov[kVC];
@@ -103,10 +108,10 @@ __global__ void __launch_bounds__(256) sfa_bwd_generic_kernel(GradArgs a) {
 #pragma unroll
                 for (int c = 0; c < kQC; ++c) {
                     dq[c] = fmaf(ds, kv[c], dq[c]);
-                    scatter_add<DET>(acc, rowoff + c * 32 + lane, sds * qv[c]);
+                    scatter_add<DET>(acc, rowoff + c * 32 + lane, sds * qv[c], fmul_k);
                 }
 #pragma unroll
-                for (int c = 0; c < kVC; ++c) scatter_add<DET>(acc, rowoff + kDK + c * 32 + lane, p * dov[c]);
+                for (int c = 0; c < kVC; ++c) scatter_add<DET>(acc, rowoff + kDK + c * 32 + lane, p * dov[c], fmul_v);
             }
         }
     }

@@ -86,6 +86,7 @@ sfa_status sfa_grad_noalloc(const void* query, const void* key, const void* valu
         return nfail(SFA_ERR_NULLPTR, "a required tensor pointer is NULL");
     if (shape->layout == SFA_LAYOUT_TND && (!actual_seq_lengths_q || !actual_seq_lengths_kv))
         return nfail(SFA_ERR_NULLPTR, "TND needs actual_seq_lengths_q and actual_seq_lengths_kv");
+    if (!(scale == scale)) return nfail(SFA_ERR_INVALID, "scale is NaN");
     const int64_t T1 = shape->layout == SFA_LAYOUT_BSND ? shape->B * shape->S1 : shape->T1;
     const int64_t T2 = shape->layout == SFA_LAYOUT_BSND ? shape->B * shape->S2 : shape->T2;
     const bool det = deterministic != 0;
@@ -113,6 +114,8 @@ sfa_status sfa_grad_noalloc(const void* query, const void* key, const void* valu
     a.dq = d_query; a.dqr = d_query_rope;
     a.dtype = shape->dtype; a.rowlist = nullptr; a.rowcap = 0;
     a.row_begin = 0; a.row_end = T1;
+    float* dmax = (float*)(w + ws.ctrl + kCtrlDmax);  // max|dOut|: the deterministic fixed-point grid
+    a.dout_absmax = dmax;
 
     cudaError_t e;
     // the accumulator must start at zero; the rest of the scratch is fully rewritten
@@ -123,9 +126,12 @@ sfa_status sfa_grad_noalloc(const void* query, const void* key, const void* valu
     if ((e = launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, (int32_t*)a.blocks, (int32_t*)a.nblk,
                             (int32_t*)a.nrows, s)) != cudaSuccess)
         return nfail(SFA_ERR_CUDA, "index compaction: %s", cudaGetErrorString(e));
+    if (det && (e = launch_absmax(shape->dtype, d_out, T1 * shape->N1 * kD, dmax, s)) != cudaSuccess)
+        return nfail(SFA_ERR_CUDA, "max|dOut|: %s", cudaGetErrorString(e));
     if ((e = launch_bwd_generic(shape->dtype, a, s)) != cudaSuccess)
         return nfail(SFA_ERR_CUDA, "backward: %s", cudaGetErrorString(e));
-    if ((e = launch_cast_dkv(shape->dtype, det, a.dkv_acc, T2, d_key, d_key_rope, d_value, s)) != cudaSuccess)
+    if ((e = launch_cast_dkv(shape->dtype, det, a.dkv_acc, T2, d_key, d_key_rope, d_value, s, dmax, scale, T1,
+                             shape->N1)) != cudaSuccess)
         return nfail(SFA_ERR_CUDA, "cast dKey/dValue: %s", cudaGetErrorString(e));
     return SFA_OK;
 }

@@ -52,30 +52,62 @@ cudaError_t launch_compact(const int32_t* idx, const SeqDesc& sd, int64_t topk, 
     return cudaGetLastError();
 }
 
+// Max-merge of a non-negative float into *dst: for x >= 0 the IEEE bit patterns
+// order like the values, so an unsigned atomicMax on the bits is a float max.
+__device__ __forceinline__ void absmax_merge(float* dst, float x) {
+    atomicMax(reinterpret_cast<unsigned int*>(dst), __float_as_uint(x));
+}
+
+// Block-wide max of one value per thread (every thread gets the result in lane 0 of warp 0).
+__device__ __forceinline__ float block_max(float v) {
+    __shared__ float red[32];
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    if (w == 0) {
+        v = l < (int)(blockDim.x >> 5) ? red[l] : 0.f;
+        for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    }
+    return v;
+}
+
 // One warp per (row, head): sum over the 512 value dims of dO * O in fp32.
+// Grid-stride over the rows; with `absmax` set, max|dO| is max-merged into it
+// (one atomic per CTA).
 template <typename T>
 __global__ void rowsum_kernel(const T* __restrict__ dout, const T* __restrict__ out, int64_t rows,
-                              float* __restrict__ res) {
+                              float* __restrict__ res, float* __restrict__ absmax) {
     const int lane = threadIdx.x & 31;
-    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (r >= rows) return;
-    const uint4* a = reinterpret_cast<const uint4*>(dout + r * kD);
-    const uint4* b = reinterpret_cast<const uint4*>(out + r * kD);
-    float s = 0.f;
+    const int64_t wpb = blockDim.x >> 5;
+    float am = 0.f;
+    for (int64_t r = (int64_t)blockIdx.x * wpb + (threadIdx.x >> 5); r < rows; r += (int64_t)gridDim.x * wpb) {
+        const uint4* a = reinterpret_cast<const uint4*>(dout + r * kD);
+        const uint4* b = reinterpret_cast<const uint4*>(out + r * kD);
+        float s = 0.f;
 #pragma unroll
-    for (int c = 0; c < kD / 8 / 32; ++c) {
-        uint4 x = a[c * 32 + lane], y = b[c * 32 + lane];
-        const T* xp = reinterpret_cast<const T*>(&x);
-        const T* yp = reinterpret_cast<const T*>(&y);
+        for (int c = 0; c < kD / 8 / 32; ++c) {
+            uint4 x = a[c * 32 + lane], y = b[c * 32 + lane];
+            const T* xp = reinterpret_cast<const T*>(&x);
+            const T* yp = reinterpret_cast<const T*>(&y);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s = fmaf(to_f(xp[e]), to_f(yp[e]), s);
+            for (int e = 0; e < 8; ++e) {
+                const float xv = to_f(xp[e]);
+                s = fmaf(xv, to_f(yp[e]), s);
+                am = fmaxf(am, fabsf(xv));
+            }
+        }
+        for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) res[r] = s;
     }
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) res[r] = s;
+    if (absmax) {
+        am = block_max(am);
+        if (threadIdx.x == 0) absmax_merge(absmax, am);
+    }
 }
 
 cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t row_begin, int64_t row_end, int64_t N1,
-                          float* rowsum, cudaStream_t st) {
+                          float* rowsum, cudaStream_t st, float* absmax) {
     const int64_t rows = (row_end - row_begin) * N1;
     const int64_t first = row_begin * N1;  // (row, head) pairs before the range
     const size_t elem = 2;                  // bf16 / fp16
@@ -83,13 +115,45 @@ cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t 
     out = (const char*)out + first * kD * elem;
     rowsum += first;
     const int warps = 8;
-    unsigned grid = (unsigned)((rows + warps - 1) / warps);
     if (rows == 0) return cudaGetLastError();
+    int64_t need = (rows + warps - 1) / warps;
+    unsigned grid = (unsigned)(need < 148 * 16 ? need : 148 * 16);
     if (dtype == SFA_DTYPE_BF16)
         rowsum_kernel<__nv_bfloat16><<<grid, warps * 32, 0, st>>>((const __nv_bfloat16*)dout,
-                                                                  (const __nv_bfloat16*)out, rows, rowsum);
+                                                                  (const __nv_bfloat16*)out, rows, rowsum, absmax);
     else
-        rowsum_kernel<__half><<<grid, warps * 32, 0, st>>>((const __half*)dout, (const __half*)out, rows, rowsum);
+        rowsum_kernel<__half><<<grid, warps * 32, 0, st>>>((const __half*)dout, (const __half*)out, rows, rowsum,
+                                                           absmax);
+    return cudaGetLastError();
+}
+
+// max|x| over n 16-bit elements (8 per 16-byte load, then a scalar tail).
+template <typename T>
+__global__ void absmax_kernel(const T* __restrict__ x, int64_t n, float* __restrict__ absmax) {
+    float am = 0.f;
+    const int64_t nv = n / 8;
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += stride) {
+        const uint4 u = xv[i];
+        const T* p = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(to_f(p[e])));
+    }
+    for (int64_t i = nv * 8 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        am = fmaxf(am, fabsf(to_f(x[i])));
+    am = block_max(am);
+    if (threadIdx.x == 0) absmax_merge(absmax, am);
+}
+
+cudaError_t launch_absmax(int dtype, const void* x, int64_t n, float* absmax, cudaStream_t st) {
+    if (n <= 0) return cudaGetLastError();
+    int64_t need = (n / 8 + 255) / 256;
+    unsigned grid = (unsigned)(need < 1 ? 1 : (need < 148 * 8 ? need : 148 * 8));
+    if (dtype == SFA_DTYPE_BF16)
+        absmax_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, n, absmax);
+    else
+        absmax_kernel<__half><<<grid, 256, 0, st>>>((const __half*)x, n, absmax);
     return cudaGetLastError();
 }
 
@@ -98,8 +162,8 @@ cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t 
 __global__ void order_kernel(int64_t row_begin, int64_t row_end, int32_t* __restrict__ order,
                              int32_t* __restrict__ ctrl) {
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    (void)ctrl;
     if (i < row_end - row_begin) order[i] = (int32_t)(row_end - 1 - i);
-    if (i < 64) ctrl[i] = 0;
 }
 
 cudaError_t launch_order(const int32_t* nrows, int64_t row_begin, int64_t row_end, int32_t* order, int32_t* ctrl,
@@ -226,9 +290,11 @@ cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblk, const SeqD
 }
 
 // [T2][1088] accumulator -> dKey [T2][512], dKeyRope [T2][64], dValue [T2][512].
+// Fixed point (deterministic mode) is scaled back by the call's grid (see fix_exponents).
 template <typename T, bool DET>
 __global__ void cast_dkv_kernel(const void* __restrict__ acc, int64_t T2, T* __restrict__ dk, T* __restrict__ dkr,
-                                T* __restrict__ dv) {
+                                T* __restrict__ dv, const float* __restrict__ dmax, float scale, int64_t T1,
+                                int64_t N1) {
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // group of 4 columns
     const int64_t per_row = kAccW / 4;
     if (i >= T2 * per_row) return;
@@ -236,9 +302,11 @@ __global__ void cast_dkv_kernel(const void* __restrict__ acc, int64_t T2, T* __r
     int c = (int)(i - r * per_row) * 4;
     float v[4];
     if (DET) {
+        const FixExp fe = fix_exponents(*dmax, scale, T1, N1);
+        const double inv = fix_inv(c < kDK ? fe.k : fe.v);  // a 4-column group never straddles 576
         const long long* a = reinterpret_cast<const long long*>(acc) + r * kAccW + c;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] = (float)((double)a[e] * kFixInv);
+        for (int e = 0; e < 4; ++e) v[e] = (float)((double)a[e] * inv);
     } else {
         float4 x = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(acc) + r * kAccW + c);
         v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
@@ -252,18 +320,19 @@ __global__ void cast_dkv_kernel(const void* __restrict__ acc, int64_t T2, T* __r
 }
 
 cudaError_t launch_cast_dkv(int dtype, bool det, const void* acc, int64_t T2, void* dk, void* dkr, void* dv,
-                            cudaStream_t st) {
+                            cudaStream_t st, const float* dmax, float scale, int64_t T1, int64_t N1) {
     int64_t n = T2 * (kAccW / 4);
     if (n == 0) return cudaGetLastError();
+    if (det && !dmax) return cudaErrorInvalidValue;
     unsigned grid = (unsigned)((n + 255) / 256);
     if (dtype == SFA_DTYPE_BF16) {
         using T = __nv_bfloat16;
-        if (det) cast_dkv_kernel<T, true><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv);
-        else cast_dkv_kernel<T, false><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv);
+        if (det) cast_dkv_kernel<T, true><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv, dmax, scale, T1, N1);
+        else cast_dkv_kernel<T, false><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv, dmax, scale, T1, N1);
     } else {
         using T = __half;
-        if (det) cast_dkv_kernel<T, true><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv);
-        else cast_dkv_kernel<T, false><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv);
+        if (det) cast_dkv_kernel<T, true><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv, dmax, scale, T1, N1);
+        else cast_dkv_kernel<T, false><<<grid, 256, 0, st>>>(acc, T2, (T*)dk, (T*)dkr, (T*)dv, dmax, scale, T1, N1);
     }
     return cudaGetLastError();
 }

@@ -5,8 +5,10 @@ The query rows are processed in chunks (sfa_grad_rows): while chunk c runs on
 the compute stream, chunk c+1's query-side inputs (query, queryRope, dOut, out,
 softmax statistics) are copied host->device on a copy stream and chunk c-1's
 dQuery / dQueryRope rows are copied device->host on a third stream.  The
-key-side inputs and the indices go first; the key-side gradients are cast from
-the accumulator and copied back at the end.  PCIe is full duplex, so a step
+key-side inputs and the indices go first (in deterministic mode followed by all
+of dOut, whose largest magnitude sets the fixed-point grid before the first
+chunk runs); the key-side gradients are cast from the accumulator and copied
+back at the end.  PCIe is full duplex, so a step
 costs about max(H2D time, compute time) plus one chunk of each, instead of
 their sum.
 """
@@ -103,10 +105,19 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
     ev_shared = torch.cuda.Event()
     ev_shared.record(pl.h2d)
     ev_in, ev_out = [], []
+    dmax = None
     with torch.cuda.stream(pl.h2d):
+        if deterministic:
+            # the fixed-point grid follows max|dOut| over every row: dOut goes over first
+            dq_["do"].copy_(d_out, non_blocking=True)
+            dmax = pl._like("dmax", torch.empty(1, dtype=torch.float32))
+            dmax.zero_()
+            ops.dout_absmax(dq_["do"], dq_["q"], ds_["k"], dq_["qr"], ds_["idx"], into=dmax, stream=pl.h2d, **kw)
         for c in range(chunks):
             a, b = bounds[c], bounds[c + 1]
             for n, x in qside.items():
+                if n == "do" and deterministic:
+                    continue
                 _rows(dq_[n], T1, a, b).copy_(_rows(x, T1, a, b), non_blocking=True)
             e = torch.cuda.Event()
             e.record(pl.h2d)
@@ -120,8 +131,8 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
         ops.sfa_grad_rows(dq_["q"], ds_["k"], ds_["k"], ds_["idx"], dq_["do"], dq_["o"], dq_["mx"], dq_["sm"],
                           dq_["qr"], ds_["kr"], row_begin=a, row_end=b, dkv_accum=acc, scale=scale,
                           sparse_block_size=sparse_block_size, sparse_mode=sparse_mode, deterministic=deterministic,
-                          actual_seq_lengths_kv=skv, workspace=ws, d_query=g_dq, d_query_rope=g_dqr, stream=comp,
-                          **kw)
+                          dout_absmax=dmax, actual_seq_lengths_kv=skv, workspace=ws, d_query=g_dq,
+                          d_query_rope=g_dqr, stream=comp, **kw)
         e = torch.cuda.Event()
         e.record(comp)
         ev_out.append(e)
@@ -130,7 +141,7 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
             _rows(h_dq, T1, a, b).copy_(_rows(g_dq, T1, a, b), non_blocking=True)
             _rows(h_dqr, T1, a, b).copy_(_rows(g_dqr, T1, a, b), non_blocking=True)
     ops.sfa_dkv_finalize(acc, dq_["q"], ds_["k"], dq_["qr"], ds_["idx"], deterministic=deterministic,
-                         outputs=(g_dk, g_dv, g_dkr), stream=comp, **kw)
+                         dout_absmax=dmax, scale=scale, outputs=(g_dk, g_dv, g_dkr), stream=comp, **kw)
     pl.d2h.wait_stream(comp)
     with torch.cuda.stream(pl.d2h):
         h_dk.copy_(g_dk, non_blocking=True)

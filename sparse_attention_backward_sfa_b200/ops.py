@@ -15,6 +15,7 @@ import torch
 from . import _native as N
 
 _DT = {torch.bfloat16: N.DTYPE_BF16, torch.float16: N.DTYPE_FP16}
+ACC_WIDTH = 1088  # key-side accumulator row: dKey 512 | dKeyRope 64 | dValue 512
 
 
 def _p(t: Optional[torch.Tensor]):
@@ -34,6 +35,42 @@ def _need(cond: bool, msg: str):
 def _check16(name, t, dtype):
     _need(t.is_cuda and t.is_contiguous(), f"{name} must be a contiguous CUDA tensor")
     _need(t.dtype == dtype, f"{name} must be {dtype}")
+
+
+def _check_numel(items):
+    """The library reads raw pointers: every tensor must hold exactly the elements its layout implies."""
+    for name, t, n in items:
+        if t is not None:
+            _need(t.numel() == n, f"{name}: {t.numel()} elements, expected {n}")
+
+
+def _check_f32(name, t):
+    _need(t.is_cuda and t.is_contiguous() and t.dtype == torch.float32, f"{name}: contiguous fp32 CUDA tensor")
+
+
+def _check_outputs(outputs, likes):
+    """Caller-supplied outputs: CUDA, contiguous, the dtype and element count of the tensor each mirrors."""
+    for (name, t), like in zip(outputs, likes):
+        if t is None:
+            continue
+        _need(t.is_cuda and t.is_contiguous(), f"{name} must be a contiguous CUDA tensor")
+        _need(t.dtype == like[0], f"{name} must be {like[0]}")
+        _need(t.numel() == like[1], f"{name}: {t.numel()} elements, expected {like[1]}")
+
+
+def _check_sfa_inputs(shape, query, key, value, sparse_indices, query_rope, key_rope, d_out=None, out=None,
+                      softmax_max=None, softmax_sum=None):
+    """Element counts of the sparse attention inputs against the sizes derived from `shape`."""
+    T1, T2, N1, N2, D, Dr = shape.T1, shape.T2, shape.N1, shape.N2, shape.D, shape.Dr
+    _need(sparse_indices.is_cuda and sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(),
+          "sparse_indices: int32 contiguous CUDA tensor")
+    for name, t in (("softmax_max", softmax_max), ("softmax_sum", softmax_sum)):
+        if t is not None:
+            _check_f32(name, t)
+    _check_numel((("key", key, T2 * N2 * D), ("value", value, T2 * N2 * D), ("key_rope", key_rope, T2 * N2 * Dr),
+                  ("query_rope", query_rope, T1 * N1 * Dr), ("sparse_indices", sparse_indices, T1 * N2 * shape.topk),
+                  ("d_out", d_out, T1 * N1 * D), ("out", out, T1 * N1 * D), ("softmax_max", softmax_max, T1 * N1),
+                  ("softmax_sum", softmax_sum, T1 * N1)))
 
 
 def sfa_shape(query: torch.Tensor, key: torch.Tensor, query_rope: torch.Tensor, sparse_indices: torch.Tensor,
@@ -70,6 +107,16 @@ def _seqlens(x, layout, B):
     return x
 
 
+def _workspace(workspace, nbytes: int, device):
+    """The caller's workspace (a contiguous uint8 CUDA tensor of at least `nbytes`), or a new one."""
+    if workspace is None:
+        return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+    _need(workspace.is_cuda and workspace.is_contiguous() and workspace.dtype == torch.uint8,
+          "workspace: contiguous uint8 CUDA tensor")
+    _need(workspace.numel() >= nbytes, f"workspace: {workspace.numel()} bytes, need {nbytes}")
+    return workspace
+
+
 def sfa_grad_workspace_size(shape: N.SfaShape, sparse_block_size: int, sparse_mode: int, deterministic: bool) -> int:
     lib = N.load()
     n = ctypes.c_size_t()
@@ -88,18 +135,20 @@ def sfa_grad(query, key, value, sparse_indices, d_out, out, softmax_max, softmax
     for name, t in (("query", query), ("key", key), ("value", value), ("d_out", d_out), ("out", out),
                     ("query_rope", query_rope), ("key_rope", key_rope)):
         _check16(name, t, dt)
-    _need(sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(), "sparse_indices: int32 contiguous")
-    _need(softmax_max.dtype == torch.float32 and softmax_sum.dtype == torch.float32, "softmax stats must be fp32")
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    _check_sfa_inputs(shape, query, key, value, sparse_indices, query_rope, key_rope, d_out, out, softmax_max,
+                      softmax_sum)
     sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
     skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
     ws_bytes = sfa_grad_workspace_size(shape, sparse_block_size, sparse_mode, deterministic)
-    if workspace is None or workspace.numel() < ws_bytes:
-        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=query.device)
+    workspace = _workspace(workspace, ws_bytes, query.device)
     if outputs is None:
         outputs = (torch.empty_like(query), torch.empty_like(key), torch.empty_like(key),
                    torch.empty_like(query_rope), torch.empty_like(key_rope))
     dq, dk, dv, dqr, dkr = outputs
+    _check_outputs((("d_query", dq), ("d_key", dk), ("d_value", dv), ("d_query_rope", dqr), ("d_key_rope", dkr)),
+                   ((dt, query.numel()), (dt, key.numel()), (dt, key.numel()), (dt, query_rope.numel()),
+                    (dt, key_rope.numel())))
     N.check(lib.sfa_grad(_p(query), _p(key), _p(value), _p(sparse_indices), _p(d_out), _p(out), _p(softmax_max),
                          _p(softmax_sum), _p(sq), _p(skv), _p(query_rope), _p(key_rope), float(scale),
                          int(sparse_block_size), int(sparse_mode), int(pre_tokens), int(next_tokens),
@@ -111,7 +160,7 @@ def sfa_grad(query, key, value, sparse_indices, d_out, out, softmax_max, softmax
 def sfa_dkv_accumulator(query, key, query_rope, sparse_indices, *, layout: str, deterministic: bool,
                         actual_seq_lengths_q=None):
     """Zeroed key-side accumulator for sfa_grad_rows: [T2, 1088] (dKey | dKeyRope | dValue), fp32,
-    or int64 fixed point (value * 2^32) when deterministic."""
+    or int64 fixed point when deterministic."""
     lib = N.load()
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
     n = ctypes.c_size_t()
@@ -120,53 +169,94 @@ def sfa_dkv_accumulator(query, key, query_rope, sparse_indices, *, layout: str, 
     return torch.zeros(shape.T2, n.value // (shape.T2 * (8 if deterministic else 4)), dtype=dt, device=query.device)
 
 
+def _check_accum(dkv_accum, shape, deterministic):
+    _need(dkv_accum.is_cuda and dkv_accum.is_contiguous() and
+          dkv_accum.dtype == (torch.int64 if deterministic else torch.float32),
+          "dkv_accum: contiguous CUDA tensor, int64 when deterministic else float32")
+    _need(dkv_accum.numel() == shape.T2 * ACC_WIDTH, f"dkv_accum: {dkv_accum.numel()} elements, expected "
+          f"{shape.T2 * ACC_WIDTH}")
+
+
+def _check_absmax(dout_absmax, deterministic):
+    if deterministic:
+        _need(dout_absmax is not None, "deterministic: dout_absmax (from dout_absmax()) is required")
+    if dout_absmax is not None:
+        _need(dout_absmax.is_cuda and dout_absmax.dtype == torch.float32 and dout_absmax.numel() == 1,
+              "dout_absmax: one fp32 CUDA element")
+
+
+def dout_absmax(d_out, query, key, query_rope, sparse_indices, *, layout: str, row_begin: int = 0,
+                row_end: Optional[int] = None, actual_seq_lengths_q=None, into: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """max|d_out| over query rows [row_begin, row_end), max-merged into `into` (a 1-element fp32 CUDA
+    tensor, zeroed here when not given).  It sets the fixed-point grid of deterministic row ranges."""
+    lib = N.load()
+    shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    _check16("d_out", d_out, query.dtype)
+    _check_numel((("d_out", d_out, shape.T1 * shape.N1 * shape.D),))
+    if into is None:
+        into = torch.zeros(1, dtype=torch.float32, device=d_out.device)
+    _check_absmax(into, False)
+    N.check(lib.sfa_dout_absmax(_p(d_out), ctypes.byref(shape), int(row_begin),
+                                int(shape.T1 if row_end is None else row_end), _stream(stream), _p(into)))
+    return into
+
+
 def sfa_grad_rows(query, key, value, sparse_indices, d_out, out, softmax_max, softmax_sum, query_rope, key_rope, *,
                   row_begin: int, row_end: int, dkv_accum: torch.Tensor, scale: float, sparse_block_size: int,
-                  layout: str, sparse_mode: int, deterministic: bool = False, actual_seq_lengths_q=None,
-                  actual_seq_lengths_kv=None, workspace: Optional[torch.Tensor] = None, d_query=None,
-                  d_query_rope=None, stream=None):
+                  layout: str, sparse_mode: int, deterministic: bool = False, dout_absmax=None,
+                  actual_seq_lengths_q=None, actual_seq_lengths_kv=None, workspace: Optional[torch.Tensor] = None,
+                  d_query=None, d_query_rope=None, stream=None):
     """Backward of query rows [row_begin, row_end) (flattened row index): writes those rows of
     (dQuery, dQueryRope) and adds their dKey / dKeyRope / dValue contributions into `dkv_accum`
-    (from sfa_dkv_accumulator). Returns (dQuery, dQueryRope)."""
+    (from sfa_dkv_accumulator).  Deterministic mode needs `dout_absmax`: max|d_out| over every row
+    that goes into the accumulator (see dout_absmax()).  Returns (dQuery, dQueryRope)."""
     lib = N.load()
     dt = query.dtype
     for name, t in (("query", query), ("key", key), ("value", value), ("d_out", d_out), ("out", out),
                     ("query_rope", query_rope), ("key_rope", key_rope)):
         _check16(name, t, dt)
-    _need(sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(), "sparse_indices: int32 contiguous")
-    _need(softmax_max.dtype == torch.float32 and softmax_sum.dtype == torch.float32, "softmax stats must be fp32")
-    _need(dkv_accum.is_contiguous() and dkv_accum.dtype == (torch.int64 if deterministic else torch.float32),
-          "dkv_accum: contiguous, int64 when deterministic else float32")
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    _check_sfa_inputs(shape, query, key, value, sparse_indices, query_rope, key_rope, d_out, out, softmax_max,
+                      softmax_sum)
+    _check_accum(dkv_accum, shape, deterministic)
+    _check_absmax(dout_absmax, deterministic)
     sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
     skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
     ws_bytes = sfa_grad_workspace_size(shape, sparse_block_size, sparse_mode, deterministic)
-    if workspace is None or workspace.numel() < ws_bytes:
-        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=query.device)
+    workspace = _workspace(workspace, ws_bytes, query.device)
     if d_query is None:
         d_query = torch.zeros_like(query)
     if d_query_rope is None:
         d_query_rope = torch.zeros_like(query_rope)
+    _check_outputs((("d_query", d_query), ("d_query_rope", d_query_rope)),
+                   ((dt, query.numel()), (dt, query_rope.numel())))
     N.check(lib.sfa_grad_rows(_p(query), _p(key), _p(value), _p(sparse_indices), _p(d_out), _p(out),
                               _p(softmax_max), _p(softmax_sum), _p(sq), _p(skv), _p(query_rope), _p(key_rope),
                               float(scale), int(sparse_block_size), int(sparse_mode), int(deterministic),
                               int(row_begin), int(row_end), ctypes.byref(shape), _p(workspace), workspace.numel(),
-                              _stream(stream), _p(dkv_accum), _p(d_query), _p(d_query_rope)))
+                              _stream(stream), _p(dkv_accum), _p(dout_absmax), _p(d_query), _p(d_query_rope)))
     return d_query, d_query_rope
 
 
 def sfa_dkv_finalize(dkv_accum, query, key, query_rope, sparse_indices, *, layout: str, deterministic: bool,
-                     actual_seq_lengths_q=None, outputs=None, stream=None):
-    """Casts a (summed) key-side accumulator into 16-bit (dKey, dValue, dKeyRope)."""
+                     dout_absmax=None, scale: float = 1.0, actual_seq_lengths_q=None, outputs=None, stream=None):
+    """Casts a (summed) key-side accumulator into 16-bit (dKey, dValue, dKeyRope).  Deterministic mode
+    needs the `dout_absmax` and `scale` the accumulator was filled with."""
     lib = N.load()
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    _check_accum(dkv_accum, shape, deterministic)
+    _check_absmax(dout_absmax, deterministic)
+    kr_shape = key.shape[:-1] + (query_rope.shape[-1],)
     if outputs is None:
-        kr_shape = key.shape[:-1] + (query_rope.shape[-1],)
         outputs = (torch.empty_like(key), torch.empty_like(key),
                    torch.empty(kr_shape, dtype=key.dtype, device=key.device))
     dk, dv, dkr = outputs
-    N.check(lib.sfa_dkv_finalize(_p(dkv_accum), ctypes.byref(shape), int(deterministic), _stream(stream), _p(dk),
-                                 _p(dv), _p(dkr)))
+    n_kr = shape.T2 * shape.N2 * shape.Dr
+    _check_outputs((("d_key", dk), ("d_value", dv), ("d_key_rope", dkr)),
+                   ((key.dtype, key.numel()), (key.dtype, key.numel()), (key.dtype, n_kr)))
+    N.check(lib.sfa_dkv_finalize(_p(dkv_accum), ctypes.byref(shape), int(deterministic), _p(dout_absmax),
+                                 float(scale), _stream(stream), _p(dk), _p(dv), _p(dkr)))
     return dk, dv, dkr
 
 
@@ -180,13 +270,12 @@ def sfa_fwd(query, key, value, sparse_indices, query_rope, key_rope, *, scale: f
                     ("key_rope", key_rope)):
         _check16(name, t, dt)
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    _check_sfa_inputs(shape, query, key, value, sparse_indices, query_rope, key_rope)
     sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
     skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
     n = ctypes.c_size_t()
     N.check(lib.sfa_fwd_workspace_size(ctypes.byref(shape), sparse_block_size, sparse_mode, ctypes.byref(n)))
-    ws = workspace
-    if ws is None or ws.numel() < n.value:
-        ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=query.device)
+    ws = _workspace(workspace, n.value, query.device)
     out = torch.empty_like(query)
     stat_shape = query.shape[:-1]
     smax = torch.empty(stat_shape, dtype=torch.float32, device=query.device)
@@ -202,6 +291,9 @@ def compact_indices(sparse_indices, key, query, query_rope, *, sparse_block_size
     """Index compaction step; returns (blocks [T1, topk], nblocks [T1], nrows [T1]) int32."""
     lib = N.load()
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    _need(sparse_indices.is_cuda and sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(),
+          "sparse_indices: int32 contiguous CUDA tensor")
+    _check_numel((("sparse_indices", sparse_indices, shape.T1 * shape.N2 * shape.topk),))
     sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
     skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
     dev = sparse_indices.device
@@ -218,6 +310,9 @@ def softmax_grad_rowsum(d_out, out, key, query_rope, sparse_indices, *, layout: 
     """FlashSoftmaxGrad(dO, O): fp32 [T1, N1] row sums of dO o O."""
     lib = N.load()
     shape = sfa_shape(d_out, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    _check16("d_out", d_out, d_out.dtype)
+    _check16("out", out, d_out.dtype)
+    _check_numel((("out", out, d_out.numel()),))
     res = torch.empty(shape.T1 * shape.N1, dtype=torch.float32, device=d_out.device)
     N.check(lib.sfa_softmax_grad_rowsum(_p(d_out), _p(out), ctypes.byref(shape), _stream(stream), _p(res)))
     return res.view(shape.T1, shape.N1)
@@ -226,11 +321,22 @@ def softmax_grad_rowsum(d_out, out, key, query_rope, sparse_indices, *, layout: 
 def _fa_shape(q, k, cu_q, cu_kv) -> N.FaShape:
     s = N.FaShape()
     _need(q.dtype in _DT, "q must be bf16 or fp16")
+    _need(q.dim() == 3 and k.dim() == 3, "TND tensors are 3-D")
+    _need(len(cu_q) == len(cu_kv), "cu_seqlens_q and cu_seqlens_kv need the same length B")
     s.dtype = _DT[q.dtype]
     s.B = len(cu_q)
     s.T1, s.Nq, s.D = q.shape
     s.T2, s.Nkv, _ = k.shape
     return s
+
+
+def _check_fa_inputs(s, k=None, v=None, dy=None, softmax_max=None, softmax_sum=None, attention_in=None):
+    for name, t in (("softmax_max", softmax_max), ("softmax_sum", softmax_sum)):
+        if t is not None:
+            _check_f32(name, t)
+    _check_numel((("k", k, s.T2 * s.Nkv * s.D), ("v", v, s.T2 * s.Nkv * s.D), ("dy", dy, s.T1 * s.Nq * s.D),
+                  ("attention_in", attention_in, s.T1 * s.Nq * s.D), ("softmax_max", softmax_max, s.T1 * s.Nq * 8),
+                  ("softmax_sum", softmax_sum, s.T1 * s.Nq * 8)))
 
 
 def _host_i64(x: Sequence[int]):
@@ -246,13 +352,15 @@ def fa_grad(q, k, v, dy, softmax_max, softmax_sum, attention_in, cu_seqlens_q, c
     for name, t in (("q", q), ("k", k), ("v", v), ("dy", dy), ("attention_in", attention_in)):
         _check16(name, t, q.dtype)
     shape = _fa_shape(q, k, cu_seqlens_q, cu_seqlens_kv)
+    _check_fa_inputs(shape, k, v, dy, softmax_max, softmax_sum, attention_in)
     n = ctypes.c_size_t()
     N.check(lib.fa_grad_workspace_size(ctypes.byref(shape), int(sparse_mode), int(deterministic), ctypes.byref(n)))
-    if workspace is None or workspace.numel() < n.value:
-        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
+    workspace = _workspace(workspace, n.value, q.device)
     if outputs is None:
         outputs = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     dq, dk, dv = outputs
+    _check_outputs((("dq", dq), ("dk", dk), ("dv", dv)),
+                   ((q.dtype, q.numel()), (q.dtype, k.numel()), (q.dtype, v.numel())))
     aq, pq = _host_i64(cu_seqlens_q)
     akv, pkv = _host_i64(cu_seqlens_kv)
     N.check(lib.fa_grad(_p(q), _p(k), _p(v), _p(dy), _p(softmax_max), _p(softmax_sum), _p(attention_in), pq, pkv,
@@ -266,7 +374,10 @@ def fa_grad(q, k, v, dy, softmax_max, softmax_sum, attention_in, cu_seqlens_q, c
 def fa_fwd(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, scale: float, sparse_mode: int, stream=None):
     """Dense varlen FA forward (TND). Returns (out, softmaxMax [T1,Nq,8], softmaxSum [T1,Nq,8])."""
     lib = N.load()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check16(name, t, q.dtype)
     shape = _fa_shape(q, k, cu_seqlens_q, cu_seqlens_kv)
+    _check_fa_inputs(shape, k, v)
     n = ctypes.c_size_t()
     N.check(lib.fa_fwd_workspace_size(ctypes.byref(shape), int(sparse_mode), ctypes.byref(n)))
     ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
@@ -333,22 +444,30 @@ def lig_kl_grad(query, key, query_index, key_index, weights, softmax_max, softma
                     ("actual_seq_lengths_key", actual_seq_lengths_key)):
         _need(t is None or (t.is_cuda and t.dtype == torch.int64 and t.is_contiguous()),
               f"{name}: int64 CUDA tensor")
+    if layout == "TND":
+        _need(actual_seq_lengths_key is not None, "TND needs actual_seq_lengths_key")
     shape = lig_shape(query, key, query_index, key_index, layout, actual_seq_lengths_query, query_rope)
     # the library sees raw pointers: every tensor must hold exactly the elements its layout implies
     T1, T2 = shape.T1, shape.T2
-    for name, t, n in (("key", key, T2 * shape.D), ("key_index", key_index, T2 * shape.Di),
+    for name, t in (("actual_seq_lengths_query", actual_seq_lengths_query),
+                    ("actual_seq_lengths_key", actual_seq_lengths_key)):
+        _need(t is None or t.numel() == shape.B, f"{name}: {shape.B} elements expected")
+    for name, t, n in (("query_index", query_index, T1 * shape.G * shape.Di),
+                       ("key", key, T2 * shape.D), ("key_index", key_index, T2 * shape.Di),
                        ("weights", weights, T1 * shape.G), ("query_rope", query_rope, T1 * shape.N1 * shape.Dr),
                        ("key_rope", key_rope, T2 * shape.Dr), ("softmax_max", softmax_max, T1 * shape.N1),
                        ("softmax_sum", softmax_sum, T1 * shape.N1), ("softmax_max_index", softmax_max_index, T1),
                        ("softmax_sum_index", softmax_sum_index, T1)):
         _need(t.numel() == n, f"{name}: {t.numel()} elements, expected {n}")
     need = lig_kl_grad_workspace_size(shape, sparse_mode)
-    if workspace is None or workspace.numel() < need:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=query.device)
+    workspace = _workspace(workspace, need, query.device)
     if outputs is None:
         outputs = (torch.empty_like(query_index), torch.empty_like(key_index), torch.empty_like(weights),
                    torch.empty(1, dtype=torch.float32, device=query.device))
     dqi, dki, dw, loss = outputs
+    dt = query.dtype
+    _check_outputs((("d_query_index", dqi), ("d_key_index", dki), ("d_weights", dw), ("loss", loss)),
+                   ((dt, T1 * shape.G * shape.Di), (dt, T2 * shape.Di), (dt, T1 * shape.G), (torch.float32, 1)))
     N.check(lib.lig_kl_grad(_p(query), _p(key), _p(query_index), _p(key_index), _p(weights), _p(softmax_max),
                             _p(softmax_sum), _p(softmax_max_index), _p(softmax_sum_index), _p(query_rope),
                             _p(key_rope), _p(actual_seq_lengths_query), _p(actual_seq_lengths_key), float(scale),

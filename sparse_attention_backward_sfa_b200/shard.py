@@ -6,8 +6,10 @@ replicated, and the ranks then sum their key-side accumulators with one
 all-reduce: dKey, dKeyRope and dValue are sums over every query row that
 selected a key (SparseFlashAttentionGrad README, 功能说明), so partial sums over
 disjoint row sets add up to the whole.  dQuery rows stay on the rank that owns
-them.  In deterministic mode the accumulator is int64 fixed point, so the
-all-reduce is exact and the result does not depend on the rank count or order.
+them.  In deterministic mode the accumulator is int64 fixed point on a grid set
+by max|dOut| over all ranks' rows (one max all-reduce of a single float first),
+so the sum all-reduce is exact and the result does not depend on the rank count
+or order.
 """
 from __future__ import annotations
 
@@ -89,14 +91,22 @@ def sfa_grad_sharded(query, key, value, sparse_indices, d_out, out, softmax_max,
     if outputs is None:
         outputs = (torch.zeros_like(query), None, None, torch.zeros_like(query_rope), None)
     dq, dk, dv, dqr, dkr = outputs
+    dmax = None
+    if deterministic:
+        # the fixed-point grid follows max|dOut| over ALL ranks' rows: every rank must use the same one
+        dmax = ops.dout_absmax(d_out, query, key, query_rope, sparse_indices, row_begin=rb, row_end=re_,
+                               stream=stream, **kw)
+        if world > 1:
+            dist.all_reduce(dmax, op=dist.ReduceOp.MAX, group=group)
     ops.sfa_grad_rows(query, key, value, sparse_indices, d_out, out, softmax_max, softmax_sum, query_rope, key_rope,
                       row_begin=rb, row_end=re_, dkv_accum=dkv_accum, scale=scale,
                       sparse_block_size=sparse_block_size, sparse_mode=sparse_mode, deterministic=deterministic,
-                      actual_seq_lengths_kv=actual_seq_lengths_kv, workspace=workspace, d_query=dq,
-                      d_query_rope=dqr, stream=stream, **kw)
+                      dout_absmax=dmax, actual_seq_lengths_kv=actual_seq_lengths_kv, workspace=workspace,
+                      d_query=dq, d_query_rope=dqr, stream=stream, **kw)
     if world > 1:
         dist.all_reduce(dkv_accum, op=dist.ReduceOp.SUM, group=group)
     key_outs = None if dk is None else (dk, dv, dkr)
     dk, dv, dkr = ops.sfa_dkv_finalize(dkv_accum, query, key, query_rope, sparse_indices,
-                                       deterministic=deterministic, outputs=key_outs, stream=stream, **kw)
+                                       deterministic=deterministic, dout_absmax=dmax, scale=scale, outputs=key_outs,
+                                       stream=stream, **kw)
     return dq, dk, dv, dqr, dkr, (rb, re_)

@@ -42,15 +42,23 @@ def sharded(dp, ranges, det, separate=False):
     accs = []
     dq = torch.zeros_like(dp.q)
     dqr = torch.zeros_like(dp.qr)
+    dmax = None
+    if det:
+        # each range's max|dOut| max-merged: what the ranks' max all-reduce computes
+        dmax = torch.zeros(1, dtype=torch.float32, device=dp.q.device)
+        for rb, re_ in ranges:
+            S.dout_absmax(dp.do, dp.q, dp.k, dp.qr, dp.idx, layout=kw["layout"], row_begin=rb, row_end=re_,
+                          actual_seq_lengths_q=dp.sq, into=dmax)
     for rb, re_ in ranges:
         a = mk() if separate else acc
         S.sfa_grad_rows(dp.q, dp.k, dp.v, dp.idx, dp.do, dp.out, dp.smax, dp.ssum, dp.qr, dp.kr, row_begin=rb,
-                        row_end=re_, dkv_accum=a, deterministic=det, d_query=dq, d_query_rope=dqr, **kw)
+                        row_end=re_, dkv_accum=a, deterministic=det, dout_absmax=dmax, d_query=dq,
+                        d_query_rope=dqr, **kw)
         accs.append(a)
     if separate:
         acc = torch.stack(accs).sum(0)  # what an all-reduce of the ranks' accumulators computes
     dk, dv, dkr = S.sfa_dkv_finalize(acc, dp.q, dp.k, dp.qr, dp.idx, layout=kw["layout"], deterministic=det,
-                                     actual_seq_lengths_q=dp.sq)
+                                     dout_absmax=dmax, scale=kw["scale"], actual_seq_lengths_q=dp.sq)
     return dq, dk, dv, dqr, dkr
 
 

@@ -93,12 +93,17 @@ def _worker(rank, world, port, results):
         ops.compact_indices = lambda *a, **k: (None, None, work.clone())
         ops.sfa_dkv_accumulator = lambda *a, **k: torch.zeros(T2, 3, dtype=torch.int64)
 
-        def fake_rows(*a, row_begin, row_end, dkv_accum, d_query, d_query_rope, **k):
+        seen_dmax = []
+
+        def fake_rows(*a, row_begin, row_end, dkv_accum, d_query, d_query_rope, dout_absmax=None, **k):
             calls.append((row_begin, row_end))
+            seen_dmax.append(None if dout_absmax is None else float(dout_absmax))
             dkv_accum[row_begin:row_end] += 1      # each row "contributes" to the key row of the same index
             d_query[row_begin:row_end] = rank + 1
             return d_query, d_query_rope
 
+        # each rank's own max|dOut| differs; the grid must use the max over ranks
+        ops.dout_absmax = lambda *a, **k: torch.tensor([float(rank + 3)])
         ops.sfa_grad_rows = fake_rows
         ops.sfa_dkv_finalize = lambda acc, *a, **k: (acc.clone(), acc.clone(), acc.clone())
         q = torch.zeros(T1, 2)
@@ -106,7 +111,7 @@ def _worker(rank, world, port, results):
                                                        None, scale=1.0, sparse_block_size=1, layout="TND",
                                                        sparse_mode=0, deterministic=True)
         expect = balanced_row_ranges(work.numpy(), world)[rank]
-        ok2 = (calls == [expect] and rng_ == expect and bool((dk == 1).all())
+        ok2 = (calls == [expect] and rng_ == expect and bool((dk == 1).all()) and seen_dmax == [float(world + 2)]
                and bool((dq[expect[0]:expect[1]] == rank + 1).all())
                and bool((dq[:expect[0]] == 0).all()) and bool((dq[expect[1]:] == 0).all()))
         results[rank] = (ok1, ok2)
