@@ -220,19 +220,21 @@ def run_ours(args, rank, world, local_rank):
     for a, b in evs:  # torch creates the CUDA event on first record; the hook needs real handles
         a.record(stream)
         b.record(stream)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # one event at every step boundary: per-step durations for the median, no extra synchronization
+    bnd = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     with ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank) as clk:
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-        t0.record(stream)
+        bnd[0].record(stream)
         for i in range(args.steps):
             step(evs[i])
-        t1.record(stream)
+            bnd[i + 1].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    ms_total = t0.elapsed_time(t1)
+    ms_total = bnd[0].elapsed_time(bnd[-1])
+    step_ms = [bnd[i].elapsed_time(bnd[i + 1]) for i in range(args.steps)]
     kern_ms = [a.elapsed_time(b) for a, b in evs]
     err = ws[:256].view(torch.int32)  # device error word of the fused kernel (first bytes of the workspace)
     ms_step = ms_total / args.steps
@@ -313,7 +315,7 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     err_word = int(err[0].item())
-    return dict(flop=flop, flop_rank=flop_rank, triples=triples, ms_step=ms_step, kern_ms=kern_ms,
+    return dict(flop=flop, flop_rank=flop_rank, triples=triples, ms_step=ms_step, kern_ms=kern_ms, step_ms=step_ms,
                 clocks=clk.summary(), e2e=e2e, ws_bytes=ws_bytes, err_word=err_word, p=p, sharded=sharded,
                 rows=(rb, re_))
 
@@ -621,21 +623,30 @@ def ctypes_ptr(ev):
     return ctypes.c_void_p(ev.cuda_event)
 
 
+class _SampledRows:
+    """Row access t -> the oracle forward's output row for a sorted sample of query rows."""
+
+    def __init__(self, arr, toks, n):
+        self._rows = {int(t): arr[i] for i, t in enumerate(toks)}
+        self._n = n
+
+    def __len__(self):
+        return self._n
+
+    def __getitem__(self, t):
+        return self._rows[int(t)]
+
+
 def cpu_baseline(workload: int, budget_s: float):
     """Time the oracle (fp64 numpy, as it stands) on a bounded sample of query
-    rows of the same workload on this host's cores."""
+    rows of the same workload on this host's cores.  O and the softmax statistics
+    of the sampled rows come from the oracle's own forward (input preparation,
+    not timed), so this arm runs no code of the library."""
     import torch
     from oracle import sfa_oracle as O
     from workloads import RowView
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     p = build_problem(workload, 0, dev)
-    import sparse_attention_backward_sfa_b200 as S
-    if dev == "cuda":
-        out, smax, ssum = S.sfa_fwd(p.q, p.k, p.k, p.indices, p.q_rope, p.k_rope, **kw(p))
-    else:
-        out = torch.zeros_like(p.q)
-        smax = torch.zeros(p.q.shape[:-1])
-        ssum = torch.ones(p.q.shape[:-1])
     rng = np.random.default_rng(12345)
     T1 = p.T1
     k = p.k.reshape(p.T2, p.D).float().cpu().numpy()
@@ -645,8 +656,10 @@ def cpu_baseline(workload: int, budget_s: float):
     n = 2
     while elapsed < budget_s and done_tokens < T1:
         toks = np.sort(rng.choice(T1, size=n, replace=False))
-        views = [RowView(x, toks, T1) for x in (p.q, p.q_rope, p.dout, out, smax, ssum, p.indices)]
-        qv, qrv, dov, ov, mv, lv, iv = views
+        qv, qrv, dov, iv = (RowView(x, toks, T1) for x in (p.q, p.q_rope, p.dout, p.indices))
+        out, m, l = O.sfa_forward(qv, k, k, iv, qrv, kr, p.scale, p.block_size, p.sparse_mode, p.layout, p.B, p.S1,
+                                  p.S2, sq, sq, tokens=toks)
+        ov, mv, lv = (_SampledRows(a, toks, T1) for a in (out, m, l))
         c0 = time.perf_counter()
         O.sfa_backward(qv, k, k, iv, dov, ov, mv, lv, qrv, kr, p.scale, p.block_size, p.sparse_mode, p.layout,
                        p.B, p.S1, p.S2, sq, sq, tokens=toks)
@@ -666,7 +679,8 @@ def cpu_baseline(workload: int, budget_s: float):
     cores = len(os.sched_getaffinity(0))
     return {"value": flop / elapsed / 1e12 if elapsed > 0 else 0.0, "unit": "TFLOP/s", "cores": cores,
             "kind": "oracle", "sample": f"{done_tokens} query rows of workload {workload} "
-                                        f"(fp64 numpy oracle, {elapsed:.1f} s)", "seconds": elapsed}
+                                        f"(fp64 numpy oracle, {elapsed:.1f} s; O and statistics of those rows "
+                                        f"from the oracle forward, not timed)", "seconds": elapsed}
 
 
 def main():
@@ -762,7 +776,9 @@ def main():
         p = r["p"]
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": r["ms_step"], "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": r["ms_step"],
+            "ms_per_step_median": statistics.median(r["step_ms"]),
+            "ms_per_step_min_max": [min(r["step_ms"]), max(r["step_ms"])], "higher_is_better": True,
             "scaling": "strong" if sharded else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "pct_of_peak": 100.0 * value / world / peak,
@@ -778,6 +794,7 @@ def main():
                          "peak_sustained": float(peaks.get("bf16_tflops_sustained", peak)),
                          "frac_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                          "kernel": "sfa_bwd_fused_kernel", "kernel_ms": kern,
+                         "kernel_ms_median": statistics.median(r["kern_ms"]),
                          "traffic": recorded_traffic(4) if args.workload == 4 and not args.seqs and not sharded
                          else None},
             "cpu_baseline": cpu,

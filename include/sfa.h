@@ -284,6 +284,27 @@ sfa_status sfa_compact_indices(const int32_t *sparse_indices, const int32_t *act
                                int32_t *nblocks_out, int32_t *nrows_out);
 
 /*
+ * The gathered key rows of every query row, as the fused kernels read them
+ * (the Gather of the SparseFlashAttentionGrad README, 功能说明: an index i selects
+ * rows [i*bs, i*bs+bs) of the token's batch / sequence, cut by S2_b and by the
+ * sparseMode 3 bound of 约束说明).  Runs the index compaction (outputs as in
+ * sfa_compact_indices), optionally sorts each row's kept blocks ascending
+ * (sorted != 0; topk <= 4096), then expands the blocks into global key-row ids
+ * (flattened [T2] view):
+ *   block_aligned == 0: rows_out[t*topk*bs + 0 .. n-1] = the kept rows in block
+ *     order, count_out[t] = n (the row count of sfa_compact_indices);
+ *   block_aligned != 0: block i of row t takes slots [i*bs, i*bs+bs) holding the
+ *     block's consecutive rows, slots past the block's kept rows carrying the row
+ *     id with bit 31 set; count_out[t] = blocks * bs.
+ * blocks_out [T1*topk], nblocks_out / count_out [T1], rows_out [T1*topk*bs]:
+ * int32, device.  Slots past count_out[t] are left unwritten.
+ */
+sfa_status sfa_key_rows(const int32_t *sparse_indices, const int32_t *actual_seq_lengths_q,
+                        const int32_t *actual_seq_lengths_kv, int64_t sparse_block_size, int64_t sparse_mode,
+                        const sfa_shape *shape, int32_t sorted, int32_t block_aligned, sfa_stream_t stream,
+                        int32_t *blocks_out, int32_t *nblocks_out, int32_t *rows_out, int32_t *count_out);
+
+/*
  * FlashSoftmaxGrad(dO, O) of stage 2 (SparseFlashAttentionGrad README): the fp32
  * row sum over the D value dims of dOut o out, one value per (query row, head):
  * rowsum_out fp32 [T1, N1] (BSND: [B*S1, N1]).

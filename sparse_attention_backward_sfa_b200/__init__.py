@@ -7,6 +7,7 @@ from .ops import (  # noqa: F401
     dout_absmax,
     fa_fwd,
     fa_grad,
+    key_rows,
     lig_kl_grad,
     lig_kl_grad_workspace_size,
     lig_shape,
@@ -28,4 +29,4 @@ __all__ = ["sfa_grad", "sfa_fwd", "fa_grad", "fa_fwd", "compact_indices", "softm
            "sfa_grad_workspace_size", "sfa_shape", "SfaError", "load", "sfa_grad_rows", "sfa_dkv_accumulator",
            "sfa_dkv_finalize", "sfa_grad_sharded", "balanced_row_ranges", "sfa_grad_host", "HostPipeline",
            "workspace_status", "set_wait_limit", "lig_kl_grad", "lig_kl_grad_workspace_size", "lig_shape",
-           "dout_absmax"]
+           "dout_absmax", "key_rows"]

@@ -66,6 +66,7 @@ SIGNATURES = {
     "sfa_fwd_workspace_size": [_PSH, _I64, _I64, _PSZ],
     "sfa_fwd": [_V, _V, _V, _V, _V, _V, _V, _V, _F, _I64, _I64, _PSH, _V, _SZ, _V, _V, _V, _V],
     "sfa_compact_indices": [_V, _V, _V, _I64, _I64, _PSH, _V, _V, _V, _V],
+    "sfa_key_rows": [_V, _V, _V, _I64, _I64, _PSH, _I32, _I32, _V, _V, _V, _V, _V],
     "sfa_softmax_grad_rowsum": [_V, _V, _PSH, _V, _V],
     "fa_grad_workspace_size": [_PFA, _I64, _I32, _PSZ],
     "fa_grad": [_V, _V, _V, _V, _V, _V, _V, _V, _V, _Dbl, _Dbl, _I64, _I64, _I64, _I64, _I32, _PFA, _V, _SZ, _V,

@@ -434,6 +434,36 @@ sfa_status sfa_compact_indices(const int32_t* sparse_indices, const int32_t* act
     return SFA_OK;
 }
 
+sfa_status sfa_key_rows(const int32_t* sparse_indices, const int32_t* actual_seq_lengths_q,
+                        const int32_t* actual_seq_lengths_kv, int64_t sparse_block_size, int64_t sparse_mode,
+                        const sfa_shape* shape, int32_t sorted, int32_t block_aligned, sfa_stream_t stream,
+                        int32_t* blocks_out, int32_t* nblocks_out, int32_t* rows_out, int32_t* count_out) {
+    g_last_error.clear();
+    Sizes z;
+    sfa_status st = check_shape(shape, sparse_block_size, sparse_mode, &z);
+    if (st != SFA_OK) return st;
+    if (!sparse_indices || !blocks_out || !nblocks_out || !rows_out || !count_out)
+        return fail(SFA_ERR_NULLPTR, "a required pointer is NULL");
+    if (shape->layout == SFA_LAYOUT_TND && (!actual_seq_lengths_q || !actual_seq_lengths_kv))
+        return fail(SFA_ERR_NULLPTR, "TND needs actual_seq_lengths_q and actual_seq_lengths_kv");
+    if (sorted && shape->topk > kSortMaxTopk)
+        return fail(SFA_ERR_INVALID, "sorted lists need topk <= %lld", (long long)kSortMaxTopk);
+    cudaStream_t s = (cudaStream_t)stream;
+    SeqDesc sd = seq_desc(shape, z, actual_seq_lengths_q, actual_seq_lengths_kv);
+    const int bs = (int)sparse_block_size;
+    const int64_t cap = shape->topk * sparse_block_size;
+    SFA_CUDA(launch_compact(sparse_indices, sd, shape->topk, bs, (int)sparse_mode, blocks_out, nblocks_out, count_out,
+                            s), "index compaction");
+    if (sorted) SFA_CUDA(launch_sort_blocks(blocks_out, nblocks_out, shape->topk, 0, z.T1, s), "block sort");
+    if (block_aligned)
+        SFA_CUDA(launch_expand_blocks(blocks_out, nblocks_out, sd, shape->topk, bs, (int)sparse_mode, cap, rows_out,
+                                      count_out, s), "key row expansion");
+    else
+        SFA_CUDA(launch_expand(blocks_out, nblocks_out, sd, shape->topk, bs, (int)sparse_mode, cap, rows_out, s),
+                 "key row expansion");
+    return SFA_OK;
+}
+
 sfa_status sfa_softmax_grad_rowsum(const void* d_out, const void* out, const sfa_shape* shape, sfa_stream_t stream,
                                    float* rowsum_out) {
     g_last_error.clear();

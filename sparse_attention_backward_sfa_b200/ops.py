@@ -305,6 +305,29 @@ def compact_indices(sparse_indices, key, query, query_rope, *, sparse_block_size
     return blocks, nb, nr
 
 
+def key_rows(sparse_indices, key, query, query_rope, *, sparse_block_size: int, layout: str, sparse_mode: int,
+             sorted_blocks: bool = False, block_aligned: bool = False, actual_seq_lengths_q=None,
+             actual_seq_lengths_kv=None, stream=None):
+    """Gathered key rows per query row (sfa_key_rows); returns (blocks [T1, topk], nblocks [T1],
+    rows [T1, topk*bs], count [T1]) int32.  Block-aligned lists flag padding slots with bit 31."""
+    lib = N.load()
+    shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
+    _need(sparse_indices.is_cuda and sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(),
+          "sparse_indices: int32 contiguous CUDA tensor")
+    _check_numel((("sparse_indices", sparse_indices, shape.T1 * shape.N2 * shape.topk),))
+    sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
+    skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
+    dev = sparse_indices.device
+    blocks = torch.full((shape.T1, shape.topk), -7, dtype=torch.int32, device=dev)
+    nb = torch.empty(shape.T1, dtype=torch.int32, device=dev)
+    rows = torch.full((shape.T1, shape.topk * sparse_block_size), -7, dtype=torch.int32, device=dev)
+    cnt = torch.empty(shape.T1, dtype=torch.int32, device=dev)
+    N.check(lib.sfa_key_rows(_p(sparse_indices), _p(sq), _p(skv), int(sparse_block_size), int(sparse_mode),
+                             ctypes.byref(shape), int(sorted_blocks), int(block_aligned), _stream(stream), _p(blocks),
+                             _p(nb), _p(rows), _p(cnt)))
+    return blocks, nb, rows, cnt
+
+
 def softmax_grad_rowsum(d_out, out, key, query_rope, sparse_indices, *, layout: str, actual_seq_lengths_q=None,
                         stream=None):
     """FlashSoftmaxGrad(dO, O): fp32 [T1, N1] row sums of dO o O."""

@@ -70,6 +70,68 @@ def test_compact_indices_bit_exact(case):
             assert nb[t] == 0 and nr[t] == 0
 
 
+KEY_ROW_CASES = {
+    "bsnd_bs5_messy": dict(layout="BSND", B=2, S1=11, S2=83, N1=1, topk=14, block_size=5, sparse_mode=3,
+                           index_mode="messy", seqlens_q=[11, 6], seqlens_kv=[83, 40]),
+    "tnd_bs16_messy": dict(layout="TND", seqlens_q=[21, 3, 30], seqlens_kv=[70, 9, 130], N1=1, topk=12,
+                           block_size=16, sparse_mode=3, index_mode="messy"),
+    "tnd_bs32_messy_mode0": dict(layout="TND", seqlens_q=[9, 17], seqlens_kv=[100, 250], N1=1, topk=10,
+                                 block_size=32, sparse_mode=0, index_mode="messy"),
+    "bsnd_bs16_q_longer": dict(layout="BSND", B=1, S1=40, S2=35, N1=1, topk=6, block_size=16, sparse_mode=3,
+                               index_mode="messy"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(KEY_ROW_CASES))
+@pytest.mark.parametrize("sorted_blocks", [False, True])
+@pytest.mark.parametrize("block_aligned", [False, True])
+def test_key_rows_bit_exact(case, sorted_blocks, block_aligned):
+    """The expanded key-row lists the fused kernels read (after the optional block sort, with the
+    block-aligned padding slots) against the oracle's selected rows: exact rows in index order
+    (unsorted), the same multiset (sorted), every padding slot flagged and every kept block whole."""
+    import sparse_attention_backward_sfa_b200 as S
+    p = tiny(29, **KEY_ROW_CASES[case])
+    dp = DevProblem(p)
+    bs = p.block_size
+    blocks, nb, rows, cnt = S.key_rows(dp.idx, dp.k, dp.q, dp.qr, sparse_block_size=bs, layout=p.layout,
+                                       sparse_mode=p.sparse_mode, sorted_blocks=sorted_blocks,
+                                       block_aligned=block_aligned, actual_seq_lengths_q=dp.sq,
+                                       actual_seq_lengths_kv=dp.skv)
+    blocks, nb, rows, cnt = (x.cpu().numpy() for x in (blocks, nb, rows, cnt))
+    flag = np.int64(1) << 31
+    seen = set()
+    for sp in O.make_spans(p.layout, p.B, p.S1, p.S2, p.seqlens_q, p.seqlens_kv):
+        for pos in range(sp.q_len):
+            t = sp.q_start + pos
+            seen.add(t)
+            ref = [sp.kv_start + j for j in O.selected_rows(p.indices[t], bs, pos, sp.q_len, sp.kv_len,
+                                                             p.sparse_mode)]
+            kept = blocks[t, :nb[t]].astype(np.int64)
+            if sorted_blocks:
+                assert (np.diff(kept) >= 0).all(), (t, kept)
+            got = rows[t, :cnt[t]].astype(np.int64) & 0xFFFFFFFF
+            if block_aligned:
+                assert cnt[t] == nb[t] * bs
+                valid = got[(got & flag) == 0]
+                for i, b in enumerate(kept.tolist()):  # every kept block whole, its cut rows flagged
+                    grp = got[i * bs:(i + 1) * bs]
+                    first = sp.kv_start + b * bs
+                    np.testing.assert_array_equal(grp & ~flag, np.arange(first, first + bs))
+                    keep = [j for j in range(b * bs, b * bs + bs) if j < sp.kv_len and
+                            (p.sparse_mode == 0 or j <= pos + sp.kv_len - sp.q_len)]
+                    np.testing.assert_array_equal((grp & flag) == 0, np.arange(bs) < len(keep))
+            else:
+                valid = got
+                assert cnt[t] == len(ref)
+            if sorted_blocks:
+                assert sorted(valid.tolist()) == sorted(ref), (t,)
+            else:
+                assert valid.tolist() == ref, (t, valid.tolist(), ref)
+    for t in range(p.T1):
+        if t not in seen:
+            assert nb[t] == 0 and cnt[t] == 0
+
+
 def test_softmax_grad_rowsum():
     import sparse_attention_backward_sfa_b200 as S
     p = tiny(3, layout="BSND", B=1, S1=37, S2=16, N1=4, topk=4)
@@ -192,6 +254,50 @@ def test_fa_small_mode0_d64():
 
 def test_fa_workload2_full():
     _fa_case(make_fa_problem())
+
+
+ODD_N1 = {
+    # the N1 values the page lists for Ascend 950 (3/6/12/24/48), served by the CUDA-core kernel
+    "n3_bsnd_bs1": dict(layout="BSND", B=2, S1=13, S2=90, N1=3, topk=40, block_size=1, sparse_mode=3,
+                        index_mode="causal", seqlens_q=[13, 8], seqlens_kv=[90, 51]),
+    "n6_tnd_bs16": dict(layout="TND", seqlens_q=[40, 7], seqlens_kv=[60, 100], N1=6, topk=6, block_size=16,
+                        sparse_mode=3, index_mode="causal"),
+    "n12_tnd_bs1": dict(layout="TND", seqlens_q=[19, 30], seqlens_kv=[19, 64], N1=12, topk=48, block_size=1,
+                        sparse_mode=3, index_mode="messy"),
+    "n24_bsnd_bs16": dict(layout="BSND", B=1, S1=21, S2=130, N1=24, topk=9, block_size=16, sparse_mode=3,
+                          index_mode="causal"),
+    "n48_tnd_bs16": dict(layout="TND", seqlens_q=[17, 5], seqlens_kv=[80, 33], N1=48, topk=6, block_size=16,
+                         sparse_mode=3, index_mode="causal"),
+    "n48_bsnd_bs1": dict(layout="BSND", B=1, S1=9, S2=64, N1=48, topk=32, block_size=1, sparse_mode=3,
+                         index_mode="causal"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(ODD_N1))
+@pytest.mark.parametrize("det", [False, True])
+def test_odd_n1_parity(case, det):
+    p = tiny(41, **ODD_N1[case])
+    dp = DevProblem(p)
+    out, m, l = prepare_oracle_forward(p, dp)
+    got = grads_np(dp.grad_gpu(deterministic=det), p)
+    compare_grads(got, oracle_backward(p, out, m, l), what=f"{case}/det={det}/")
+
+
+@pytest.mark.parametrize("case", ["n6_tnd_bs16", "n48_bsnd_bs1"])
+def test_odd_n1_forward_parity(case):
+    p = tiny(43, **ODD_N1[case])
+    dp = DevProblem(p)
+    out, m, l = (x.float().cpu().numpy() for x in dp.forward_gpu())
+    ro, rm, rl = oracle_forward(p)
+    assert_close(f"{case} out", out.reshape(ro.shape), ro)
+    np.testing.assert_allclose(m.reshape(rm.shape), rm, rtol=1e-4, atol=1e-4)
+    np.testing.assert_allclose(l.reshape(rl.shape), rl, rtol=1e-4, atol=1e-6)
+
+
+@pytest.mark.parametrize("D", [192, 256])
+@pytest.mark.parametrize("det", [False, True])
+def test_fa_large_head_dims_gqa(D, det):
+    _fa_case(make_fa_problem(seed=7 + D, lens=(29, 50), N=6, Nkv=2, D=D, sparse_mode=3, kv_lens=(41, 50)), det)
 
 
 def test_fa_page2_worked_example():
