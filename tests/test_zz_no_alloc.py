@@ -51,6 +51,7 @@ def test_noalloc_matches_sfa_grad_two_calls_in_a_row():
         (tiny_problem(802, D=512, Dr=64, layout="BSND", B=2, S1=9, S2=500, N1=64, topk=200, block_size=1,
                       sparse_mode=0, seqlens_q=[9, 5], seqlens_kv=[500, 260]), False),
     ]
+    devs = []
     for p, det in problems:
         dp = DevProblem(p)
         prepare_oracle_forward(p, dp)
@@ -58,6 +59,17 @@ def test_noalloc_matches_sfa_grad_two_calls_in_a_row():
         got = grads_np(_noalloc(lib, dp, det), p)
         torch.cuda.synchronize()
         compare_grads(got, ref, what=f"noalloc/{p.name}/")
+        devs.append((dp, det))
+    # deterministic calls are bit-identical run to run, also after another problem has
+    # left its contents in the shared scratch
+    dp, det = devs[0]
+    assert det
+    first = [x.clone() for x in _noalloc(lib, dp, True)]
+    _noalloc(lib, devs[1][0], devs[1][1])
+    again = _noalloc(lib, dp, True)
+    torch.cuda.synchronize()
+    for name, a, b in zip(("dQuery", "dKey", "dValue", "dQueryRope", "dKeyRope"), first, again):
+        assert torch.equal(a, b), f"noalloc deterministic {name} differs between calls"
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
