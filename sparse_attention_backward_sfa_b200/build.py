@@ -12,7 +12,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SOURCES = ["sfa_api.cu", "sfa_prep.cu", "sfa_generic.cu", "fa_generic.cu", "sfa_fused.cu", "sfa_noalloc.cu", "fa_fused.cu",
-           "sfa_fwd_fused.cu", "lig_fused.cu"]
+           "sfa_fwd_fused.cu", "lig_fused.cu", "sfa_pair.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
          "-shared", "-Xptxas", "-warn-spills"]
 

@@ -211,6 +211,7 @@ sfa_status grad_impl(const void* query, const void* key, const void* value, cons
     char* w = (char*)workspace;
 
     GradArgs a;
+    memset(&a, 0, sizeof a);
     a.q = query; a.qr = query_rope; a.k = key; a.kr = key_rope; a.v = value;
     a.dout = d_out; a.out = out; a.smax = softmax_max; a.ssum = softmax_sum; a.idx = sparse_indices;
     a.sd = seq_desc(shape, z, actual_seq_lengths_q, actual_seq_lengths_kv);
@@ -244,7 +245,26 @@ sfa_status grad_impl(const void* query, const void* key, const void* value, cons
             SFA_CUDA(launch_sort_blocks((int32_t*)a.blocks, a.nblk, a.topk, row_begin, row_end, s), "block sort");
         SFA_CUDA(launch_expand(a.blocks, a.nblk, a.sd, a.topk, a.bs, a.mode, a.rowcap, (int32_t*)a.rowlist, s),
                  "key row expansion");
-        {
+        if (shape->N1 == 128) {
+            // adjacent rows with identical block lists go to the paired kernel (two CTAs of a
+            // cluster share each key tile); the other rows, if any, to the single-row kernel
+            int32_t* counts = (int32_t*)(w + ws.ctrl + kCtrlCounts);
+            int32_t* pairs = (int32_t*)(w + ws.pairs);
+            SFA_CUDA(launch_pair_lists(a.blocks, a.nblk, a.sd, a.topk, row_begin, row_end, (int32_t*)(w + ws.pflags),
+                                       pairs, (int32_t*)a.order, counts, s), "row pairs");
+            PairArgs pa;
+            memset(&pa, 0, sizeof pa);
+            pa.q = query; pa.qr = query_rope; pa.k = key; pa.kr = key_rope; pa.dout = d_out;
+            pa.sd = a.sd; pa.topk = a.topk; pa.bs = a.bs; pa.mode = a.mode; pa.scale = scale; pa.det = det;
+            pa.dtype = shape->dtype; pa.blocks = a.blocks; pa.nblk = a.nblk; pa.pairs = pairs; pa.npairs = counts;
+            pa.smax = softmax_max; pa.ssum = softmax_sum; pa.rowsum = a.rowsum; pa.dkv_acc = a.dkv_acc;
+            pa.dq_acc = a.dq_acc; pa.dq = d_query; pa.dqr = d_query_rope; pa.err = a.ctrl;
+            pa.dout_absmax = a.dout_absmax;
+            a.nwork_dev = counts + 1;
+            KernelEvents ev(s);
+            SFA_CUDA(launch_bwd_pair(shape->dtype, pa, s), "paired backward");
+            SFA_CUDA(launch_bwd_fused(shape->dtype, a, s), "fused backward");
+        } else {
             KernelEvents ev(s);
             SFA_CUDA(launch_bwd_fused(shape->dtype, a, s), "fused backward");
         }

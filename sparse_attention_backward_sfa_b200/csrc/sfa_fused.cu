@@ -83,6 +83,7 @@ struct FusedParams {
     const float* dmax;       // deterministic mode: max|dOut| that sets the fixed-point grid
     int64_t T1;
     int64_t nwork;           // entries of `order` (query rows processed by this launch)
+    const int32_t* nwork_dev;  // when set: the entry count, read on the device
     int64_t cap;
     float scale;
     int det;
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
     const uint32_t T_S = tmem, T_DP = tmem + 128;
     auto T_STG = [&](int s) { return tmem + 256u + 128u * s; };
 
-    const int nwork = (int)prm.nwork;
+    const int nwork = prm.nwork_dev ? *prm.nwork_dev : (int)prm.nwork;
     const float scale = prm.scale;
 
     if (warp == 12) {
@@ -693,6 +694,7 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
     p.dmax = a.dout_absmax;
     p.T1 = T1;
     p.nwork = a.row_end - a.row_begin;
+    p.nwork_dev = a.nwork_dev;
     p.cap = a.rowcap;
     p.scale = a.scale;
     p.det = DET ? 1 : 0;
@@ -704,7 +706,7 @@ cudaError_t launch_t(const GradArgs& a, cudaStream_t st) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int grid = (int)(p.nwork < sms ? p.nwork : sms);
+    int grid = (int)(p.nwork < sms ? p.nwork : sms);  // (an upper bound when the count is on the device)
     if (grid > kMaxFusedGrid) grid = kMaxFusedGrid;
     if (grid < 1) return cudaSuccess;
     kern<<<grid, kThreads, Cfg<N1>::kSmem, st>>>(p);

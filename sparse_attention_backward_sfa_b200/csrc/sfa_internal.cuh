@@ -164,6 +164,8 @@ struct GradWs {
     size_t order;   // [T1] int32 work order (longest first)
     size_t rowsum;  // [T1][N1] fp32 FlashSoftmaxGrad
     size_t rowlist; // [T1][topk*bs] int32 gathered key rows, fused path only
+    size_t pflags;  // [T1/2+1] int32 pair flags of adjacent rows (N1 = 128 fused path)
+    size_t pairs;   // [T1/2+1] int32 first rows of the row pairs (N1 = 128 fused path)
     size_t ctrl;    // 256 B of counters / flags (offset 0: the device error word)
     size_t total;
 };
@@ -173,6 +175,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // Offset of the fp32 max|dOut| inside a workspace's 256-byte control area (the
 // error word is at offset 0; the area is zeroed at the start of every call).
 constexpr size_t kCtrlDmax = 128;
+// Offset of the int32 [2] (row pairs, remaining rows) counts of the paired backward.
+constexpr size_t kCtrlCounts = 64;
 
 constexpr int kMaxFusedGrid = 256;  // persistent CTAs of the fused kernel (one per SM)
 
@@ -188,6 +192,9 @@ inline GradWs grad_ws_layout(int64_t T1, int64_t T2, int64_t N1, int64_t topk, i
     w.order = o;  o = align256(o + (size_t)T1 * 4);
     w.rowsum = o; o = align256(o + (size_t)T1 * N1 * 4);
     w.rowlist = o; o = align256(o + (fused ? (size_t)T1 * topk * bs * 4 : 0));
+    const bool pair = fused && N1 == 128;
+    w.pflags = o;  o = align256(o + (pair ? (size_t)(T1 / 2 + 1) * 4 : 0));
+    w.pairs = o;   o = align256(o + (pair ? (size_t)(T1 / 2 + 1) * 4 : 0));
     w.total = o;
     return w;
 }
@@ -251,7 +258,27 @@ struct GradArgs {
     int dtype; const int32_t* rowlist; int64_t rowcap;
     int64_t row_begin, row_end;  // query rows [row_begin, row_end) of the flattened [T1] view are processed
     const float* dout_absmax;    // deterministic mode: max|dOut| over every row added into dkv_acc (device)
+    const int32_t* nwork_dev;    // fused kernel: when set, the device count of `order` entries to process
 };
+
+// Paired-row tensor-core backward (N1 = 128, value == key): rows t, t + 1 of each pair share
+// their kept blocks; the two CTAs of a cluster exchange P / dS (sfa_pair.cu).
+struct PairArgs {
+    const void* q; const void* qr; const void* k; const void* kr; const void* dout;
+    SeqDesc sd; int64_t topk; int bs; int mode; float scale; bool det; int dtype;
+    const int32_t* blocks; const int32_t* nblk;
+    const int32_t* pairs; const int32_t* npairs;  // first rows of the pairs, device count
+    const float* smax; const float* ssum; const float* rowsum;
+    void* dkv_acc; float* dq_acc; void* dq; void* dqr; int* err;
+    const float* dout_absmax;
+};
+// Pairs of adjacent rows (row_begin + 2m, + 1) with identical non-empty block lists in one
+// batch / sequence; pair first rows and the other rows listed in descending order, counts
+// [pairs, rows] in counts[0..1] (device).
+cudaError_t launch_pair_lists(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk,
+                              int64_t row_begin, int64_t row_end, int32_t* flags, int32_t* pairs, int32_t* solo,
+                              int32_t* counts, cudaStream_t st);
+cudaError_t launch_bwd_pair(int dtype, const PairArgs& a, cudaStream_t st);
 cudaError_t launch_bwd_generic(int dtype, const GradArgs& a, cudaStream_t st);
 cudaError_t launch_bwd_fused(int dtype, const GradArgs& a, cudaStream_t st);
 bool fused_supported(int64_t N1);

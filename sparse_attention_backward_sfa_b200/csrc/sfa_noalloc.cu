@@ -15,6 +15,7 @@
 // contents; the accumulator is cleared on the call's stream before use.
 #include <cstdarg>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include "sfa_internal.cuh"
@@ -102,6 +103,7 @@ sfa_status sfa_grad_noalloc(const void* query, const void* key, const void* valu
     char* w = (char*)scratch;
 
     GradArgs a;
+    memset(&a, 0, sizeof a);
     a.q = query; a.qr = query_rope; a.k = key; a.kr = key_rope; a.v = value;
     a.dout = d_out; a.out = out; a.smax = softmax_max; a.ssum = softmax_sum; a.idx = sparse_indices;
     a.sd.layout = shape->layout; a.sd.B = (int32_t)shape->B; a.sd.S1 = shape->S1; a.sd.S2 = shape->S2;
