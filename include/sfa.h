@@ -172,7 +172,11 @@ sfa_status sfa_dkv_accum_size(const sfa_shape *shape, int32_t deterministic, siz
  *     zeroes it before the first range and may add accumulators of other ranges
  *     (other GPUs) element-wise before sfa_dkv_finalize.  With deterministic == 1
  *     the accumulator is integer, so that element-wise addition is exact and
- *     order-independent and the final outputs are bit-identical to sfa_grad's.
+ *     order-independent; when every range boundary is an even row the final
+ *     outputs are bit-identical to sfa_grad's (N1 = 128 processes rows 2m and
+ *     2m + 1 with identical block lists as one pair, whose key-side sums are
+ *     formed together: a boundary between them changes the rounding, not the
+ *     tolerance).
  *   - dout_absmax (device fp32, deterministic mode only; may be NULL otherwise):
  *     max|d_out| over EVERY row whose contributions go into this accumulator (on
  *     every GPU), which fixes the fixed-point grid: zero it, add each range with

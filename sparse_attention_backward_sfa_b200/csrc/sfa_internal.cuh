@@ -164,7 +164,7 @@ struct GradWs {
     size_t order;   // [T1] int32 work order (longest first)
     size_t rowsum;  // [T1][N1] fp32 FlashSoftmaxGrad
     size_t rowlist; // [T1][topk*bs] int32 gathered key rows, fused path only
-    size_t pflags;  // [T1/2+1] int32 pair flags of adjacent rows (N1 = 128 fused path)
+    size_t pflags;  // [T1/2+1] int32 flags of the candidate pairs (2m, 2m+1) (N1 = 128 fused path)
     size_t pairs;   // [T1/2+1] int32 first rows of the row pairs (N1 = 128 fused path)
     size_t ctrl;    // 256 B of counters / flags (offset 0: the device error word)
     size_t total;
@@ -272,9 +272,9 @@ struct PairArgs {
     void* dkv_acc; float* dq_acc; void* dq; void* dqr; int* err;
     const float* dout_absmax;
 };
-// Pairs of adjacent rows (row_begin + 2m, + 1) with identical non-empty block lists in one
-// batch / sequence; pair first rows and the other rows listed in descending order, counts
-// [pairs, rows] in counts[0..1] (device).
+// Pairs of rows (2m, 2m + 1) inside [row_begin, row_end) with identical non-empty block lists in
+// one batch / sequence; pair first rows and the other rows listed in descending order, counts
+// [pairs, rows] in counts[0..1] (device).  `flags` holds one entry per candidate pair.
 cudaError_t launch_pair_lists(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk,
                               int64_t row_begin, int64_t row_end, int32_t* flags, int32_t* pairs, int32_t* solo,
                               int32_t* counts, cudaStream_t st);

@@ -757,29 +757,32 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
 // ---------------------------------------------------------------------------
 // Pairing of adjacent rows with identical block lists, and the work lists
 // ---------------------------------------------------------------------------
-// Candidate m = rows (row_begin + 2m, row_begin + 2m + 1): a pair when both are valid rows of the
-// same batch / sequence with the same non-empty list of kept blocks (in the order the kernels read).
+// Candidate m = rows (2m, 2m + 1) of the flattened row index, for the candidates that meet
+// [row_begin, row_end): a pair when both rows lie in the range and are valid rows of the same
+// batch / sequence with the same non-empty list of kept blocks (in the order the kernels read).
+// Pairs depend on the row index only, so row ranges whose boundaries are even rows form the
+// pairs of the whole call.
 __global__ void pair_flags_kernel(const int32_t* __restrict__ blocks, const int32_t* __restrict__ nblk, SeqDesc sd,
                                   int64_t topk, int64_t row_begin, int64_t row_end, int32_t* __restrict__ flags) {
     const int lane = threadIdx.x & 31;
-    const int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int64_t t0 = row_begin + 2 * m;
+    const int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t t0 = 2 * ((row_begin >> 1) + i);
     if (t0 >= row_end) return;
-    bool ok = t0 + 1 < row_end;
+    bool ok = t0 >= row_begin && t0 + 1 < row_end;
     if (ok) {
         const TokInfo a = tok_info(sd, t0), b = tok_info(sd, t0 + 1);
         ok = a.valid && b.valid && a.kv_start == b.kv_start && a.kv_len == b.kv_len && a.q_len == b.q_len;
     }
-    const int n0 = nblk[t0];
-    ok = ok && n0 > 0 && n0 == nblk[t0 + 1];
+    ok = ok && nblk[t0] > 0 && nblk[t0] == nblk[t0 + 1];
     if (ok) {
+        const int n0 = nblk[t0];
         bool diff = false;
         const int32_t* x = blocks + t0 * topk;
         const int32_t* y = x + topk;
-        for (int i = lane; i < n0; i += 32) diff |= x[i] != y[i];
+        for (int k = lane; k < n0; k += 32) diff |= x[k] != y[k];
         ok = !__any_sync(0xffffffffu, diff);
     }
-    if (lane == 0) flags[m] = ok ? 1 : 0;
+    if (lane == 0) flags[i] = ok ? 1 : 0;
 }
 
 // Exclusive block-wide prefix sums of two counters (1024 threads); totals returned in *ta / *tb.
@@ -813,29 +816,29 @@ __device__ __forceinline__ void scan2(int a, int b, int& ea, int& eb, int& ta, i
     __syncthreads();
 }
 
-// One CTA of 1024 threads: the pair list (first rows) and the list of the remaining rows, both in
-// descending row order (under the causal masks later rows carry more keys: the longest work first).
+// One CTA of 1024 threads: the pair list (first rows) and the list of the remaining rows of the
+// range, both in descending row order (under the causal masks later rows carry more keys: the
+// longest work first).
 __global__ void __launch_bounds__(1024) pair_lists_kernel(const int32_t* __restrict__ flags, int64_t row_begin,
                                                           int64_t row_end, int32_t* __restrict__ pairs,
                                                           int32_t* __restrict__ solo, int32_t* __restrict__ counts) {
-    const int64_t M = (row_end - row_begin + 1) / 2;
+    const int64_t m0 = row_begin >> 1;
+    const int64_t M = ((row_end + 1) >> 1) - m0;  // candidates meeting the range
     int np = 0, ns = 0;
     for (int64_t base = 0; base < M; base += 1024) {
-        const int64_t i = base + threadIdx.x;
-        const bool valid = i < M;
-        const int64_t m = M - 1 - i;
-        const int64_t t0 = row_begin + 2 * m;
-        const int f = valid ? flags[m] : 0;
-        const int nrow = valid ? (int)(row_end - t0 < 2 ? row_end - t0 : 2) : 0;
-        const int a = f, b = f ? 0 : nrow;
+        const int64_t i = M - 1 - (base + threadIdx.x);
+        const bool valid = base + threadIdx.x < M;
+        const int64_t t0 = 2 * (m0 + i);
+        const int f = valid ? flags[i] : 0;
+        const bool in0 = valid && t0 >= row_begin, in1 = valid && t0 + 1 < row_end;
+        const int a = f, b = f ? 0 : (int)in0 + (int)in1;
         int ea, eb, ta, tb;
         scan2(a, b, ea, eb, ta, tb);
         if (a) pairs[np + ea] = (int32_t)t0;
-        if (b == 2) {
-            solo[ns + eb] = (int32_t)(t0 + 1);
-            solo[ns + eb + 1] = (int32_t)t0;
-        } else if (b == 1) {
-            solo[ns + eb] = (int32_t)t0;
+        if (!f) {
+            int o = ns + eb;
+            if (in1) solo[o++] = (int32_t)(t0 + 1);
+            if (in0) solo[o] = (int32_t)t0;
         }
         np += ta;
         ns += tb;
@@ -918,7 +921,7 @@ cudaError_t launch_pair_t(const PairArgs& a, cudaStream_t st) {
 cudaError_t launch_pair_lists(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk,
                               int64_t row_begin, int64_t row_end, int32_t* flags, int32_t* pairs, int32_t* solo,
                               int32_t* counts, cudaStream_t st) {
-    const int64_t M = (row_end - row_begin + 1) / 2;
+    const int64_t M = ((row_end + 1) >> 1) - (row_begin >> 1);
     if (M > 0) {
         const int warps = 8;
         pair_flags_kernel<<<(unsigned)((M + warps - 1) / warps), warps * 32, 0, st>>>(blocks, nblk, sd, topk,

@@ -96,7 +96,9 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
     h_dq, h_dk, h_dv, h_dqr, h_dkr = outputs
 
     chunks = max(1, min(chunks, T1))
-    bounds = [(T1 * c) // chunks for c in range(chunks + 1)]
+    # chunk boundaries on even rows: rows (2m, 2m + 1) that share their blocks stay one pair, as in
+    # the single call (deterministic results are then bit-identical to it)
+    bounds = [min(T1, 2 * ((T1 * c) // (2 * chunks))) for c in range(chunks)] + [T1]
     # the copy stream starts after whatever the caller queued before this call
     pl.h2d.wait_stream(comp)
     with torch.cuda.stream(pl.h2d):

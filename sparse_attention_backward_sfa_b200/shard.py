@@ -20,15 +20,20 @@ import numpy as np
 Range = Tuple[int, int]
 
 
-def balanced_row_ranges(row_work: Sequence[float], parts: int) -> List[Range]:
+def balanced_row_ranges(row_work: Sequence[float], parts: int, align: int = 2) -> List[Range]:
     """Splits rows 0..len(row_work) into `parts` contiguous ranges of about equal total work.
 
     Boundary k sits at the row edge whose cumulative work is closest to k/parts of the
-    total (the last range ends at the last row); ranges may be empty when rows are few or
-    work is concentrated.
+    total (the last range ends at the last row), rounded to a multiple of `align`: the
+    backward processes rows (2m, 2m + 1) with identical block lists as one pair, so
+    even boundaries keep every pair of the whole call together (deterministic results
+    then equal the unsharded call bit for bit).  Ranges may be empty when rows are few
+    or work is concentrated.
     """
     if parts < 1:
         raise ValueError("parts must be >= 1")
+    if align < 1:
+        raise ValueError("align must be >= 1")
     w = np.asarray(row_work, dtype=np.float64)
     if w.ndim != 1 or (w.size and w.min() < 0):
         raise ValueError("row_work must be a 1-D sequence of non-negative numbers")
@@ -45,6 +50,7 @@ def balanced_row_ranges(row_work: Sequence[float], parts: int) -> List[Range]:
             b = lo if lo > 0 and target - cum[lo - 1] <= cum[hi - 1] - target else hi
         else:
             b = (n * k) // parts
+        b = int(round(b / align)) * align
         bounds.append(min(max(b, bounds[-1]), n))
     bounds.append(n)
     return [(bounds[k], bounds[k + 1]) for k in range(parts)]

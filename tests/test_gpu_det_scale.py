@@ -90,9 +90,9 @@ def test_fa_deterministic_small_gradient(s):
 
 @pytest.mark.parametrize("case", ["fused_n128", "generic_n8"])
 def test_rows_path_small_gradient(case):
-    """Three row ranges, each into its own accumulator, summed (what the ranks' all-reduce does),
-    with the grid from the max of the ranges' max|dOut|: bit-identical to sfa_grad and within the
-    tolerance of the oracle at dOut x 1e-8."""
+    """Three row ranges (boundaries on even rows), each into its own accumulator, summed (what the
+    ranks' all-reduce does), with the grid from the max of the ranges' max|dOut|: bit-identical
+    to sfa_grad and within the tolerance of the oracle at dOut x 1e-8."""
     import sparse_attention_backward_sfa_b200 as S
     p = scaled_problem(case, 1e-8, seed=919)
     dp = DevProblem(p)
@@ -100,7 +100,8 @@ def test_rows_path_small_gradient(case):
     full = dp.grad_gpu(deterministic=True)
     kw = dp.kw()
     T1 = p.T1
-    ranges = [(0, T1 // 3), (T1 // 3, (2 * T1) // 3 + 1), ((2 * T1) // 3 + 1, T1)]
+    a, b = 2 * (T1 // 6), 2 * (T1 // 3) + 2  # even boundaries: the pairs of rows of the whole call
+    ranges = [(0, a), (a, b), (b, T1)]
     dmax = torch.zeros(1, dtype=torch.float32, device="cuda")
     for rb, re_ in ranges:
         S.dout_absmax(dp.do, dp.q, dp.k, dp.qr, dp.idx, layout=p.layout, row_begin=rb, row_end=re_,

@@ -63,7 +63,9 @@ def sharded(dp, ranges, det, separate=False):
 
 
 def three_ranges(T1):
-    a, b = T1 // 3, (2 * T1) // 3 + 1
+    """Three ranges with boundaries on even rows (pairs of rows stay together, as in the whole call)."""
+    a, b = 2 * (T1 // 6), 2 * (T1 // 3) + 2
+    b = min(b, T1)
     return [(0, a), (a, b), (b, T1)]
 
 

@@ -22,15 +22,19 @@ def test_balanced_row_ranges_properties():
         n = int(rng.integers(0, 60))
         parts = int(rng.integers(1, 9))
         w = rng.integers(0, 50, size=n).astype(np.float64)
-        r = balanced_row_ranges(w, parts)
-        assert len(r) == parts
-        assert r[0][0] == 0 and r[-1][1] == n
-        assert all(a <= b for a, b in r) and all(r[i][1] == r[i + 1][0] for i in range(parts - 1))
-        if n and w.sum() > 0:
-            sums = np.array([w[a:b].sum() for a, b in r])
-            assert sums.sum() == w.sum()
-            # every boundary sits at the row edge nearest its target, so no share is off by more than one row
-            assert np.abs(sums - w.sum() / parts).max() <= w.max() + 1e-9
+        for align in (1, 2):
+            r = balanced_row_ranges(w, parts, align=align)
+            assert len(r) == parts
+            assert r[0][0] == 0 and r[-1][1] == n
+            assert all(a <= b for a, b in r) and all(r[i][1] == r[i + 1][0] for i in range(parts - 1))
+            # inner boundaries on multiples of `align` (pairs of rows 2m, 2m + 1 stay together)
+            assert all(b % align == 0 or b == n for _, b in r[:-1])
+            if n and w.sum() > 0:
+                sums = np.array([w[a:b].sum() for a, b in r])
+                assert sums.sum() == w.sum()
+                # every boundary sits at the row edge nearest its target, then moves at most align - 1
+                # rows to its multiple of `align`: no share is off by more than 2 * align - 1 rows
+                assert np.abs(sums - w.sum() / parts).max() <= (2 * align - 1) * w.max() + 1e-9
 
 
 def test_balanced_row_ranges_edges():
@@ -38,6 +42,8 @@ def test_balanced_row_ranges_edges():
     assert balanced_row_ranges([0, 0, 0, 0], 2) == [(0, 2), (2, 4)]
     assert balanced_row_ranges([3, 1], 1) == [(0, 2)]
     assert balanced_row_ranges([1, 1, 1, 1, 4], 2) == [(0, 4), (4, 5)]
+    assert balanced_row_ranges([1, 1, 1, 1, 1, 1], 2, align=1) == [(0, 3), (3, 6)]
+    assert balanced_row_ranges([1, 1, 1, 1, 1, 1], 2) in ([(0, 2), (2, 6)], [(0, 4), (4, 6)])
     with pytest.raises(ValueError):
         balanced_row_ranges([1, -1], 2)
     with pytest.raises(ValueError):
