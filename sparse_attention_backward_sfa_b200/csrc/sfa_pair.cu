@@ -127,11 +127,13 @@ __device__ __forceinline__ void sdp_item(int j, int& kind, int& c) {
 // Gradient blocks of a tile: k < 5 dQ~ block k of the own row (one key chunk); k >= 5 the rank's
 // key-side block k - 5 (rank 0 dV, rank 1 dK~) over both rows (the own row's chunk, then the partner's).
 __device__ __forceinline__ int num_blocks(uint32_t rank) { return rank ? 10 : 9; }
-// The next tile's S / dP items follow the last five gradient blocks as whole groups (K_g, Q_g,
-// dO_g), the last group (K4, Q4): a key chunk is then never held in the 4-slot ring across a
-// two-chunk gradient block (two items per block, as in the single-row kernel, would deadlock it).
-constexpr int kGroups = 5;
-__device__ __forceinline__ int interleave_start(uint32_t rank) { return num_blocks(rank) - kGroups; }
+// The next tile's S / dP items follow gradient blocks 4..8 as whole groups (K_g, Q_g, dO_g), the
+// last group (K4, Q4): a key chunk is then never held in the 4-slot ring across a two-chunk
+// gradient block (two items per block, as in the single-row kernel, would deadlock it).  The
+// same blocks on both ranks keep the two rows' next S / dP (and so their softmax) in step; the
+// placement was measured on workload 4 (blocks 4..8: 86.5 ms; the last five: 87.9; 3..7: 88.0;
+// 2..6: 88.1; 0..4: 91.4).
+__device__ __forceinline__ int interleave_start(uint32_t) { return 4; }
 __device__ __forceinline__ int group_end(int g) { return 3 * g + 3 < 14 ? 3 * g + 3 : 14; }
 
 __device__ __forceinline__ bool softmax_all(bool v) {

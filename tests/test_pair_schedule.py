@@ -1,8 +1,8 @@
 """Deadlock check of the paired-row backward's schedule (two CTAs of a cluster), on the CPU.
 
 Each CTA runs a cross-tile pipeline over its own 4-slot ring (the next tile's 14 S / dP
-items interleaved as whole (K, Q, dO) triples, one triple after each of the last five
-gradient blocks, so a key chunk is never held across a gradient block's loads) with its own
+items interleaved as whole (K, Q, dO) triples, one triple after each of gradient blocks
+4..8, so a key chunk is never held across a gradient block's loads) with its own
 gradient blocks: dQ~ 0-4 (one chunk each), then the key-side blocks over both rows (rank 0
 dV 0-3, rank 1 dK~ 0-4; two chunks each: the own row's, then the partner's).  The CTAs are
 coupled through the exchanged P / dS tile:
@@ -16,9 +16,6 @@ The model replays both CTAs against these dependencies and the ring / staging / 
 rules of the single-row model and checks that every role of both CTAs finishes.
 """
 import pytest
-
-GROUPS = 5  # gradient blocks followed by a group of next-tile S / dP items
-
 
 def group_items(g):
     """S / dP items of group g: (K_g, Q_g, dO_g), the last group (K4, Q4)."""
@@ -34,10 +31,13 @@ def sdp_item(j):
     return j - 3 * c, c
 
 
+INTER = 4  # first gradient block followed by a group (the same on both ranks)
+
+
 def schedule(rank, ntiles):
     """Events (tile, kind, index, half) in issue order: ("S", j, 0) and ("G", k, h)."""
     nb = nblocks(rank)
-    inter = nb - GROUPS
+    inter = INTER
     ev = [(0, "S", j, 0) for j in range(14)]
     for i in range(ntiles):
         for k in range(nb):
@@ -139,15 +139,8 @@ def step(c, peer, grant_before_wait=True):
     return progress
 
 
-def simulate(ntiles, slots=4, grant_before_wait=True, groups=None):
-    global GROUPS
-    saved = GROUPS
-    if groups is not None:
-        GROUPS = groups
-    try:
-        a, b = Cta(0, ntiles, slots), Cta(1, ntiles, slots)
-    finally:
-        GROUPS = saved
+def simulate(ntiles, slots=4, grant_before_wait=True):
+    a, b = Cta(0, ntiles, slots), Cta(1, ntiles, slots)
     progress = True
     while progress:
         progress = step(a, b, grant_before_wait) | step(b, a, grant_before_wait)
@@ -167,6 +160,19 @@ def test_schedule_covers_every_item_once():
 @pytest.mark.parametrize("ntiles", [1, 2, 3, 8])
 def test_pair_schedule_is_deadlock_free(ntiles):
     assert simulate(ntiles)
+
+
+@pytest.mark.parametrize("inter", [0, 1, 2, 3, 4])
+def test_every_group_placement_is_deadlock_free(inter):
+    """Whole triples after any five consecutive blocks keep the ring live (the placement is a
+    performance choice only)."""
+    global INTER
+    saved = INTER
+    INTER = inter
+    try:
+        assert all(simulate(n) for n in (1, 2, 3, 8))
+    finally:
+        INTER = saved
 
 
 def test_model_detects_a_deadlock():
