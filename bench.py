@@ -43,7 +43,7 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 
 # committed ncu summaries: (summary file, kernel sources whose hash it records)
 PROFILE_SUMMARIES = {
-    4: ("sfa_bwd_fused_kernel_workload4.md", ("sfa_fused.cu", "tc_common.cuh")),
+    4: ("sfa_bwd_pair_kernel_workload4.md", ("sfa_pair.cu", "tc_common.cuh")),
     2: ("fa_bwd_fused_kernel_workload2.md", ("fa_fused.cu", "tc_common.cuh")),
     "fwd4": ("sfa_fwd_fused_kernel_workload4.md", ("sfa_fwd_fused.cu", "tc_common.cuh")),
     "lig": ("lig_fused_kernel_indexer.md", ("lig_fused.cu", "tc_common.cuh")),
@@ -577,13 +577,13 @@ def run_fa(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     lib = N.load()
-    fp = make_fa_problem(seed=1002 + 7919 * rank)
+    fp = make_fa_problem(seed=1002 + 7919 * rank, D=args.fa_d)
     t = lambda a: torch.from_numpy(a).to(device=dev, dtype=torch.bfloat16)
     q, k, v, dy = t(fp.q), t(fp.k), t(fp.v), t(fp.dy)
     out, smax, ssum = S.fa_fwd(q, k, v, fp.cu_seqlens_q, fp.cu_seqlens_kv, scale=fp.scale, sparse_mode=3)
     lens = np.diff(np.concatenate([[0], fp.cu_seqlens_q]))
     triples = int(sum(L * (L + 1) // 2 for L in lens)) * fp.Nq
-    flop = triples * 1280
+    flop = triples * 10 * fp.D  # five GEMMs of 2*D FLOP per triple (1280 at D = 128)
     outs = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     stream = torch.cuda.current_stream(dev)
 
@@ -690,6 +690,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
+    ap.add_argument("--fa-d", type=int, default=128, help="workload 2: head dim (128 as configured; 64 a variant)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--fwd", action="store_true",
@@ -762,14 +763,15 @@ def main():
         cpu = cpu_baseline(args.workload, args.cpu_budget)
         cpu.pop("seconds", None)
     if rank == 0 and args.workload == 2:
-        line = {"metric": "dense varlen FA backward TFLOP/s (bf16, 5-GEMM count, D=128)", "value": value,
+        line = {"metric": f"dense varlen FA backward TFLOP/s (bf16, 5-GEMM count, D={args.fa_d})", "value": value,
                 "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": r["ms_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": WORKLOADS[2], "valid_triples": r["triples"], "gflop_per_step": r["flop"] / 1e9},
+                "config": {"workload": WORKLOADS[2] if args.fa_d == 128 else WORKLOADS[2].replace("d128", f"d{args.fa_d}"),
+                           "valid_triples": r["triples"], "gflop_per_step": r["flop"] / 1e9},
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                              "frac": achieved / peak, "kernel": "fa_bwd_fused_kernel", "kernel_ms": kern,
-                             "traffic": recorded_traffic(2)},
+                             "traffic": recorded_traffic(2) if args.fa_d == 128 else None},
                 "gpu_launches": 3 * args.steps, "clocks": r["clocks"]}
         print(json.dumps(line), flush=True)
     elif rank == 0:
@@ -793,14 +795,16 @@ def main():
                          "frac": achieved / peak, "peak_source": f"{src} bf16 burst",
                          "peak_sustained": float(peaks.get("bf16_tflops_sustained", peak)),
                          "frac_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
-                         "kernel": "sfa_bwd_fused_kernel", "kernel_ms": kern,
+                         "kernel": "sfa_bwd_pair_kernel" if p.N1 == 128 else "sfa_bwd_fused_kernel",
+                         "kernel_ms": kern,
                          "kernel_ms_median": statistics.median(r["kern_ms"]),
                          "traffic": recorded_traffic(4) if args.workload == 4 and not args.seqs and not sharded
                          else None},
             "cpu_baseline": cpu,
             "e2e": r["e2e"],
-            # compact, rowsum, order, block sort (block-sparse lists of topk <= 4096), expand, fused, cast
-            "gpu_launches": (6 + int(p.block_size > 1 and p.topk <= 4096)) * args.steps,
+            # compact, rowsum, order, block sort (block-sparse lists of topk <= 4096), expand, [N1 = 128:
+            # pair flags, pair lists, paired kernel], single-row kernel, cast
+            "gpu_launches": (6 + int(p.block_size > 1 and p.topk <= 4096) + (3 if p.N1 == 128 else 0)) * args.steps,
             "clocks": r["clocks"],
             "device_error_word": r["err_word"],
         }

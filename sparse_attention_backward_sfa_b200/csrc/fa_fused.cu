@@ -1,4 +1,4 @@
-// Tensor-core dense varlen FlashAttention backward for sm_100a, head dim 128
+// Tensor-core dense varlen FlashAttention backward for sm_100a, head dims 64 and 128
 // (aclnnFlashAttentionUnpaddingScoreGrad, 计算公式: dV = P^T.dY, dQ = scale*dS.K,
 // dK = scale*dS^T.Q with dS = P o (dY.V^T - rowsum(dY o attentionIn)) and
 // P = exp(scale*Q.K^T - softmaxMax) / softmaxSum; TND layout, GQA, sparseMode 0 / 3).
@@ -20,6 +20,10 @@
 // Warps: 0-7 softmax (two per TMEM lane quarter, each taking half of the query
 // columns), 0-3 also the dK/dV write-out, 4-11 dQ flush (two per lane quarter,
 // halves of the query columns), 12 TMA producer, 13 MMA.
+// Head dim 64 runs the same schedule with half-width K / V / Q / dY tiles (one SW128
+// half each), S^T / dP^T over 4 K-steps, dK / dV accumulators of 64 TMEM columns, and
+// dQ^T formed with M = 128 over the key block's 64 valid dims (the upper 64 TMEM lanes
+// are not written out).
 #include <cuda.h>
 
 #include <algorithm>
@@ -36,7 +40,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kFaD = 128;
+constexpr int kFaDMax = 128;  // largest head dim of the tensor-core path (the smem / TMEM plan)
 constexpr int kBlk = 128;
 constexpr int kFaThreads = 448;
 // K, V, then Q / dY of slot x at kOffQ / kOffO + x * 65536, dS, constants, barriers
@@ -59,8 +63,8 @@ struct FaParams {
     const float* smax;    // [T1][Nq][8]
     const float* ssum;
     const float* rowsum;  // [T1][Nq]
-    void* dq_acc;         // [T1][Nq][128] fp32 or int64
-    void* dk;             // [T2][Nkv][128]
+    void* dq_acc;         // [T1][Nq][D] fp32 or int64
+    void* dk;             // [T2][Nkv][D]
     void* dv;
     int* err;
     const float* dmax;    // deterministic mode: max|dY| that sets the dQ fixed-point grid
@@ -88,9 +92,12 @@ __device__ __forceinline__ int first_qb(const Seq& s, int kb, int mode) {
     return lo <= 0 ? 0 : (int)(lo / kBlk);
 }
 
-template <typename T, bool DET>
+template <typename T, bool DET, int D>
 __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __grid_constant__ FaParams prm) {
+    static_assert(D == 64 || D == 128, "head dims 64 and 128");
     constexpr bool kF16 = std::is_same<T, __half>::value;
+    constexpr int kHalves = D / 64;       // SW128 halves (64 dims each) of a K / V / Q / dY tile
+    constexpr uint32_t kTileTx = kHalves * kBlk * 128u;  // bytes of one such tile
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -156,11 +163,11 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
             if (lane == 0) {
                 ok = WAIT(KV_EMPTY, (item_ctr & 1) ^ 1, 21);
                 if (ok) {
-                    mbar_expect_tx(KV_FULL, 4 * kBlk * 128);
+                    mbar_expect_tx(KV_FULL, 2 * kTileTx);
                     const int row = (int)(s.ks + (int64_t)it.kb * kBlk);
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_2d(sbase + kOffK + h * 16384, &prm.mapK, it.hk * kFaD + h * 64, row, KV_FULL);
-                        tma_load_2d(sbase + kOffV + h * 16384, &prm.mapV, it.hk * kFaD + h * 64, row, KV_FULL);
+                    for (int h = 0; h < kHalves; ++h) {
+                        tma_load_2d(sbase + kOffK + h * 16384, &prm.mapK, it.hk * D + h * 64, row, KV_FULL);
+                        tma_load_2d(sbase + kOffV + h * 16384, &prm.mapV, it.hk * D + h * 64, row, KV_FULL);
                     }
                 }
             }
@@ -172,12 +179,12 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                     if (lane == 0) {
                         ok = WAIT(QDO_EMPTY(x), ((pair_ctr >> 1) & 1) ^ 1, 22);
                         if (ok) {
-                            mbar_expect_tx(QDO_FULL(x), 4 * kBlk * 128);
+                            mbar_expect_tx(QDO_FULL(x), 2 * kTileTx);
                             const int row = (int)(s.qs + (int64_t)qb * kBlk);
-                            for (int hh = 0; hh < 2; ++hh) {
-                                tma_load_2d(sbase + kOffQ + x * 65536 + hh * 16384, &prm.mapQ, h * kFaD + hh * 64, row,
+                            for (int hh = 0; hh < kHalves; ++hh) {
+                                tma_load_2d(sbase + kOffQ + x * 65536 + hh * 16384, &prm.mapQ, h * D + hh * 64, row,
                                             QDO_FULL(x));
-                                tma_load_2d(sbase + kOffO + x * 65536 + hh * 16384, &prm.mapO, h * kFaD + hh * 64, row,
+                                tma_load_2d(sbase + kOffO + x * 65536 + hh * 16384, &prm.mapO, h * D + hh * 64, row,
                                             QDO_FULL(x));
                             }
                         }
@@ -201,8 +208,10 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
     } else if (warp == 13) {
         // =================== MMA issuer ===================
         const uint32_t ID_S = idesc(128, 128, false, false, kF16);  // S^T, dP^T (A = K/V, B = Q/dY, both K-major)
-        const uint32_t ID_A = idesc(128, 128, false, true, kF16);   // dV (A = P in TMEM), dK (A = dS K-major); B MN-major
-        const uint32_t ID_Q = idesc(128, 128, true, true, kF16);    // dQ^T (A = K MN-major, B = dS MN-major)
+        const uint32_t ID_A = idesc(128, D, false, true, kF16);     // dV (A = P in TMEM), dK (A = dS K-major); B MN-major
+        // dQ^T (A = K MN-major, B = dS MN-major); M = 128 also for head dim 64 (its upper 64 rows
+        // read the unused second half of the K tile and are never written out)
+        const uint32_t ID_Q = idesc(128, 128, true, true, kF16);
         const uint32_t sK = sbase + kOffK, sV = sbase + kOffV, sDS = sbase + kOffDS;
         int item_ctr = 0, pair_ctr = 0;
         bool ok = true;
@@ -229,7 +238,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                     if (!ok) break;
                     tc_fence_after();
                     if (lane == 0) {
-                        for (int ks = 0; ks < 8; ++ks) {
+                        for (int ks = 0; ks < D / 16; ++ks) {
                             const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
                             mma(T_S, sdesc(sK + off, 16, 1024), sdesc(sQ + off, 16, 1024), ID_S, ks > 0);
                         }
@@ -237,7 +246,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                         ok = WAIT(DQ_FREE, (pair_ctr & 1) ^ 1, 33);
                         if (ok) {
                             tc_fence_after();
-                            for (int ks = 0; ks < 8; ++ks) {
+                            for (int ks = 0; ks < D / 16; ++ks) {
                                 const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
                                 mma(T_DP, sdesc(sV + off, 16, 1024), sdesc(sO + off, 16, 1024), ID_S, ks > 0);
                             }
@@ -386,16 +395,17 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
                         if (!ok) break;
                         tc_fence_after();
                         const int dim = j;
+                        const bool dim_ok = quarter * 32 < D;  // (warp-uniform) lane quarter holds real dims
                         const int64_t nq = min((int64_t)kBlk, s.ql - (int64_t)qb * kBlk);
                         const int64_t row0 = s.qs + (int64_t)qb * kBlk;
 #pragma unroll 1
-                        for (int cc = 2 * hsel; cc < 2 * hsel + 2; ++cc) {
+                        for (int cc = 2 * hsel; cc < 2 * hsel + 2 && dim_ok; ++cc) {
                             float v[32];
                             tmem_ld32(T_DP + lane_base + cc * 32, v);
                             tmem_wait_ld();
                             const int lim = (int)min((int64_t)32, nq - cc * 32);
-                            const size_t base = ((size_t)(row0 + cc * 32) * prm.Nq + h) * kFaD + dim;
-                            const uint32_t step = (uint32_t)prm.Nq * kFaD;  // elements between query rows
+                            const size_t base = ((size_t)(row0 + cc * 32) * prm.Nq + h) * D + dim;
+                            const uint32_t step = (uint32_t)prm.Nq * D;  // elements between query rows
                             // one running pointer (not 32 precomputed addresses) keeps the loop in registers
                             if (DET) {
                                 unsigned long long* d = reinterpret_cast<unsigned long long*>(prm.dq_acc) + base;
@@ -420,13 +430,13 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
             ok = __all_sync(0xffffffffu, WAIT(ACC_FULL, item_ctr & 1, 30));
             if (!ok) break;
             tc_fence_after();
-            const int64_t orow = ((s.ks + jl) * prm.Nkv + it.hk) * kFaD;
+            const int64_t orow = ((s.ks + jl) * prm.Nkv + it.hk) * D;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
                 T* dst = reinterpret_cast<T*>(which ? prm.dv : prm.dk) + orow;
                 const uint32_t src = which ? T_DV : T_DK;
 #pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
+                for (int cc = 0; cc < D / 32; ++cc) {
                     float v[32];
                     tmem_ld32(src + lane_base + cc * 32, v);
                     tmem_wait_ld();
@@ -454,19 +464,18 @@ __global__ void __launch_bounds__(kFaThreads, 1) fa_bwd_fused_kernel(const __gri
     }
 }
 
-template <typename T>
+template <typename T, int D>
 __global__ void fa_rowsum_kernel(const T* __restrict__ dy, const T* __restrict__ o, int64_t rows,
                                  float* __restrict__ res) {
     const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (r >= rows) return;
-    const uint2 a = reinterpret_cast<const uint2*>(dy + r * kFaD)[lane];
-    const uint2 b = reinterpret_cast<const uint2*>(o + r * kFaD)[lane];
-    const T* ap = reinterpret_cast<const T*>(&a);
-    const T* bp = reinterpret_cast<const T*>(&b);
+    constexpr int kPer = D / 32;  // elements per lane
+    const T* ap = dy + r * D + lane * kPer;
+    const T* bp = o + r * D + lane * kPer;
     float sum = 0.f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) sum = fmaf(to_f(ap[e]), to_f(bp[e]), sum);
+    for (int e = 0; e < kPer; ++e) sum = fmaf(to_f(ap[e]), to_f(bp[e]), sum);
 #pragma unroll
     for (int k = 16; k; k >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, k);
     if (lane == 0) res[r] = sum;
@@ -483,11 +492,11 @@ __global__ void fa_cast_dq_kernel(const void* __restrict__ acc, int64_t n, T* __
     dq[i] = from_f<T>(x);
 }
 
-template <typename T, bool DET>
+template <typename T, bool DET, int D>
 cudaError_t launch_fa_t(const FaFusedArgs& a, cudaStream_t st) {
     FaParams p;
     memset(&p, 0, sizeof p);
-    const uint64_t qcols = (uint64_t)a.Nq * kFaD, kcols = (uint64_t)a.Nkv * kFaD;
+    const uint64_t qcols = (uint64_t)a.Nq * D, kcols = (uint64_t)a.Nkv * D;
     if (!make_map(&p.mapQ, a.q, a.dtype, qcols, a.T1, qcols, kBlk) ||
         !make_map(&p.mapO, a.dy, a.dtype, qcols, a.T1, qcols, kBlk) ||
         !make_map(&p.mapK, a.k, a.dtype, kcols, a.T2, kcols, kBlk) ||
@@ -514,9 +523,9 @@ cudaError_t launch_fa_t(const FaFusedArgs& a, cudaStream_t st) {
     p.wait_ns = wait_limit_ns();
     const int64_t rows = a.T1 * a.Nq;
     if (rows > 0)
-        fa_rowsum_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>((const T*)a.dy, (const T*)a.o, rows,
-                                                                        (float*)a.rowsum);
-    auto kern = fa_bwd_fused_kernel<T, DET>;
+        fa_rowsum_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>((const T*)a.dy, (const T*)a.o, rows,
+                                                                           (float*)a.rowsum);
+    auto kern = fa_bwd_fused_kernel<T, DET, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFaSmem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -525,7 +534,7 @@ cudaError_t launch_fa_t(const FaFusedArgs& a, cudaStream_t st) {
     const int grid = std::min(sms, a.nitems);
     if (grid > 0) kern<<<grid, kFaThreads, kFaSmem, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int64_t n = a.T1 * a.Nq * kFaD;
+    const int64_t n = a.T1 * a.Nq * D;
     if (n > 0)
         fa_cast_dq_kernel<T, DET><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.dq_acc, n, (T*)a.dq, a.dout_absmax,
                                                                             a.scale, a.T1, a.Nq / a.Nkv);
@@ -563,11 +572,17 @@ size_t fa_fused_items(const int64_t* cu_q, const int64_t* cu_kv, int64_t B, int6
     return items.size();
 }
 
-bool fa_fused_supported(int64_t D) { return D == kFaD; }
+bool fa_fused_supported(int64_t D) { return D == 64 || D == kFaDMax; }
+
+template <typename T, int D>
+cudaError_t launch_fa_d(const FaFusedArgs& a, cudaStream_t st) {
+    return a.det ? launch_fa_t<T, true, D>(a, st) : launch_fa_t<T, false, D>(a, st);
+}
 
 cudaError_t launch_fa_bwd_fused(int dtype, const FaFusedArgs& a, cudaStream_t st) {
-    if (dtype == SFA_DTYPE_BF16) return a.det ? launch_fa_t<__nv_bfloat16, true>(a, st) : launch_fa_t<__nv_bfloat16, false>(a, st);
-    return a.det ? launch_fa_t<__half, true>(a, st) : launch_fa_t<__half, false>(a, st);
+    if (dtype == SFA_DTYPE_BF16)
+        return a.D == 64 ? launch_fa_d<__nv_bfloat16, 64>(a, st) : launch_fa_d<__nv_bfloat16, 128>(a, st);
+    return a.D == 64 ? launch_fa_d<__half, 64>(a, st) : launch_fa_d<__half, 128>(a, st);
 }
 
 }  // namespace sfa

@@ -531,7 +531,7 @@ static sfa_status check_cu(const int64_t* cu, int64_t B, int64_t T, const char* 
 constexpr size_t kCtrl = 256;
 static size_t fa_cu_bytes(int64_t B) { return kCtrl + 2 * align256((size_t)B * 8); }
 
-// Workspace of the tensor-core dense backward (head dim 128): cumulative lengths,
+// Workspace of the tensor-core dense backward (head dims 64 and 128): cumulative lengths,
 // work list, rowsum(dY o O), dQ accumulator, control word.
 struct FaFusedWs {
     size_t items, rowsum, dq, ctrl, total;
@@ -609,7 +609,7 @@ sfa_status fa_grad(const void* q, const void* k, const void* v, const void* dy, 
         memset(&f, 0, sizeof f);
         f.q = q; f.k = k; f.v = v; f.dy = dy; f.o = attention_in; f.smax = softmax_max; f.ssum = softmax_sum;
         f.cu_q = cuq; f.cu_kv = cukv; f.B = shape->B; f.T1 = shape->T1; f.T2 = shape->T2; f.Nq = shape->Nq;
-        f.Nkv = shape->Nkv; f.mode = (int)sparse_mode; f.scale = (float)scale; f.det = det; f.dtype = shape->dtype;
+        f.Nkv = shape->Nkv; f.D = shape->D; f.mode = (int)sparse_mode; f.scale = (float)scale; f.det = det; f.dtype = shape->dtype;
         f.items = w + fw.items; f.nitems = (int)nitems; f.rowsum = (float*)(w + fw.rowsum); f.dq_acc = w + fw.dq;
         f.err = (int*)(w + fw.ctrl); f.dq = dq; f.dk = dk; f.dv = dv;
         f.dout_absmax = (const float*)(w + fw.ctrl + kCtrlDmax);

@@ -314,16 +314,16 @@ struct FaArgs {
 };
 cudaError_t launch_fa_bwd(int dtype, const FaArgs& a, cudaStream_t st);
 
-// Tensor-core dense backward (head dim 128): work list of (sequence, kv head,
+// Tensor-core dense backward (head dims 64 and 128): work list of (sequence, kv head,
 // 128-key block) items, built on the host and copied into the workspace.
 struct FaFusedArgs {
     const void* q; const void* k; const void* v; const void* dy; const void* o;
     const float* smax; const float* ssum;
     const int64_t* cu_q; const int64_t* cu_kv;
-    int64_t B, T1, T2, Nq, Nkv; int mode; float scale; bool det; int dtype;
+    int64_t B, T1, T2, Nq, Nkv, D; int mode; float scale; bool det; int dtype;
     const void* items; int nitems;
     float* rowsum;   // [T1][Nq]
-    void* dq_acc;    // [T1][Nq][128] fp32 or int64 (zeroed by the caller)
+    void* dq_acc;    // [T1][Nq][D] fp32 or int64 (zeroed by the caller)
     int* err;
     void* dq; void* dk; void* dv;
     const float* dout_absmax;  // deterministic mode: max|dY| (device)

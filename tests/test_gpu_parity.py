@@ -252,6 +252,35 @@ def test_fa_small_mode0_d64():
     _fa_case(make_fa_problem(seed=6, lens=(20, 45), N=4, Nkv=4, D=64, sparse_mode=0))
 
 
+@pytest.mark.parametrize("det", [False, True])
+def test_fa_d64_gqa_bottom_right(det):
+    """Head dim 64 on the tensor-core kernel: GQA, several 128-key blocks with ragged tails,
+    sequences with fewer queries than keys (bottom-right causal), an empty query span."""
+    _fa_case(make_fa_problem(seed=8, lens=(150, 0, 77, 300), N=8, Nkv=2, D=64, sparse_mode=3,
+                             kv_lens=(200, 30, 77, 300)), det)
+
+
+def test_fa_d64_workload2_shape():
+    """Workload 2's sequences and heads at head dim 64."""
+    _fa_case(make_fa_problem(seed=9, D=64))
+
+
+def test_fa_d64_fp16():
+    import sparse_attention_backward_sfa_b200 as S
+    fp = make_fa_problem(seed=10, lens=(64, 190), N=4, Nkv=1, D=64, sparse_mode=3)
+    d = DevFA(fp, dtype=torch.float16)
+    d.forward_gpu()
+    out = d.out.float().cpu().numpy()
+    sm = d.smax.cpu().numpy().astype(np.float64)
+    ss = d.ssum.cpu().numpy().astype(np.float64)
+    dq, dk, dv = (x.float().cpu().numpy() for x in d.grad_gpu())
+    rq, rk, rv = O.fa_backward(fp.q, fp.k, fp.v, fp.dy, sm, ss, out, fp.cu_seqlens_q, fp.cu_seqlens_kv, fp.scale,
+                               fp.sparse_mode)
+    assert_close("fa16 dq", dq, rq)
+    assert_close("fa16 dk", dk, rk)
+    assert_close("fa16 dv", dv, rv)
+
+
 def test_fa_workload2_full():
     _fa_case(make_fa_problem())
 
