@@ -127,14 +127,12 @@ __device__ __forceinline__ void sdp_item(int j, int& kind, int& c) {
 // Gradient blocks of a tile: k < 5 dQ~ block k of the own row (one key chunk); k >= 5 the rank's
 // key-side block k - 5 (rank 0 dV, rank 1 dK~) over both rows (the own row's chunk, then the partner's).
 __device__ __forceinline__ int num_blocks(uint32_t rank) { return rank ? 10 : 9; }
-// The next tile's S / dP items follow gradient blocks 4..8 as whole groups (K_g, Q_g, dO_g), the
-// last group (K4, Q4): a key chunk is then never held in the 4-slot ring across a two-chunk
-// gradient block (two items per block, as in the single-row kernel, would deadlock it).  The
-// same blocks on both ranks keep the two rows' next S / dP (and so their softmax) in step; the
-// placement was measured on workload 4 (blocks 4..8: 86.5 ms; the last five: 87.9; 3..7: 88.0;
-// 2..6: 88.1; 0..4: 91.4).
-__device__ __forceinline__ int interleave_start(uint32_t) { return 4; }
-__device__ __forceinline__ int group_end(int g) { return 3 * g + 3 < 14 ? 3 * g + 3 : 14; }
+// Per tile: the five dQ~ blocks, then for c = 0..4 the key-side block c (if the rank has it)
+// followed by the next tile's S item c (K_c, q_c) and dP item c (c < 4: K_c, dO_c).  When the
+// next tile belongs to the same pair, the own row's chunk of key-side block c is also the next
+// tile's q_c (rank 1) or dO_c (rank 0): it is loaded once and released after its second use
+// (23 / 24 chunk loads per tile instead of 27 / 29).  A key chunk is held only across its own
+// S / dP items, so the 4-slot ring cannot deadlock (checked by a CPU model of both CTAs).
 
 __device__ __forceinline__ bool softmax_all(bool v) {
     uint32_t r;
@@ -309,8 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
     const int npairs = *prm.npairs;
     const int bs = prm.bs;
     const float scale = prm.scale;
-    const int nblocks = num_blocks(rank);
-    const int kInter = interleave_start(rank);
+    const int nblocks = num_blocks(rank);  // gradient blocks per tile: 5 dQ~ + the key-side ones
+    const int nkey = nblocks - 5;
 
     if (warp == 12) {
         // =================== TMA producer ===================
@@ -427,20 +425,26 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
         };
         Tile cur, nxt;
         bool have = next_tile(cur);
-        for (int j = 0; j < 14 && have && ok; ++j) ok = sdp_load(cur, j);
+        for (int j = 0; j < 14 && have && ok; ++j) ok = sdp_load(cur, j);  // the first tile's S / dP
         const int gkind = rank ? 1 : 2;  // the key-side blocks' A operand: q (dK~) or dO (dV)
         while (have && ok) {
+            for (int c = 0; c < 5 && ok; ++c) ok = load(cur, 0, c, 0);  // dQ~ blocks: the tile's key chunks
             bool have_next = false;
-            for (int k = 0; k < nblocks && ok; ++k) {
-                if (k < 5) {
-                    ok = load(cur, 0, k, 0);
-                } else {
-                    ok = load(cur, gkind, k - 5, cur.t0 + (int)rank);
-                    if (ok) ok = load(cur, gkind, k - 5, cur.t0 + (int)peer);
+            if (ok) have_next = next_tile(nxt);
+            // the next tile of the same pair reads the same row chunks: rank 1's own q chunk of dK~
+            // block c is also the next S item's B, rank 0's own dO chunk of dV block c the next dP item's
+            const bool same = have_next && nxt.t0 == cur.t0;
+            for (int c = 0; c < 5 && ok; ++c) {
+                if (c < nkey) {
+                    ok = load(cur, gkind, c, cur.t0 + (int)rank);
+                    if (ok) ok = load(cur, gkind, c, cur.t0 + (int)peer);
                 }
-                if (ok && k == kInter) have_next = next_tile(nxt);
-                if (ok && have_next && k >= kInter)
-                    for (int jj = 3 * (k - kInter); jj < group_end(k - kInter) && ok; ++jj) ok = sdp_load(nxt, jj);
+                if (ok && have_next) {
+                    const int t = nxt.t0 + (int)rank;
+                    ok = load(nxt, 0, c, 0);
+                    if (ok && !(rank == 1 && same)) ok = load(nxt, 1, c, t);
+                    if (ok && c < 4 && !(rank == 0 && same)) ok = load(nxt, 2, c, t);
+                }
             }
             cur = nxt;
             have = have_next;
@@ -502,8 +506,9 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
             advance();
             return true;
         };
-        // K = 128 half of a key-side block: A = the chunk in the current slot, B = P or dS in bsrc
-        auto grad_half = [&](uint32_t dst, uint32_t bsrc, bool first, int code) -> bool {
+        // K = 128 half of a key-side block: A = the chunk in the current slot, B = P or dS in bsrc;
+        // the slot is released after these MMAs unless another MMA still reads it
+        auto grad_half = [&](uint32_t dst, uint32_t bsrc, bool first, bool release, int code) -> bool {
             if (!wait_full(code)) return false;
             const uint32_t sa = sbase + slot * kSlotBytes;
             if (lane == 0) {
@@ -512,14 +517,14 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                     const uint64_t bd = sdesc(bsrc + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
                     mma(dst, a, bd, ID_G, (!first || ks > 0) ? 1u : 0u);
                 }
-                mma_commit(EMPTY(slot));
+                if (release) mma_commit(EMPTY(slot));
             }
             __syncwarp();
             advance();
             return true;
         };
         int w_next = cid, tile_next = 0;
-        auto next_tile = [&]() -> bool {
+        auto next_tile = [&](int& w_of) -> bool {
             while (w_next < npairs) {
                 const int nslots = prm.nblk[prm.pairs[w_next]] * bs;
                 if (tile_next * kKeys >= nslots) {
@@ -528,41 +533,65 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                     continue;
                 }
                 ++tile_next;
+                w_of = w_next;
                 return true;
             }
             return false;
         };
-        bool have = next_tile();
-        for (int j = 0; j < 14 && have && ok; ++j) ok = sdp(j);
+        // S^T (c-th q chunk in sB) or dP^T (dO chunk) item c of a tile against the key chunk in sK
+        auto sdp_mma = [&](uint32_t dst, uint32_t sK, uint32_t sB, int c) {
+            const int ksteps = c < 4 ? 8 : 4;
+            for (int ks = 0; ks < ksteps; ++ks) {
+                const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                mma(dst, sdesc(sK + off, 16, 1024), sdesc(sB + off, 16, 1024), ID_S, (c > 0 || ks > 0) ? 1u : 0u);
+            }
+        };
+        auto slot_addr = [&]() { return sbase + slot * kSlotBytes; };
+        int cur_w = 0;
+        bool have = next_tile(cur_w);
+        for (int j = 0; j < 14 && have && ok; ++j) ok = sdp(j);  // the first tile's S / dP
         while (have && ok) {
             if (lane == 0) ok = WAIT(PDS_FULL, tile_ctr & 1, 104);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
-            bool have_next = false;
-            for (int k = 0; k < nblocks && ok; ++k, ++blk_ctr) {
+            // ---- dQ~ blocks 0..4 of the own row: A = key chunk [128 dims x 128 keys] (MN), B = dS (MN) ----
+            for (int c = 0; c < 5 && ok; ++c, ++blk_ctr) {
                 const int stg = blk_ctr & 1;
                 if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 105);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t dst = T_STG(stg);
-                if (k < 5) {
-                    // dQ~^T of the own row: A = key chunk [128 dims x 128 keys] (MN), B = dS [heads x keys] (MN)
-                    if (!(ok = wait_full(106))) break;
-                    const uint32_t sa = sbase + slot * kSlotBytes;
-                    if (lane == 0) {
-                        for (int ks = 0; ks < kKeys / 16; ++ks)
-                            mma(dst, sdesc(sa + ks * 2048, kHalf, 1024), sdesc(sY + ks * 2048, kHalf, 1024), ID_Q,
-                                ks > 0 ? 1u : 0u);
-                        mma_commit(EMPTY(slot));
-                    }
-                    __syncwarp();
-                    advance();
-                } else {
-                    // dV^T (rank 0: A = dO chunks, B = P) or dK~^T (rank 1: A = q chunks, B = dS) over both rows
-                    if (!(ok = grad_half(dst, bOwn, true, 107))) break;
-                    if (k == 5) {  // the partner's P / dS of this tile has landed in R
+                if (!(ok = wait_full(106))) break;
+                const uint32_t sa = slot_addr();
+                if (lane == 0) {
+                    for (int ks = 0; ks < kKeys / 16; ++ks)
+                        mma(T_STG(stg), sdesc(sa + ks * 2048, kHalf, 1024), sdesc(sY + ks * 2048, kHalf, 1024), ID_Q,
+                            ks > 0 ? 1u : 0u);
+                    mma_commit(EMPTY(slot));
+                    mma_commit(STG_FULL(stg));
+                }
+                __syncwarp();
+                advance();
+            }
+            if (!ok) break;
+            int nxt_w = 0;
+            const bool have_next = next_tile(nxt_w);
+            const bool same = have_next && nxt_w == cur_w;
+            // ---- key-side block c over both rows, then the next tile's S / dP item c ----
+            for (int c = 0; c < 5 && ok; ++c) {
+                int sOwn = -1;  // slot of the own row's chunk of block c
+                if (c < nkey) {
+                    const int stg = blk_ctr & 1;
+                    if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 105);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    tc_fence_after();
+                    // the own chunk stays for the next tile's S (rank 1) / dP (rank 0) item when shared
+                    const bool keep = same && (rank == 1 || c < 4);
+                    sOwn = slot;
+                    if (!(ok = grad_half(T_STG(stg), bOwn, true, !keep, 107))) break;
+                    if (c == 0) {  // the partner's P / dS of this tile has landed in R
                         if (lane == 0)
                             ok = wait_cluster(RECV, recv_done & 1, abort_flag, prm.err, 108, prm.wait_ns);
                         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -570,19 +599,49 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                         ++recv_done;
                         tc_fence_after();
                     }
-                    if (!(ok = grad_half(dst, sR, false, 109))) break;
+                    if (!(ok = grad_half(T_STG(stg), sR, false, true, 109))) break;
+                    if (lane == 0) {
+                        mma_commit(STG_FULL(stg));
+                        if (c == nkey - 1) mma_commit(PDS_FREE);  // the last reads of P, dS and R
+                    }
+                    __syncwarp();
+                    ++blk_ctr;
+                }
+                if (!have_next) continue;
+                if (!(ok = wait_full(103))) break;
+                const int sK = slot;
+                advance();
+                int sQ = sOwn;
+                if (!(rank == 1 && same)) {
+                    if (!(ok = wait_full(103))) break;
+                    sQ = slot;
+                    advance();
+                }
+                int sO = -1;
+                if (c < 4) {
+                    sO = sOwn;
+                    if (!(rank == 0 && same)) {
+                        if (!(ok = wait_full(103))) break;
+                        sO = slot;
+                        advance();
+                    }
                 }
                 if (lane == 0) {
-                    mma_commit(STG_FULL(stg));
-                    if (k == nblocks - 1) mma_commit(PDS_FREE);
+                    const uint32_t aK = sbase + sK * kSlotBytes;
+                    sdp_mma(T_S, aK, sbase + sQ * kSlotBytes, c);
+                    mma_commit(EMPTY(sQ));
+                    if (c < 4) {
+                        sdp_mma(T_DP, aK, sbase + sO * kSlotBytes, c);
+                        mma_commit(EMPTY(sO));
+                    }
+                    mma_commit(EMPTY(sK));
+                    if (c == 4) mma_commit(SDP_FULL);
                 }
                 __syncwarp();
-                if (k == kInter) have_next = next_tile();
-                if (have_next && k >= kInter)
-                    for (int jj = 3 * (k - kInter); jj < group_end(k - kInter) && ok; ++jj) ok = sdp(jj);
             }
             ++tile_ctr;
             have = have_next;
+            cur_w = nxt_w;
         }
         if (lane == 0) {
             *consumed = recv_done;

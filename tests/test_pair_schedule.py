@@ -204,3 +204,141 @@ def test_pairs_of_items_deadlock_a_four_slot_ring():
     finally:
         schedule = saved
     assert simulate(3)
+
+
+# ---------------------------------------------------------------------------
+# The merged schedule: the next tile's S / dP items share the own row's chunk
+# ---------------------------------------------------------------------------
+# Per tile after the five dQ~ blocks, for c = 0..4: the key-side block c (rank 0 dV c < 4,
+# rank 1 dK~ c < 5; loads: own chunk, partner chunk) followed by the next tile's S item c
+# (K_c', own q chunk) and dP item c (c < 4: K_c', own dO chunk).  When the next tile belongs
+# to the same pair, the own chunk of the key-side block is also the S item's q chunk (rank 1)
+# or the dP item's dO chunk (rank 0): it is loaded once and its slot is released after its
+# second use.  Loads are FIFO in the ring; a slot is freed after the last MMA that reads it.
+
+def merged_ops(rank, ntiles, same=True):
+    """(loads, mmas): loads in issue order; mmas in issue order as (kind, tile, block, [load ids]).
+    kind: 'S' (an S / dP item; 'S13' marks the tile's last), 'G' (first half of a gradient block,
+    needs staging, and for block 0 the tile's P / dS), 'H' (second half), 'Gq' (a one-chunk dQ~ block)."""
+    nkey = 5 if rank else 4
+    loads, mmas = [], []
+
+    def ld(tag):
+        loads.append(tag)
+        return len(loads) - 1
+
+    def sdp_items(i, c, sq=None, so=None):
+        k = ld(("K", i, c))
+        q = sq if sq is not None else ld(("Q", i, c))
+        mmas.append(("S", i, 2 * c, [k, q]))
+        if c < 4:
+            o = so if so is not None else ld(("O", i, c))
+            mmas.append(("S", i, 2 * c + 1, [k, o]))
+        if c == 4:
+            mmas[-1] = ("S13", i, 2 * c, [k, q])
+
+    for c in range(5):  # the first tile's S / dP, standalone
+        sdp_items(0, c)
+    for i in range(ntiles):
+        nxt = i + 1 < ntiles
+        for c in range(5):
+            mmas.append(("Gq", i, c, [ld(("Kq", i, c))]))
+        for c in range(5):
+            own = None
+            if c < nkey:
+                own = ld(("own", i, c))
+                par = ld(("par", i, c))
+                mmas.append(("G", i, 5 + c, [own]))
+                mmas.append(("H", i, 5 + c, [par]))
+            if nxt:
+                share = same and own is not None
+                if rank == 1:
+                    sdp_items(i + 1, c, sq=own if share else None)
+                else:
+                    sdp_items(i + 1, c, so=own if share and c < 4 else None)
+    return loads, mmas
+
+
+def simulate_merged(ntiles, slots=4, same=True):
+    """Both CTAs' merged schedules against the ring, staging, softmax / exchange and flush rules."""
+    class C:
+        pass
+
+    ctas = []
+    for rank in (0, 1):
+        c = C()
+        c.rank = rank
+        c.loads, c.mmas = merged_ops(rank, ntiles, same)
+        last_use = {}
+        for mi, (_, _, _, ids) in enumerate(c.mmas):
+            for l in ids:
+                last_use[l] = mi
+        c.release_at = last_use
+        c.nb = 9 if rank == 0 else 10
+        c.loaded = c.issued = c.flushed = c.blocks = 0
+        c.freed = set()
+        c.started = c.written = c.sdp_done = c.grad_done = -1
+        ctas.append(c)
+
+    def step(c, peer):
+        progress = False
+        if c.loaded < len(c.loads):  # producer: FIFO ring
+            if c.loaded < slots or (c.loaded - slots) in c.freed:
+                c.loaded += 1
+                progress = True
+        if c.issued < len(c.mmas):  # MMA
+            kind, i, b, ids = c.mmas[c.issued]
+            ready = all(l < c.loaded for l in ids)
+            if kind in ("G", "Gq"):
+                if b == 0 and c.written < i:
+                    ready = False
+                if c.blocks >= 2 and c.flushed < c.blocks - 1:
+                    ready = False
+            if kind == "H" and b == 5 and peer.written < i:
+                ready = False
+            if ready:
+                if kind in ("G", "Gq"):
+                    c.blocks += 1
+                if kind in ("H", "Gq") and b == c.nb - 1:
+                    c.grad_done = i
+                if kind == "S13":
+                    c.sdp_done = i
+                c.freed.update(l for l, at in c.release_at.items() if at == c.issued)
+                c.issued += 1
+                progress = True
+        t = c.started + 1
+        if t < ntiles and c.sdp_done >= t and c.grad_done >= t - 1 and c.started == c.written:
+            c.started = t
+            progress = True
+        t = c.written + 1
+        if t <= c.started and (t == 0 or peer.started >= t):
+            c.written = t
+            progress = True
+        if c.flushed < c.blocks:
+            c.flushed += 1
+            progress = True
+        return progress
+
+    a, b = ctas
+    progress = True
+    while progress:
+        progress = step(a, b) | step(b, a)
+    return all(c.loaded == len(c.loads) and c.issued == len(c.mmas) and c.written == ntiles - 1 for c in ctas)
+
+
+@pytest.mark.parametrize("ntiles", [1, 2, 3, 8])
+@pytest.mark.parametrize("same", [True, False])
+def test_merged_schedule_is_deadlock_free(ntiles, same):
+    assert simulate_merged(ntiles, same=same)
+
+
+def test_merged_schedule_loads():
+    """Per tile: rank 0 23 chunk loads (27 without sharing), rank 1 24 (29)."""
+    for rank, shared, unshared in ((0, 23, 27), (1, 24, 29)):
+        n2 = len(merged_ops(rank, 2, True)[0]) - len(merged_ops(rank, 1, True)[0])
+        u2 = len(merged_ops(rank, 2, False)[0]) - len(merged_ops(rank, 1, False)[0])
+        assert (n2, u2) == (shared, unshared)
+
+
+def test_merged_model_detects_a_deadlock():
+    assert not simulate_merged(3, slots=2)
