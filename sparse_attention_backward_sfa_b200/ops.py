@@ -33,8 +33,15 @@ def _need(cond: bool, msg: str):
 
 
 def _check16(name, t, dtype):
-    _need(t.is_cuda and t.is_contiguous(), f"{name} must be a contiguous CUDA tensor")
+    _need(t.is_contiguous(), f"{name} must be contiguous")
     _need(t.dtype == dtype, f"{name} must be {dtype}")
+
+
+def _check_cuda(named):
+    """Device placement, checked after every size check (so a wrong size is reported as such)."""
+    for name, t in named:
+        if t is not None:
+            _need(t.is_cuda, f"{name} must be a CUDA tensor")
 
 
 def _check_numel(items):
@@ -45,7 +52,7 @@ def _check_numel(items):
 
 
 def _check_f32(name, t):
-    _need(t.is_cuda and t.is_contiguous() and t.dtype == torch.float32, f"{name}: contiguous fp32 CUDA tensor")
+    _need(t.is_contiguous() and t.dtype == torch.float32, f"{name}: contiguous fp32 tensor")
 
 
 def _check_outputs(outputs, likes):
@@ -53,17 +60,18 @@ def _check_outputs(outputs, likes):
     for (name, t), like in zip(outputs, likes):
         if t is None:
             continue
-        _need(t.is_cuda and t.is_contiguous(), f"{name} must be a contiguous CUDA tensor")
+        _need(t.is_contiguous(), f"{name} must be contiguous")
         _need(t.dtype == like[0], f"{name} must be {like[0]}")
         _need(t.numel() == like[1], f"{name}: {t.numel()} elements, expected {like[1]}")
+        _need(t.is_cuda, f"{name} must be a CUDA tensor")
 
 
 def _check_sfa_inputs(shape, query, key, value, sparse_indices, query_rope, key_rope, d_out=None, out=None,
                       softmax_max=None, softmax_sum=None):
     """Element counts of the sparse attention inputs against the sizes derived from `shape`."""
     T1, T2, N1, N2, D, Dr = shape.T1, shape.T2, shape.N1, shape.N2, shape.D, shape.Dr
-    _need(sparse_indices.is_cuda and sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(),
-          "sparse_indices: int32 contiguous CUDA tensor")
+    _need(sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(),
+          "sparse_indices: int32 contiguous tensor")
     for name, t in (("softmax_max", softmax_max), ("softmax_sum", softmax_sum)):
         if t is not None:
             _check_f32(name, t)
@@ -71,6 +79,13 @@ def _check_sfa_inputs(shape, query, key, value, sparse_indices, query_rope, key_
                   ("query_rope", query_rope, T1 * N1 * Dr), ("sparse_indices", sparse_indices, T1 * N2 * shape.topk),
                   ("d_out", d_out, T1 * N1 * D), ("out", out, T1 * N1 * D), ("softmax_max", softmax_max, T1 * N1),
                   ("softmax_sum", softmax_sum, T1 * N1)))
+
+
+def _sfa_named(query, key, value, sparse_indices, query_rope, key_rope, d_out=None, out=None, softmax_max=None,
+               softmax_sum=None):
+    return (("query", query), ("key", key), ("value", value), ("sparse_indices", sparse_indices),
+            ("query_rope", query_rope), ("key_rope", key_rope), ("d_out", d_out), ("out", out),
+            ("softmax_max", softmax_max), ("softmax_sum", softmax_sum))
 
 
 def sfa_shape(query: torch.Tensor, key: torch.Tensor, query_rope: torch.Tensor, sparse_indices: torch.Tensor,
@@ -138,6 +153,8 @@ def sfa_grad(query, key, value, sparse_indices, d_out, out, softmax_max, softmax
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
     _check_sfa_inputs(shape, query, key, value, sparse_indices, query_rope, key_rope, d_out, out, softmax_max,
                       softmax_sum)
+    _check_cuda(_sfa_named(query, key, value, sparse_indices, query_rope, key_rope, d_out, out, softmax_max,
+                           softmax_sum))
     sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
     skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
     ws_bytes = sfa_grad_workspace_size(shape, sparse_block_size, sparse_mode, deterministic)
@@ -170,9 +187,8 @@ def sfa_dkv_accumulator(query, key, query_rope, sparse_indices, *, layout: str, 
 
 
 def _check_accum(dkv_accum, shape, deterministic):
-    _need(dkv_accum.is_cuda and dkv_accum.is_contiguous() and
-          dkv_accum.dtype == (torch.int64 if deterministic else torch.float32),
-          "dkv_accum: contiguous CUDA tensor, int64 when deterministic else float32")
+    _need(dkv_accum.is_contiguous() and dkv_accum.dtype == (torch.int64 if deterministic else torch.float32),
+          "dkv_accum: contiguous, int64 when deterministic else float32")
     _need(dkv_accum.numel() == shape.T2 * ACC_WIDTH, f"dkv_accum: {dkv_accum.numel()} elements, expected "
           f"{shape.T2 * ACC_WIDTH}")
 
@@ -181,8 +197,7 @@ def _check_absmax(dout_absmax, deterministic):
     if deterministic:
         _need(dout_absmax is not None, "deterministic: dout_absmax (from dout_absmax()) is required")
     if dout_absmax is not None:
-        _need(dout_absmax.is_cuda and dout_absmax.dtype == torch.float32 and dout_absmax.numel() == 1,
-              "dout_absmax: one fp32 CUDA element")
+        _need(dout_absmax.dtype == torch.float32 and dout_absmax.numel() == 1, "dout_absmax: one fp32 element")
 
 
 def dout_absmax(d_out, query, key, query_rope, sparse_indices, *, layout: str, row_begin: int = 0,
@@ -194,9 +209,11 @@ def dout_absmax(d_out, query, key, query_rope, sparse_indices, *, layout: str, r
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
     _check16("d_out", d_out, query.dtype)
     _check_numel((("d_out", d_out, shape.T1 * shape.N1 * shape.D),))
+    _check_cuda((("d_out", d_out),))
     if into is None:
         into = torch.zeros(1, dtype=torch.float32, device=d_out.device)
     _check_absmax(into, False)
+    _check_cuda((("into", into),))
     N.check(lib.sfa_dout_absmax(_p(d_out), ctypes.byref(shape), int(row_begin),
                                 int(shape.T1 if row_end is None else row_end), _stream(stream), _p(into)))
     return into
@@ -221,6 +238,8 @@ def sfa_grad_rows(query, key, value, sparse_indices, d_out, out, softmax_max, so
                       softmax_sum)
     _check_accum(dkv_accum, shape, deterministic)
     _check_absmax(dout_absmax, deterministic)
+    _check_cuda(_sfa_named(query, key, value, sparse_indices, query_rope, key_rope, d_out, out, softmax_max,
+                           softmax_sum) + (("dkv_accum", dkv_accum), ("dout_absmax", dout_absmax)))
     sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
     skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
     ws_bytes = sfa_grad_workspace_size(shape, sparse_block_size, sparse_mode, deterministic)
@@ -247,6 +266,7 @@ def sfa_dkv_finalize(dkv_accum, query, key, query_rope, sparse_indices, *, layou
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
     _check_accum(dkv_accum, shape, deterministic)
     _check_absmax(dout_absmax, deterministic)
+    _check_cuda((("dkv_accum", dkv_accum), ("dout_absmax", dout_absmax)))
     kr_shape = key.shape[:-1] + (query_rope.shape[-1],)
     if outputs is None:
         outputs = (torch.empty_like(key), torch.empty_like(key),
@@ -271,6 +291,7 @@ def sfa_fwd(query, key, value, sparse_indices, query_rope, key_rope, *, scale: f
         _check16(name, t, dt)
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
     _check_sfa_inputs(shape, query, key, value, sparse_indices, query_rope, key_rope)
+    _check_cuda(_sfa_named(query, key, value, sparse_indices, query_rope, key_rope))
     sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
     skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
     n = ctypes.c_size_t()
@@ -291,9 +312,10 @@ def compact_indices(sparse_indices, key, query, query_rope, *, sparse_block_size
     """Index compaction step; returns (blocks [T1, topk], nblocks [T1], nrows [T1]) int32."""
     lib = N.load()
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
-    _need(sparse_indices.is_cuda and sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(),
-          "sparse_indices: int32 contiguous CUDA tensor")
+    _need(sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(),
+          "sparse_indices: int32 contiguous tensor")
     _check_numel((("sparse_indices", sparse_indices, shape.T1 * shape.N2 * shape.topk),))
+    _check_cuda((("sparse_indices", sparse_indices),))
     sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
     skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
     dev = sparse_indices.device
@@ -312,9 +334,10 @@ def key_rows(sparse_indices, key, query, query_rope, *, sparse_block_size: int, 
     rows [T1, topk*bs], count [T1]) int32.  Block-aligned lists flag padding slots with bit 31."""
     lib = N.load()
     shape = sfa_shape(query, key, query_rope, sparse_indices, layout, actual_seq_lengths_q)
-    _need(sparse_indices.is_cuda and sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(),
-          "sparse_indices: int32 contiguous CUDA tensor")
+    _need(sparse_indices.dtype == torch.int32 and sparse_indices.is_contiguous(),
+          "sparse_indices: int32 contiguous tensor")
     _check_numel((("sparse_indices", sparse_indices, shape.T1 * shape.N2 * shape.topk),))
+    _check_cuda((("sparse_indices", sparse_indices),))
     sq = _seqlens(actual_seq_lengths_q, layout, shape.B)
     skv = _seqlens(actual_seq_lengths_kv, layout, shape.B)
     dev = sparse_indices.device
@@ -336,6 +359,7 @@ def softmax_grad_rowsum(d_out, out, key, query_rope, sparse_indices, *, layout: 
     _check16("d_out", d_out, d_out.dtype)
     _check16("out", out, d_out.dtype)
     _check_numel((("out", out, d_out.numel()),))
+    _check_cuda((("d_out", d_out), ("out", out)))
     res = torch.empty(shape.T1 * shape.N1, dtype=torch.float32, device=d_out.device)
     N.check(lib.sfa_softmax_grad_rowsum(_p(d_out), _p(out), ctypes.byref(shape), _stream(stream), _p(res)))
     return res.view(shape.T1, shape.N1)
@@ -353,13 +377,15 @@ def _fa_shape(q, k, cu_q, cu_kv) -> N.FaShape:
     return s
 
 
-def _check_fa_inputs(s, k=None, v=None, dy=None, softmax_max=None, softmax_sum=None, attention_in=None):
+def _check_fa_inputs(s, q, k=None, v=None, dy=None, softmax_max=None, softmax_sum=None, attention_in=None):
     for name, t in (("softmax_max", softmax_max), ("softmax_sum", softmax_sum)):
         if t is not None:
             _check_f32(name, t)
     _check_numel((("k", k, s.T2 * s.Nkv * s.D), ("v", v, s.T2 * s.Nkv * s.D), ("dy", dy, s.T1 * s.Nq * s.D),
                   ("attention_in", attention_in, s.T1 * s.Nq * s.D), ("softmax_max", softmax_max, s.T1 * s.Nq * 8),
                   ("softmax_sum", softmax_sum, s.T1 * s.Nq * 8)))
+    _check_cuda((("q", q), ("k", k), ("v", v), ("dy", dy), ("attention_in", attention_in),
+                 ("softmax_max", softmax_max), ("softmax_sum", softmax_sum)))
 
 
 def _host_i64(x: Sequence[int]):
@@ -375,7 +401,7 @@ def fa_grad(q, k, v, dy, softmax_max, softmax_sum, attention_in, cu_seqlens_q, c
     for name, t in (("q", q), ("k", k), ("v", v), ("dy", dy), ("attention_in", attention_in)):
         _check16(name, t, q.dtype)
     shape = _fa_shape(q, k, cu_seqlens_q, cu_seqlens_kv)
-    _check_fa_inputs(shape, k, v, dy, softmax_max, softmax_sum, attention_in)
+    _check_fa_inputs(shape, q, k, v, dy, softmax_max, softmax_sum, attention_in)
     n = ctypes.c_size_t()
     N.check(lib.fa_grad_workspace_size(ctypes.byref(shape), int(sparse_mode), int(deterministic), ctypes.byref(n)))
     workspace = _workspace(workspace, n.value, q.device)
@@ -400,7 +426,7 @@ def fa_fwd(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, scale: float, sparse_mode: i
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check16(name, t, q.dtype)
     shape = _fa_shape(q, k, cu_seqlens_q, cu_seqlens_kv)
-    _check_fa_inputs(shape, k, v)
+    _check_fa_inputs(shape, q, k, v)
     n = ctypes.c_size_t()
     N.check(lib.fa_fwd_workspace_size(ctypes.byref(shape), int(sparse_mode), ctypes.byref(n)))
     ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
@@ -462,11 +488,10 @@ def lig_kl_grad(query, key, query_index, key_index, weights, softmax_max, softma
         _check16(name, t, query.dtype)
     for name, t in (("softmax_max", softmax_max), ("softmax_sum", softmax_sum),
                     ("softmax_max_index", softmax_max_index), ("softmax_sum_index", softmax_sum_index)):
-        _need(t.is_cuda and t.is_contiguous() and t.dtype == torch.float32, f"{name}: contiguous fp32 CUDA tensor")
+        _check_f32(name, t)
     for name, t in (("actual_seq_lengths_query", actual_seq_lengths_query),
                     ("actual_seq_lengths_key", actual_seq_lengths_key)):
-        _need(t is None or (t.is_cuda and t.dtype == torch.int64 and t.is_contiguous()),
-              f"{name}: int64 CUDA tensor")
+        _need(t is None or (t.dtype == torch.int64 and t.is_contiguous()), f"{name}: int64 tensor")
     if layout == "TND":
         _need(actual_seq_lengths_key is not None, "TND needs actual_seq_lengths_key")
     shape = lig_shape(query, key, query_index, key_index, layout, actual_seq_lengths_query, query_rope)
@@ -482,6 +507,12 @@ def lig_kl_grad(query, key, query_index, key_index, weights, softmax_max, softma
                        ("softmax_sum", softmax_sum, T1 * shape.N1), ("softmax_max_index", softmax_max_index, T1),
                        ("softmax_sum_index", softmax_sum_index, T1)):
         _need(t.numel() == n, f"{name}: {t.numel()} elements, expected {n}")
+    _check_cuda((("query", query), ("key", key), ("query_index", query_index), ("key_index", key_index),
+                 ("weights", weights), ("query_rope", query_rope), ("key_rope", key_rope),
+                 ("softmax_max", softmax_max), ("softmax_sum", softmax_sum),
+                 ("softmax_max_index", softmax_max_index), ("softmax_sum_index", softmax_sum_index),
+                 ("actual_seq_lengths_query", actual_seq_lengths_query),
+                 ("actual_seq_lengths_key", actual_seq_lengths_key)))
     need = lig_kl_grad_workspace_size(shape, sparse_mode)
     workspace = _workspace(workspace, need, query.device)
     if outputs is None:
