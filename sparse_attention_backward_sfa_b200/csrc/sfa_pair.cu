@@ -25,21 +25,24 @@
 //    each block contracts over both rows' heads (K = 256) in one TMEM
 //    accumulator, so the reduction of a key tile into dKey / dValue carries both
 //    rows: half the reduction bytes per (row, key) pair of the single-row kernel.
-//    For that, rank 1 sends its P and rank 0 its dS (32 KB per tile each) with a
-//    bulk copy shared::cta -> shared::cluster that completes on the receiver's
-//    mbarrier; each also loads the partner row's dO (rank 0) or q (rank 1) chunks.
+//    For that, rank 0 sends its dS (32 KB per tile) with a bulk copy shared::cta
+//    -> shared::cluster that completes on rank 1's mbarrier, and rank 1 stores its
+//    P straight into rank 0's receive buffer (distributed shared memory stores,
+//    a proxy fence, one remote arrive): rank 1 keeps no P of its own, and that
+//    buffer is a fifth slot of its operand ring.  Each rank also loads the partner
+//    row's dO (rank 0) or q (rank 1) chunks.
 //    dQ~ stays per row: each rank forms dQ~^T = K~^T.dS^T of its own row and
 //    accumulates it across the row's tiles in its per-CTA fp32 scratch.
-//  * Shared memory: a 4-slot ring of 32 KB operand chunks, P (X), dS (Y) and the
-//    received tile (R), 32 KB each, row ids and masks, constants, barriers: the
+//  * Shared memory: a ring of 32 KB operand chunks (4 slots on rank 0, 5 on rank
+//    1), P (X, rank 0 only), dS (Y) and the received tile (R), 32 KB each, row ids and masks, constants, barriers: the
 //    same offsets in both CTAs, so an offset names the same object in the peer.
 //  * Hand-over of the single received buffer R: a rank grants its partner the
 //    next tile's copy (remote arrive on the partner's PEER_FREE) once its own
 //    gradient MMAs of the previous tile completed (they read R); the sender
 //    overwrites its copy source only after that grant, which also proves the
-//    previous copy was consumed.  The receiver arms its RECV barrier with the
-//    expected bytes when it grants, and its MMA warp waits on RECV before the
-//    first MMA that reads R.
+//    previous copy was consumed.  Rank 1 arms its RECV barrier with the expected
+//    bytes when it grants; rank 0's RECV completes on the partner's arrive; each
+//    MMA warp waits on RECV before the first MMA that reads R.
 //  * Warp roles per CTA: 0-3 softmax/dS, 4-11 flush, 12 TMA producer, 13 MMA
 //    issuer; the producer and MMA warps run a cross-tile software pipeline (the
 //    next tile's S^T / dP^T items interleaved, a (K, Q, dO) group at a time, into
@@ -61,14 +64,15 @@ namespace {
 using namespace tc;
 
 constexpr int kThreads = 448;       // 4 softmax + 8 flush + 1 TMA + 1 MMA warps
-constexpr int kSlots = 4;           // operand ring
+constexpr int kSlots = 4;           // operand ring of rank 0
+constexpr int kSlotsMax = 5;        // rank 1: its P goes straight to the partner, X is a fifth slot
 constexpr int kSlotBytes = 32768;
 constexpr int kHalf = 16384;
 constexpr int kKeys = 128;          // key rows per tile (MMA M)
 constexpr int kN1 = 128;            // query heads (MMA N of S^T / dP^T, K of the gradient blocks per row)
 constexpr uint32_t kTileBytes = 32768;  // P or dS of one row and one tile, bf16 [128 keys x 128 heads]
 
-constexpr int kOffX = kSlots * kSlotBytes;        // P of the own row (rank 1: staged for the copy)
+constexpr int kOffX = kSlots * kSlotBytes;        // P of the own row (rank 0); rank 1: ring slot 4
 constexpr int kOffY = kOffX + 32768;              // dS of the own row
 constexpr int kOffR = kOffY + 32768;              // the partner's P (rank 0) or dS (rank 1)
 constexpr int kOffRows = kOffR + 32768;           // int32 [2][128] key row ids, bit 31: invalid for both rows
@@ -77,8 +81,8 @@ constexpr int kOffConst = kOffMask + 2 * 4 * 4;   // float [3][128] max*log2e, 1
 constexpr int kOffBar = kOffConst + 3 * kN1 * 4;
 enum {
     BAR_FULL = 0,
-    BAR_EMPTY = BAR_FULL + kSlots,
-    BAR_SDP = BAR_EMPTY + kSlots,
+    BAR_EMPTY = BAR_FULL + kSlotsMax,
+    BAR_SDP = BAR_EMPTY + kSlotsMax,
     BAR_PDS_FULL,
     BAR_PDS_FREE,
     BAR_STG_FULL,
@@ -272,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
     };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kSlots; ++s) {
+        for (int s = 0; s < kSlotsMax; ++s) {
             mbar_init(FULL(s), 1);
             mbar_init(EMPTY(s), 1);
         }
@@ -309,6 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
     const float scale = prm.scale;
     const int nblocks = num_blocks(rank);  // gradient blocks per tile: 5 dQ~ + the key-side ones
     const int nkey = nblocks - 5;
+    const int ring_slots = rank ? kSlotsMax : kSlots;  // ring slots of this rank
 
     if (warp == 12) {
         // =================== TMA producer ===================
@@ -415,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                     tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, t * kN1, FULL(slot));
             }
             if (lane == 0) issued_mask |= 1u << slot;
-            if (++slot == kSlots) { slot = 0; sphase ^= 1; }
+            if (++slot == ring_slots) { slot = 0; sphase ^= 1; }
             return true;
         };
         auto sdp_load = [&](const Tile& x, int j) -> bool {
@@ -451,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
         }
         // drain: every issued load must land before the CTA can exit
         if (lane == 0) {
-            for (int k = 0; k < kSlots; ++k) {
-                const int s = (slot + k) % kSlots;
+            for (int k = 0; k < ring_slots; ++k) {
+                const int s = (slot + k) % ring_slots;
                 const uint32_t ph = s < slot ? sphase : sphase ^ 1;
                 if (issued_mask & (1u << s)) {
                     uint64_t t0 = globaltimer();
@@ -482,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
             return r;
         };
         auto advance = [&]() {
-            if (++slot == kSlots) { slot = 0; sphase ^= 1; }
+            if (++slot == ring_slots) { slot = 0; sphase ^= 1; }
         };
         auto sdp = [&](int j) -> bool {
             int kind, c;
@@ -598,6 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                         if (!ok) break;
                         ++recv_done;
                         tc_fence_after();
+                        if (!rank) fence_view_async_shared();  // R was written by the partner's stores
                     }
                     if (!(ok = grad_half(T_STG(stg), sR, false, true, 109))) break;
                     if (lane == 0) {
@@ -659,7 +665,6 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
         const uint32_t peer_free_remote = mapa(PEER_FREE, peer);
         const uint32_t recv_remote = mapa(RECV, peer);
         const uint32_t r_remote = mapa(sbase + kOffR, peer);
-        const uint32_t copy_src = sbase + (rank ? kOffX : kOffY);  // rank 1 sends P, rank 0 sends dS
         int tile_ctr = 0;
         uint32_t grants = 0;
         bool ok = true;
@@ -683,12 +688,15 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                 if (ok) ok = WAIT(ROWS_FULL(tile_ctr & 1), (tile_ctr >> 1) & 1, 115);
                 if (ok && tile_ctr > 0) ok = WAIT(PDS_FREE, (tile_ctr - 1) & 1, 111);
                 if (ok && threadIdx.x == 0) {
-                    // R is free again (this CTA's MMAs of the previous tile completed): arm it for this
-                    // tile's copy and grant it to the partner; then wait for the partner's grant, which
-                    // also means this CTA's previous copy has been consumed, before overwriting its source
-                    mbar_expect_tx(RECV, kTileBytes);
-                    ++grants;
-                    *granted = grants;
+                    // R is free again (this CTA's MMAs of the previous tile completed): grant it to the
+                    // partner (rank 1 first arms it for the bulk copy of rank 0's dS; rank 0 receives
+                    // rank 1's P as stores and one remote arrive); then wait for the partner's grant,
+                    // which also means this CTA's previous tile has been consumed there, before writing
+                    if (rank) {
+                        mbar_expect_tx(RECV, kTileBytes);
+                        ++grants;
+                        *granted = grants;
+                    }
                     if (tile_ctr > 0) {
                         mbar_arrive_remote(peer_free_remote);
                         ok = wait_cluster(PEER_FREE, (tile_ctr - 1) & 1, abort_flag, prm.err, 112, prm.wait_ns);
@@ -732,17 +740,24 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const uint32_t off = half * kHalf + j * 128 + (((u0 + u) ^ (j & 7)) << 4);
-                        *reinterpret_cast<uint4*>(sPp + off) =
-                            make_uint4(pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
+                        if (rank)  // rank 1's P is only read by rank 0: stored straight into its R
+                            st_cluster_v4(r_remote + off, pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
+                        else
+                            *reinterpret_cast<uint4*>(sPp + off) =
+                                make_uint4(pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
                         *reinterpret_cast<uint4*>(sDSp + off) =
                             make_uint4(dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
                     }
                 }
                 fence_view_async_shared();
+                if (rank) fence_view_async_cluster();
                 tc_fence_before();
                 mbar_arrive(PDS_FULL);
                 asm volatile("bar.sync 1, 128;" ::: "memory");  // the whole tile is written and fenced
-                if (threadIdx.x == 0) bulk_copy_to_peer(r_remote, copy_src, kTileBytes, recv_remote);
+                if (threadIdx.x == 0) {
+                    if (rank) mbar_arrive_remote(recv_remote);  // rank 0's R holds this tile's P
+                    else bulk_copy_to_peer(r_remote, sbase + kOffY, kTileBytes, recv_remote);  // dS to rank 1
+                }
             }
         }
     } else {

@@ -259,8 +259,12 @@ def merged_ops(rank, ntiles, same=True):
     return loads, mmas
 
 
-def simulate_merged(ntiles, slots=4, same=True):
-    """Both CTAs' merged schedules against the ring, staging, softmax / exchange and flush rules."""
+def simulate_merged(ntiles, slots=(4, 5), same=True):
+    """Both CTAs' merged schedules against the ring, staging, softmax / exchange and flush rules.
+    `slots`: ring slots of rank 0 and rank 1 (rank 1 stores its P straight into the partner's
+    receive buffer, so its own P buffer serves as a fifth slot); an int gives both the same."""
+    if isinstance(slots, int):
+        slots = (slots, slots)
     class C:
         pass
 
@@ -268,6 +272,7 @@ def simulate_merged(ntiles, slots=4, same=True):
     for rank in (0, 1):
         c = C()
         c.rank = rank
+        c.slots = slots[rank]
         c.loads, c.mmas = merged_ops(rank, ntiles, same)
         last_use = {}
         for mi, (_, _, _, ids) in enumerate(c.mmas):
@@ -283,7 +288,7 @@ def simulate_merged(ntiles, slots=4, same=True):
     def step(c, peer):
         progress = False
         if c.loaded < len(c.loads):  # producer: FIFO ring
-            if c.loaded < slots or (c.loaded - slots) in c.freed:
+            if c.loaded < c.slots or (c.loaded - c.slots) in c.freed:
                 c.loaded += 1
                 progress = True
         if c.issued < len(c.mmas):  # MMA
@@ -328,8 +333,9 @@ def simulate_merged(ntiles, slots=4, same=True):
 
 @pytest.mark.parametrize("ntiles", [1, 2, 3, 8])
 @pytest.mark.parametrize("same", [True, False])
-def test_merged_schedule_is_deadlock_free(ntiles, same):
-    assert simulate_merged(ntiles, same=same)
+@pytest.mark.parametrize("slots", [(4, 5), 4])
+def test_merged_schedule_is_deadlock_free(ntiles, same, slots):
+    assert simulate_merged(ntiles, slots=slots, same=same)
 
 
 def test_merged_schedule_loads():
@@ -342,3 +348,4 @@ def test_merged_schedule_loads():
 
 def test_merged_model_detects_a_deadlock():
     assert not simulate_merged(3, slots=2)
+    assert not simulate_merged(3, slots=(2, 5))
