@@ -328,11 +328,34 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
             int32_t my[4];  // this lane's four key rows for gather4 (clamped into the key tensor)
             int32_t run0;   // row of slot 0 (the 2-D tile's first row when contiguous)
         };
+        // The pair's tile count and spans are read once per pair, and the block ids of the
+        // pair's next tile are fetched one tile ahead: under the reduction traffic a dependent
+        // global read costs about a microsecond, and this warp's reads sit between its loads.
         int w_next = cid, tile_next = 0;
+        int pw = -1, pt0 = 0, pnslots = 0;  // the pair the cached fields describe
+        TokInfo ti0{}, ti1{};
+        int32_t pre[4] = {0, 0, 0, 0};  // block ids of this lane's slots in tile pre_tile of pair pw
+        int pre_tile = -1;
+        auto fetch_blocks = [&](int tile, int32_t (&blk)[4]) {
+            const int32_t* bl = prm.blocks + (int64_t)pt0 * prm.topk;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int g = tile * kKeys + 4 * lane + e;
+                blk[e] = g < pnslots ? bl[g / bs] : 0;
+            }
+        };
         auto next_tile = [&](Tile& x) -> bool {
             while (w_next < npairs) {
-                const int t0 = prm.pairs[w_next];
-                const int nslots = prm.nblk[t0] * bs;
+                if (pw != w_next) {
+                    pw = w_next;
+                    pt0 = prm.pairs[w_next];
+                    pnslots = prm.nblk[pt0] * bs;
+                    ti0 = tok_info(prm.sd, pt0);
+                    ti1 = tok_info(prm.sd, (int64_t)pt0 + 1);
+                    pre_tile = -1;
+                }
+                const int t0 = pt0;
+                const int nslots = pnslots;
                 if (tile_next * kKeys >= nslots) {
                     w_next += ncl;
                     tile_next = 0;
@@ -340,8 +363,17 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                 }
                 x.t0 = t0;
                 x.tile = tile_next++;
-                const TokInfo ti0 = tok_info(prm.sd, t0), ti1 = tok_info(prm.sd, (int64_t)t0 + 1);
-                const int32_t* bl = prm.blocks + (int64_t)t0 * prm.topk;
+                int32_t blkv[4];
+                if (pre_tile == x.tile) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) blkv[e] = pre[e];
+                } else {
+                    fetch_blocks(x.tile, blkv);
+                }
+                if (tile_next * kKeys < nslots) {  // the pair's next tile: its reads are issued now
+                    fetch_blocks(tile_next, pre);
+                    pre_tile = tile_next;
+                }
                 const int rb = tile_ctr & 1;
                 if (lane == 0) ok = WAIT(ROWS_EMPTY(rb), ((tile_ctr >> 1) & 1) ^ 1, 101);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -357,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                     bool own = false, any = false;
                     if (g < nslots) {
                         const int i = g / bs, o = g - i * bs;
-                        const int64_t blk = bl[i];
+                        const int64_t blk = blkv[e];
                         row = ti0.kv_start + blk * bs + o;
                         const int k0 = block_rows(blk, bs, ti0, prm.mode), k1 = block_rows(blk, bs, ti1, prm.mode);
                         own = o < (rank ? k1 : k0);
@@ -529,9 +561,14 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
             return true;
         };
         int w_next = cid, tile_next = 0;
+        int pw = -1, pnslots = 0;  // key slots of pair pw (read once per pair)
         auto next_tile = [&](int& w_of) -> bool {
             while (w_next < npairs) {
-                const int nslots = prm.nblk[prm.pairs[w_next]] * bs;
+                if (pw != w_next) {
+                    pw = w_next;
+                    pnslots = prm.nblk[prm.pairs[w_next]] * bs;
+                }
+                const int nslots = pnslots;
                 if (tile_next * kKeys >= nslots) {
                     w_next += ncl;
                     tile_next = 0;
