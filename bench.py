@@ -155,12 +155,14 @@ def kw(p):
 
 def paired_work_fraction(p, S):
     """Share of the valid (row, key) pairs in rows the paired kernel takes: rows (2m, 2m + 1) of
-    one sequence whose sorted block lists are identical and non-empty (the library's pairing
-    rule); the rest run on the single-row kernel."""
+    one sequence whose block lists (sorted where the library sorts them) are identical and
+    non-empty (the library's pairing rule); the rest run on the single-row kernel."""
     import numpy as np
     import torch
+    # the library sorts block-sparse lists of topk <= 4096 before pairing; others pair as compacted
+    sort = p.block_size > 1 and p.topk <= 4096
     blocks, nb, _, cnt = S.key_rows(p.indices, p.k, p.q, p.q_rope, sparse_block_size=p.block_size,
-                                    layout=p.layout, sparse_mode=p.sparse_mode, sorted_blocks=True,
+                                    layout=p.layout, sparse_mode=p.sparse_mode, sorted_blocks=sort,
                                     actual_seq_lengths_q=p.seqlens_q, actual_seq_lengths_kv=p.seqlens_kv)
     T1 = nb.numel()
     M = T1 // 2
