@@ -53,18 +53,27 @@ constexpr int kSlotBytes = 32768;
 constexpr int kHalf = 16384;
 constexpr int kKeys = 128;          // key rows per tile (MMA M)
 
+// N1 = 128: every chunk streams through a 5-slot ring of 32 KB.  N1 = 64: the tile's key rows stay
+// resident (5 chunks, 144 KB) from the S^T / dP^T items to the dQ~ blocks, so each tile gathers
+// them once instead of twice (gathered loads are the slowest TMA operations); q / dO chunks
+// (16 KB at 64 heads) stream through a 3-slot ring of 16 KB.
 template <int N1> struct Cfg {
-    static constexpr int kSlots = N1 == 128 ? 5 : 6;
-    static constexpr int kRing = kSlots * kSlotBytes;
-    static constexpr int kOffP = kRing;
+    static constexpr bool kResident = N1 == 64;
+    static constexpr int kKeyBytes = 4 * kSlotBytes + kHalf;                // resident key tile
+    static constexpr int kSlots = N1 == 128 ? 5 : 3;
+    static constexpr int kRingSlot = N1 == 128 ? kSlotBytes : 16384;
+    static constexpr int kQHalf = N1 * 128;                                 // 64-dim halves of a q / dO chunk
+    static constexpr int kOffRing = kResident ? kKeyBytes : 0;
+    static constexpr int kOffP = kOffRing + kSlots * kRingSlot;
     static constexpr int kOffDS = kOffP + (N1 == 128 ? 32768 : 16384);
     static constexpr int kOffRows = kOffDS + (N1 == 128 ? 32768 : 16384);  // int32 [2][128]
     static constexpr int kOffConst = kOffRows + 2 * kKeys * 4;              // float [3][128]
     static constexpr int kOffBar = kOffConst + 3 * 128 * 4;
-    static constexpr int kNumBars = 2 * kSlots + 12;
+    static constexpr int kNumBars = 2 * kSlots + 12 + (kResident ? 10 : 0);
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmem = kOffMisc + 16;
 };
+static_assert(Cfg<64>::kSmem <= 232448 && Cfg<128>::kSmem <= 232448, "shared memory per CTA");
 
 struct FusedParams {
     CUtensorMap mapQ, mapQr, mapO, mapK, mapKr;  // dO shares mapO; key maps: 1-row boxes (gather4)
@@ -234,6 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
     auto ROWS_FULL = [&](int s) { return bar0 + 8u * (2 * C::kSlots + 7 + s); };
     auto ROWS_EMPTY = [&](int s) { return bar0 + 8u * (2 * C::kSlots + 9 + s); };
     const uint32_t DONE = bar0 + 8u * (2 * C::kSlots + 11);
+    // resident key tile (N1 = 64): chunk c loaded / free for the next tile's load
+    auto KFULL = [&](int c) { return bar0 + 8u * (2 * C::kSlots + 12 + c); };
+    auto KEMPTY = [&](int c) { return bar0 + 8u * (2 * C::kSlots + 17 + c); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     // bounded mbarrier wait: past prm.wait_ns it records `code` in the error word and every role exits
@@ -256,6 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
             mbar_init(ROWS_EMPTY(s), 256);
         }
         mbar_init(DONE, 1);
+        if (C::kResident)
+            for (int c = 0; c < 5; ++c) {
+                mbar_init(KFULL(c), 1);
+                mbar_init(KEMPTY(c), 1);
+            }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -281,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
         int tile_ctr = 0;  // tiles whose row ids have been staged
         bool ok = true;
         uint32_t issued_mask = 0;  // slots that have received loads
+        uint32_t kbits = 0;        // resident key chunks: parity of their loads so far
         // the CTA's tiles in order: row w (stepping by gridDim.x, rows without keys skipped), tile
         struct Tile {
             int t, n, tile, first, run0;
@@ -332,35 +350,43 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
         };
         // one chunk of tile x into the next ring slot
         auto load = [&](const Tile& x, int kind, int c) -> bool {
-            if (lane == 0) ok = WAIT(EMPTY(slot), sphase ^ 1, 2);
+            const bool resident = C::kResident && kind == 0;  // into the key tile's chunk c
+            if (lane == 0)
+                ok = resident ? WAIT(KEMPTY(c), ((kbits >> c) & 1u) ^ 1u, 12) : WAIT(EMPTY(slot), sphase ^ 1, 2);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) return false;
-            const uint32_t dst = sbase + slot * kSlotBytes;
+            const uint32_t dst = resident ? sbase + c * kSlotBytes : sbase + C::kOffRing + slot * C::kRingSlot;
+            const uint32_t bar = resident ? KFULL(c) : FULL(slot);
             const int halves = c < 4 ? 2 : 1;
             if (lane == 0) {
                 const uint32_t rows = kind == 0 ? kKeys : N1;
-                mbar_expect_tx(FULL(slot), halves * rows * 128u);
+                mbar_expect_tx(bar, halves * rows * 128u);
             }
             __syncwarp();
             if (kind == 0 && x.contig) {
                 if (lane == 0) {
                     const CUtensorMap* map = c < 4 ? &prm.mapK128 : &prm.mapKr128;
                     for (int h = 0; h < halves; ++h)
-                        tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, x.run0, FULL(slot));
+                        tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, x.run0, bar);
                 }
             } else if (kind == 0) {
                 // key rows: every lane gathers its own four rows, in parallel
                 const CUtensorMap* map = c < 4 ? &prm.mapK : &prm.mapKr;
                 for (int h = 0; h < halves; ++h)
                     tma_gather4(dst + h * kHalf + lane * 512, map, c < 4 ? c * 128 + h * 64 : 0, x.my[0], x.my[1],
-                                x.my[2], x.my[3], FULL(slot));
+                                x.my[2], x.my[3], bar);
             } else if (lane == 0) {
                 const CUtensorMap* map = kind == 1 ? (c < 4 ? &prm.mapQ : &prm.mapQr) : &prm.mapO;
                 for (int h = 0; h < halves; ++h)
-                    tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, x.t * N1, FULL(slot));
+                    tma_load_2d(dst + h * C::kQHalf, map, c < 4 ? c * 128 + h * 64 : 0, x.t * N1, bar);
             }
-            if (lane == 0) issued_mask |= 1u << slot;
-            if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+            if (resident) {
+                kbits ^= 1u << c;
+                if (lane == 0) issued_mask |= 1u << (16 + c);
+            } else {
+                if (lane == 0) issued_mask |= 1u << slot;
+                if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+            }
             return true;
         };
         Tile cur, nxt;
@@ -375,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
             for (int k = 0; k < 14 && ok; ++k) {
                 int kind, b;
                 block_of(k, kind, b);
-                ok = load(cur, kind, b);
+                if (!(C::kResident && kind == 0)) ok = load(cur, kind, b);  // dQ~ blocks read the key tile
                 if (ok && k == kInterleave) have_next = next_tile(nxt);
                 if (ok && have_next && k >= kInterleave) {
                     for (int q = 0; q < 2 && ok; ++q) {
@@ -400,6 +426,12 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                     }
                 }
             }
+            for (int c = 0; c < 5; ++c)  // resident key chunks: their last load
+                if (issued_mask & (1u << (16 + c))) {
+                    const uint64_t t0 = globaltimer();
+                    while (!mbar_try(KFULL(c), ((kbits >> c) & 1u) ^ 1u) && globaltimer() - t0 < 1000000000ull) {
+                    }
+                }
         }
     } else if (warp == 13) {
         // =================== MMA issuer ===================
@@ -413,6 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
         int blk_ctr = 0;
         bool ok = true;
         uint32_t slotK = 0;  // key chunk of the S / dP item pair in progress
+        int sdp_tiles = 0;   // tiles whose S / dP items were issued (resident key tile: load parity)
+        auto ring_addr = [&](int s) { return sbase + C::kOffRing + (uint32_t)s * C::kRingSlot; };
         auto wait_full = [&](int code) -> bool {
             bool r = true;
             if (lane == 0) r = WAIT(FULL(slot), sphase, code);
@@ -424,22 +458,36 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
         auto sdp = [&](int j) -> bool {
             int kind, c;
             sdp_item(j, kind, c);
+            if (C::kResident && kind == 0) {  // the key chunk lands in the resident key tile
+                bool r = true;
+                if (lane == 0) r = WAIT(KFULL(c), (uint32_t)sdp_tiles & 1u, 13);
+                r = __shfl_sync(0xffffffffu, r, 0);
+                if (!r) return false;
+                tc_fence_after();
+                slotK = sbase + (uint32_t)c * kSlotBytes;
+                return true;
+            }
             if (!wait_full(3)) return false;
-            const uint32_t sa = sbase + slot * kSlotBytes;
+            const uint32_t sa = ring_addr(slot);
             if (kind == 0) slotK = sa;
             if (lane == 0 && kind != 0) {
                 const uint32_t dst = kind == 1 ? T_S : T_DP;
                 const int ksteps = c < 4 ? 8 : 4;
                 for (int ks = 0; ks < ksteps; ++ks) {
-                    const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-                    mma(dst, sdesc(slotK + off, 16, 1024), sdesc(sa + off, 16, 1024), ID_S, (c > 0 || ks > 0) ? 1u : 0u);
+                    const uint32_t offk = (ks >> 2) * kHalf + (ks & 3) * 32;      // key chunk halves
+                    const uint32_t offq = (ks >> 2) * C::kQHalf + (ks & 3) * 32;  // q / dO chunk halves
+                    mma(dst, sdesc(slotK + offk, 16, 1024), sdesc(sa + offq, 16, 1024), ID_S,
+                        (c > 0 || ks > 0) ? 1u : 0u);
                 }
-                // a slot is released once the MMAs that read it have completed
+                // a slot is released once the MMAs that read it have completed; a resident key
+                // chunk stays for the dQ~ block that reads it again
                 mma_commit(EMPTY(slot));
-                if (kind == 2 || c == 4) mma_commit(EMPTY((slotK - sbase) / kSlotBytes));
+                if (!C::kResident && (kind == 2 || c == 4))
+                    mma_commit(EMPTY((slotK - sbase - C::kOffRing) / C::kRingSlot));
                 if (j == 13) mma_commit(SDP_FULL);
             }
             __syncwarp();
+            if (j == 13) ++sdp_tiles;
             if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
             return true;
         };
@@ -471,19 +519,20 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                 const int stg = blk_ctr & 1;
                 int kind, b;
                 block_of(k, kind, b);
+                const bool resident = C::kResident && kind == 0;  // A = the resident key chunk b
                 if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 5);
-                if (lane == 0 && ok) ok = WAIT(FULL(slot), sphase, 6);
+                if (lane == 0 && ok && !resident) ok = WAIT(FULL(slot), sphase, 6);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t sa = sbase + slot * kSlotBytes;
+                const uint32_t sa = resident ? sbase + (uint32_t)b * kSlotBytes : ring_addr(slot);
                 if (lane == 0) {
                     const uint32_t dst = T_STG(stg);
                     if (kind != 0) {
                         // dV^T (A = dO chunk) or dK~^T (A = q chunk): [128 dims x 128 keys], K = heads
                         const uint32_t bsrc = kind == 2 ? sP : sDS;
                         for (int ks = 0; ks < N1 / 16; ++ks) {
-                            const uint64_t a = sdesc(sa + ks * 2048, kHalf, 1024);
+                            const uint64_t a = sdesc(sa + ks * 2048, C::kQHalf, 1024);
                             const uint64_t bd = sdesc(bsrc + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
                             mma(dst, a, bd, ID_G, ks > 0 ? 1u : 0u);
                         }
@@ -495,12 +544,12 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_fused_kernel(const __grid
                             mma(dst, a, bd, ID_Q, ks > 0 ? 1u : 0u);
                         }
                     }
-                    mma_commit(EMPTY(slot));
+                    mma_commit(resident ? KEMPTY(b) : EMPTY(slot));  // the key chunk's last read
                     mma_commit(STG_FULL(stg));
                     if (k == 13) mma_commit(PDS_FREE);
                 }
                 __syncwarp();
-                if (++slot == C::kSlots) { slot = 0; sphase ^= 1; }
+                if (!resident && ++slot == C::kSlots) { slot = 0; sphase ^= 1; }
                 // the next tile's S^T / dP^T overwrite this tile's: the softmax warps have read
                 // them (PDS_FULL above), and P / dS stay in shared memory until PDS_FREE
                 if (k == kInterleave) have_next = next_tile();
