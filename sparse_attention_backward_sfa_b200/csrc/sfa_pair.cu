@@ -33,8 +33,8 @@
 //    row's dO (rank 0) or q (rank 1) chunks.
 //    dQ~ stays per row: each rank forms dQ~^T = K~^T.dS^T of its own row and
 //    accumulates it across the row's tiles in its per-CTA fp32 scratch.
-//  * Shared memory: a ring of 32 KB operand chunks (4 slots on rank 0, 5 on rank
-//    1), P (X, rank 0 only), dS (Y) and the received tile (R), 32 KB each, row ids and masks, constants, barriers: the
+//  * Shared memory: 32 KB operand slots (4 on rank 0, 5 on rank 1) split into the
+//    two rings, P (X, rank 0 only), dS (Y) and the received tile (R), 32 KB each, row ids and masks, constants, barriers: the
 //    same offsets in both CTAs, so an offset names the same object in the peer.
 //  * Hand-over of the single received buffer R: a rank grants its partner the
 //    next tile's copy (remote arrive on the partner's PEER_FREE) once its own
@@ -43,10 +43,10 @@
 //    previous copy was consumed.  Rank 1 arms its RECV barrier with the expected
 //    bytes when it grants; rank 0's RECV completes on the partner's arrive; each
 //    MMA warp waits on RECV before the first MMA that reads R.
-//  * Warp roles per CTA: 0-3 softmax/dS, 4-11 flush, 12 TMA producer, 13 MMA
-//    issuer; the producer and MMA warps run a cross-tile software pipeline (the
-//    next tile's S^T / dP^T items interleaved, a (K, Q, dO) group at a time, into
-//    this tile's last five gradient blocks).  Every wait is bounded; on timeout the CTA records an
+//  * Warp roles per CTA: 0-3 softmax/dS, 4-11 flush, 12 / 14 TMA producers and
+//    13 / 15 MMA issuers of the gradient blocks / the S^T and dP^T items, each
+//    pair with its own ring, so the next tile's S^T / dP^T are formed while this
+//    tile's gradient blocks run.  Every wait is bounded; on timeout the CTA records an
 //    error word and leaves, after waiting (bounded) for copies still addressed to
 //    it and meeting its partner at the final cluster barrier.
 #include <cuda.h>
@@ -63,9 +63,10 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 448;       // 4 softmax + 8 flush + 1 TMA + 1 MMA warps
-constexpr int kSlots = 4;           // operand ring of rank 0
+constexpr int kThreads = 512;       // 4 softmax + 8 flush + 2 TMA + 2 MMA warps
+constexpr int kSlots = 4;           // operand slots of rank 0
 constexpr int kSlotsMax = 5;        // rank 1: its P goes straight to the partner, X is a fifth slot
+constexpr int kSRing0 = 3, kSRing1 = 3;  // S / dP ring slots of rank 0 / 1 (the rest carry the gradient blocks)
 constexpr int kSlotBytes = 32768;
 constexpr int kHalf = 16384;
 constexpr int kKeys = 128;          // key rows per tile (MMA M)
@@ -123,20 +124,20 @@ struct PairParams {
     uint64_t wait_ns;
 };
 
-// S / dP items j = 0..13 of a tile: K0 Q0 O0 K1 Q1 O1 K2 Q2 O2 K3 Q3 O3 K4 Q4 (kind 0 key, 1 q, 2 dO)
-__device__ __forceinline__ void sdp_item(int j, int& kind, int& c) {
-    c = j / 3;
-    kind = j - 3 * c;
-}
 // Gradient blocks of a tile: k < 5 dQ~ block k of the own row (one key chunk); k >= 5 the rank's
 // key-side block k - 5 (rank 0 dV, rank 1 dK~) over both rows (the own row's chunk, then the partner's).
 __device__ __forceinline__ int num_blocks(uint32_t rank) { return rank ? 10 : 9; }
-// Per tile: the five dQ~ blocks, then for c = 0..4 the key-side block c (if the rank has it)
-// followed by the next tile's S item c (K_c, q_c) and dP item c (c < 4: K_c, dO_c).  When the
-// next tile belongs to the same pair, the own row's chunk of key-side block c is also the next
-// tile's q_c (rank 1) or dO_c (rank 0): it is loaded once and released after its second use
-// (23 / 24 chunk loads per tile instead of 27 / 29).  A key chunk is held only across its own
-// S / dP items, so the 4-slot ring cannot deadlock (checked by a CPU model of both CTAs).
+// Two rings and two MMA warps per CTA.  The gradient ring (1 slot on rank 0, 2 on rank 1) carries,
+// per tile, the five key chunks of the dQ~ blocks, then each key-side block's own-row and partner
+// chunk, consumed in that order by the gradient MMA warp.  The S / dP ring (3 slots) carries each
+// tile's S items (K_c, q_c) and dP items (the same K_c, dO_c), consumed by the S / dP MMA warp, which
+// starts a tile's items once the softmax has read the previous tile's S^T / dP^T.  So the gradient
+// blocks never wait for the next tile's S / dP operands, and the flush (the reductions, the
+// throughput bound of the gradient phase) is fed back to back; per tile 27 (rank 0) / 29 (rank 1)
+// chunks are loaded.  A ring slot holds a chunk only until the MMAs of its item or block complete,
+// so neither ring can deadlock (checked by a CPU model of both CTAs).  Slot splits measured on the
+// 16K-token block-sparse workload: gradient / S 1+3 and 2+3 (rank 0, rank 1) 73.8 ms, 2+2 and 2+3
+// (key chunk reloaded for the dP item) 74.6-75.8 ms, one ring for both 78.3 ms.
 
 __device__ __forceinline__ bool softmax_all(bool v) {
     uint32_t r;
@@ -289,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
             mbar_init(ROWS_FULL(s), 1);
             mbar_init(ROWS_EMPTY(s), 256);
         }
-        mbar_init(DONE, 1);
+        mbar_init(DONE, 2);
         mbar_init(RECV, 1);
         mbar_init(PEER_FREE, 1);
         misc[1] = misc[2] = misc[3] = 0;
@@ -313,11 +314,16 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
     const float scale = prm.scale;
     const int nblocks = num_blocks(rank);  // gradient blocks per tile: 5 dQ~ + the key-side ones
     const int nkey = nblocks - 5;
-    const int ring_slots = rank ? kSlotsMax : kSlots;  // ring slots of this rank
+    // two rings: slots [0, g_slots) carry the gradient blocks' chunks, the next two slots the S / dP
+    // items' chunks (rank 1's fifth slot is its P buffer, which it never uses)
+    const int s_slots = rank ? kSRing1 : kSRing0;
+    const int g_slots = (rank ? kSlotsMax : kSlots) - s_slots;
 
-    if (warp == 12) {
-        // =================== TMA producer ===================
-        int slot = 0;
+    if (warp == 12 || warp == 14) {
+        // =================== TMA producers: 12 the gradient ring, 14 the S / dP ring ===================
+        const bool srole = warp == 14;  // also stages each tile's key row ids and masks
+        const int ring0 = srole ? g_slots : 0, ring_n = srole ? s_slots : g_slots;
+        int slot = 0;  // position in this producer's ring
         uint32_t sphase = 0;
         int tile_ctr = 0;
         bool ok = true;
@@ -375,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                     pre_tile = tile_next;
                 }
                 const int rb = tile_ctr & 1;
-                if (lane == 0) ok = WAIT(ROWS_EMPTY(rb), ((tile_ctr >> 1) & 1) ^ 1, 101);
+                if (srole && lane == 0) ok = WAIT(ROWS_EMPTY(rb), ((tile_ctr >> 1) & 1) ^ 1, 101);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) return false;
                 // lane L owns slots 4L..4L+3 of the tile; a slot is block i = g / bs, row o = g % bs of it
@@ -396,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                         any = o < (k0 > k1 ? k0 : k1);
                     }
                     rowv[e] = (int32_t)row;
-                    rowids[rb * kKeys + 4 * lane + e] = any ? (int32_t)row : (int32_t)0x80000000;
+                    if (srole) rowids[rb * kKeys + 4 * lane + e] = any ? (int32_t)row : (int32_t)0x80000000;
                     if (own) ownbits |= 1u << e;
                 }
                 // slot 0's row, then a contiguity vote (slots past the list's end do not count)
@@ -412,15 +418,17 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                 }
                 x.run0 = run0;
                 x.contig = __all_sync(0xffffffffu, contig);
-                // own-row validity bits: word w covers slots 32w..32w+31 (lanes 8w..8w+7)
+                if (srole) {
+                    // own-row validity bits: word w covers slots 32w..32w+31 (lanes 8w..8w+7)
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const uint32_t part = (lane >> 3) == w ? ownbits << (4 * (lane & 7)) : 0u;
-                    const uint32_t word = __reduce_or_sync(0xffffffffu, part);
-                    if (lane == 0) masks[rb * 4 + w] = word;
+                    for (int w = 0; w < 4; ++w) {
+                        const uint32_t part = (lane >> 3) == w ? ownbits << (4 * (lane & 7)) : 0u;
+                        const uint32_t word = __reduce_or_sync(0xffffffffu, part);
+                        if (lane == 0) masks[rb * 4 + w] = word;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(ROWS_FULL(rb));
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(ROWS_FULL(rb));
                 ++tile_ctr;
                 return true;
             }
@@ -428,133 +436,108 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
         };
         // one chunk into the next ring slot: kind 0 key chunk c of tile x, 1 / 2 q / dO chunk c of row t
         auto load = [&](const Tile& x, int kind, int c, int t) -> bool {
-            if (lane == 0) ok = WAIT(EMPTY(slot), sphase ^ 1, 102);
+            const int gs = ring0 + slot;  // the slot's index in shared memory
+            if (lane == 0) ok = WAIT(EMPTY(gs), sphase ^ 1, 102);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) return false;
-            const uint32_t dst = sbase + slot * kSlotBytes;
+            const uint32_t dst = sbase + gs * kSlotBytes;
             const int halves = c < 4 ? 2 : 1;
-            if (lane == 0) mbar_expect_tx(FULL(slot), halves * 128u * 128u);
+            if (lane == 0) mbar_expect_tx(FULL(gs), halves * 128u * 128u);
             __syncwarp();
             if (kind == 0 && x.contig) {
                 if (lane == 0) {
                     const CUtensorMap* map = c < 4 ? &prm.mapK128 : &prm.mapKr128;
                     for (int h = 0; h < halves; ++h)
-                        tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, x.run0, FULL(slot));
+                        tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, x.run0, FULL(gs));
                 }
             } else if (kind == 0) {
                 const CUtensorMap* map = c < 4 ? &prm.mapK : &prm.mapKr;
                 for (int h = 0; h < halves; ++h)
                     tma_gather4(dst + h * kHalf + lane * 512, map, c < 4 ? c * 128 + h * 64 : 0, x.my[0], x.my[1],
-                                x.my[2], x.my[3], FULL(slot));
+                                x.my[2], x.my[3], FULL(gs));
             } else if (lane == 0) {
                 const CUtensorMap* map = kind == 1 ? (c < 4 ? &prm.mapQ : &prm.mapQr) : &prm.mapO;
                 for (int h = 0; h < halves; ++h)
-                    tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, t * kN1, FULL(slot));
+                    tma_load_2d(dst + h * kHalf, map, c < 4 ? c * 128 + h * 64 : 0, t * kN1, FULL(gs));
             }
-            if (lane == 0) issued_mask |= 1u << slot;
-            if (++slot == ring_slots) { slot = 0; sphase ^= 1; }
+            if (lane == 0) issued_mask |= 1u << gs;
+            if (++slot == ring_n) { slot = 0; sphase ^= 1; }
             return true;
         };
-        auto sdp_load = [&](const Tile& x, int j) -> bool {
-            int kind, c;
-            sdp_item(j, kind, c);
-            return load(x, kind, c, x.t0 + (int)rank);
-        };
-        Tile cur, nxt;
-        bool have = next_tile(cur);
-        for (int j = 0; j < 14 && have && ok; ++j) ok = sdp_load(cur, j);  // the first tile's S / dP
-        const int gkind = rank ? 1 : 2;  // the key-side blocks' A operand: q (dK~) or dO (dV)
-        while (have && ok) {
-            for (int c = 0; c < 5 && ok; ++c) ok = load(cur, 0, c, 0);  // dQ~ blocks: the tile's key chunks
-            bool have_next = false;
-            if (ok) have_next = next_tile(nxt);
-            // the next tile of the same pair reads the same row chunks: rank 1's own q chunk of dK~
-            // block c is also the next S item's B, rank 0's own dO chunk of dV block c the next dP item's
-            const bool same = have_next && nxt.t0 == cur.t0;
-            for (int c = 0; c < 5 && ok; ++c) {
-                if (c < nkey) {
+        Tile cur;
+        if (srole) {
+            // every tile's S / dP items: S item c (K_c, q_c), then dP item c (c < 4: dO_c with K_c,
+            // which a ring of three or more slots keeps from the S item and a smaller one reloads)
+            const bool holdK = ring_n >= 3;
+            while (ok && next_tile(cur)) {
+                const int t = cur.t0 + (int)rank;
+                for (int c = 0; c < 5 && ok; ++c) {
+                    ok = load(cur, 0, c, 0);
+                    if (ok) ok = load(cur, 1, c, t);
+                    if (ok && c < 4 && !holdK) ok = load(cur, 0, c, 0);
+                    if (ok && c < 4) ok = load(cur, 2, c, t);
+                }
+            }
+        } else {
+            // every tile's gradient blocks: the five key chunks of the dQ~ blocks, then per key-side
+            // block the own row's chunk and the partner's (q for dK~, dO for dV)
+            const int gkind = rank ? 1 : 2;
+            while (ok && next_tile(cur)) {
+                for (int c = 0; c < 5 && ok; ++c) ok = load(cur, 0, c, 0);
+                for (int c = 0; c < nkey && ok; ++c) {
                     ok = load(cur, gkind, c, cur.t0 + (int)rank);
                     if (ok) ok = load(cur, gkind, c, cur.t0 + (int)peer);
                 }
-                if (ok && have_next) {
-                    const int t = nxt.t0 + (int)rank;
-                    ok = load(nxt, 0, c, 0);
-                    if (ok && !(rank == 1 && same)) ok = load(nxt, 1, c, t);
-                    if (ok && c < 4 && !(rank == 0 && same)) ok = load(nxt, 2, c, t);
-                }
             }
-            cur = nxt;
-            have = have_next;
         }
         // drain: every issued load must land before the CTA can exit
         if (lane == 0) {
-            for (int k = 0; k < ring_slots; ++k) {
-                const int s = (slot + k) % ring_slots;
+            for (int k = 0; k < ring_n; ++k) {
+                const int s = (slot + k) % ring_n;
                 const uint32_t ph = s < slot ? sphase : sphase ^ 1;
-                if (issued_mask & (1u << s)) {
+                if (issued_mask & (1u << (ring0 + s))) {
                     uint64_t t0 = globaltimer();
-                    while (!mbar_try(FULL(s), ph) && globaltimer() - t0 < 1000000000ull) {
+                    while (!mbar_try(FULL(ring0 + s), ph) && globaltimer() - t0 < 1000000000ull) {
                     }
                 }
             }
         }
-    } else if (warp == 13) {
-        // =================== MMA issuer ===================
+    } else if (warp == 13 || warp == 15) {
+        // =================== MMA issuers: 13 the gradient blocks, 15 the S / dP items ===================
+        const bool srole = warp == 15;
         const uint32_t ID_S = idesc(128, kN1, false, false, kF16);  // S^T, dP^T
         const uint32_t ID_G = idesc(128, 128, true, false, kF16);   // dV^T, dK~^T (N = keys)
         const uint32_t ID_Q = idesc(128, kN1, true, true, kF16);    // dQ~^T (N = heads)
         const uint32_t sX = sbase + kOffX, sY = sbase + kOffY, sR = sbase + kOffR;
         const uint32_t bOwn = rank ? sY : sX;  // B of the own row's half: dS (dK~) or P (dV)
+        const int ring0 = srole ? g_slots : 0, ring_n = srole ? s_slots : g_slots;
         int slot = 0;
         uint32_t sphase = 0;
         int tile_ctr = 0, blk_ctr = 0;
         uint32_t recv_done = 0;
         bool ok = true;
-        uint32_t slotK = 0;
+        auto gslot = [&]() { return ring0 + slot; };  // the current chunk's slot in shared memory
         auto wait_full = [&](int code) -> bool {
             bool r = true;
-            if (lane == 0) r = WAIT(FULL(slot), sphase, code);
+            if (lane == 0) r = WAIT(FULL(gslot()), sphase, code);
             r = __shfl_sync(0xffffffffu, r, 0);
             if (r) tc_fence_after();
             return r;
         };
         auto advance = [&]() {
-            if (++slot == ring_slots) { slot = 0; sphase ^= 1; }
+            if (++slot == ring_n) { slot = 0; sphase ^= 1; }
         };
-        auto sdp = [&](int j) -> bool {
-            int kind, c;
-            sdp_item(j, kind, c);
-            if (!wait_full(103)) return false;
-            const uint32_t sa = sbase + slot * kSlotBytes;
-            if (kind == 0) slotK = sa;
-            if (lane == 0 && kind != 0) {
-                const uint32_t dst = kind == 1 ? T_S : T_DP;
-                const int ksteps = c < 4 ? 8 : 4;
-                for (int ks = 0; ks < ksteps; ++ks) {
-                    const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-                    mma(dst, sdesc(slotK + off, 16, 1024), sdesc(sa + off, 16, 1024), ID_S,
-                        (c > 0 || ks > 0) ? 1u : 0u);
-                }
-                mma_commit(EMPTY(slot));
-                if (kind == 2 || c == 4) mma_commit(EMPTY((slotK - sbase) / kSlotBytes));
-                if (j == 13) mma_commit(SDP_FULL);
-            }
-            __syncwarp();
-            advance();
-            return true;
-        };
-        // K = 128 half of a key-side block: A = the chunk in the current slot, B = P or dS in bsrc;
-        // the slot is released after these MMAs unless another MMA still reads it
-        auto grad_half = [&](uint32_t dst, uint32_t bsrc, bool first, bool release, int code) -> bool {
+        // K = 128 half of a key-side block: A = the chunk in the current slot, B = P or dS in bsrc
+        auto grad_half = [&](uint32_t dst, uint32_t bsrc, bool first, int code) -> bool {
             if (!wait_full(code)) return false;
-            const uint32_t sa = sbase + slot * kSlotBytes;
+            const uint32_t sa = sbase + gslot() * kSlotBytes;
             if (lane == 0) {
                 for (int ks = 0; ks < kN1 / 16; ++ks) {
                     const uint64_t a = sdesc(sa + ks * 2048, kHalf, 1024);
                     const uint64_t bd = sdesc(bsrc + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
                     mma(dst, a, bd, ID_G, (!first || ks > 0) ? 1u : 0u);
                 }
-                if (release) mma_commit(EMPTY(slot));
+                mma_commit(EMPTY(gslot()));
             }
             __syncwarp();
             advance();
@@ -562,77 +545,109 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
         };
         int w_next = cid, tile_next = 0;
         int pw = -1, pnslots = 0;  // key slots of pair pw (read once per pair)
-        auto next_tile = [&](int& w_of) -> bool {
+        auto next_tile = [&]() -> bool {
             while (w_next < npairs) {
                 if (pw != w_next) {
                     pw = w_next;
                     pnslots = prm.nblk[prm.pairs[w_next]] * bs;
                 }
-                const int nslots = pnslots;
-                if (tile_next * kKeys >= nslots) {
+                if (tile_next * kKeys >= pnslots) {
                     w_next += ncl;
                     tile_next = 0;
                     continue;
                 }
                 ++tile_next;
-                w_of = w_next;
                 return true;
             }
             return false;
         };
-        // S^T (c-th q chunk in sB) or dP^T (dO chunk) item c of a tile against the key chunk in sK
-        auto sdp_mma = [&](uint32_t dst, uint32_t sK, uint32_t sB, int c) {
-            const int ksteps = c < 4 ? 8 : 4;
-            for (int ks = 0; ks < ksteps; ++ks) {
-                const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-                mma(dst, sdesc(sK + off, 16, 1024), sdesc(sB + off, 16, 1024), ID_S, (c > 0 || ks > 0) ? 1u : 0u);
+        if (srole) {
+            // ---- every tile's S / dP items: S item c (K_c, q_c) accumulates S^T, dP item c (K_c,
+            // dO_c) dP^T; a tile's items start once the softmax has read the previous tile's ----
+            while (ok && next_tile()) {
+                if (tile_ctr > 0) {
+                    if (lane == 0) ok = WAIT(PDS_FULL, (tile_ctr - 1) & 1, 119);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                const bool holdK = ring_n >= 3;  // the key chunk stays from S item c to dP item c
+                auto item = [&](uint32_t dst, int sK, int sB, int c) {
+                    const int ksteps = c < 4 ? 8 : 4;
+                    for (int ks = 0; ks < ksteps; ++ks) {
+                        const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                        mma(dst, sdesc(sbase + sK * kSlotBytes + off, 16, 1024),
+                            sdesc(sbase + sB * kSlotBytes + off, 16, 1024), ID_S, (c > 0 || ks > 0) ? 1u : 0u);
+                    }
+                };
+                for (int c = 0; c < 5 && ok; ++c) {
+                    if (!(ok = wait_full(103))) break;
+                    const int sK = gslot();
+                    advance();
+                    if (!(ok = wait_full(103))) break;
+                    const int sQ = gslot();
+                    advance();
+                    const bool keepK = holdK && c < 4;
+                    if (lane == 0) {
+                        item(T_S, sK, sQ, c);
+                        mma_commit(EMPTY(sQ));
+                        if (!keepK) mma_commit(EMPTY(sK));
+                        if (c == 4) mma_commit(SDP_FULL);
+                    }
+                    __syncwarp();
+                    if (c == 4) break;
+                    int sK2 = sK;
+                    if (!holdK) {
+                        if (!(ok = wait_full(103))) break;
+                        sK2 = gslot();
+                        advance();
+                    }
+                    if (!(ok = wait_full(103))) break;
+                    const int sO = gslot();
+                    advance();
+                    if (lane == 0) {
+                        item(T_DP, sK2, sO, c);
+                        mma_commit(EMPTY(sO));
+                        mma_commit(EMPTY(sK2));
+                    }
+                    __syncwarp();
+                }
+                ++tile_ctr;
             }
-        };
-        auto slot_addr = [&]() { return sbase + slot * kSlotBytes; };
-        int cur_w = 0;
-        bool have = next_tile(cur_w);
-        for (int j = 0; j < 14 && have && ok; ++j) ok = sdp(j);  // the first tile's S / dP
-        while (have && ok) {
-            if (lane == 0) ok = WAIT(PDS_FULL, tile_ctr & 1, 104);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            tc_fence_after();
-            // ---- dQ~ blocks 0..4 of the own row: A = key chunk [128 dims x 128 keys] (MN), B = dS (MN) ----
-            for (int c = 0; c < 5 && ok; ++c, ++blk_ctr) {
-                const int stg = blk_ctr & 1;
-                if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 105);
+        } else {
+            while (ok && next_tile()) {
+                if (lane == 0) ok = WAIT(PDS_FULL, tile_ctr & 1, 104);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after();
-                if (!(ok = wait_full(106))) break;
-                const uint32_t sa = slot_addr();
-                if (lane == 0) {
-                    for (int ks = 0; ks < kKeys / 16; ++ks)
-                        mma(T_STG(stg), sdesc(sa + ks * 2048, kHalf, 1024), sdesc(sY + ks * 2048, kHalf, 1024), ID_Q,
-                            ks > 0 ? 1u : 0u);
-                    mma_commit(EMPTY(slot));
-                    mma_commit(STG_FULL(stg));
-                }
-                __syncwarp();
-                advance();
-            }
-            if (!ok) break;
-            int nxt_w = 0;
-            const bool have_next = next_tile(nxt_w);
-            const bool same = have_next && nxt_w == cur_w;
-            // ---- key-side block c over both rows, then the next tile's S / dP item c ----
-            for (int c = 0; c < 5 && ok; ++c) {
-                int sOwn = -1;  // slot of the own row's chunk of block c
-                if (c < nkey) {
+                // ---- dQ~ blocks 0..4 of the own row: A = key chunk [128 dims x 128 keys] (MN), B = dS (MN) ----
+                for (int c = 0; c < 5 && ok; ++c, ++blk_ctr) {
                     const int stg = blk_ctr & 1;
                     if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 105);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     tc_fence_after();
-                    // the own chunk stays for the next tile's S (rank 1) / dP (rank 0) item when shared
-                    const bool keep = same && (rank == 1 || c < 4);
-                    sOwn = slot;
-                    if (!(ok = grad_half(T_STG(stg), bOwn, true, !keep, 107))) break;
+                    if (!(ok = wait_full(106))) break;
+                    const uint32_t sa = sbase + gslot() * kSlotBytes;
+                    if (lane == 0) {
+                        for (int ks = 0; ks < kKeys / 16; ++ks)
+                            mma(T_STG(stg), sdesc(sa + ks * 2048, kHalf, 1024), sdesc(sY + ks * 2048, kHalf, 1024),
+                                ID_Q, ks > 0 ? 1u : 0u);
+                        mma_commit(EMPTY(gslot()));
+                        mma_commit(STG_FULL(stg));
+                    }
+                    __syncwarp();
+                    advance();
+                }
+                if (!ok) break;
+                // ---- key-side block c over both rows: the own row's chunk, then the partner's ----
+                for (int c = 0; c < nkey && ok; ++c) {
+                    const int stg = blk_ctr & 1;
+                    if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 105);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (!(ok = grad_half(T_STG(stg), bOwn, true, 107))) break;
                     if (c == 0) {  // the partner's P / dS of this tile has landed in R
                         if (lane == 0)
                             ok = wait_cluster(RECV, recv_done & 1, abort_flag, prm.err, 108, prm.wait_ns);
@@ -642,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                         tc_fence_after();
                         if (!rank) fence_view_async_shared();  // R was written by the partner's stores
                     }
-                    if (!(ok = grad_half(T_STG(stg), sR, false, true, 109))) break;
+                    if (!(ok = grad_half(T_STG(stg), sR, false, 109))) break;
                     if (lane == 0) {
                         mma_commit(STG_FULL(stg));
                         if (c == nkey - 1) mma_commit(PDS_FREE);  // the last reads of P, dS and R
@@ -650,45 +665,12 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                     __syncwarp();
                     ++blk_ctr;
                 }
-                if (!have_next) continue;
-                if (!(ok = wait_full(103))) break;
-                const int sK = slot;
-                advance();
-                int sQ = sOwn;
-                if (!(rank == 1 && same)) {
-                    if (!(ok = wait_full(103))) break;
-                    sQ = slot;
-                    advance();
-                }
-                int sO = -1;
-                if (c < 4) {
-                    sO = sOwn;
-                    if (!(rank == 0 && same)) {
-                        if (!(ok = wait_full(103))) break;
-                        sO = slot;
-                        advance();
-                    }
-                }
-                if (lane == 0) {
-                    const uint32_t aK = sbase + sK * kSlotBytes;
-                    sdp_mma(T_S, aK, sbase + sQ * kSlotBytes, c);
-                    mma_commit(EMPTY(sQ));
-                    if (c < 4) {
-                        sdp_mma(T_DP, aK, sbase + sO * kSlotBytes, c);
-                        mma_commit(EMPTY(sO));
-                    }
-                    mma_commit(EMPTY(sK));
-                    if (c == 4) mma_commit(SDP_FULL);
-                }
-                __syncwarp();
+                ++tile_ctr;
             }
-            ++tile_ctr;
-            have = have_next;
-            cur_w = nxt_w;
         }
         if (lane == 0) {
-            *consumed = recv_done;
-            mma_commit(DONE);
+            if (!srole) *consumed = recv_done;
+            mma_commit(DONE);  // both MMA warps arrive: every MMA of the CTA has completed
             uint64_t t0 = globaltimer();
             while (!mbar_try(DONE, 0) && globaltimer() - t0 < 1000000000ull) {
             }
