@@ -126,7 +126,22 @@ struct PairParams {
 
 // Gradient blocks of a tile: k < 5 dQ~ block k of the own row (one key chunk); k >= 5 the rank's
 // key-side block k - 5 (rank 0 dV, rank 1 dK~) over both rows (the own row's chunk, then the partner's).
-__device__ __forceinline__ int num_blocks(uint32_t rank) { return rank ? 10 : 9; }
+// dQ~ block (dims 384-511) of rank 0's row that rank 1 computes: rank 1 holds that row's dS (it
+// receives it for dK~) and the tile's key chunk, so the block costs it no load, and rank 0, the
+// rank that waits at the exchange, gets one block less.  Rank 1 also keeps those dims' partial
+// sums, in rank 0's scratch (which rank 0 leaves unused there) and writes them to dQuery.
+constexpr int kDqMoved = 3;
+__device__ __forceinline__ int num_blocks(uint32_t rank) { return rank ? 11 : 8; }
+// Block bi of a tile in the flush order: dQ~ blocks first (rank 0: chunks 0, 1, 2, 4; rank 1:
+// chunks 0-3, then rank 0's chunk 3, then chunk 4), then the key-side blocks.
+__device__ __forceinline__ void block_of(uint32_t rank, int bi, bool& dq, bool& moved, int& b) {
+    const int ndq = rank ? 6 : 4;
+    dq = bi < ndq;
+    moved = rank && bi == kDqMoved + 1;
+    if (!dq) b = bi - ndq;
+    else if (rank) b = bi <= kDqMoved ? bi : (bi == kDqMoved + 1 ? kDqMoved : bi - 1);
+    else b = bi < kDqMoved ? bi : bi + 1;
+}
 // Two rings and two MMA warps per CTA.  The gradient ring (1 slot on rank 0, 2 on rank 1) carries,
 // per tile, the five key chunks of the dQ~ blocks, then each key-side block's own-row and partner
 // chunk, consumed in that order by the gradient MMA warp.  The S / dP ring (3 slots) carries each
@@ -185,8 +200,8 @@ __device__ __noinline__ bool wait_cluster(uint32_t bar, uint32_t parity, volatil
 enum { DQ_SINGLE = 0, DQ_FIRST = 1, DQ_MID = 2, DQ_LAST = 3 };
 template <typename T>
 __device__ __forceinline__ void flush_dq(const float (&v)[32], int mode, int cc, int t, int dim,
-                                         const PairParams& prm) {
-    float* sc = prm.dq_scratch + ((size_t)blockIdx.x * kN1 + cc * 32) * kDK + dim;
+                                         const PairParams& prm, int cta) {
+    float* sc = prm.dq_scratch + ((size_t)cta * kN1 + cc * 32) * kDK + dim;
     if (mode == DQ_FIRST) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) st_relaxed(sc + e * kDK, v[e]);
@@ -312,8 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
     const int npairs = *prm.npairs;
     const int bs = prm.bs;
     const float scale = prm.scale;
-    const int nblocks = num_blocks(rank);  // gradient blocks per tile: 5 dQ~ + the key-side ones
-    const int nkey = nblocks - 5;
+    const int nblocks = num_blocks(rank);  // gradient blocks per tile: the dQ~ and key-side ones
+    const int nkey = rank ? 5 : 4;
     // two rings: slots [0, g_slots) carry the gradient blocks' chunks, the next two slots the S / dP
     // items' chunks (rank 1's fifth slot is its P buffer, which it never uses)
     const int s_slots = rank ? kSRing1 : kSRing0;
@@ -483,7 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
             // block the own row's chunk and the partner's (q for dK~, dO for dV)
             const int gkind = rank ? 1 : 2;
             while (ok && next_tile(cur)) {
-                for (int c = 0; c < 5 && ok; ++c) ok = load(cur, 0, c, 0);
+                for (int c = 0; c < 5 && ok; ++c)
+                    if (rank || c != kDqMoved) ok = load(cur, 0, c, 0);
                 for (int c = 0; c < nkey && ok; ++c) {
                     ok = load(cur, gkind, c, cur.t0 + (int)rank);
                     if (ok) ok = load(cur, gkind, c, cur.t0 + (int)peer);
@@ -620,23 +636,41 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after();
-                // ---- dQ~ blocks 0..4 of the own row: A = key chunk [128 dims x 128 keys] (MN), B = dS (MN) ----
-                for (int c = 0; c < 5 && ok; ++c, ++blk_ctr) {
+                // ---- dQ~ blocks: A = key chunk [128 dims x 128 keys] (MN), B = dS (MN) of the own row;
+                // rank 1 also forms rank 0's block kDqMoved from the received dS, same key chunk ----
+                auto dq_block = [&](uint32_t bsrc, bool release) -> bool {
                     const int stg = blk_ctr & 1;
-                    if (lane == 0) ok = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 105);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
+                    bool r = true;
+                    if (lane == 0) r = WAIT(STG_EMPTY(stg), ((blk_ctr >> 1) & 1) ^ 1, 105);
+                    r = __shfl_sync(0xffffffffu, r, 0);
+                    if (!r) return false;
                     tc_fence_after();
-                    if (!(ok = wait_full(106))) break;
                     const uint32_t sa = sbase + gslot() * kSlotBytes;
                     if (lane == 0) {
                         for (int ks = 0; ks < kKeys / 16; ++ks)
-                            mma(T_STG(stg), sdesc(sa + ks * 2048, kHalf, 1024), sdesc(sY + ks * 2048, kHalf, 1024),
+                            mma(T_STG(stg), sdesc(sa + ks * 2048, kHalf, 1024), sdesc(bsrc + ks * 2048, kHalf, 1024),
                                 ID_Q, ks > 0 ? 1u : 0u);
-                        mma_commit(EMPTY(gslot()));
+                        if (release) mma_commit(EMPTY(gslot()));
                         mma_commit(STG_FULL(stg));
                     }
                     __syncwarp();
+                    ++blk_ctr;
+                    return true;
+                };
+                for (int c = 0; c < 5 && ok; ++c) {
+                    if (!rank && c == kDqMoved) continue;
+                    if (!(ok = wait_full(106))) break;
+                    const bool moved = rank && c == kDqMoved;
+                    if (!(ok = dq_block(sY, !moved))) break;
+                    if (moved) {  // rank 0's dS of this tile has landed in R
+                        if (lane == 0)
+                            ok = wait_cluster(RECV, recv_done & 1, abort_flag, prm.err, 108, prm.wait_ns);
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
+                        if (!ok) break;
+                        ++recv_done;
+                        tc_fence_after();
+                        if (!(ok = dq_block(sR, true))) break;
+                    }
                     advance();
                 }
                 if (!ok) break;
@@ -648,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                     if (!ok) break;
                     tc_fence_after();
                     if (!(ok = grad_half(T_STG(stg), bOwn, true, 107))) break;
-                    if (c == 0) {  // the partner's P / dS of this tile has landed in R
+                    if (c == 0 && !rank) {  // rank 1's P of this tile has landed in R (rank 1 waited above)
                         if (lane == 0)
                             ok = wait_cluster(RECV, recv_done & 1, abort_flag, prm.err, 108, prm.wait_ns);
                         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -809,7 +843,9 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                     ok = __all_sync(0xffffffffu, WAIT(STG_FULL(stg), (blk_ctr >> 1) & 1, 114));
                     if (!ok) break;
                     tc_fence_after();
-                    const int b = bi < 5 ? bi : bi - 5;
+                    bool dq, moved;
+                    int b;
+                    block_of(rank, bi, dq, moved, b);
                     const bool active = b < 4 || q < 2;  // rope blocks: 64 valid dims
                     const int dim = (b < 4 ? b * 128 : kD) + q * 32 + lane;
                     if (active) {
@@ -817,7 +853,9 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_bwd_pair_kernel(const __grid_
                             float v[32];
                             tmem_ld32(T_STG(stg) + lane_base + cc * 32, v);
                             tmem_wait_ld();
-                            if (bi < 5) flush_dq<T>(v, dqmode, cc, t, dim, prm);
+                            if (dq)  // the moved block: rank 0's row, in rank 0's scratch
+                                flush_dq<T>(v, dqmode, cc, moved ? t0 : t, dim, prm,
+                                            (int)blockIdx.x - (moved ? (int)rank : 0));
                             else flush_keys<DET>(v, rank ? (size_t)dim : (size_t)(kDK + dim), rid + cc * 32, prm,
                                                  fmul);
                         }

@@ -28,11 +28,16 @@ def two_ring_ops(rank, ntiles, hold_k=False):
     of two chunks, or with hold_k (an S ring of 3+ slots keeps K_c from S item c to dP item c) one
     op per c of three chunks (c < 4) or two (c = 4); `last` marks the tile's last op."""
     nkey = 5 if rank else 4
-    grad = []
+    grad = []  # (kind, tile, block, chunks needed present, chunks released)
     for i in range(ntiles):
-        grad += [("Gq", i, c, 1) for c in range(5)]
+        if rank:  # own dQ~ 0-3, rank 0's dQ~ 3 (same key chunk, needs rank 0's dS), own dQ~ 4
+            grad += [("Gq", i, c, 1, 1) for c in range(3)]
+            grad += [("Gq", i, 3, 1, 0), ("Gm", i, 4, 1, 1), ("Gq", i, 5, 1, 1)]
+        else:     # dQ~ 0, 1, 2, 4
+            grad += [("Gq", i, c, 1, 1) for c in range(4)]
+        nq = 6 if rank else 4
         for c in range(nkey):
-            grad += [("G", i, 5 + c, 1), ("H", i, 5 + c, 1)]
+            grad += [("G", i, nq + c, 1, 1), ("H", i, nq + c, 1, 1)]
     if hold_k:
         sdp = [(i, c == 4, 3 if c < 4 else 2) for i in range(ntiles) for c in range(5)]
     else:
@@ -50,8 +55,9 @@ def simulate_two_rings(ntiles, gslots=(2, 3), sslots=(2, 2)):
         c.rank = rank
         c.gs, c.ss = gslots[rank], sslots[rank]
         c.grad, c.sdp = two_ring_ops(rank, ntiles, hold_k=c.ss >= 3)
-        c.nb = 9 if rank == 0 else 10
-        c.gl = c.gi = 0  # gradient chunks loaded / consumed (each op consumes one chunk, released at use)
+        c.nb = 8 if rank == 0 else 11
+        c.gl = c.gi = 0  # gradient chunks loaded / ops issued
+        c.gused = 0      # gradient chunks released
         c.sl = c.si = 0  # S chunks loaded / S ops issued
         c.sused = 0      # S chunks released
         c.flushed = c.blocks = 0
@@ -62,27 +68,31 @@ def simulate_two_rings(ntiles, gslots=(2, 3), sslots=(2, 2)):
 
     def step(c, peer):
         progress = False
-        if c.gl < len(c.grad) and c.gl - c.gi < c.gs:  # gradient producer
+        if c.gl < sum(op[4] for op in c.grad) and c.gl - c.gused < c.gs:  # gradient producer
             c.gl += 1
             progress = True
         if c.sl < sum(n for _, _, n in c.sdp) and c.sl - c.sused < c.ss:  # S producer
             c.sl += 1
             progress = True
         if c.gi < len(c.grad):  # gradient MMA warp
-            kind, i, b, _ = c.grad[c.gi]
-            ready = c.gl > c.gi
-            if kind in ("G", "Gq"):
+            kind, i, b, need, rel = c.grad[c.gi]
+            ready = c.gl >= c.gused + need
+            if kind in ("G", "Gq", "Gm"):
                 if b == 0 and c.written < i:
                     ready = False
                 if c.blocks >= 2 and c.flushed < c.blocks - 1:
                     ready = False
-            if kind == "H" and b == 5 and peer.written < i:
+            nq = 6 if c.rank else 4
+            if kind == "Gm" and peer.written < i:  # rank 0's dS of tile i
+                ready = False
+            if kind == "H" and b == nq and c.rank == 0 and peer.written < i:  # rank 1's P of tile i
                 ready = False
             if ready:
-                if kind in ("G", "Gq"):
+                if kind in ("G", "Gq", "Gm"):
                     c.blocks += 1
                 if kind == "H" and b == c.nb - 1:
                     c.grad_done = i
+                c.gused += rel
                 c.gi += 1
                 progress = True
         if c.si < len(c.sdp):  # S MMA warp: tile i's items after the softmax read tile i - 1's
