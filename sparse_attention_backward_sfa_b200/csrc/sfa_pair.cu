@@ -29,13 +29,15 @@
 //    -> shared::cluster that completes on rank 1's mbarrier, and rank 1 stores its
 //    P straight into rank 0's receive buffer (distributed shared memory stores,
 //    a proxy fence, one remote arrive): rank 1 keeps no P of its own, and that
-//    buffer is a fifth slot of its operand ring.  Each rank also loads the partner
-//    row's dO (rank 0) or q (rank 1) chunks.
-//    dQ~ stays per row: each rank forms dQ~^T = K~^T.dS^T of its own row and
-//    accumulates it across the row's tiles in its per-CTA fp32 scratch.
+//    buffer is a fifth operand slot.  Each rank also loads the partner row's dO
+//    (rank 0) or q (rank 1) chunks.
+//    dQ~ is formed per row, dQ~^T = K~^T.dS^T, and accumulated across the row's
+//    tiles in a per-CTA fp32 scratch: rank 0 its row's dims 0-383 and the rope,
+//    rank 1 its whole row and rank 0's dims 384-511 (from the dS it receives).
 //  * Shared memory: 32 KB operand slots (4 on rank 0, 5 on rank 1) split into the
-//    two rings, P (X, rank 0 only), dS (Y) and the received tile (R), 32 KB each, row ids and masks, constants, barriers: the
-//    same offsets in both CTAs, so an offset names the same object in the peer.
+//    two rings, P (X, rank 0 only), dS (Y) and the received tile (R), 32 KB each,
+//    row ids and masks, constants, barriers: the same offsets in both CTAs, so an
+//    offset names the same object in the peer.
 //  * Hand-over of the single received buffer R: a rank grants its partner the
 //    next tile's copy (remote arrive on the partner's PEER_FREE) once its own
 //    gradient MMAs of the previous tile completed (they read R); the sender
@@ -46,9 +48,9 @@
 //  * Warp roles per CTA: 0-3 softmax/dS, 4-11 flush, 12 / 14 TMA producers and
 //    13 / 15 MMA issuers of the gradient blocks / the S^T and dP^T items, each
 //    pair with its own ring, so the next tile's S^T / dP^T are formed while this
-//    tile's gradient blocks run.  Every wait is bounded; on timeout the CTA records an
-//    error word and leaves, after waiting (bounded) for copies still addressed to
-//    it and meeting its partner at the final cluster barrier.
+//    tile's gradient blocks run.  Every wait is bounded; on timeout the CTA
+//    records an error word and leaves, after waiting (bounded) for copies still
+//    addressed to it and meeting its partner at the final cluster barrier.
 #include <cuda.h>
 
 #include <cstring>
