@@ -44,6 +44,7 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 # committed ncu summaries: (summary file, kernel sources whose hash it records)
 PROFILE_SUMMARIES = {
     4: ("sfa_bwd_pair_kernel_workload4.md", ("sfa_pair.cu", "tc_common.cuh")),
+    3: ("sfa_bwd_fused_kernel_workload3.md", ("sfa_fused.cu", "tc_common.cuh")),
     2: ("fa_bwd_fused_kernel_workload2.md", ("fa_fused.cu", "tc_common.cuh")),
     "fwd4": ("sfa_fwd_fused_kernel_workload4.md", ("sfa_fwd_fused.cu", "tc_common.cuh")),
     "lig": ("lig_fused_kernel_indexer.md", ("lig_fused.cu", "tc_common.cuh")),
@@ -835,8 +836,7 @@ def main():
                          "paired_work_fraction": r["paired"],
                          "kernel_ms": kern,
                          "kernel_ms_median": statistics.median(r["kern_ms"]),
-                         "traffic": recorded_traffic(4) if args.workload == 4 and not args.seqs and not sharded
-                         else None},
+                         "traffic": recorded_traffic(args.workload) if not args.seqs and not sharded else None},
             "cpu_baseline": cpu,
             "e2e": r["e2e"],
             # compact, rowsum, order, block sort (block-sparse lists of topk <= 4096), expand, [N1 = 128:
