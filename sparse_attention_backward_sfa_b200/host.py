@@ -46,7 +46,7 @@ class HostPipeline:
 def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, softmax_max, softmax_sum, query_rope,
                   key_rope, *, scale: float, sparse_block_size: int, layout: str, sparse_mode: int,
                   deterministic: bool = False, actual_seq_lengths_q=None, actual_seq_lengths_kv=None,
-                  outputs=None, chunks: int = 8, pipeline: Optional[HostPipeline] = None, device=None):
+                  outputs=None, chunks: int = 16, pipeline: Optional[HostPipeline] = None, device=None):
     """sfa_grad on pinned host tensors; returns host (dQuery, dKey, dValue, dQueryRope, dKeyRope).
 
     value == key is the only layout the pages support (`value_is_key` must be True).  `outputs`
