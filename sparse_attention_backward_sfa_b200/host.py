@@ -1,9 +1,9 @@
 """Sparse attention backward for host-resident (pinned) tensors, with the copies
 overlapped with the computation.
 
-The query rows are processed in chunks (sfa_grad_rows): while chunk c runs on
-the compute stream, chunk c+1's query-side inputs (query, queryRope, dOut, out,
-softmax statistics) are copied host->device on a copy stream and chunk c-1's
+The query rows are processed in chunks (sfa_grad_rows), last rows first: while one chunk runs
+on the compute stream, the next chunk's query-side inputs (query, queryRope, dOut, out,
+softmax statistics) are copied host->device on a copy stream and the previous chunk's
 dQuery / dQueryRope rows are copied device->host on a third stream.  The
 key-side inputs and the indices go first (in deterministic mode followed by all
 of dOut, whose largest magnitude sets the fixed-point grid before the first
@@ -99,6 +99,9 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
     # chunk boundaries on even rows: rows (2m, 2m + 1) that share their blocks stay one pair, as in
     # the single call (deterministic results are then bit-identical to it)
     bounds = [min(T1, 2 * ((T1 * c) // (2 * chunks))) for c in range(chunks)] + [T1]
+    # last rows first: under a causal mask they select the most keys, so the call ends on its
+    # lightest chunk (the compute left after the last host->device copy is the smallest)
+    order = range(chunks - 1, -1, -1)
     # the copy stream starts after whatever the caller queued before this call
     pl.h2d.wait_stream(comp)
     with torch.cuda.stream(pl.h2d):
@@ -115,7 +118,7 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
             dmax = pl._like("dmax", torch.empty(1, dtype=torch.float32))
             dmax.zero_()
             ops.dout_absmax(dq_["do"], dq_["q"], ds_["k"], dq_["qr"], ds_["idx"], into=dmax, stream=pl.h2d, **kw)
-        for c in range(chunks):
+        for c in order:
             a, b = bounds[c], bounds[c + 1]
             for n, x in qside.items():
                 if n == "do" and deterministic:
@@ -127,9 +130,9 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
     comp.wait_event(ev_shared)
     acc.zero_()
     pl.d2h.wait_stream(comp)
-    for c in range(chunks):
+    for i, c in enumerate(order):
         a, b = bounds[c], bounds[c + 1]
-        comp.wait_event(ev_in[c])
+        comp.wait_event(ev_in[i])
         ops.sfa_grad_rows(dq_["q"], ds_["k"], ds_["k"], ds_["idx"], dq_["do"], dq_["o"], dq_["mx"], dq_["sm"],
                           dq_["qr"], ds_["kr"], row_begin=a, row_end=b, dkv_accum=acc, scale=scale,
                           sparse_block_size=sparse_block_size, sparse_mode=sparse_mode, deterministic=deterministic,
