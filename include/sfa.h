@@ -165,6 +165,9 @@ sfa_status sfa_dkv_accum_size(const sfa_shape *shape, int32_t deterministic, siz
  * flattened [T1] row index (BSND: b * S1 + s; TND: the token index).
  *   - Same inputs, workspace and validation as sfa_grad; 0 <= row_begin <=
  *     row_end <= T1, else SFA_ERR_INVALID before any device work.
+ *   - Of sparse_indices, query, query_rope, d_out, out, softmax_max and
+ *     softmax_sum only the range's rows are read (a pipeline may copy the other
+ *     rows while this call runs); key / key_rope are read whole.
  *   - d_query / d_query_rope: the rows in the range are written (zero for rows
  *     with no selected key); rows outside the range are not touched.
  *   - dkv_accum (caller-owned, 256-byte aligned, sfa_dkv_accum_size bytes): the

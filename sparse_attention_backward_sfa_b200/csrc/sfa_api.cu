@@ -234,7 +234,7 @@ sfa_status grad_impl(const void* query, const void* key, const void* value, cons
         SFA_CUDA(cudaMemsetAsync(a.dkv_acc, 0, (size_t)z.T2 * kAccW * (det ? 8 : 4), s), "zero dK/dV accumulator");
     float* rowsum_dmax = own_acc && det ? own_dmax : nullptr;  // max|dO| taken by the rowsum pass
     SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, (int32_t*)a.blocks, (int32_t*)a.nblk,
-                            (int32_t*)a.nrows, s), "index compaction");
+                            (int32_t*)a.nrows, row_begin, row_end, s), "index compaction");
     const bool fused = fused_shape && value == key;
     if (fused) {
         SFA_CUDA(launch_rowsum(shape->dtype, d_out, out, row_begin, row_end, shape->N1, (float*)a.rowsum, s,
@@ -243,7 +243,8 @@ sfa_status grad_impl(const void* query, const void* key, const void* value, cons
         // block-sparse lists sorted: consecutive selected blocks become contiguous key tiles
         if (a.bs > 1 && a.topk <= kSortMaxTopk)
             SFA_CUDA(launch_sort_blocks((int32_t*)a.blocks, a.nblk, a.topk, row_begin, row_end, s), "block sort");
-        SFA_CUDA(launch_expand(a.blocks, a.nblk, a.sd, a.topk, a.bs, a.mode, a.rowcap, (int32_t*)a.rowlist, s),
+        SFA_CUDA(launch_expand(a.blocks, a.nblk, a.sd, a.topk, a.bs, a.mode, a.rowcap, (int32_t*)a.rowlist, row_begin,
+                               row_end, s),
                  "key row expansion");
         if (shape->N1 == 128) {
             // adjacent rows with identical block lists go to the paired kernel (two CTAs of a
@@ -404,7 +405,8 @@ sfa_status sfa_fwd(const void* query, const void* key, const void* value, const 
     SFA_CUDA(cudaMemsetAsync(w + ws.ctrl, 0, 256, s), "zero control word");
     a.blocks = blocks; a.nblk = nblk;
     a.out = out; a.smax = softmax_max; a.ssum = softmax_sum;
-    SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, blocks, nblk, nrows, s), "index compaction");
+    SFA_CUDA(launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, blocks, nblk, nrows, 0, z.T1, s),
+             "index compaction");
     if (ws.rowlist && value == key) {
         // tensor-core path: expanded key-row lists, longest rows first
         FwdFusedArgs f;
@@ -422,7 +424,7 @@ sfa_status sfa_fwd(const void* query, const void* key, const void* value, const 
             SFA_CUDA(launch_expand_blocks(blocks, nblk, a.sd, a.topk, a.bs, a.mode, f.rowcap, (int32_t*)f.rowlist,
                                           (int32_t*)f.nrows, s), "key row expansion");
         } else {
-            SFA_CUDA(launch_expand(blocks, nblk, a.sd, a.topk, a.bs, a.mode, f.rowcap, (int32_t*)f.rowlist, s),
+            SFA_CUDA(launch_expand(blocks, nblk, a.sd, a.topk, a.bs, a.mode, f.rowcap, (int32_t*)f.rowlist, 0, z.T1, s),
                      "key row expansion");
         }
         KernelEvents ev(s);
@@ -450,7 +452,7 @@ sfa_status sfa_compact_indices(const int32_t* sparse_indices, const int32_t* act
         return fail(SFA_ERR_NULLPTR, "TND needs actual_seq_lengths_q and actual_seq_lengths_kv");
     SeqDesc sd = seq_desc(shape, z, actual_seq_lengths_q, actual_seq_lengths_kv);
     SFA_CUDA(launch_compact(sparse_indices, sd, shape->topk, (int)sparse_block_size, (int)sparse_mode, blocks_out,
-                            nblocks_out, nrows_out, (cudaStream_t)stream), "index compaction");
+                            nblocks_out, nrows_out, 0, z.T1, (cudaStream_t)stream), "index compaction");
     return SFA_OK;
 }
 
@@ -473,13 +475,13 @@ sfa_status sfa_key_rows(const int32_t* sparse_indices, const int32_t* actual_seq
     const int bs = (int)sparse_block_size;
     const int64_t cap = shape->topk * sparse_block_size;
     SFA_CUDA(launch_compact(sparse_indices, sd, shape->topk, bs, (int)sparse_mode, blocks_out, nblocks_out, count_out,
-                            s), "index compaction");
+                            0, z.T1, s), "index compaction");
     if (sorted) SFA_CUDA(launch_sort_blocks(blocks_out, nblocks_out, shape->topk, 0, z.T1, s), "block sort");
     if (block_aligned)
         SFA_CUDA(launch_expand_blocks(blocks_out, nblocks_out, sd, shape->topk, bs, (int)sparse_mode, cap, rows_out,
                                       count_out, s), "key row expansion");
     else
-        SFA_CUDA(launch_expand(blocks_out, nblocks_out, sd, shape->topk, bs, (int)sparse_mode, cap, rows_out, s),
+        SFA_CUDA(launch_expand(blocks_out, nblocks_out, sd, shape->topk, bs, (int)sparse_mode, cap, rows_out, 0, z.T1, s),
                  "key row expansion");
     return SFA_OK;
 }

@@ -222,8 +222,10 @@ inline FwdWs fwd_ws_layout(int64_t T1, int64_t N1, int64_t topk, int64_t bs) {
 // ---------------------------------------------------------------------------
 // Launchers (defined in the .cu files; all return cudaGetLastError())
 // ---------------------------------------------------------------------------
+// index compaction of query rows [row_begin, row_end) (only those rows' indices are read and
+// only their entries of blocks / nblk / nrows written)
 cudaError_t launch_compact(const int32_t* idx, const SeqDesc& sd, int64_t topk, int bs, int mode, int32_t* blocks,
-                           int32_t* nblk, int32_t* nrows, cudaStream_t st);
+                           int32_t* nblk, int32_t* nrows, int64_t row_begin, int64_t row_end, cudaStream_t st);
 // rowsum(dO o O) of query rows [row_begin, row_end) (rows outside are not written)
 // (when `absmax` is non-null, max|dO| over the range is max-merged into it too)
 cudaError_t launch_rowsum(int dtype, const void* dout, const void* out, int64_t row_begin, int64_t row_end, int64_t N1,
@@ -236,8 +238,9 @@ cudaError_t launch_order(const int32_t* nrows, int64_t row_begin, int64_t row_en
 constexpr int64_t kSortMaxTopk = 4096;
 cudaError_t launch_sort_blocks(int32_t* blocks, const int32_t* nblk, int64_t topk, int64_t row_begin, int64_t row_end,
                                cudaStream_t st);
+// key-row lists of query rows [row_begin, row_end)
 cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs, int mode,
-                          int64_t cap, int32_t* rowlist, cudaStream_t st);
+                          int64_t cap, int32_t* rowlist, int64_t row_begin, int64_t row_end, cudaStream_t st);
 // block-aligned key-row lists for sparse_block_size % 16 == 0 (invalid slots: bit 31 set)
 cudaError_t launch_expand_blocks(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs,
                                  int mode, int64_t cap, int32_t* rowlist, int32_t* nslots, cudaStream_t st);

@@ -126,7 +126,7 @@ sfa_status sfa_grad_noalloc(const void* query, const void* key, const void* valu
     if ((e = cudaMemsetAsync(a.dkv_acc, 0, (size_t)T2 * kAccW * (det ? 8 : 4), s)) != cudaSuccess)
         return nfail(SFA_ERR_CUDA, "clear scratch: %s", cudaGetErrorString(e));
     if ((e = launch_compact(sparse_indices, a.sd, a.topk, a.bs, a.mode, (int32_t*)a.blocks, (int32_t*)a.nblk,
-                            (int32_t*)a.nrows, s)) != cudaSuccess)
+                            (int32_t*)a.nrows, 0, T1, s)) != cudaSuccess)
         return nfail(SFA_ERR_CUDA, "index compaction: %s", cudaGetErrorString(e));
     if (det && (e = launch_absmax(shape->dtype, d_out, T1 * shape->N1 * kD, dmax, s)) != cudaSuccess)
         return nfail(SFA_ERR_CUDA, "max|dOut|: %s", cudaGetErrorString(e));

@@ -8,13 +8,14 @@
 
 namespace sfa {
 
-// One warp per query row: keep the valid block indices in their original order.
+// One warp per query row of [row_begin, row_end): keep the valid block indices in their original
+// order (no other row's indices are read).
 __global__ void compact_kernel(const int32_t* __restrict__ idx, SeqDesc sd, int64_t topk, int bs, int mode,
                                int32_t* __restrict__ blocks, int32_t* __restrict__ nblk,
-                               int32_t* __restrict__ nrows) {
+                               int32_t* __restrict__ nrows, int64_t row_begin, int64_t row_end) {
     const int lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= sd.T1) return;
+    const int64_t t = row_begin + (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= row_end) return;
     TokInfo ti = tok_info(sd, t);
     int count = 0, rows = 0;
     if (ti.valid) {
@@ -45,10 +46,12 @@ __global__ void compact_kernel(const int32_t* __restrict__ idx, SeqDesc sd, int6
 }
 
 cudaError_t launch_compact(const int32_t* idx, const SeqDesc& sd, int64_t topk, int bs, int mode, int32_t* blocks,
-                           int32_t* nblk, int32_t* nrows, cudaStream_t st) {
+                           int32_t* nblk, int32_t* nrows, int64_t row_begin, int64_t row_end, cudaStream_t st) {
     const int warps = 8;
-    int64_t grid = (sd.T1 + warps - 1) / warps;
-    if (grid > 0) compact_kernel<<<(unsigned)grid, warps * 32, 0, st>>>(idx, sd, topk, bs, mode, blocks, nblk, nrows);
+    int64_t grid = (row_end - row_begin + warps - 1) / warps;
+    if (grid > 0)
+        compact_kernel<<<(unsigned)grid, warps * 32, 0, st>>>(idx, sd, topk, bs, mode, blocks, nblk, nrows, row_begin,
+                                                              row_end);
     return cudaGetLastError();
 }
 
@@ -178,10 +181,11 @@ cudaError_t launch_order(const int32_t* nrows, int64_t row_begin, int64_t row_en
 // Expand each query row's compacted block list into its gathered key rows
 // (global row ids, in index order), one warp per query row.
 __global__ void expand_kernel(const int32_t* __restrict__ blocks, const int32_t* __restrict__ nblk, SeqDesc sd,
-                              int64_t topk, int bs, int mode, int64_t cap, int32_t* __restrict__ rowlist) {
+                              int64_t topk, int bs, int mode, int64_t cap, int32_t* __restrict__ rowlist,
+                              int64_t row_begin, int64_t row_end) {
     const int lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= sd.T1) return;
+    const int64_t t = row_begin + (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= row_end) return;
     const TokInfo ti = tok_info(sd, t);
     const int nb = nblk[t];
     int32_t* dst = rowlist + t * cap;
@@ -282,10 +286,12 @@ cudaError_t launch_sort_blocks(int32_t* blocks, const int32_t* nblk, int64_t top
 }
 
 cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblk, const SeqDesc& sd, int64_t topk, int bs, int mode,
-                          int64_t cap, int32_t* rowlist, cudaStream_t st) {
+                          int64_t cap, int32_t* rowlist, int64_t row_begin, int64_t row_end, cudaStream_t st) {
     const int warps = 8;
-    int64_t grid = (sd.T1 + warps - 1) / warps;
-    if (grid > 0) expand_kernel<<<(unsigned)grid, warps * 32, 0, st>>>(blocks, nblk, sd, topk, bs, mode, cap, rowlist);
+    int64_t grid = (row_end - row_begin + warps - 1) / warps;
+    if (grid > 0)
+        expand_kernel<<<(unsigned)grid, warps * 32, 0, st>>>(blocks, nblk, sd, topk, bs, mode, cap, rowlist, row_begin,
+                                                             row_end);
     return cudaGetLastError();
 }
 

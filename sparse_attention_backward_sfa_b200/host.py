@@ -3,9 +3,9 @@ overlapped with the computation.
 
 The query rows are processed in chunks (sfa_grad_rows), last rows first: while one chunk runs
 on the compute stream, the next chunk's query-side inputs (query, queryRope, dOut, out,
-softmax statistics) are copied host->device on a copy stream and the previous chunk's
-dQuery / dQueryRope rows are copied device->host on a third stream.  The
-key-side inputs and the indices go first (in deterministic mode followed by all
+softmax statistics, sparse indices) are copied host->device on a copy stream and the previous
+chunk's dQuery / dQueryRope rows are copied device->host on a third stream.  The
+key-side inputs go first (in deterministic mode followed by all
 of dOut, whose largest magnitude sets the fixed-point grid before the first
 chunk runs); the key-side gradients are cast from the accumulator and copied
 back at the end.  PCIe is full duplex, so a step
@@ -63,8 +63,10 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
     T1 = 1
     for d in lead:
         T1 *= d
-    qside = {"q": query, "qr": query_rope, "do": d_out, "o": out, "mx": softmax_max, "sm": softmax_sum}
-    shared = {"k": key, "kr": key_rope, "idx": sparse_indices}
+    # a row range reads only its own rows of these (the indices included), so they go over per chunk
+    qside = {"q": query, "qr": query_rope, "do": d_out, "o": out, "mx": softmax_max, "sm": softmax_sum,
+             "idx": sparse_indices}
+    shared = {"k": key, "kr": key_rope}
     if actual_seq_lengths_q is not None:
         shared["sq"] = actual_seq_lengths_q
     if actual_seq_lengths_kv is not None and actual_seq_lengths_kv is not actual_seq_lengths_q:
@@ -82,10 +84,10 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
     kw = dict(layout=layout, actual_seq_lengths_q=sq)
     acc = pl.buf.get("acc")
     if acc is None or acc.dtype != (torch.int64 if deterministic else torch.float32):
-        acc = ops.sfa_dkv_accumulator(dq_["q"], ds_["k"], dq_["qr"], ds_["idx"], deterministic=deterministic, **kw)
+        acc = ops.sfa_dkv_accumulator(dq_["q"], ds_["k"], dq_["qr"], dq_["idx"], deterministic=deterministic, **kw)
         pl.buf["acc"] = acc
     ws = pl.buf.get("ws")
-    shape = ops.sfa_shape(dq_["q"], ds_["k"], dq_["qr"], ds_["idx"], layout, sq)
+    shape = ops.sfa_shape(dq_["q"], ds_["k"], dq_["qr"], dq_["idx"], layout, sq)
     need = ops.sfa_grad_workspace_size(shape, sparse_block_size, sparse_mode, deterministic)
     if ws is None or ws.numel() < need:
         ws = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -117,7 +119,7 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
             dq_["do"].copy_(d_out, non_blocking=True)
             dmax = pl._like("dmax", torch.empty(1, dtype=torch.float32))
             dmax.zero_()
-            ops.dout_absmax(dq_["do"], dq_["q"], ds_["k"], dq_["qr"], ds_["idx"], into=dmax, stream=pl.h2d, **kw)
+            ops.dout_absmax(dq_["do"], dq_["q"], ds_["k"], dq_["qr"], dq_["idx"], into=dmax, stream=pl.h2d, **kw)
         for c in order:
             a, b = bounds[c], bounds[c + 1]
             for n, x in qside.items():
@@ -133,7 +135,7 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
     for i, c in enumerate(order):
         a, b = bounds[c], bounds[c + 1]
         comp.wait_event(ev_in[i])
-        ops.sfa_grad_rows(dq_["q"], ds_["k"], ds_["k"], ds_["idx"], dq_["do"], dq_["o"], dq_["mx"], dq_["sm"],
+        ops.sfa_grad_rows(dq_["q"], ds_["k"], ds_["k"], dq_["idx"], dq_["do"], dq_["o"], dq_["mx"], dq_["sm"],
                           dq_["qr"], ds_["kr"], row_begin=a, row_end=b, dkv_accum=acc, scale=scale,
                           sparse_block_size=sparse_block_size, sparse_mode=sparse_mode, deterministic=deterministic,
                           dout_absmax=dmax, actual_seq_lengths_kv=skv, workspace=ws, d_query=g_dq,
@@ -145,7 +147,7 @@ def sfa_grad_host(query, key, value_is_key: bool, sparse_indices, d_out, out, so
         with torch.cuda.stream(pl.d2h):
             _rows(h_dq, T1, a, b).copy_(_rows(g_dq, T1, a, b), non_blocking=True)
             _rows(h_dqr, T1, a, b).copy_(_rows(g_dqr, T1, a, b), non_blocking=True)
-    ops.sfa_dkv_finalize(acc, dq_["q"], ds_["k"], dq_["qr"], ds_["idx"], deterministic=deterministic,
+    ops.sfa_dkv_finalize(acc, dq_["q"], ds_["k"], dq_["qr"], dq_["idx"], deterministic=deterministic,
                          dout_absmax=dmax, scale=scale, outputs=(g_dk, g_dv, g_dkr), stream=comp, **kw)
     pl.d2h.wait_stream(comp)
     with torch.cuda.stream(pl.d2h):

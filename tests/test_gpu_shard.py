@@ -109,6 +109,50 @@ def test_rows_outside_range_untouched_and_range_checked():
                         row_end=p.T1 + 1, dkv_accum=acc, d_query=dq, d_query_rope=dqr, **kw)
 
 
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_rows_range_reads_only_its_rows(case):
+    """A row range reads only its own rows of the indices and of the query-side inputs (the host
+    pipeline copies them chunk by chunk): with every other row poisoned (NaN inputs, scrambled
+    indices) the range's dQuery rows and key-side sums are bit-identical to the clean call's."""
+    import sparse_attention_backward_sfa_b200 as S
+    p = tiny_problem(319, D=512, Dr=64, **CASES[case])
+    dp = DevProblem(p)
+    prepare_oracle_forward(p, dp)
+    kw = dp.kw()
+    T1 = p.T1
+    a, b = 2 * (T1 // 4), min(T1, 2 * (T1 // 4) + 4)
+
+    def run(q, qr, do, out, smax, ssum, idx):
+        acc = S.sfa_dkv_accumulator(q, dp.k, qr, idx, layout=kw["layout"], deterministic=True,
+                                    actual_seq_lengths_q=dp.sq)
+        dmax = torch.zeros(1, dtype=torch.float32, device=q.device)
+        S.dout_absmax(do, q, dp.k, qr, idx, layout=kw["layout"], row_begin=a, row_end=b,
+                      actual_seq_lengths_q=dp.sq, into=dmax)
+        dq, dqr = torch.zeros_like(q), torch.zeros_like(qr)
+        S.sfa_grad_rows(q, dp.k, dp.v, idx, do, out, smax, ssum, qr, dp.kr, row_begin=a, row_end=b, dkv_accum=acc,
+                        deterministic=True, dout_absmax=dmax, d_query=dq, d_query_rope=dqr, **kw)
+        torch.cuda.synchronize()
+        return dq.reshape(T1, -1)[a:b], dqr.reshape(T1, -1)[a:b], acc
+
+    clean = run(dp.q, dp.qr, dp.do, dp.out, dp.smax, dp.ssum, dp.idx)
+    g = torch.Generator(device="cpu").manual_seed(5)
+
+    def poison(x):
+        y = x.clone()
+        flat = y.reshape(T1, -1)
+        keep = flat[a:b].clone()
+        if y.dtype == torch.int32:
+            flat.copy_(torch.randint(-1, 1 << 20, flat.shape, generator=g, dtype=torch.int32).to(y.device))
+        else:
+            flat.fill_(float("nan"))
+        flat[a:b] = keep
+        return y
+
+    got = run(*(poison(x) for x in (dp.q, dp.qr, dp.do, dp.out, dp.smax, dp.ssum, dp.idx)))
+    for name, x, y in zip(("dQuery rows", "dQueryRope rows", "key-side accumulator"), got, clean):
+        assert torch.equal(x, y), f"{case}: {name} depend on rows outside the range"
+
+
 def test_balanced_split_of_real_counts():
     """The bench's work split on a causal problem: contiguous, covering, boundaries on even rows
     (row pairs stay together) and balanced within three rows."""
