@@ -45,6 +45,7 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 PROFILE_SUMMARIES = {
     4: ("sfa_bwd_pair_kernel_workload4.md", ("sfa_pair.cu", "tc_common.cuh")),
     3: ("sfa_bwd_fused_kernel_workload3.md", ("sfa_fused.cu", "tc_common.cuh")),
+    5: ("sfa_bwd_fused_kernel_workload5.md", ("sfa_fused.cu", "tc_common.cuh")),
     2: ("fa_bwd_fused_kernel_workload2.md", ("fa_fused.cu", "tc_common.cuh")),
     "fwd4": ("sfa_fwd_fused_kernel_workload4.md", ("sfa_fwd_fused.cu", "tc_common.cuh")),
     "lig": ("lig_fused_kernel_indexer.md", ("lig_fused.cu", "tc_common.cuh")),
@@ -138,14 +139,14 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-SEQS = None  # optional override of workload 4's sequence lengths (--seqs, for profiling captures)
+SEQS = None  # optional smaller case of workload 4 or 5 (--seqs, for profiling captures)
 
 
 def build_problem(workload: int, seed_offset: int, device):
     from workloads import make_device_problem
     p = make_device_problem(workload, device=device,
                             seed=None if seed_offset == 0 else 2000 + workload + 7919 * seed_offset,
-                            seqs=SEQS if workload == 4 else None)
+                            seqs=SEQS if workload in (4, 5) else None)
     return p
 
 
@@ -734,7 +735,8 @@ def main():
                     help="time the dense lightning-indexer gradient with KL loss (lig_kl_grad)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqs", default=None,
-                    help="comma-separated sequence lengths replacing workload 4's (smaller profiling case)")
+                    help="smaller profiling case: comma-separated sequence lengths replacing workload 4's, "
+                         "or workload 5's sequence length (topk scaled with it)")
     args = ap.parse_args()
     global SEQS
     if args.seqs:

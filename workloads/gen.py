@@ -302,8 +302,9 @@ def make_device_problem(cfg: int, device="cuda", seed: Optional[int] = None, seq
     """Workloads 3, 4, 5 generated directly on the device as torch tensors in the
     library's layouts (q [B,S1,N1,D] or [T1,N1,D], key [..,1,D], indices
     [..,1,topk]); value is key.  Seed defaults to 2000 + cfg.  `seqs` replaces
-    workload 4's sequence lengths (a smaller case of the same shape, used for
-    profiling captures)."""
+    workload 4's sequence lengths, or workload 5's sequence length S (topk scaled
+    with it, 8192 * S / 32768, so every row keeps its share of selected keys): a
+    smaller case of the same shape, used for profiling captures."""
     gen = torch.Generator(device=device)
     gen.manual_seed(2000 + cfg if seed is None else seed)
     D, Dr = 512, 64
@@ -316,6 +317,9 @@ def make_device_problem(cfg: int, device="cuda", seed: Optional[int] = None, seq
         layout = "TND"
     elif cfg == 5:
         B, S, N1, topk, bs = 1, 32768, 128, 8192, 1
+        if seqs is not None:
+            S = int(seqs[0])
+            topk = max(1, 8192 * S // 32768)
         layout, lens = "BSND", None
     else:
         raise ValueError(cfg)
