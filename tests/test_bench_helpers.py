@@ -36,3 +36,22 @@ def test_pairs_need_identical_live_blocks_in_one_sequence():
 def test_empty_rows_never_pair():
     S = fake([[0], [0]], [0, 0], [0, 0])
     assert bench.paired_work_fraction(problem("BSND", S1=2, topk=1), S) == 0.0
+
+
+def test_smaller_workload5_case_keeps_each_rows_share():
+    """`bench.py --workload 5 --seqs S` (profiling captures): S1 = S2 = S and topk scaled with S, so
+    row t still selects min(t + 1, topk) distinct causal keys, padded with -1 — the full workload's
+    recipe at a quarter (or any fraction) of its size."""
+    from workloads import make_device_problem
+    S = 1024
+    p = make_device_problem(5, device="cpu", seqs=[S])
+    topk = 8192 * S // 32768
+    assert p.layout == "BSND" and p.block_size == 1 and not p.deterministic
+    assert tuple(p.indices.shape) == (1, S, 1, topk) and tuple(p.q.shape) == (1, S, 128, 512)
+    idx = p.indices.reshape(S, topk)
+    for t in (0, 1, topk - 2, topk - 1, topk, S // 2, S - 1):
+        row = idx[t]
+        live = row[row >= 0]
+        assert live.numel() == min(t + 1, topk), t
+        assert bool((row[live.numel():] == -1).all()), t
+        assert int(live.max()) <= t and live.unique().numel() == live.numel(), t
